@@ -1,0 +1,154 @@
+/*
+ * dsa.h — C ABI of the B200 (sm_100a) DeepSeek Sparse Attention hot path.
+ *
+ * The method (DeepSeek-V3.2-Exp): a lightning indexer scores every causal
+ * (query t, key s) pair with a few FP8 heads, a fine-grained selection keeps
+ * the top-k keys per query, and multi-query attention runs over only those
+ * entries of the MLA latent cache ("DeepSeek-V3.2-Exp解析", dtcms.com, section
+ * 一.1, the three-stage workflow; "Lightning Indexer 的计算过程", adg.csdn.net/
+ * 695234..., steps 1-4).
+ *
+ * Conventions for every call:
+ *  - All array arguments are DEVICE pointers (CUDA global memory of the
+ *    current device), row-major, owned by the caller. The library never
+ *    allocates, frees or keeps them. Arrays must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream). Calls only
+ *    enqueue work; they return before it runs.
+ *  - The return value reports argument validation and launch errors; nothing
+ *    is enqueued unless it is DSA_OK. A kernel that gives up on an internal
+ *    wait (bounded, about a second) records a code that dsa_get_device_error()
+ *    reads. Indices outside [0, rows) given to the attention calls are
+ *    skipped and reported the same way.
+ *  - e4m3 = OCP FP8 E4M3 ("fn": no infinities), one byte per value.
+ *    bf16 = bfloat16 bits, two bytes per value.
+ *  - Supported shapes: H_I in {8, 64} and d_I in {64, 128} for prefill,
+ *    H_I = 64 and d_I in {64, 128} for decode; 1 <= topk <= 2048;
+ *    Hq in [1, 128]; the latent row is 576 values (512 + 64 RoPE) and the
+ *    value is its first 512. Other shapes return DSA_ERR_UNSUPPORTED.
+ */
+#ifndef DSA_B200_H
+#define DSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = -1, /* null pointer, negative size, misaligned array */
+  DSA_ERR_UNSUPPORTED = -2, /* shape outside the supported set */
+  DSA_ERR_CUDA = -3,        /* a CUDA call or launch failed (see dsa_last_error) */
+  DSA_ERR_TIMEOUT = -4,     /* reported by dsa_get_device_error: a kernel gave up on a wait */
+  DSA_ERR_WORKSPACE = -5,   /* workspace null or smaller than the *_workspace_size() result */
+  DSA_ERR_BAD_INDEX = -6    /* reported by dsa_get_device_error: an index outside its cache */
+} dsa_status;
+
+/* Latent row geometry of the MLA cache (576 = 512 latent + 64 RoPE values). */
+#define DSA_D_QK 576
+#define DSA_D_V 512
+#define DSA_MAX_TOPK 2048
+
+/* ------------------------------------------------------------------------
+ * Prefill indexer + top-k.
+ *
+ * For one causal sequence of L tokens ("Lightning Indexer 的计算过程" steps 3-4;
+ * deepseek.csdn.net section 2.2 细粒度词元选择):
+ *   I[t,s] = q_scale[t] * k_scale[s] * sum_j w[t,j] * ReLU(e4m3(q_I[t,j,:]) . e4m3(k_cache[s,:]))
+ * for s <= t, and idx[t, 0..topk) = the min(topk, t+1) keys s <= t with the
+ * largest I[t,s], ordered by (I descending, s ascending), then -1.
+ *
+ *   q_I      [L, H_I, d_I] e4m3     indexer queries (post-RoPE, quantised per token)
+ *   q_scale  [L] f32 (> 0)          per-token query scale
+ *   w        [L, H_I] f32           per-head weights (any sign)
+ *   k_cache  [L, d_I] e4m3          indexer keys (one key shared by all heads)
+ *   k_scale  [L] f32 (> 0)          per-token key scale
+ *   idx      [L, topk] int32        output
+ *   workspace, ws_bytes             device scratch of at least
+ *                                   dsa_index_topk_workspace_size(L, H_I, d_I, topk)
+ *                                   bytes; its contents are not kept between calls.
+ * The L x L score matrix is never formed: scores are streamed into per-row
+ * candidate lists bounded by the workspace size.
+ * ------------------------------------------------------------------------ */
+size_t dsa_index_topk_workspace_size(int L, int H_I, int d_I, int topk);
+
+dsa_status dsa_index_topk(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
+                          const float* k_scale, int L, int H_I, int d_I, int topk, int32_t* idx, void* workspace,
+                          size_t ws_bytes, void* stream);
+
+/* Test hook: the same kernel's fp32 scores for query rows [row0, row0+nrows),
+ * written to scores[nrows, L] (row r is query t = row0 + r; entries s > t are
+ * -INFINITY). Bit-identical to the values the selection of dsa_index_topk
+ * ranks. Needs no workspace. */
+dsa_status dsa_index_scores(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
+                            const float* k_scale, int L, int H_I, int d_I, int row0, int nrows, float* scores,
+                            void* stream);
+
+/* ------------------------------------------------------------------------
+ * Sparse MQA attention over the MLA latent cache (prefill).
+ *
+ * For every query token t and head h (deepseek.csdn.net section 2.2; the
+ * 576-value latent row of yudonglee.me "DeepSeek-V3.2 explained" section 2.4):
+ *   z_s = scale * q[t,h,:] . kv[s,:]          for s in idx[t,:], s >= 0
+ *   out[t,h,:] = sum_s softmax(z)_s * kv[s, 0:512]   (bf16 out, fp32 math)
+ *   lse[t,h] = log(sum_s exp(z_s))            (natural log; -inf if no entry)
+ * All heads share each selected row. Entries < 0 are skipped.
+ *
+ *   q        [T, Hq, 576] bf16
+ *   kv       [L, 576] bf16         latent cache rows
+ *   idx      [T, topk] int32       rows of kv (-1 = none)
+ *   out      [T, Hq, 512] bf16     output
+ *   lse      [T, Hq] f32 or NULL
+ * No workspace.
+ * ------------------------------------------------------------------------ */
+dsa_status dsa_sparse_mla_attn(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int T, int L, int Hq,
+                               int topk, float scale, uint16_t* out, float* lse, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Decode: B sequences, one new query each, at position t = lens[b]-1 of its
+ * own cache (the new token's key and latent row are already cached). Caches
+ * are strided by L_max tokens per sequence. Same definitions as prefill with
+ * t = lens[b]-1 (the decode curve of adg.csdn.net/695234..., figure (b)).
+ *
+ *   q_I      [B, H_I, d_I] e4m3     q_scale [B] f32     w [B, H_I] f32
+ *   k_cache  [B, L_max, d_I] e4m3   k_scale [B, L_max] f32
+ *   lens     [B] int32 (device), 1 <= lens[b] <= L_max
+ *   idx      [B, topk] int32 out    (rows of sequence b's own cache)
+ *   workspace                       >= dsa_index_topk_decode_workspace_size(B, L_max, topk)
+ *                                   bytes: the per-key scores and the selection.
+ * ------------------------------------------------------------------------ */
+size_t dsa_index_topk_decode_workspace_size(int B, int L_max, int topk);
+
+dsa_status dsa_index_topk_decode(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
+                                 const float* k_scale, const int32_t* lens, int B, int L_max, int H_I, int d_I,
+                                 int topk, int32_t* idx, void* workspace, size_t ws_bytes, void* stream);
+
+/* Test hook: decode scores[B, L_max] f32 (entries s >= lens[b] untouched). */
+dsa_status dsa_index_scores_decode(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
+                                   const float* k_scale, const int32_t* lens, int B, int L_max, int H_I, int d_I,
+                                   float* scores, void* stream);
+
+/*   q [B, Hq, 576] bf16, kv [B, L_max, 576] bf16, idx [B, topk] int32 (rows of
+ *   sequence b's cache, -1 = none), out [B, Hq, 512] bf16, lse [B, Hq] f32 or NULL. */
+dsa_status dsa_sparse_mla_attn_decode(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int L_max,
+                                      int Hq, int topk, float scale, uint16_t* out, float* lse, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Errors.
+ * ------------------------------------------------------------------------ */
+/* Synchronises `stream`, then reads and clears the device error word of the
+ * current device: DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_BAD_INDEX (*detail gets
+ * the raw word, may be NULL); DSA_ERR_CUDA if the synchronisation fails. */
+dsa_status dsa_get_device_error(void* stream, unsigned int* detail);
+
+const char* dsa_status_string(dsa_status s);
+/* Message of the last failing call on this host thread ("" if none). */
+const char* dsa_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_B200_H */

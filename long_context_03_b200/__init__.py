@@ -1,0 +1,244 @@
+"""B200 (sm_100a) DeepSeek Sparse Attention hot path: thin Python binding.
+
+Every call here marshals torch CUDA tensors into the C ABI of
+libdsa_b200.so (declared in include/dsa.h) and nothing else: the indexer, the
+selection and the attention all run in the library's CUDA kernels. PyTorch
+only provides device memory and the current stream. There is no CPU fallback:
+if the library is missing or fails to load, every call raises.
+
+Build the library first with `python -m long_context_03_b200.build` (or
+`__graft_entry__.build()`).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdsa_b200.so")
+
+D_QK = 576
+D_V = 512
+MAX_TOPK = 2048
+
+STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported shape", -3: "CUDA error",
+          -4: "device wait timed out", -5: "workspace too small", -6: "index outside the cache"}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class DSAError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded CUDA library (raises if it was not built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m long_context_03_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            P, I, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+            L.dsa_index_topk_workspace_size.argtypes = [I, I, I, I]
+            L.dsa_index_topk_workspace_size.restype = SZ
+            L.dsa_index_topk.argtypes = [P, P, P, P, P, I, I, I, I, P, P, SZ, P]
+            L.dsa_index_scores.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P]
+            L.dsa_sparse_mla_attn.argtypes = [P, P, P, I, I, I, I, F, P, P, P]
+            L.dsa_index_topk_decode_workspace_size.argtypes = [I, I, I]
+            L.dsa_index_topk_decode_workspace_size.restype = SZ
+            L.dsa_index_topk_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P, P, SZ, P]
+            L.dsa_index_scores_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, P, P]
+            L.dsa_sparse_mla_attn_decode.argtypes = [P, P, P, I, I, I, I, F, P, P, P]
+            L.dsa_get_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_uint)]
+            L.dsa_status_string.argtypes = [I]
+            L.dsa_status_string.restype = ctypes.c_char_p
+            L.dsa_last_error.argtypes = []
+            L.dsa_last_error.restype = ctypes.c_char_p
+            for name in ("dsa_index_topk", "dsa_index_scores", "dsa_sparse_mla_attn", "dsa_index_topk_decode",
+                         "dsa_index_scores_decode", "dsa_sparse_mla_attn_decode", "dsa_get_device_error"):
+                getattr(L, name).restype = I
+            _lib = L
+    return _lib
+
+
+def _check(status: int):
+    if status != 0:
+        raise DSAError(status, lib().dsa_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _req(t: torch.Tensor, name: str, dtype, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _u8(t: torch.Tensor) -> torch.Tensor:
+    return t.view(torch.uint8) if t.dtype == torch.float8_e4m3fn else t
+
+
+# ----------------------------------------------------------------- prefill
+
+def index_topk_workspace_size(L: int, H_I: int, d_I: int, topk: int) -> int:
+    return int(lib().dsa_index_topk_workspace_size(L, H_I, d_I, topk))
+
+
+def index_topk(q_I, q_scale, w, k_cache, k_scale, topk: int, *, idx=None, workspace=None) -> torch.Tensor:
+    """Prefill indexer + top-k: idx [L, topk] int32 (ranked, -1 padded)."""
+    q_I, k_cache = _u8(q_I), _u8(k_cache)
+    L, H_I, d_I = q_I.shape
+    _req(q_I, "q_I", torch.uint8)
+    _req(q_scale, "q_scale", torch.float32, (L,))
+    _req(w, "w", torch.float32, (L, H_I))
+    _req(k_cache, "k_cache", torch.uint8, (L, d_I))
+    _req(k_scale, "k_scale", torch.float32, (L,))
+    if idx is None:
+        idx = torch.empty((L, topk), dtype=torch.int32, device=q_I.device)
+    _req(idx, "idx", torch.int32, (L, topk))
+    need = index_topk_workspace_size(L, H_I, d_I, topk)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q_I.device)
+    _check(lib().dsa_index_topk(_ptr(q_I), _ptr(q_scale), _ptr(w), _ptr(k_cache), _ptr(k_scale), L, H_I, d_I,
+                                topk, _ptr(idx), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _stream(q_I.device)))
+    return idx
+
+
+def index_scores(q_I, q_scale, w, k_cache, k_scale, row0: int = 0, nrows: Optional[int] = None,
+                 *, scores=None) -> torch.Tensor:
+    """Test hook: the GPU's own fp32 scores [nrows, L] for rows row0.. (-inf for s > t)."""
+    q_I, k_cache = _u8(q_I), _u8(k_cache)
+    L, H_I, d_I = q_I.shape
+    if nrows is None:
+        nrows = L - row0
+    _req(q_I, "q_I", torch.uint8)
+    _req(q_scale, "q_scale", torch.float32, (L,))
+    _req(w, "w", torch.float32, (L, H_I))
+    _req(k_cache, "k_cache", torch.uint8, (L, d_I))
+    _req(k_scale, "k_scale", torch.float32, (L,))
+    if scores is None:
+        scores = torch.empty((nrows, L), dtype=torch.float32, device=q_I.device)
+    _req(scores, "scores", torch.float32, (nrows, L))
+    _check(lib().dsa_index_scores(_ptr(q_I), _ptr(q_scale), _ptr(w), _ptr(k_cache), _ptr(k_scale), L, H_I, d_I,
+                                  row0, nrows, _ptr(scores), _stream(q_I.device)))
+    return scores
+
+
+def sparse_mla_attn(q, kv, idx, scale: float, *, out=None, lse=None, want_lse: bool = False
+                    ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Sparse MQA over the latent cache: out [T, Hq, 512] bf16 (and lse [T, Hq] f32)."""
+    T, Hq, D = q.shape
+    L = kv.shape[0]
+    topk = idx.shape[1]
+    _req(q, "q", torch.bfloat16, (T, Hq, D_QK))
+    _req(kv, "kv", torch.bfloat16, (L, D_QK))
+    _req(idx, "idx", torch.int32, (T, topk))
+    if out is None:
+        out = torch.empty((T, Hq, D_V), dtype=torch.bfloat16, device=q.device)
+    _req(out, "out", torch.bfloat16, (T, Hq, D_V))
+    if lse is None and want_lse:
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _req(lse, "lse", torch.float32, (T, Hq))
+    _check(lib().dsa_sparse_mla_attn(_ptr(q), _ptr(kv), _ptr(idx), T, L, Hq, topk, float(scale), _ptr(out),
+                                     _ptr(lse), _stream(q.device)))
+    return out, lse
+
+
+# ------------------------------------------------------------------ decode
+
+def index_topk_decode_workspace_size(B: int, L_max: int, topk: int) -> int:
+    return int(lib().dsa_index_topk_decode_workspace_size(B, L_max, topk))
+
+
+def _req_decode(q_I, q_scale, w, k_cache, k_scale, lens):
+    B, H_I, d_I = q_I.shape
+    L_max = k_cache.shape[1]
+    _req(q_I, "q_I", torch.uint8)
+    _req(q_scale, "q_scale", torch.float32, (B,))
+    _req(w, "w", torch.float32, (B, H_I))
+    _req(k_cache, "k_cache", torch.uint8, (B, L_max, d_I))
+    _req(k_scale, "k_scale", torch.float32, (B, L_max))
+    _req(lens, "lens", torch.int32, (B,))
+    return B, H_I, d_I, L_max
+
+
+def index_topk_decode(q_I, q_scale, w, k_cache, k_scale, lens, topk: int, *, idx=None, workspace=None):
+    """Decode indexer + top-k: idx [B, topk] int32 (rows of each sequence's cache)."""
+    q_I, k_cache = _u8(q_I), _u8(k_cache)
+    B, H_I, d_I, L_max = _req_decode(q_I, q_scale, w, k_cache, k_scale, lens)
+    if idx is None:
+        idx = torch.empty((B, topk), dtype=torch.int32, device=q_I.device)
+    _req(idx, "idx", torch.int32, (B, topk))
+    need = index_topk_decode_workspace_size(B, L_max, topk)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q_I.device)
+    _check(lib().dsa_index_topk_decode(_ptr(q_I), _ptr(q_scale), _ptr(w), _ptr(k_cache), _ptr(k_scale),
+                                       _ptr(lens), B, L_max, H_I, d_I, topk, _ptr(idx), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _stream(q_I.device)))
+    return idx
+
+
+def index_scores_decode(q_I, q_scale, w, k_cache, k_scale, lens, *, scores=None) -> torch.Tensor:
+    """Test hook: decode fp32 scores [B, L_max] (entries s >= lens[b] are left as allocated)."""
+    q_I, k_cache = _u8(q_I), _u8(k_cache)
+    B, H_I, d_I, L_max = _req_decode(q_I, q_scale, w, k_cache, k_scale, lens)
+    if scores is None:
+        scores = torch.full((B, L_max), float("-inf"), dtype=torch.float32, device=q_I.device)
+    _req(scores, "scores", torch.float32, (B, L_max))
+    _check(lib().dsa_index_scores_decode(_ptr(q_I), _ptr(q_scale), _ptr(w), _ptr(k_cache), _ptr(k_scale),
+                                         _ptr(lens), B, L_max, H_I, d_I, _ptr(scores), _stream(q_I.device)))
+    return scores
+
+
+def sparse_mla_attn_decode(q, kv, idx, scale: float, *, out=None, lse=None, want_lse: bool = False):
+    """Decode sparse MQA: q [B, Hq, 576], kv [B, L_max, 576] -> out [B, Hq, 512] bf16 (and lse)."""
+    B, Hq, D = q.shape
+    L_max = kv.shape[1]
+    topk = idx.shape[1]
+    _req(q, "q", torch.bfloat16, (B, Hq, D_QK))
+    _req(kv, "kv", torch.bfloat16, (B, L_max, D_QK))
+    _req(idx, "idx", torch.int32, (B, topk))
+    if out is None:
+        out = torch.empty((B, Hq, D_V), dtype=torch.bfloat16, device=q.device)
+    _req(out, "out", torch.bfloat16, (B, Hq, D_V))
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _req(lse, "lse", torch.float32, (B, Hq))
+    _check(lib().dsa_sparse_mla_attn_decode(_ptr(q), _ptr(kv), _ptr(idx), B, L_max, Hq, topk, float(scale),
+                                            _ptr(out), _ptr(lse), _stream(q.device)))
+    return out, lse
+
+
+def device_error(device=None) -> Tuple[int, int]:
+    """Synchronise the current stream and read/clear the device error word: (status, raw word)."""
+    detail = ctypes.c_uint(0)
+    st = lib().dsa_get_device_error(_stream(device), ctypes.byref(detail))
+    return int(st), int(detail.value)
+
+
+def check_device_error(device=None):
+    st, raw = device_error(device)
+    if st != 0:
+        raise DSAError(st, f"{lib().dsa_last_error().decode()} (raw {raw:#x})")

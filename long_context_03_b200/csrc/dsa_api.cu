@@ -1,0 +1,421 @@
+// C ABI of the DSA hot path (see include/dsa.h): argument checks, workspace
+// carving, TMA descriptors and kernel launches. One translation unit holds
+// every kernel so the device error word is a single symbol.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/dsa.h"
+#include "dsa_common.cuh"
+#include "indexer_decode.cuh"
+#include "indexer_prefill.cuh"
+#include "sparse_mla.cuh"
+#include "topk_select.cuh"
+
+using namespace dsa;
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+dsa_status fail(dsa_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+dsa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(DSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int num_sms() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int n = 0;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 1;
+}
+
+// ---- TMA descriptor encoding through the driver entry point ----
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D byte tensor [outer, inner] (row-major, rows of `inner` bytes), box
+// [box_outer, box_inner], swizzled to match the tensor-core layouts.
+dsa_status make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                       uint32_t box_outer) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw = (inner == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return DSA_OK;
+}
+
+template <typename K>
+dsa_status set_smem(K kernel, int bytes) {
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  return DSA_OK;
+}
+
+dsa_status check_launch(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return DSA_OK;
+}
+
+// ---- prefill indexer ----
+constexpr int kNetPrefill = 8 * 32;  // epilogue threads of the prefill indexer
+
+int select_maxper(int topk) { return (topk <= 128) ? 2 : 17; }
+int select_cap(int topk) { return select_maxper(topk) * kNetPrefill; }
+
+int rows_per_block(int H_I) { return 2 * (256 / H_I); }
+
+bool prefill_shape_ok(int H_I, int d_I) { return (H_I == 8 || H_I == 64) && (d_I == 64 || d_I == 128); }
+
+struct WsPrefill {
+  uint64_t* cand;
+  uint64_t* sel;
+  size_t bytes;
+};
+
+WsPrefill prefill_ws_layout(void* base, int L, int H_I, int topk, int grid) {
+  WsPrefill w;
+  const size_t cand_bytes = static_cast<size_t>(grid) * rows_per_block(H_I) * select_cap(topk) * 8;
+  const size_t sel_bytes = static_cast<size_t>(L) * topk * 8;
+  w.cand = reinterpret_cast<uint64_t*>(base);
+  w.sel = reinterpret_cast<uint64_t*>(reinterpret_cast<char*>(base) + cand_bytes);
+  w.bytes = cand_bytes + sel_bytes;
+  return w;
+}
+
+template <int HI, int DI, bool kSelect, int MAXPER>
+dsa_status launch_prefill(const uint8_t* q_I, const uint8_t* k_cache, const IdxPrefillParams& p, int grid,
+                          cudaStream_t st) {
+  using C = IdxPrefillCfg<HI, DI>;
+  CUtensorMap tmQ, tmK;
+  dsa_status s = make_map_u8(&tmQ, q_I, DI, static_cast<uint64_t>(p.L) * HI, DI, C::NCOL);
+  if (s != DSA_OK) return s;
+  s = make_map_u8(&tmK, k_cache, DI, static_cast<uint64_t>(p.L), DI, C::BM);
+  if (s != DSA_OK) return s;
+  auto kern = indexer_prefill_kernel<HI, DI, kSelect, MAXPER>;
+  s = set_smem(kern, C::SMEM_BYTES);
+  if (s != DSA_OK) return s;
+  kern<<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(tmQ, tmK, p);
+  return check_launch("indexer_prefill_kernel");
+}
+
+template <bool kSelect, int MAXPER>
+dsa_status dispatch_prefill(int H_I, int d_I, const uint8_t* q_I, const uint8_t* k_cache, const IdxPrefillParams& p,
+                            int grid, cudaStream_t st) {
+  if (H_I == 64 && d_I == 128) return launch_prefill<64, 128, kSelect, MAXPER>(q_I, k_cache, p, grid, st);
+  if (H_I == 64 && d_I == 64) return launch_prefill<64, 64, kSelect, MAXPER>(q_I, k_cache, p, grid, st);
+  if (H_I == 8 && d_I == 128) return launch_prefill<8, 128, kSelect, MAXPER>(q_I, k_cache, p, grid, st);
+  if (H_I == 8 && d_I == 64) return launch_prefill<8, 64, kSelect, MAXPER>(q_I, k_cache, p, grid, st);
+  return fail(DSA_ERR_UNSUPPORTED, "H_I=%d d_I=%d not supported", H_I, d_I);
+}
+
+dsa_status launch_rank_sort(const uint64_t* keys, int32_t* idx, int K, int rows, cudaStream_t st) {
+  if (rows <= 0) return DSA_OK;
+  if (K <= 64) rank_sort_kernel<64><<<rows, 256, 0, st>>>(keys, idx, K, rows);
+  else if (K <= 128) rank_sort_kernel<128><<<rows, 256, 0, st>>>(keys, idx, K, rows);
+  else if (K <= 256) rank_sort_kernel<256><<<rows, 256, 0, st>>>(keys, idx, K, rows);
+  else if (K <= 512) rank_sort_kernel<512><<<rows, 256, 0, st>>>(keys, idx, K, rows);
+  else if (K <= 1024) rank_sort_kernel<1024><<<rows, 256, 0, st>>>(keys, idx, K, rows);
+  else rank_sort_kernel<2048><<<rows, 256, 0, st>>>(keys, idx, K, rows);
+  return check_launch("rank_sort_kernel");
+}
+
+__global__ void fill_f32_kernel(float* p, size_t n, float v) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    p[i] = v;
+}
+
+// ---- decode ----
+
+template <int HI, int DI>
+dsa_status launch_decode_scores(const uint8_t* q_I, const uint8_t* k_cache, int B, const IdxDecodeParams& p,
+                                cudaStream_t st) {
+  using C = IdxDecodeCfg<HI, DI>;
+  CUtensorMap tmQ, tmK;
+  dsa_status s = make_map_u8(&tmQ, q_I, DI, static_cast<uint64_t>(B) * HI, DI, HI);
+  if (s != DSA_OK) return s;
+  s = make_map_u8(&tmK, k_cache, DI, static_cast<uint64_t>(B) * p.L_max, DI, C::BM);
+  if (s != DSA_OK) return s;
+  auto kern = indexer_decode_kernel<HI, DI>;
+  s = set_smem(kern, C::SMEM_BYTES);
+  if (s != DSA_OK) return s;
+  dim3 grid((p.L_max + C::CHUNK - 1) / C::CHUNK, B);
+  kern<<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(tmQ, tmK, p);
+  return check_launch("indexer_decode_kernel");
+}
+
+dsa_status decode_scores(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
+                         const float* k_scale, const int32_t* lens, int B, int L_max, int H_I, int d_I, float* scores,
+                         cudaStream_t st) {
+  IdxDecodeParams p;
+  p.q_scale = q_scale;
+  p.w = w;
+  p.k_scale = k_scale;
+  p.lens = lens;
+  p.L_max = L_max;
+  p.scores = scores;
+  if (H_I == 64 && d_I == 128) return launch_decode_scores<64, 128>(q_I, k_cache, B, p, st);
+  if (H_I == 64 && d_I == 64) return launch_decode_scores<64, 64>(q_I, k_cache, B, p, st);
+  return fail(DSA_ERR_UNSUPPORTED, "decode: H_I=%d d_I=%d not supported", H_I, d_I);
+}
+
+dsa_status check_decode_args(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
+                             const float* k_scale, const int32_t* lens, int B, int L_max, int H_I, int d_I) {
+  if (!q_I || !q_scale || !w || !k_cache || !k_scale || !lens) return fail(DSA_ERR_INVALID_ARG, "null pointer");
+  if (B <= 0 || L_max <= 0) return fail(DSA_ERR_INVALID_ARG, "B=%d L_max=%d", B, L_max);
+  if (!aligned16(q_I) || !aligned16(k_cache)) return fail(DSA_ERR_INVALID_ARG, "q_I / k_cache not 16-byte aligned");
+  if (!(H_I == 64 && (d_I == 64 || d_I == 128)))
+    return fail(DSA_ERR_UNSUPPORTED, "decode: H_I=%d d_I=%d not supported", H_I, d_I);
+  if (static_cast<long long>(B) * L_max >= (1ll << 31)) return fail(DSA_ERR_UNSUPPORTED, "B*L_max too large");
+  return DSA_OK;
+}
+
+// ---- attention ----
+dsa_status launch_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int T, int rows, long long kv_stride,
+                      int Hq, int topk, float scale, uint16_t* out, float* lse, cudaStream_t st) {
+  MlaParams p;
+  p.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  p.kv = reinterpret_cast<const __nv_bfloat16*>(kv);
+  p.idx = idx;
+  p.out = reinterpret_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.kv_token_stride = kv_stride;
+  p.rows = rows;
+  p.T = T;
+  p.Hq = Hq;
+  p.K = topk;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  dsa_status s = set_smem(sparse_mla_kernel, MlaCfg::SMEM_BYTES);
+  if (s != DSA_OK) return s;
+  static int max_clusters = 0;
+  if (max_clusters == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * 512, 1, 1);
+    cfg.blockDim = dim3(MlaCfg::NTHREADS, 1, 1);
+    cfg.dynamicSmemBytes = MlaCfg::SMEM_BYTES;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, sparse_mla_kernel, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = num_sms() / 2;
+    }
+    max_clusters = n;
+  }
+  const int nclusters = T < max_clusters ? T : max_clusters;
+  sparse_mla_kernel<<<2 * nclusters, MlaCfg::NTHREADS, MlaCfg::SMEM_BYTES, st>>>(p);
+  return check_launch("sparse_mla_kernel");
+}
+
+dsa_status check_mla_args(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int T, int L, int Hq, int topk,
+                          float scale, const uint16_t* out) {
+  if (!q || !kv || !idx || !out) return fail(DSA_ERR_INVALID_ARG, "null pointer");
+  if (T < 0 || L <= 0) return fail(DSA_ERR_INVALID_ARG, "T=%d L=%d", T, L);
+  if (!aligned16(q) || !aligned16(kv) || !aligned16(out) || !aligned16(idx))
+    return fail(DSA_ERR_INVALID_ARG, "q / kv / idx / out not 16-byte aligned");
+  if (Hq < 1 || Hq > 128) return fail(DSA_ERR_UNSUPPORTED, "Hq=%d not in [1, 128]", Hq);
+  if (topk < 1 || topk > DSA_MAX_TOPK) return fail(DSA_ERR_UNSUPPORTED, "topk=%d not in [1, %d]", topk, DSA_MAX_TOPK);
+  if (!std::isfinite(scale)) return fail(DSA_ERR_INVALID_ARG, "scale is not finite");
+  return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t dsa_index_topk_workspace_size(int L, int H_I, int d_I, int topk) {
+  if (L <= 0 || topk <= 0 || !prefill_shape_ok(H_I, d_I)) return 0;
+  const int nrb = (L + rows_per_block(H_I) - 1) / rows_per_block(H_I);
+  const int grid = nrb < num_sms() ? nrb : num_sms();
+  return prefill_ws_layout(nullptr, L, H_I, topk, grid).bytes;
+}
+
+dsa_status dsa_index_topk(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
+                          const float* k_scale, int L, int H_I, int d_I, int topk, int32_t* idx, void* workspace,
+                          size_t ws_bytes, void* stream) {
+  if (!q_I || !q_scale || !w || !k_cache || !k_scale || !idx) return fail(DSA_ERR_INVALID_ARG, "null pointer");
+  if (L <= 0) return fail(DSA_ERR_INVALID_ARG, "L=%d", L);
+  if (!prefill_shape_ok(H_I, d_I)) return fail(DSA_ERR_UNSUPPORTED, "H_I=%d d_I=%d not supported", H_I, d_I);
+  if (topk < 1 || topk > DSA_MAX_TOPK) return fail(DSA_ERR_UNSUPPORTED, "topk=%d not in [1, %d]", topk, DSA_MAX_TOPK);
+  if (static_cast<long long>(L) * H_I >= (1ll << 31)) return fail(DSA_ERR_UNSUPPORTED, "L*H_I too large");
+  if (!aligned16(q_I) || !aligned16(k_cache)) return fail(DSA_ERR_INVALID_ARG, "q_I / k_cache not 16-byte aligned");
+  const int rb = rows_per_block(H_I);
+  const int nrb = (L + rb - 1) / rb;
+  const int grid = nrb < num_sms() ? nrb : num_sms();
+  const WsPrefill ws = prefill_ws_layout(workspace, L, H_I, topk, grid);
+  if (!workspace || ws_bytes < ws.bytes)
+    return fail(DSA_ERR_WORKSPACE, "workspace %zu bytes, need %zu", ws_bytes, ws.bytes);
+  if (!aligned16(workspace)) return fail(DSA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  IdxPrefillParams p = {};
+  p.q_scale = q_scale;
+  p.w = w;
+  p.k_scale = k_scale;
+  p.L = L;
+  p.topk = topk;
+  p.rb_begin = 0;
+  p.rb_end = nrb;
+  p.cand = ws.cand;
+  p.cap = select_cap(topk);
+  p.sel_keys = ws.sel;
+  dsa_status s = (select_maxper(topk) == 2) ? dispatch_prefill<true, 2>(H_I, d_I, q_I, k_cache, p, grid, st)
+                                            : dispatch_prefill<true, 17>(H_I, d_I, q_I, k_cache, p, grid, st);
+  if (s != DSA_OK) return s;
+  return launch_rank_sort(ws.sel, idx, topk, L, st);
+}
+
+dsa_status dsa_index_scores(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
+                            const float* k_scale, int L, int H_I, int d_I, int row0, int nrows, float* scores,
+                            void* stream) {
+  if (!q_I || !q_scale || !w || !k_cache || !k_scale || !scores) return fail(DSA_ERR_INVALID_ARG, "null pointer");
+  if (L <= 0 || row0 < 0 || nrows < 0 || row0 + nrows > L)
+    return fail(DSA_ERR_INVALID_ARG, "L=%d row0=%d nrows=%d", L, row0, nrows);
+  if (!prefill_shape_ok(H_I, d_I)) return fail(DSA_ERR_UNSUPPORTED, "H_I=%d d_I=%d not supported", H_I, d_I);
+  if (!aligned16(q_I) || !aligned16(k_cache)) return fail(DSA_ERR_INVALID_ARG, "q_I / k_cache not 16-byte aligned");
+  if (nrows == 0) return DSA_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t n = static_cast<size_t>(nrows) * L;
+  fill_f32_kernel<<<1024, 256, 0, st>>>(scores, n, -INFINITY);
+  dsa_status s = check_launch("fill_f32_kernel");
+  if (s != DSA_OK) return s;
+  const int rb = rows_per_block(H_I);
+  IdxPrefillParams p = {};
+  p.q_scale = q_scale;
+  p.w = w;
+  p.k_scale = k_scale;
+  p.L = L;
+  p.topk = 1;
+  p.rb_begin = row0 / rb;
+  p.rb_end = (row0 + nrows + rb - 1) / rb;
+  p.scores = scores;
+  p.row0 = row0;
+  p.nrows = nrows;
+  const int nrb = p.rb_end - p.rb_begin;
+  const int grid = nrb < num_sms() ? nrb : num_sms();
+  return dispatch_prefill<false, 1>(H_I, d_I, q_I, k_cache, p, grid, st);
+}
+
+dsa_status dsa_sparse_mla_attn(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int T, int L, int Hq,
+                               int topk, float scale, uint16_t* out, float* lse, void* stream) {
+  dsa_status s = check_mla_args(q, kv, idx, T, L, Hq, topk, scale, out);
+  if (s != DSA_OK) return s;
+  if (T == 0) return DSA_OK;
+  return launch_mla(q, kv, idx, T, L, 0, Hq, topk, scale, out, lse, static_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_index_topk_decode_workspace_size(int B, int L_max, int topk) {
+  if (B <= 0 || L_max <= 0 || topk <= 0) return 0;
+  const size_t scores = (static_cast<size_t>(B) * L_max * 4 + 255) / 256 * 256;
+  return scores + static_cast<size_t>(B) * topk * 8;
+}
+
+dsa_status dsa_index_topk_decode(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
+                                 const float* k_scale, const int32_t* lens, int B, int L_max, int H_I, int d_I,
+                                 int topk, int32_t* idx, void* workspace, size_t ws_bytes, void* stream) {
+  dsa_status s = check_decode_args(q_I, q_scale, w, k_cache, k_scale, lens, B, L_max, H_I, d_I);
+  if (s != DSA_OK) return s;
+  if (!idx) return fail(DSA_ERR_INVALID_ARG, "null pointer");
+  if (topk < 1 || topk > DSA_MAX_TOPK) return fail(DSA_ERR_UNSUPPORTED, "topk=%d not in [1, %d]", topk, DSA_MAX_TOPK);
+  const size_t need = dsa_index_topk_decode_workspace_size(B, L_max, topk);
+  if (!workspace || ws_bytes < need) return fail(DSA_ERR_WORKSPACE, "workspace %zu bytes, need %zu", ws_bytes, need);
+  if (!aligned16(workspace)) return fail(DSA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* scores = reinterpret_cast<float*>(workspace);
+  uint64_t* sel = reinterpret_cast<uint64_t*>(reinterpret_cast<char*>(workspace) +
+                                              (static_cast<size_t>(B) * L_max * 4 + 255) / 256 * 256);
+  s = decode_scores(q_I, q_scale, w, k_cache, k_scale, lens, B, L_max, H_I, d_I, scores, st);
+  if (s != DSA_OK) return s;
+  decode_select_kernel<1024><<<B, 1024, 0, st>>>(scores, lens, L_max, topk, sel);
+  s = check_launch("decode_select_kernel");
+  if (s != DSA_OK) return s;
+  return launch_rank_sort(sel, idx, topk, B, st);
+}
+
+dsa_status dsa_index_scores_decode(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
+                                   const float* k_scale, const int32_t* lens, int B, int L_max, int H_I, int d_I,
+                                   float* scores, void* stream) {
+  dsa_status s = check_decode_args(q_I, q_scale, w, k_cache, k_scale, lens, B, L_max, H_I, d_I);
+  if (s != DSA_OK) return s;
+  if (!scores) return fail(DSA_ERR_INVALID_ARG, "null pointer");
+  return decode_scores(q_I, q_scale, w, k_cache, k_scale, lens, B, L_max, H_I, d_I, scores,
+                       static_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_sparse_mla_attn_decode(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int L_max,
+                                      int Hq, int topk, float scale, uint16_t* out, float* lse, void* stream) {
+  dsa_status s = check_mla_args(q, kv, idx, B, L_max, Hq, topk, scale, out);
+  if (s != DSA_OK) return s;
+  if (B == 0) return DSA_OK;
+  return launch_mla(q, kv, idx, B, L_max, static_cast<long long>(L_max) * DSA_D_QK, Hq, topk, scale, out, lse,
+                    static_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_get_device_error(void* stream, unsigned int* detail) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned int h = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&h, g_device_error, sizeof(h), 0, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "dsa_get_device_error");
+  if (detail) *detail = h;
+  if (h == 0) return DSA_OK;
+  const unsigned int zero = 0;
+  e = cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "dsa_get_device_error (clear)");
+  const unsigned int code = h & 0xFFu;
+  if (code == kErrTimeout) return fail(DSA_ERR_TIMEOUT, "a kernel gave up waiting (site %u)", h >> 8);
+  return fail(DSA_ERR_BAD_INDEX, "an attention index was outside its cache (site %u)", h >> 8);
+}
+
+const char* dsa_status_string(dsa_status s) {
+  switch (s) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARG: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED: return "unsupported shape";
+    case DSA_ERR_CUDA: return "CUDA error";
+    case DSA_ERR_TIMEOUT: return "device wait timed out";
+    case DSA_ERR_WORKSPACE: return "workspace too small";
+    case DSA_ERR_BAD_INDEX: return "index outside the cache";
+  }
+  return "unknown status";
+}
+
+const char* dsa_last_error(void) { return g_last_error; }
+
+}  // extern "C"

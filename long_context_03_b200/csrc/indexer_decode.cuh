@@ -1,0 +1,276 @@
+// Decode lightning indexer: B sequences, one new query token each, scored
+// against that sequence's cached FP8 keys, then an exact per-sequence top-k.
+//
+// Same score as the prefill indexer ("Lightning Indexer 的计算过程", step 3,
+// adg.csdn.net/695234...), for the single row t = lens[b]-1:
+//     I[b,s] = q_scale[b] * k_scale[b,s] * sum_j w[b,j] * ReLU(q8[b,j,:] . k8[b,s,:]),  s < lens[b].
+// The decode cost curve of "DeepSeek-V3.2-Exp" (adg.csdn.net/695234..., figure
+// (b) Decoding) is the regime here: one query per sequence, so the work is a
+// single pass over the key cache and HBM bandwidth is the bound.
+//
+// Scoring kernel: a CTA takes 1024 keys of one sequence, streams its 8 key
+// tiles through a 4-stage TMA ring, multiplies each against the sequence's
+// [H_I x d_I] query on the tensor core (M = 128 keys, N = H_I heads) and the
+// epilogue reduces the heads per key, writing one fp32 score per key to the
+// scores buffer. Several CTAs share an SM so enough loads are in flight to
+// cover HBM latency.
+//
+// Selection kernel: one CTA per sequence runs an exact radix select over the
+// 64-bit ranking keys (score, then lower index) of its scores and writes the
+// top-k keys unordered; rank_sort_kernel orders them.
+#pragma once
+
+#include "dsa_common.cuh"
+#include "topk_select.cuh"
+
+namespace dsa {
+
+template <int HI, int DI>
+struct IdxDecodeCfg {
+  static constexpr int BM = 128;
+  static constexpr int CHUNK = 1024;           // keys per CTA
+  static constexpr int NKT = CHUNK / BM;
+  static constexpr int KST = 4;
+  static constexpr int NACC = 2;
+  static constexpr int QBYTES = HI * DI;
+  static constexpr int KTILE_BYTES = BM * DI;
+  static constexpr int NTHREADS = 6 * 32;      // producer, MMA, 4 epilogue warps
+  static constexpr SwizzleMode SW = (DI == 128) ? kSw128 : kSw64;
+  static constexpr uint32_t SBO = 8 * DI;
+  static constexpr uint32_t IDESC = instr_desc(kFmtE4M3, 128, HI, false, false);
+  static constexpr int KSTEPS = DI / 32;
+  static constexpr int TMEM_COLS = 128;        // 2 x HI (<= 128) rounded to a power of two >= 32
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_Q = OFF_K + KST * KTILE_BYTES;
+  static constexpr int OFF_W = OFF_Q + ((QBYTES + 1023) / 1024) * 1024;
+  static constexpr int OFF_BAR = OFF_W + HI * 4;
+  static constexpr int NBAR = 1 + 2 * KST + 2 * NACC;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static_assert(HI % 16 == 0 && HI <= 64, "decode indexer: H_I must be 16, 32, 48 or 64");
+};
+
+struct IdxDecodeParams {
+  const float* q_scale;  // [B]
+  const float* w;        // [B, HI]
+  const float* k_scale;  // [B, L_max]
+  const int32_t* lens;   // [B]
+  int L_max;
+  float* scores;         // [B, L_max]; entries s >= lens[b] untouched
+};
+
+template <int HI, int DI>
+__global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS)
+    indexer_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                          const IdxDecodeParams p) {
+  using C = IdxDecodeCfg<HI, DI>;
+  const int b = blockIdx.y;
+  const int s0 = blockIdx.x * C::CHUNK;
+  const int n = p.lens[b];
+  if (s0 >= n) return;  // whole CTA, before any barrier or TMEM allocation
+  const int nkt = min(C::NKT, (n - s0 + C::BM - 1) / C::BM);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* k_s = smem + C::OFF_K;
+  uint8_t* q_s = smem + C::OFF_Q;
+  float* w_s = reinterpret_cast<float*>(smem + C::OFF_W);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = bars + 1 + C::KST;
+  uint64_t* acc_full = bars + 1 + 2 * C::KST;
+  uint64_t* acc_empty = bars + 1 + 2 * C::KST + C::NACC;
+  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  int* abort_s = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
+  const AbortFlag ab{abort_s};
+  const uint32_t warp = warp_id();
+  const uint32_t lane = lane_id();
+
+  if (threadIdx.x == 0) {
+    *abort_s = 0;
+    mbar_init(q_full, 1);
+    for (int i = 0; i < C::KST; ++i) {
+      mbar_init(k_full + i, 1);
+      mbar_init(k_empty + i, 1);
+    }
+    for (int i = 0; i < C::NACC; ++i) {
+      mbar_init(acc_full + i, 1);
+      mbar_init(acc_empty + i, 4);
+    }
+    fence_mbar_init();
+  }
+  for (int i = threadIdx.x; i < HI; i += blockDim.x) w_s[i] = p.w[static_cast<size_t>(b) * HI + i];
+  if (warp == 1) tmem_alloc(tmem_base_s, C::TMEM_COLS);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_s;
+  const size_t row0 = static_cast<size_t>(b) * p.L_max + s0;  // first key row of this CTA
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, C::QBYTES);
+      tma_load_2d(q_s, &tmQ, q_full, 0, b * HI);
+      for (int kt = 0; kt < nkt; ++kt) {
+        const int slot = kt % C::KST;
+        if (!mbar_wait(k_empty + slot, ((kt / C::KST) & 1) ^ 1, ab, 11)) break;
+        mbar_arrive_expect_tx(k_full + slot, C::KTILE_BYTES);
+        tma_load_2d(k_s + slot * C::KTILE_BYTES, &tmK, k_full + slot, 0, static_cast<int>(row0) + kt * C::BM);
+      }
+      // wait until the MMA has consumed every issued tile (copies landed)
+      for (int kt = max(0, nkt - C::KST); kt < nkt && !ab.raised(); ++kt)
+        mbar_wait(k_empty + kt % C::KST, (kt / C::KST) & 1, ab, 12);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      bool ok = mbar_wait(q_full, 0, ab, 13);
+      const uint32_t q_addr = smem_u32(q_s);
+      for (int kt = 0; kt < nkt && ok; ++kt) {
+        const int slot = kt % C::KST;
+        const int buf = kt % C::NACC;
+        if (!mbar_wait(k_full + slot, (kt / C::KST) & 1, ab, 14)) break;
+        if (!mbar_wait(acc_empty + buf, ((kt / C::NACC) & 1) ^ 1, ab, 15)) break;
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(k_s + slot * C::KTILE_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < C::KSTEPS; ++kk) {
+          const uint64_t ad = smem_desc(a_addr + kk * 32, 16, C::SBO, C::SW);
+          const uint64_t bd = smem_desc(q_addr + kk * 32, 16, C::SBO, C::SW);
+          mma_f8(tmem + buf * HI, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(acc_full + buf);
+        tc_commit(k_empty + slot);
+      }
+    }
+  } else {
+    const int quarter = static_cast<int>(warp & 3);
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    const float qs = p.q_scale[b];
+    for (int kt = 0; kt < nkt; ++kt) {
+      const int buf = kt % C::NACC;
+      const int s = s0 + kt * C::BM + quarter * 32 + static_cast<int>(lane);
+      const float ks = (s < n) ? p.k_scale[static_cast<size_t>(b) * p.L_max + s] : 0.f;
+      if (!mbar_wait(acc_full + buf, (kt / C::NACC) & 1, ab, 16)) break;
+      tc_fence_after();
+      float acc = 0.f;
+      if constexpr (HI % 32 == 0) {
+#pragma unroll
+        for (int h = 0; h < HI / 32; ++h) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_addr + buf * HI + h * 32, r);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) acc = __fmaf_rn(w_s[h * 32 + j], fmaxf(__uint_as_float(r[j]), 0.f), acc);
+        }
+      } else {
+        uint32_t r[16];
+        tmem_ld16(tmem + lane_addr + buf * HI, r);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) acc = __fmaf_rn(w_s[j], fmaxf(__uint_as_float(r[j]), 0.f), acc);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty + buf);
+      if (s < n) p.scores[static_cast<size_t>(b) * p.L_max + s] = __fmul_rn(__fmul_rn(acc, qs), ks);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// Exact top-k of one sequence's scores (one CTA of kThreads per sequence).
+// Radix select over ranking keys recomputed from (score, s) on every pass;
+// the scores stay in L2 between passes. Writes the k best keys of sequence b
+// (unordered, 0 where lens[b] < k) to sel_keys[b, 0..k).
+template <int kThreads>
+__global__ void __launch_bounds__(kThreads)
+    decode_select_kernel(const float* __restrict__ scores, const int32_t* __restrict__ lens, int L_max, int K,
+                         uint64_t* __restrict__ sel_keys) {
+  __shared__ int hist[256];
+  __shared__ int misc[4];
+  __shared__ unsigned long long mm[2];
+  const int b = blockIdx.x;
+  const int n = lens[b];
+  const float* sc = scores + static_cast<size_t>(b) * L_max;
+  uint64_t* dst = sel_keys + static_cast<size_t>(b) * K;
+  const int tid = threadIdx.x;
+  if (n <= K) {
+    for (int i = tid; i < K; i += kThreads) dst[i] = (i < n) ? rank_key(sc[i], static_cast<uint32_t>(i)) : 0ull;
+    return;
+  }
+  // common prefix of all keys
+  unsigned long long kmin = ~0ull, kmax = 0ull;
+  for (int i = tid; i < n; i += kThreads) {
+    const uint64_t k = rank_key(sc[i], static_cast<uint32_t>(i));
+    kmin = k < kmin ? k : kmin;
+    kmax = k > kmax ? k : kmax;
+  }
+  if (tid == 0) {
+    mm[0] = ~0ull;
+    mm[1] = 0ull;
+  }
+  __syncthreads();
+  atomicMin(&mm[0], kmin);
+  atomicMax(&mm[1], kmax);
+  __syncthreads();
+  const uint64_t diff = mm[0] ^ mm[1];
+  const int hi_bit = diff ? 63 - __clzll(static_cast<long long>(diff)) : 0;
+  int shift = hi_bit & ~7;
+  uint64_t prefix = (shift + 8 >= 64) ? 0ull : (static_cast<uint64_t>(mm[1]) >> (shift + 8)) << (shift + 8);
+  int remaining = K;
+  while (true) {
+    for (int i = tid; i < 256; i += kThreads) hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < n; i += kThreads) {
+      const uint64_t x = rank_key(sc[i], static_cast<uint32_t>(i));
+      if ((shift + 8 >= 64) || ((x >> (shift + 8)) == (prefix >> (shift + 8))))
+        atomicAdd(&hist[(x >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    if (tid < 32) {
+      int c[8];
+      int tot = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        c[i] = hist[255 - 8 * tid - i];
+        tot += c[i];
+      }
+      int incl = tot;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (tid >= off) incl += y;
+      }
+      const uint32_t ball = __ballot_sync(0xffffffffu, incl >= remaining);
+      if (tid == __ffs(ball) - 1) {
+        int cum = incl - tot;
+        for (int i = 0; i < 8; ++i) {
+          if (cum + c[i] >= remaining) {
+            misc[0] = 255 - 8 * tid - i;
+            misc[1] = cum;
+            misc[2] = c[i];
+            break;
+          }
+          cum += c[i];
+        }
+      }
+    }
+    __syncthreads();
+    const int d = misc[0], above = misc[1], inb = misc[2];
+    remaining -= above;
+    prefix |= static_cast<uint64_t>(d) << shift;
+    __syncthreads();
+    if (inb == remaining || shift == 0) break;
+    shift -= 8;
+  }
+  if (tid == 0) misc[3] = 0;
+  __syncthreads();
+  for (int i = tid; i < n; i += kThreads) {
+    const uint64_t x = rank_key(sc[i], static_cast<uint32_t>(i));
+    if (x >= prefix) dst[atomicAdd(&misc[3], 1)] = x;
+  }
+}
+
+}  // namespace dsa

@@ -1,0 +1,350 @@
+// Prefill lightning indexer with the top-k selection streamed into its
+// epilogue, for one causal sequence of L tokens.
+//
+// The score ("Lightning Indexer 的计算过程", step 3 <1>-<2>, adg.csdn.net/695234...;
+// "DeepSeek-V3.2-Exp解析" section 一.1, dtcms.com):
+//     I[t,s] = q_scale[t] * k_scale[s] * sum_j w[t,j] * ReLU(q8[t,j,:] . k8[s,:]),  s <= t.
+// Scales are positive, so they are applied after the ReLU (equal in real
+// arithmetic to dequantising first). The FP8 products are exact and summed in
+// fp32 by the tensor core.
+//
+// Mapping onto tcgen05 (kind::f8f6f4, fp32 accumulator in TMEM):
+//   D[key, (token, head)] = K_tile[128 keys x d_I] * Q_half[(token, head) x d_I]^T
+// i.e. keys in M (128 TMEM lanes) and (token, head) in N (256 columns). Each
+// epilogue thread owns one key (one TMEM lane) and reduces the H_I heads of a
+// token inside its own registers: no shuffles. Two 256-column accumulators
+// alternate so the tensor core fills one while the epilogue drains the other.
+//
+// A CTA is persistent and owns "row blocks" of RB = 2 * 256 / H_I consecutive
+// query tokens, taken longest-first. For a row block it streams every key tile
+// up to the block's last token (TMA, 4-stage ring), so each key tile is reused
+// by RB tokens from shared memory.
+//
+// Selection (same page, step 4 <1>; deepseek.csdn.net section 2.2): each row
+// keeps a candidate list in the workspace, admitting a key only if its 64-bit
+// ranking key beats the row's threshold. When a list nears capacity it is cut
+// to exactly topk keys by a cooperative radix select and the threshold rises
+// to the cut. Nothing that could still rank in the top-k is ever dropped, and
+// the L x L score matrix never exists anywhere. At the end of a row block each
+// row's exact top-k keys go to `sel_keys` (unordered); rank_sort_kernel then
+// orders them.
+#pragma once
+
+#include "dsa_common.cuh"
+#include "topk_select.cuh"
+
+namespace dsa {
+
+template <int HI, int DI>
+struct IdxPrefillCfg {
+  static constexpr int BM = 128;               // keys per tile (MMA M, TMEM lanes)
+  static constexpr int NCOL = 256;             // accumulator columns per buffer (MMA N)
+  static constexpr int TB = NCOL / HI;         // tokens per accumulator buffer
+  static constexpr int NACC = 2;               // accumulator buffers
+  static constexpr int RB = TB * NACC;         // tokens per row block
+  static constexpr int KST = 4;                // key-tile ring depth
+  static constexpr int QBUF_BYTES = NCOL * DI; // one Q half: 256 (token, head) rows x d_I bytes
+  static constexpr int KTILE_BYTES = BM * DI;
+  static constexpr int NEPI = 8;               // epilogue warps (2 per TMEM lane quarter)
+  static constexpr int NTHREADS = (2 + NEPI) * 32;
+  static constexpr int NET = NEPI * 32;        // epilogue threads
+  static constexpr int TOK_PER_WARP = TB / 2;  // tokens of a buffer per epilogue warp
+  static constexpr SwizzleMode SW = (DI == 128) ? kSw128 : kSw64;
+  static constexpr uint32_t SBO = 8 * DI;      // bytes between 8-row core groups
+  static constexpr uint32_t IDESC = instr_desc(kFmtE4M3, 128, NCOL, false, false);
+  static constexpr int KSTEPS = DI / 32;       // MMA K = 32 for 8-bit inputs
+
+  // shared memory carve-up (offsets from a 1024-byte aligned base)
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + NACC * QBUF_BYTES;
+  static constexpr int OFF_W = OFF_K + KST * KTILE_BYTES;  // f32 [RB][HI]
+  static constexpr int OFF_QS = OFF_W + RB * HI * 4;       // f32 [RB]
+  static constexpr int OFF_THR = OFF_QS + RB * 4;          // u64 [RB]
+  static constexpr int OFF_CNT = OFF_THR + RB * 8;         // i32 [RB]
+  static constexpr int OFF_SCR = OFF_CNT + RB * 4;         // i32 [272] select scratch
+  static constexpr int OFF_BAR = (OFF_SCR + 272 * 4 + 7) / 8 * 8;
+  static constexpr int NBAR = 2 + 2 * KST + 2 * NACC;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;      // tmem base, abort flag
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+
+  static_assert(HI * TB == NCOL, "heads must divide 256");
+  static_assert(TB % 2 == 0, "two epilogue warps per lane quarter split a buffer's tokens");
+};
+
+struct IdxPrefillParams {
+  const float* q_scale;  // [L]
+  const float* w;        // [L, HI]
+  const float* k_scale;  // [L]
+  int L;
+  int topk;
+  int rb_begin, rb_end;  // row blocks [rb_begin, rb_end) of RB tokens
+  // selection mode
+  uint64_t* cand;        // [gridDim.x][RB][cap] candidate lists
+  int cap;
+  uint64_t* sel_keys;    // [L][topk] exact top-k keys per row, unordered, 0-padded
+  // score mode (test hook)
+  float* scores;         // [nrows][L]; rows t in [row0, row0 + nrows)
+  int row0, nrows;
+};
+
+// sum_j w[j] * max(x_j, 0) over the H_I accumulator columns of one token,
+// j ascending. Shared by both modes so their scores are bit-identical.
+template <int HI>
+__device__ __forceinline__ float relu_weighted_head_sum(uint32_t taddr, const float* __restrict__ w) {
+  float acc = 0.f;
+  if constexpr (HI % 32 == 0) {
+#pragma unroll
+    for (int h = 0; h < HI / 32; ++h) {
+      uint32_t r[32];
+      tmem_ld32(taddr + h * 32, r);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) acc = __fmaf_rn(w[h * 32 + j], fmaxf(__uint_as_float(r[j]), 0.f), acc);
+    }
+  } else {
+    static_assert(HI == 8, "H_I must be 8 or a multiple of 32");
+    uint32_t r[8];
+    tmem_ld8(taddr, r);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc = __fmaf_rn(w[j], fmaxf(__uint_as_float(r[j]), 0.f), acc);
+  }
+  return acc;
+}
+
+template <int HI, int DI, bool kSelect, int MAXPER>
+__global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
+    indexer_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                           const IdxPrefillParams p) {
+  using C = IdxPrefillCfg<HI, DI>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* q_s = smem + C::OFF_Q;
+  uint8_t* k_s = smem + C::OFF_K;
+  float* w_s = reinterpret_cast<float*>(smem + C::OFF_W);
+  float* qs_s = reinterpret_cast<float*>(smem + C::OFF_QS);
+  uint64_t* thr_s = reinterpret_cast<uint64_t*>(smem + C::OFF_THR);
+  int* cnt_s = reinterpret_cast<int*>(smem + C::OFF_CNT);
+  int* scr_s = reinterpret_cast<int*>(smem + C::OFF_SCR);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* k_full = bars + 2;
+  uint64_t* k_empty = bars + 2 + C::KST;
+  uint64_t* acc_full = bars + 2 + 2 * C::KST;
+  uint64_t* acc_empty = bars + 2 + 2 * C::KST + C::NACC;
+  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  int* abort_s = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
+  const AbortFlag ab{abort_s};
+
+  const uint32_t warp = warp_id();
+  const uint32_t lane = lane_id();
+
+  if (threadIdx.x == 0) {
+    *abort_s = 0;
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int i = 0; i < C::KST; ++i) {
+      mbar_init(k_full + i, 1);
+      mbar_init(k_empty + i, 1);
+    }
+    for (int i = 0; i < C::NACC; ++i) {
+      mbar_init(acc_full + i, 1);
+      mbar_init(acc_empty + i, C::NEPI);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+  }
+  if (warp == 1) tmem_alloc(tmem_base_s, 512);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_s;
+
+  const int nrb = p.rb_end - p.rb_begin;
+  const int G = gridDim.x;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      uint32_t qe_phase = 1;
+      int kslot = 0;
+      uint32_t ke_phase = 1;
+      for (int j = blockIdx.x; j < nrb; j += G) {
+        const int rb = p.rb_end - 1 - j;
+        const int t0 = rb * C::RB;
+        const int tlast = min(t0 + C::RB, p.L) - 1;
+        const int nkt = tlast / C::BM + 1;
+        if (!mbar_wait(q_empty, qe_phase, ab, 1)) break;
+        qe_phase ^= 1;
+        mbar_arrive_expect_tx(q_full, C::NACC * C::QBUF_BYTES);
+        for (int b = 0; b < C::NACC; ++b)
+          tma_load_2d(q_s + b * C::QBUF_BYTES, &tmQ, q_full, 0, (t0 + b * C::TB) * HI);
+        bool ok = true;
+        for (int kt = 0; kt < nkt; ++kt) {
+          if (!mbar_wait(k_empty + kslot, ke_phase, ab, 2)) { ok = false; break; }
+          mbar_arrive_expect_tx(k_full + kslot, C::KTILE_BYTES);
+          tma_load_2d(k_s + kslot * C::KTILE_BYTES, &tmK, k_full + kslot, 0, kt * C::BM);
+          if (++kslot == C::KST) { kslot = 0; ke_phase ^= 1; }
+        }
+        if (!ok) break;
+      }
+      // Drain: do not leave the CTA while a copy may still land in its
+      // shared memory (bounded, like every wait here).
+      for (int i = 0; i < C::KST; ++i) {
+        if (ab.raised()) break;
+        mbar_wait(k_empty + kslot, ke_phase, ab, 3);
+        if (++kslot == C::KST) { kslot = 0; ke_phase ^= 1; }
+      }
+      if (!ab.raised()) mbar_wait(q_empty, qe_phase, ab, 4);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      uint32_t qf_phase = 0;
+      int kslot = 0;
+      uint32_t kf_phase = 0;
+      uint32_t ae_phase[C::NACC];
+      for (int b = 0; b < C::NACC; ++b) ae_phase[b] = 1;
+      const uint32_t q_base = smem_u32(q_s);
+      const uint32_t k_base = smem_u32(k_s);
+      for (int j = blockIdx.x; j < nrb; j += G) {
+        const int rb = p.rb_end - 1 - j;
+        const int t0 = rb * C::RB;
+        const int tlast = min(t0 + C::RB, p.L) - 1;
+        const int nkt = tlast / C::BM + 1;
+        if (!mbar_wait(q_full, qf_phase, ab, 5)) break;
+        qf_phase ^= 1;
+        bool ok = true;
+        for (int kt = 0; kt < nkt && ok; ++kt) {
+          if (!mbar_wait(k_full + kslot, kf_phase, ab, 6)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = k_base + kslot * C::KTILE_BYTES;
+          for (int b = 0; b < C::NACC; ++b) {
+            if (!mbar_wait(acc_empty + b, ae_phase[b], ab, 7)) { ok = false; break; }
+            ae_phase[b] ^= 1;
+            tc_fence_after();
+            const uint32_t b_addr = q_base + b * C::QBUF_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < C::KSTEPS; ++kk) {
+              const uint64_t ad = smem_desc(a_addr + kk * 32, 16, C::SBO, C::SW);
+              const uint64_t bd = smem_desc(b_addr + kk * 32, 16, C::SBO, C::SW);
+              mma_f8(tmem + b * C::NCOL, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(acc_full + b);
+          }
+          tc_commit(k_empty + kslot);
+          if (++kslot == C::KST) { kslot = 0; kf_phase ^= 1; }
+        }
+        tc_commit(q_empty);
+        if (!ok) break;
+      }
+    }
+  } else {
+    // ---------------- epilogue: scores, threshold filter, selection ----------------
+    const int e = static_cast<int>(warp) - 2;          // 0..NEPI-1
+    const int et = e * 32 + static_cast<int>(lane);    // 0..NET-1
+    const int quarter = static_cast<int>(warp & 3);    // TMEM lane quarter this warp may access
+    const int half = e / 4;                            // which half of a buffer's tokens
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    uint32_t af_phase[C::NACC];
+    for (int b = 0; b < C::NACC; ++b) af_phase[b] = 0;
+    uint64_t* my_cand = p.cand + static_cast<size_t>(blockIdx.x) * C::RB * p.cap;
+
+    for (int j = blockIdx.x; j < nrb; j += G) {
+      const int rb = p.rb_end - 1 - j;
+      const int t0 = rb * C::RB;
+      const int tlast = min(t0 + C::RB, p.L) - 1;
+      const int nkt = tlast / C::BM + 1;
+      // per-row-block state
+      for (int i = et; i < C::RB * HI; i += C::NET) {
+        const int t = t0 + i / HI;
+        w_s[i] = (t < p.L) ? p.w[static_cast<size_t>(t) * HI + (i % HI)] : 0.f;
+      }
+      for (int i = et; i < C::RB; i += C::NET) {
+        const int t = t0 + i;
+        qs_s[i] = (t < p.L) ? p.q_scale[t] : 0.f;
+        thr_s[i] = 0ull;
+        cnt_s[i] = 0;
+      }
+      named_bar_sync(1, C::NET);
+      bool ok = true;
+      for (int kt = 0; kt < nkt && ok; ++kt) {
+        const int s = kt * C::BM + quarter * 32 + static_cast<int>(lane);
+        const float ks = (s < p.L) ? p.k_scale[s] : 0.f;
+        for (int b = 0; b < C::NACC; ++b) {
+          if (!mbar_wait(acc_full + b, af_phase[b], ab, 8)) { ok = false; break; }
+          af_phase[b] ^= 1;
+          tc_fence_after();
+#pragma unroll 1
+          for (int q = 0; q < C::TOK_PER_WARP; ++q) {
+            const int tt = half * C::TOK_PER_WARP + q;   // token within the buffer
+            const int tl = b * C::TB + tt;               // token within the row block
+            const int t = t0 + tl;
+            const float acc = relu_weighted_head_sum<HI>(tmem + lane_addr + b * C::NCOL + tt * HI, w_s + tl * HI);
+            const float score = __fmul_rn(__fmul_rn(acc, qs_s[tl]), ks);
+            const bool valid = (t < p.L) && (s <= t);
+            if constexpr (kSelect) {
+              const uint64_t key = rank_key(score, static_cast<uint32_t>(s));
+              const bool pred = valid && key > thr_s[tl];
+              const uint32_t m = __ballot_sync(0xffffffffu, pred);
+              if (m) {
+                const int leader = __ffs(m) - 1;
+                int base = 0;
+                if (static_cast<int>(lane) == leader) base = atomicAdd(cnt_s + tl, __popc(m));
+                base = __shfl_sync(0xffffffffu, base, leader);
+                if (pred) my_cand[static_cast<size_t>(tl) * p.cap + base + __popc(m & ((1u << lane) - 1u))] = key;
+              }
+            } else {
+              if (valid && t >= p.row0 && t < p.row0 + p.nrows)
+                p.scores[static_cast<size_t>(t - p.row0) * p.L + s] = score;
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(acc_empty + b);
+        }
+        if constexpr (kSelect) {
+          // Cut any list that could overflow on the next tile (at most BM
+          // appends per row per tile).
+          named_bar_sync(1, C::NET);
+          for (int tl = 0; tl < C::RB; ++tl) {
+            const int n = cnt_s[tl];
+            if (n > p.cap - C::BM) {
+              const uint64_t floor =
+                  compact_top_k<C::NET, MAXPER>(my_cand + static_cast<size_t>(tl) * p.cap, n, p.topk, scr_s, et, 1);
+              if (et == 0) {
+                cnt_s[tl] = p.topk;
+                thr_s[tl] = floor - 1;
+              }
+              named_bar_sync(1, C::NET);
+            }
+          }
+        }
+      }
+      if (!ok) break;
+      if constexpr (kSelect) {
+        named_bar_sync(1, C::NET);
+        for (int tl = 0; tl < C::RB; ++tl) {
+          const int t = t0 + tl;
+          if (t >= p.L) break;
+          uint64_t* c = my_cand + static_cast<size_t>(tl) * p.cap;
+          int n = cnt_s[tl];
+          if (n > p.topk) {
+            compact_top_k<C::NET, MAXPER>(c, n, p.topk, scr_s, et, 1);
+            n = p.topk;
+          }
+          uint64_t* dst = p.sel_keys + static_cast<size_t>(t) * p.topk;
+          for (int i = et; i < p.topk; i += C::NET) dst[i] = (i < n) ? c[i] : 0ull;
+        }
+      }
+      named_bar_sync(1, C::NET);
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace dsa

@@ -1,0 +1,538 @@
+// Sparse MQA attention over the selected rows of the MLA latent cache.
+//
+// For a query token t with heads h and selected rows S_t ("细粒度词元选择",
+// deepseek.csdn.net section 2.2: attention only over the top-k entries {c_s},
+// shared by every head; the 576-value latent row of yudonglee.me
+// "DeepSeek-V3.2 explained" section 2.4):
+//     z[h,s] = scale * Q[t,h,0:576] . C[s,0:576],   s in S_t
+//     u[t,h,:] = sum_s softmax_s(z[h,:]) * C[s, 0:512]
+// with fp32 softmax and accumulation, bf16 tensor-core inputs and a bf16 output.
+//
+// The fp32 output tile of one token (128 heads x 512 values) needs all 512
+// TMEM columns of an SM, so each token runs on a 2-CTA cluster:
+//   CTA 0 (score CTA): Q[t] lives in TMEM (288 columns, bf16 pairs) as the A
+//     operand. Per chunk of 32 selected rows it gathers the rows (cp.async,
+//     128-byte swizzled), runs S = Q C^T (M = 128 heads, N = 32 rows, K = 576),
+//     and its softmax warps (one thread per head) turn S into bf16
+//     probabilities P with a running reference max. The max is only moved
+//     when a chunk exceeds it by more than 2^8, so P <= 256 and the
+//     accumulator rarely needs rescaling. P, the per-head rescale factors and,
+//     after the last chunk, the row sums and maxima go to CTA 1 by a bulk
+//     shared-memory copy across the cluster.
+//   CTA 1 (value CTA): gathers the value part (first 512 values) of the same
+//     rows, rescales O when told to, and runs O += P V (M = 128 heads,
+//     N = 2 x 256 values, K = 32 rows) into its full TMEM. Its MMA commit
+//     signals CTA 0 directly (multicast commit) that the P buffer is free.
+//     After the last chunk it writes u = O / l in bf16 and the log-sum-exp.
+// A cluster is persistent over tokens. Work per chunk is balanced: 2*128*576
+// flops per row for QK^T, 2*128*512 for PV.
+//
+// Entries idx < 0 are skipped (probability 0). Entries >= the row bound are
+// also skipped and reported through the device error word.
+#pragma once
+
+#include "dsa_common.cuh"
+
+namespace dsa {
+
+struct MlaCfg {
+  static constexpr int D = 576;               // QK dims
+  static constexpr int DV = 512;              // value dims
+  static constexpr int NK = 32;               // selected rows per chunk
+  static constexpr int M = 128;               // heads per MMA (rows >= Hq are zero)
+  static constexpr int SLAB = 64;             // bf16 values per 128-byte swizzle row
+  static constexpr int NSLAB_QK = D / SLAB;   // 9
+  static constexpr int NSLAB_V = DV / SLAB;   // 8
+  static constexpr int SLAB_BYTES = NK * 128; // one slab of a chunk: 32 rows x 128 B
+  static constexpr int C_BYTES = NSLAB_QK * SLAB_BYTES;  // 36 KB
+  static constexpr int V_BYTES = NSLAB_V * SLAB_BYTES;   // 32 KB
+  static constexpr int NCST = 4;              // gather ring depth (score CTA)
+  static constexpr int NVST = 5;              // gather ring depth (value CTA)
+  static constexpr int NSB = 4;               // S buffers in TMEM
+  static constexpr int NPB = 2;               // P message buffers
+  static constexpr int P_BYTES = M * NK * 2;  // 8 KB, K-major, 64-byte swizzle
+  static constexpr int MSG_ALPHA = P_BYTES;           // f32 [128]
+  static constexpr int MSG_CTRL = MSG_ALPHA + M * 4;  // u32 [4]: any_rescale
+  static constexpr int MSG_L = MSG_CTRL + 16;         // f32 [128] (last chunk only)
+  static constexpr int MSG_M = MSG_L + M * 4;         // f32 [128] (last chunk only)
+  static constexpr int MSG_BYTES_MID = MSG_L;         // 8720
+  static constexpr int MSG_BYTES_LAST = MSG_M + M * 4;  // 9744
+  static constexpr int MSG_STRIDE = (MSG_BYTES_LAST + 1023) / 1024 * 1024;
+  static constexpr int NPROD = 4;             // producer warps
+  static constexpr int W_MMA = 4;
+  static constexpr int W_SM0 = 5;             // first softmax / epilogue warp
+  static constexpr int NTHREADS = 9 * 32;
+  static constexpr int S_COL = 0;             // S buffers: columns [0, NSB*NK)
+  static constexpr int Q_COL = 128;           // Q: columns [128, 416)
+  static constexpr uint32_t IDESC_QK = instr_desc(kFmtBF16, M, NK, false, false);
+  static constexpr uint32_t IDESC_PV = instr_desc(kFmtBF16, M, 256, false, true);
+  // shared memory (offsets from a 1024-aligned base); the two CTAs share the
+  // layout so barrier offsets match across the cluster
+  static constexpr int OFF_RING = 0;          // score CTA: NCST x C_BYTES; value CTA: NVST x V_BYTES
+  static constexpr int RING_BYTES = (NCST * C_BYTES > NVST * V_BYTES) ? NCST * C_BYTES : NVST * V_BYTES;
+  static constexpr int OFF_MSG = OFF_RING + RING_BYTES;  // NPB x MSG_STRIDE (staging / receive)
+  static constexpr int OFF_BAR = OFF_MSG + NPB * MSG_STRIDE;
+  // barriers
+  static constexpr int B_RING_FULL = 0;                  // [NVST]
+  static constexpr int B_RING_EMPTY = B_RING_FULL + NVST;  // [NVST]
+  static constexpr int B_S_FULL = B_RING_EMPTY + NVST;   // [NSB]  (score CTA)
+  static constexpr int B_S_EMPTY = B_S_FULL + NSB;       // [NSB]  (score CTA)
+  static constexpr int B_Q_READY = B_S_EMPTY + NSB;      // score CTA
+  static constexpr int B_Q_FREE = B_Q_READY + 1;         // score CTA
+  static constexpr int B_P_FREE = B_Q_FREE + 1;          // [NPB] score CTA, arrived by the value CTA's MMA
+  static constexpr int B_P_FULL = B_P_FREE + NPB;        // [NPB] value CTA, completed by the bulk copy
+  static constexpr int B_O_READY = B_P_FULL + NPB;       // [NPB] value CTA: correction done
+  static constexpr int B_PV_DONE = B_O_READY + NPB;      // value CTA: a token's last PV is done
+  static constexpr int B_STAGE = B_PV_DONE + 1;          // score CTA: softmax warps wrote the staging buffer
+  static constexpr int B_QUIESCE = B_STAGE + 1;          // value CTA: all PV issued so far complete
+  static constexpr int NBAR = B_QUIESCE + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 32;
+};
+
+struct MlaParams {
+  const __nv_bfloat16* q;    // [T, Hq, 576]
+  const __nv_bfloat16* kv;   // latent rows; token i reads kv + i*kv_token_stride
+  const int32_t* idx;        // [T, K]
+  __nv_bfloat16* out;        // [T, Hq, 512]
+  float* lse;                // [T, Hq] or null
+  long long kv_token_stride; // elements between consecutive tokens' caches (0: one shared cache)
+  int rows;                  // valid row bound of a token's cache
+  int T, Hq, K;
+  float scale_log2;          // softmax scale * log2(e)
+};
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t map_to_peer(uint32_t local_saddr, uint32_t peer) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_saddr), "r"(peer));
+  return r;
+}
+// Bulk copy local shared memory -> a cluster peer's shared memory, completing
+// (complete_tx) on the peer's mbarrier. Addresses 16-byte aligned, size % 16 == 0.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
+                                                  uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst_cluster),
+      "r"(src_cta), "r"(bytes), "r"(bar_cluster)
+      : "memory");
+}
+// Commit that arrives on the barrier at the same offset in each CTA of `mask`.
+__device__ __forceinline__ void tc_commit_mc(uint64_t* bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Gather rows [j*NK, j*NK+NK) of a token's selection into a 128-byte-swizzled
+// ring slot: slab s of row r at slot + s*SLAB_BYTES + r*128, 16-byte chunk c
+// stored at position c ^ (r & 7). `nslab` slabs (9 = full row, 8 = values).
+__device__ __forceinline__ void gather_chunk(uint32_t slot, const __nv_bfloat16* __restrict__ kv_tok,
+                                             const int32_t* __restrict__ idx_tok, int j, int K, int rows,
+                                             int nslab, int ptid) {
+  // 128 producer threads: 4 per row, each thread takes every 4th 16-byte chunk of its row
+  const int r = ptid >> 2;
+  const int e = j * MlaCfg::NK + r;
+  int row = (e < K) ? __ldg(idx_tok + e) : -1;
+  bool valid = row >= 0;
+  if (row >= rows) {
+    set_device_error(kErrBadIndex, 0);
+    valid = false;
+  }
+  const char* src_row = reinterpret_cast<const char*>(kv_tok + static_cast<long long>(valid ? row : 0) * MlaCfg::D);
+  const int nchunks = nslab * 8;
+  for (int c = (ptid & 3); c < nchunks; c += 4) {
+    const int s = c >> 3, cc = c & 7;
+    const uint32_t dst = slot + s * MlaCfg::SLAB_BYTES + r * 128 + ((cc ^ (r & 7)) << 4);
+    cp_async_16_zfill(dst, src_row + c * 16, valid);
+  }
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
+    sparse_mla_kernel(const MlaParams p) {
+  using C = MlaCfg;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  int* abort_s = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
+  int* rescale_s = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
+  const AbortFlag ab{abort_s};
+  const uint32_t rank = cluster_ctarank();
+  const uint32_t warp = warp_id();
+  const uint32_t lane = lane_id();
+  const int cluster_id = blockIdx.x >> 1;
+  const int nclusters = gridDim.x >> 1;
+  const int nchunk = (p.K + C::NK - 1) / C::NK;
+
+  if (threadIdx.x == 0) {
+    *abort_s = 0;
+    rescale_s[0] = 0;
+    rescale_s[1] = 0;
+    for (int i = 0; i < C::NVST; ++i) {
+      mbar_init(bars + C::B_RING_FULL + i, C::NPROD * 32);
+      mbar_init(bars + C::B_RING_EMPTY + i, 1);
+    }
+    for (int i = 0; i < C::NSB; ++i) {
+      mbar_init(bars + C::B_S_FULL + i, 1);
+      mbar_init(bars + C::B_S_EMPTY + i, 4);
+    }
+    mbar_init(bars + C::B_Q_READY, 4);
+    mbar_init(bars + C::B_Q_FREE, 1);
+    for (int i = 0; i < C::NPB; ++i) {
+      mbar_init(bars + C::B_P_FREE + i, 1);
+      mbar_init(bars + C::B_P_FULL + i, 1);
+      mbar_init(bars + C::B_O_READY + i, 4);
+    }
+    mbar_init(bars + C::B_PV_DONE, 1);
+    mbar_init(bars + C::B_STAGE, 4);
+    mbar_init(bars + C::B_QUIESCE, 1);
+    fence_mbar_init();
+  }
+  if (warp == C::W_MMA) tmem_alloc(tmem_base_s, 512);
+  __syncthreads();
+  // Value CTA: arm the first use of each P receive buffer before the peer can send.
+  if (rank == 1 && threadIdx.x == 0) {
+    const int total = ((p.T - 1 - cluster_id) / nclusters + 1) * nchunk;  // messages this cluster receives
+    for (int i = 0; i < C::NPB && i < total; ++i) {
+      const bool last = ((i % nchunk) == nchunk - 1);
+      mbar_arrive_expect_tx(bars + C::B_P_FULL + i, last ? C::MSG_BYTES_LAST : C::MSG_BYTES_MID);
+    }
+  }
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_s;
+  const uint32_t ring = smem_u32(smem + C::OFF_RING);
+  const uint32_t msg = smem_u32(smem + C::OFF_MSG);
+
+  if (rank == 0) {
+    // =========================== score CTA ===========================
+    if (warp < C::NPROD) {
+      const int ptid = threadIdx.x;
+      int slot = 0;
+      uint32_t ph = 1;
+      for (int tk = cluster_id; tk < p.T; tk += nclusters) {
+        const __nv_bfloat16* kv_tok = p.kv + tk * p.kv_token_stride;
+        const int32_t* idx_tok = p.idx + static_cast<size_t>(tk) * p.K;
+        bool ok = true;
+        for (int j = 0; j < nchunk; ++j) {
+          if (!mbar_wait(bars + C::B_RING_EMPTY + slot, ph, ab, 31)) { ok = false; break; }
+          gather_chunk(ring + slot * C::C_BYTES, kv_tok, idx_tok, j, p.K, p.rows, C::NSLAB_QK, ptid);
+          cp_async_mbar_arrive(bars + C::B_RING_FULL + slot);
+          if (++slot == C::NCST) { slot = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+      }
+      asm volatile("cp.async.wait_all;" ::: "memory");
+    } else if (warp == C::W_MMA) {
+      if (lane == 0) {
+        int slot = 0;
+        uint32_t ph = 0;
+        int sb = 0;
+        uint32_t sph = 1;
+        uint32_t qph = 0;
+        bool ok = true;
+        for (int tk = cluster_id; tk < p.T && ok; tk += nclusters) {
+          if (!mbar_wait(bars + C::B_Q_READY, qph, ab, 32)) break;
+          qph ^= 1;
+          tc_fence_after();
+          for (int j = 0; j < nchunk; ++j) {
+            if (!mbar_wait(bars + C::B_RING_FULL + slot, ph, ab, 33)) { ok = false; break; }
+            if (!mbar_wait(bars + C::B_S_EMPTY + sb, sph, ab, 34)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t cbase = ring + slot * C::C_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < C::D / 16; ++kk) {
+              const uint32_t baddr = cbase + (kk >> 2) * C::SLAB_BYTES + (kk & 3) * 32;
+              const uint64_t bd = smem_desc(baddr, 16, 1024, kSw128);
+              mma_bf16_ts(tmem + C::S_COL + sb * C::NK, tmem + C::Q_COL + kk * 8, bd, C::IDESC_QK,
+                          kk > 0 ? 1u : 0u);
+            }
+            tc_commit(bars + C::B_S_FULL + sb);
+            tc_commit(bars + C::B_RING_EMPTY + slot);
+            if (++slot == C::NCST) { slot = 0; ph ^= 1; }
+            if (++sb == C::NSB) { sb = 0; sph ^= 1; }
+          }
+          tc_commit(bars + C::B_Q_FREE);
+        }
+      }
+    } else {
+      // softmax warps: thread = head row (TMEM lane)
+      const int quarter = static_cast<int>(warp & 3);
+      const int h = quarter * 32 + static_cast<int>(lane);
+      const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+      const uint32_t peer_msg = map_to_peer(msg, 1);
+      const uint32_t peer_pfull = map_to_peer(smem_u32(bars + C::B_P_FULL), 1);
+      int sb = 0;
+      uint32_t sph = 0;
+      uint32_t qfree_ph = 1;
+      int pb = 0;
+      uint32_t pfree_ph = 1;
+      uint32_t stage_ph = 0;
+      bool ok = true;
+      for (int tk = cluster_id; tk < p.T && ok; tk += nclusters) {
+        // --- load Q[tk] into TMEM once the previous token's QK^T is done ---
+        if (!mbar_wait(bars + C::B_Q_FREE, qfree_ph, ab, 35)) break;
+        qfree_ph ^= 1;
+        tc_fence_after();
+        {
+          const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(tk) * p.Hq + h) * C::D);
+#pragma unroll 1
+          for (int cb = 0; cb < C::D / 64; ++cb) {  // 9 blocks of 32 columns (64 values)
+            uint32_t r[32];
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              uint4 x = make_uint4(0, 0, 0, 0);
+              if (h < p.Hq) x = __ldg(qrow + cb * 8 + v);
+              r[4 * v + 0] = x.x;
+              r[4 * v + 1] = x.y;
+              r[4 * v + 2] = x.z;
+              r[4 * v + 3] = x.w;
+            }
+            tmem_st32(tmem + lane_addr + C::Q_COL + cb * 32, r);
+          }
+          tmem_st_wait();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + C::B_Q_READY);
+        if (tk + nclusters < p.T && h == 0) {
+          // warm L2 with the next token's queries
+          const char* nq = reinterpret_cast<const char*>(p.q + static_cast<size_t>(tk + nclusters) * p.Hq * C::D);
+          const uint32_t qbytes = static_cast<uint32_t>(p.Hq) * C::D * 2;
+          asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(nq), "r"(qbytes) : "memory");
+        }
+        const int32_t* idx_tok = p.idx + static_cast<size_t>(tk) * p.K;
+        float m_ref = -INFINITY;
+        float l_sum = 0.f;
+        for (int j = 0; j < nchunk; ++j) {
+          if (!mbar_wait(bars + C::B_S_FULL + sb, sph, ab, 36)) { ok = false; break; }
+          tc_fence_after();
+          uint32_t sr[32];
+          tmem_ld32(tmem + lane_addr + C::S_COL + sb * C::NK, sr);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bars + C::B_S_EMPTY + sb);
+          if (++sb == C::NSB) { sb = 0; sph ^= 1; }
+          // validity of the chunk's 32 entries (same for every head)
+          const int e_l = j * C::NK + static_cast<int>(lane);
+          const int my_idx = (e_l < p.K) ? __ldg(idx_tok + e_l) : -1;
+          const uint32_t vmask = __ballot_sync(0xffffffffu, my_idx >= 0 && my_idx < p.rows);
+          float x[32];
+          float mc = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            x[c] = ((vmask >> c) & 1u) ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
+            mc = fmaxf(mc, x[c]);
+          }
+          float alpha = 1.f;
+          if (mc > -INFINITY && (m_ref == -INFINITY || mc > m_ref + 8.f)) {
+            alpha = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - mc);
+            m_ref = mc;
+            l_sum *= alpha;
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float p0 = (x[2 * c] == -INFINITY) ? 0.f : exp2f(x[2 * c] - m_ref);
+            const float p1 = (x[2 * c + 1] == -INFINITY) ? 0.f : exp2f(x[2 * c + 1] - m_ref);
+            pk[c] = pack_bf16x2(p0, p1);
+            const __nv_bfloat162 b2 = *reinterpret_cast<__nv_bfloat162*>(&pk[c]);
+            l_sum += __low2float(b2) + __high2float(b2);
+          }
+          const bool last = (j == nchunk - 1);
+          // staging buffer pb is free once the value CTA's MMA consumed its previous message
+          if (!mbar_wait(bars + C::B_P_FREE + pb, pfree_ph, ab, 37)) { ok = false; break; }
+          uint8_t* st = smem + C::OFF_MSG + pb * C::MSG_STRIDE;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int pc = c ^ ((h >> 1) & 3);
+            *reinterpret_cast<uint4*>(st + h * 64 + pc * 16) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          }
+          reinterpret_cast<float*>(st + C::MSG_ALPHA)[h] = alpha;
+          const uint32_t any_rs = __ballot_sync(0xffffffffu, alpha != 1.f);
+          if (lane == 0 && any_rs) atomicOr(rescale_s + (pb & 1), 1);
+          if (last) {
+            reinterpret_cast<float*>(st + C::MSG_L)[h] = l_sum;
+            reinterpret_cast<float*>(st + C::MSG_M)[h] = m_ref;
+          }
+          fence_async_shared();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bars + C::B_STAGE);
+          if (warp == C::W_SM0 && lane == 0) {
+            // all four softmax warps have written the staging buffer
+            if (!mbar_wait(bars + C::B_STAGE, stage_ph, ab, 38)) { ok = false; }
+            if (ok) {
+              uint32_t* ctrl = reinterpret_cast<uint32_t*>(st + C::MSG_CTRL);
+              ctrl[0] = static_cast<uint32_t>(rescale_s[pb & 1]);
+              rescale_s[pb & 1] = 0;
+              fence_async_shared();
+              const uint32_t bytes = last ? C::MSG_BYTES_LAST : C::MSG_BYTES_MID;
+              bulk_copy_to_peer(peer_msg + pb * C::MSG_STRIDE, smem_u32(st), bytes, peer_pfull + pb * 8);
+            }
+          }
+          stage_ph ^= 1;
+          if (++pb == C::NPB) { pb = 0; pfree_ph ^= 1; }
+          if (!ok) break;
+        }
+      }
+    }
+  } else {
+    // =========================== value CTA ===========================
+    if (warp < C::NPROD) {
+      const int ptid = threadIdx.x;
+      int slot = 0;
+      uint32_t ph = 1;
+      for (int tk = cluster_id; tk < p.T; tk += nclusters) {
+        const __nv_bfloat16* kv_tok = p.kv + tk * p.kv_token_stride;
+        const int32_t* idx_tok = p.idx + static_cast<size_t>(tk) * p.K;
+        bool ok = true;
+        for (int j = 0; j < nchunk; ++j) {
+          if (!mbar_wait(bars + C::B_RING_EMPTY + slot, ph, ab, 41)) { ok = false; break; }
+          gather_chunk(ring + slot * C::V_BYTES, kv_tok, idx_tok, j, p.K, p.rows, C::NSLAB_V, ptid);
+          cp_async_mbar_arrive(bars + C::B_RING_FULL + slot);
+          if (++slot == C::NVST) { slot = 0; ph ^= 1; }
+        }
+        if (!ok) break;
+      }
+      asm volatile("cp.async.wait_all;" ::: "memory");
+    } else if (warp == C::W_MMA) {
+      if (lane == 0) {
+        int slot = 0;
+        uint32_t ph = 0;
+        int pb = 0;
+        uint32_t pph = 0;
+        int use = 0;  // messages consumed, to arm the receive barriers ahead
+        const int total = ((p.T - 1 - cluster_id) / nclusters + 1) * nchunk;
+        bool ok = true;
+        for (int tk = cluster_id; tk < p.T && ok; tk += nclusters) {
+          for (int j = 0; j < nchunk; ++j) {
+            if (!mbar_wait(bars + C::B_RING_FULL + slot, ph, ab, 42)) { ok = false; break; }
+            if (!mbar_wait(bars + C::B_P_FULL + pb, pph, ab, 43)) { ok = false; break; }
+            const uint32_t any_rs =
+                reinterpret_cast<const volatile uint32_t*>(smem + C::OFF_MSG + pb * C::MSG_STRIDE + C::MSG_CTRL)[0];
+            // A rescale needs O quiescent: commit everything issued so far to
+            // QUIESCE; the correction warps wait on it, rescale, then signal O_READY.
+            if (any_rs && j > 0) tc_commit(bars + C::B_QUIESCE);
+            if (!mbar_wait(bars + C::B_O_READY + pb, pph, ab, 44)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t vbase = ring + slot * C::V_BYTES;
+            const uint32_t pbase = msg + pb * C::MSG_STRIDE;
+#pragma unroll
+            for (int kk = 0; kk < C::NK / 16; ++kk) {
+              const uint64_t ad = smem_desc(pbase + kk * 32, 16, 512, kSw64);
+#pragma unroll
+              for (int nh = 0; nh < 2; ++nh) {
+                const uint64_t bd = smem_desc(vbase + nh * 4 * C::SLAB_BYTES + kk * 2048, C::SLAB_BYTES, 1024, kSw128);
+                mma_bf16_ss(tmem + nh * 256, ad, bd, C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+              }
+            }
+            tc_commit(bars + C::B_RING_EMPTY + slot);
+            tc_commit_mc(bars + C::B_P_FREE + pb, 0x1);  // the score CTA's buffer pb is free
+            if (j == nchunk - 1) tc_commit(bars + C::B_PV_DONE);
+            // re-arm this receive buffer for message use + NPB
+            const int nxt = use + C::NPB;
+            if (nxt < total) {
+              const bool last = ((nxt % nchunk) == nchunk - 1);
+              mbar_arrive_expect_tx(bars + C::B_P_FULL + pb, last ? C::MSG_BYTES_LAST : C::MSG_BYTES_MID);
+            }
+            ++use;
+            if (++slot == C::NVST) { slot = 0; ph ^= 1; }
+            if (++pb == C::NPB) { pb = 0; pph ^= 1; }
+          }
+        }
+      }
+    } else {
+      // correction + epilogue warps: thread = head row
+      const int quarter = static_cast<int>(warp & 3);
+      const int h = quarter * 32 + static_cast<int>(lane);
+      const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+      int pb = 0;
+      uint32_t pph = 0;
+      uint32_t pv_ph = 0;
+      uint32_t qz_ph = 0;
+      bool ok = true;
+      for (int tk = cluster_id; tk < p.T && ok; tk += nclusters) {
+        float l_fin = 0.f, m_fin = -INFINITY;
+        for (int j = 0; j < nchunk; ++j) {
+          if (!mbar_wait(bars + C::B_P_FULL + pb, pph, ab, 45)) { ok = false; break; }
+          const uint8_t* mb = smem + C::OFF_MSG + pb * C::MSG_STRIDE;
+          const uint32_t any_rs = reinterpret_cast<const volatile uint32_t*>(mb + C::MSG_CTRL)[0];
+          if (j == nchunk - 1) {
+            l_fin = reinterpret_cast<const float*>(mb + C::MSG_L)[h];
+            m_fin = reinterpret_cast<const float*>(mb + C::MSG_M)[h];
+          }
+          if (any_rs && j > 0) {
+            const float alpha = reinterpret_cast<const float*>(mb + C::MSG_ALPHA)[h];
+            if (!mbar_wait(bars + C::B_QUIESCE, qz_ph, ab, 46)) { ok = false; break; }
+            qz_ph ^= 1;
+            tc_fence_after();
+#pragma unroll 1
+            for (int cb = 0; cb < C::DV / 32; ++cb) {
+              uint32_t r[32];
+              tmem_ld32(tmem + lane_addr + cb * 32, r);
+#pragma unroll
+              for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
+              tmem_st32(tmem + lane_addr + cb * 32, r);
+            }
+            tmem_st_wait();
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bars + C::B_O_READY + pb);
+          if (++pb == C::NPB) { pb = 0; pph ^= 1; }
+        }
+        if (!ok) break;
+        // the token's last PV has landed in TMEM
+        if (!mbar_wait(bars + C::B_PV_DONE, pv_ph, ab, 47)) break;
+        pv_ph ^= 1;
+        tc_fence_after();
+        const bool empty = !(l_fin > 0.f);
+        const float inv = empty ? 0.f : 1.f / l_fin;
+        uint4* orow = reinterpret_cast<uint4*>(p.out + (static_cast<size_t>(tk) * p.Hq + (h < p.Hq ? h : 0)) * C::DV);
+#pragma unroll 1
+        for (int cb = 0; cb < C::DV / 32; ++cb) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_addr + cb * 32, r);  // whole warp (aligned op); only real heads store
+          if (h < p.Hq) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 o;
+              o.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]) * inv, __uint_as_float(r[8 * v + 1]) * inv);
+              o.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]) * inv, __uint_as_float(r[8 * v + 3]) * inv);
+              o.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]) * inv, __uint_as_float(r[8 * v + 5]) * inv);
+              o.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]) * inv, __uint_as_float(r[8 * v + 7]) * inv);
+              orow[cb * 4 + v] = o;
+            }
+          }
+        }
+        if (h < p.Hq && p.lse)
+          p.lse[static_cast<size_t>(tk) * p.Hq + h] = empty ? -INFINITY : (m_fin + log2f(l_fin)) * 0.69314718055994531f;
+        tc_fence_before();
+      }
+    }
+  }
+
+  __syncthreads();
+  cluster_sync_all();
+  if (warp == C::W_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace dsa

@@ -1,0 +1,56 @@
+"""The C ABI library: builds, loads, exports every declared symbol, and
+rejects bad arguments before touching the GPU (runs without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dsa_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from long_context_03_b200 import build
+    build.build()
+    import long_context_03_b200 as m
+    return m.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert "dsa_index_topk" in names and "dsa_sparse_mla_attn" in names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_null_pointers_are_rejected(lib):
+    st = lib.dsa_index_topk(None, None, None, None, None, 16, 64, 128, 8, None, None, 0, None)
+    assert st == -1
+    assert b"null" in lib.dsa_last_error()
+    st = lib.dsa_sparse_mla_attn(None, None, None, 1, 1, 1, 1, ctypes.c_float(1.0), None, None, None)
+    assert st == -1
+
+
+def test_unsupported_shapes_are_rejected(lib):
+    p = ctypes.c_void_p(16)  # never dereferenced: validation fails first
+    assert lib.dsa_index_topk(p, p, p, p, p, 16, 32, 128, 8, p, p, 1 << 30, None) == -2
+    assert lib.dsa_index_topk(p, p, p, p, p, 16, 64, 128, 4096, p, p, 1 << 30, None) == -2
+    assert lib.dsa_sparse_mla_attn(p, p, p, 1, 1, 129, 8, ctypes.c_float(1.0), p, None, None) == -2
+    assert lib.dsa_index_topk_decode(p, p, p, p, p, p, 1, 16, 8, 128, 8, p, p, 1 << 30, None) == -2
+
+
+def test_misaligned_arrays_are_rejected(lib):
+    p, bad = ctypes.c_void_p(256), ctypes.c_void_p(257)
+    assert lib.dsa_sparse_mla_attn(bad, p, p, 1, 1, 16, 8, ctypes.c_float(1.0), p, None, None) == -1
+
+
+def test_status_strings(lib):
+    assert lib.dsa_status_string(0) == b"ok"
+    assert lib.dsa_status_string(-5) == b"workspace too small"

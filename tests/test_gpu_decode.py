@@ -1,0 +1,44 @@
+"""Decode indexer, top-k and attention on the GPU against the float64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from gpu_helpers import attn_close, cpu_topk_of, overlap_excluding_ties, score_tolerance_ok
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dsa():
+    import long_context_03_b200 as m
+    m.lib()
+    return m
+
+
+@pytest.mark.parametrize("d_I", [128, 64])
+def test_decode_path(dsa, d_I):
+    B, L, k = 6, 5000, 2048
+    lens = [5000, 4999, 1, 2048, 2049, 3333]
+    inp = workloads.make_decode(B, L, 64, d_I, 128, k, seed=31, lens=lens)
+    d = inp.to("cuda")
+    sc = dsa.index_scores_decode(d.q_I, d.q_scale, d.w, d.k_cache, d.k_scale, d.lens).cpu().numpy()
+    idx = dsa.index_topk_decode(d.q_I, d.q_scale, d.w, d.k_cache, d.k_scale, d.lens, k)
+    out, lse = dsa.sparse_mla_attn_decode(d.q, d.kv, idx, inp.scale, want_lse=True)
+    dsa.check_device_error()
+    idx = idx.cpu().numpy()
+    res = oracle.decode_seqs(inp, range(B))
+    for b in range(B):
+        n = lens[b]
+        t = n - 1
+        ref_sc, ref_idx, ref_out, ref_lse = res[b]
+        ok, worst = score_tolerance_ok(sc[b:b + 1, :n], ref_sc[None], [t])
+        assert ok, (b, worst)
+        assert np.array_equal(idx[b], cpu_topk_of(sc[b:b + 1, :n], [t], k)[0])
+        assert overlap_excluding_ties(idx[b:b + 1], ref_idx[None], ref_sc[None], [t], k) >= 0.999
+        # attention over the GPU's own selection, checked against the oracle on that selection
+        ref_o, ref_l = oracle.sparse_mla(oracle._bf16_bits(inp.q[b:b + 1]), inp.kv[b, :n], idx[b:b + 1], inp.scale)
+        ok, mx, rl = attn_close(out[b:b + 1], ref_o)
+        assert ok, (b, mx, rl)
+        np.testing.assert_allclose(lse[b].cpu().numpy(), ref_l[0], rtol=1e-4, atol=1e-4)
