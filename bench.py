@@ -1,0 +1,400 @@
+"""Benchmark of the DSA hot path on B200: prefill tokens/s at L = 131072 and
+decode tokens/s for 64 sequences x 65536 cached tokens.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+a 131072-token causal prefill (indexer + top-2048 selection + sparse MQA over
+the latent cache) and one decode batch (64 queries, each against its own
+65536-token caches). Inputs are seeded, generated on the device and resident
+in HBM before timing; they are far larger than L2 (the queries alone are
+19 GB), so no flush is needed between steps. `value` is prefill tokens/s
+summed over ranks; decode tokens/s is reported beside it.
+
+With N > 1 (torchrun), every rank runs the same workload independently on
+its own GPU (replicas: the path has no exchange step); times are the max over
+ranks and `value` counts every rank's tokens.
+
+--impl reference times the float64 CPU oracle (the checker, not a competing
+system) on a bounded sample of the same workload on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "DSA prefill tokens/s @128K & decode tok/s, % of FP8/BF16/HBM roofline"
+D_QK, D_V = 576, 512
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--prefill-L", type=int, default=131072)
+    ap.add_argument("--decode-B", type=int, default=64)
+    ap.add_argument("--decode-L", type=int, default=65536)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-rows", type=int, default=24)
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------- helpers
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        m = json.load(open(p))
+        return {"hbm_gbs": m["hbm_gbs"], "bf16_tflops": m["bf16_tflops"],
+                "bf16_tflops_sustained": m["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def prefill_work(L, H_I, d_I, Hq, topk):
+    """Algorithmic work of one prefill pass (causal pairs only)."""
+    pairs = L * (L + 1) // 2
+    idx_flop = 2.0 * H_I * d_I * pairs
+    sel = sum(min(topk, t + 1) for t in range(min(L, topk))) + max(0, L - topk) * topk
+    attn_flop = sel * Hq * 2.0 * (D_QK + D_V)
+    return idx_flop, attn_flop
+
+
+def decode_bytes(B, L, H_I, d_I, Hq, topk):
+    """Compulsory HBM bytes of one decode step."""
+    keys = B * L * (d_I + 4)
+    gather = B * min(topk, L) * D_QK * 2
+    small = B * (H_I * d_I + 4 + H_I * 4 + Hq * D_QK * 2 + Hq * D_V * 2 + topk * 4)
+    return keys, gather, small
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(5)
+        except Exception:
+            self.p.kill()
+        self.f.flush()
+        rows = []
+        for line in open(self.f.name):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.f.name)
+        if not rows:
+            return None
+        sm = [r[0] for r in rows]
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[2]) if v.lower() == "active"})
+        return {"sm_mhz": float(np.median(loaded)), "sm_max_mhz": rows[0][1], "reasons": reasons,
+                "samples": len(rows)}
+
+
+def dist_setup(gpus):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                             device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------- CPU baseline
+
+def cpu_oracle_prefill(inp_dev, n_rows, seed=1):
+    """Oracle on a uniform sample of query rows of the prefill workload.
+
+    Returns (tokens/s estimate for the whole prefill, seconds, rows, threads).
+    The per-row cost grows with t, so rows are drawn uniformly over [0, L).
+    """
+    import oracle
+    L = inp_dev.L
+    n_rows = max(n_rows, oracle.num_threads())
+    g = np.random.default_rng(seed)
+    rows = np.sort(g.choice(L, size=n_rows, replace=False))
+    host = dict(q_I=inp_dev.q_I[rows].cpu(), q_scale=inp_dev.q_scale[rows].cpu(), w=inp_dev.w[rows].cpu(),
+                k_cache=inp_dev.k_cache.cpu(), k_scale=inp_dev.k_scale.cpu(), q=inp_dev.q[rows].cpu(),
+                kv=inp_dev.kv.cpu())
+    t0 = time.perf_counter()
+    sc = oracle.index_scores(host["q_I"], host["q_scale"], host["w"], host["k_cache"], host["k_scale"], rows,
+                             query_rows=np.arange(n_rows))
+    ix = oracle.topk(sc, rows, inp_dev.topk)
+    oracle.sparse_mla(host["q"], host["kv"], ix, inp_dev.scale)
+    dt = time.perf_counter() - t0
+    return n_rows / dt, dt, rows, min(n_rows, oracle.num_threads())
+
+
+def cpu_oracle_decode(dec_dev, n_seq):
+    import oracle
+    sub = workloads.DecodeInputs(n_seq, dec_dev.L, dec_dev.H_I, dec_dev.d_I, dec_dev.Hq, dec_dev.topk, dec_dev.scale,
+                                 dec_dev.q_I[:n_seq].cpu(), dec_dev.q_scale[:n_seq].cpu(), dec_dev.w[:n_seq].cpu(),
+                                 dec_dev.k_cache[:n_seq].cpu(), dec_dev.k_scale[:n_seq].cpu(),
+                                 dec_dev.q[:n_seq].cpu(), dec_dev.kv[:n_seq].cpu(), dec_dev.lens[:n_seq].cpu())
+    t0 = time.perf_counter()
+    oracle.decode_seqs(sub, range(n_seq))
+    dt = time.perf_counter() - t0
+    return n_seq / dt, dt
+
+
+# -------------------------------------------------------------- our path
+
+def run_ours(a, ws, rank):
+    import long_context_03_b200 as dsa
+    dev = torch.device("cuda", torch.cuda.current_device())
+    cfgP = dict(workloads.CONFIGS["prefill_L131072"])
+    cfgP["L"] = a.prefill_L
+    cfgD = dict(workloads.CONFIGS["decode_B64_L65536"])
+    cfgD["B"], cfgD["L"] = a.decode_B, a.decode_L
+    P = workloads.make_prefill(cfgP["L"], cfgP["H_I"], cfgP["d_I"], cfgP["Hq"], cfgP["topk"], seed=rank,
+                               device=dev)
+    D = workloads.make_decode(cfgD["B"], cfgD["L"], cfgD["H_I"], cfgD["d_I"], cfgD["Hq"], cfgD["topk"], seed=rank,
+                              device=dev)
+    L, k = P.L, P.topk
+    idx = torch.empty((L, k), dtype=torch.int32, device=dev)
+    out = torch.empty((L, P.Hq, D_V), dtype=torch.bfloat16, device=dev)
+    ws_p = torch.empty(dsa.index_topk_workspace_size(L, P.H_I, P.d_I, k), dtype=torch.uint8, device=dev)
+    didx = torch.empty((D.B, k), dtype=torch.int32, device=dev)
+    dout = torch.empty((D.B, D.Hq, D_V), dtype=torch.bfloat16, device=dev)
+    ws_d = torch.empty(dsa.index_topk_decode_workspace_size(D.B, D.L, k), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        dsa.index_topk(P.q_I, P.q_scale, P.w, P.k_cache, P.k_scale, k, idx=idx, workspace=ws_p)
+        if ev:
+            ev[1].record(stream)
+        dsa.sparse_mla_attn(P.q, P.kv, idx, P.scale, out=out)
+        if ev:
+            ev[2].record(stream)
+        dsa.index_topk_decode(D.q_I, D.q_scale, D.w, D.k_cache, D.k_scale, D.lens, k, idx=didx, workspace=ws_d)
+        if ev:
+            ev[3].record(stream)
+        dsa.sparse_mla_attn_decode(D.q, D.kv, didx, D.scale, out=dout)
+        if ev:
+            ev[4].record(stream)
+
+    for _ in range(a.warmup):
+        step()
+    torch.cuda.synchronize()
+    dsa.check_device_error()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(a.steps)]
+    clk = ClockSampler(dev.index)
+    barrier(ws)
+    torch.cuda.synchronize()
+    clk.start()
+    t_wall = time.perf_counter()
+    for s in range(a.steps):
+        step(evs[s])
+    torch.cuda.synchronize()
+    barrier(ws)
+    t_wall = time.perf_counter() - t_wall
+    clocks = clk.stop()
+    dsa.check_device_error()
+    seg = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in evs])  # ms
+    t_idx, t_attn, t_didx, t_dattn = [max_over_ranks(float(seg[:, i].mean()), ws) for i in range(4)]
+    t_prefill = t_idx + t_attn
+    t_decode = t_didx + t_dattn
+
+    pk = peaks()
+    fp8_peak = 2.0 * pk["bf16_tflops_sustained"]
+    idx_flop, attn_flop = prefill_work(L, P.H_I, P.d_I, P.Hq, k)
+    keys_b, gather_b, small_b = decode_bytes(D.B, D.L, D.H_I, D.d_I, D.Hq, k)
+    idx_tf = idx_flop / (t_idx * 1e-3) / 1e12
+    attn_tf = attn_flop / (t_attn * 1e-3) / 1e12
+    dec_gbs = (keys_b + gather_b + small_b) / (t_decode * 1e-3) / 1e9
+    dec_idx_gbs = (keys_b + D.B * (D.H_I * D.d_I + 8 + D.H_I * 4)) / (t_didx * 1e-3) / 1e9
+    rl = {
+        "prefill_indexer": {"bound": "tensor", "achieved": idx_tf, "peak": fp8_peak, "unit": "TFLOP/s",
+                            "frac": idx_tf / fp8_peak, "traffic": None,
+                            "note": "FP8 peak = 2 x measured sustained bf16 (nominal fp8:bf16 ratio); time includes the rank sort"},
+        "prefill_attention": {"bound": "tensor", "achieved": attn_tf, "peak": pk["bf16_tflops_sustained"],
+                              "unit": "TFLOP/s", "frac": attn_tf / pk["bf16_tflops_sustained"], "traffic": None},
+        "decode_step": {"bound": "hbm", "achieved": dec_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                        "frac": dec_gbs / pk["hbm_gbs"], "traffic": None},
+        "decode_indexer": {"bound": "hbm", "achieved": dec_idx_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                           "frac": dec_idx_gbs / pk["hbm_gbs"], "traffic": None},
+    }
+    dom = "prefill_indexer" if t_idx >= t_attn else "prefill_attention"
+    value = ws * L / (t_prefill * 1e-3)
+    dec_tps = ws * D.B / (t_decode * 1e-3)
+    res = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": a.steps, "warmup": a.warmup,
+        "ms_per_step": t_prefill + t_decode, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8-e4m3 indexer / bf16 attention (fp32 accumulate)", "data": "synthetic",
+        "config": {"workload": f"prefill L={L} (H_I={P.H_I}, d_I={P.d_I}, topk={k}, Hq={P.Hq}) + "
+                               f"decode B={D.B} x L={D.L}", "parallelism": "replicas" if ws > 1 else "single",
+                   "l2": "inputs larger than L2 (no flush needed)", "seed": "rank"},
+        "prefill": {"tokens_per_s": value, "ms": t_prefill, "indexer_ms": t_idx, "attention_ms": t_attn},
+        "decode": {"tokens_per_s": dec_tps, "ms": t_decode, "indexer_ms": t_didx, "attention_ms": t_dattn},
+        "roofline": dict(rl[dom], kernel=dom),
+        "roofline_all": rl,
+        "peaks": {"source": pk["source"], "fp8": "2 x bf16_tflops_sustained"},
+        "gpu_launches": 7 * a.steps,
+        "clocks": clocks,
+        "wall_s_timed": t_wall,
+    }
+    if not a.no_e2e:
+        res["e2e"] = run_e2e(a, dsa, P, idx, out, ws_p, ws, dev)
+    if rank == 0 and not a.no_cpu_baseline:
+        tps, dt, rows, cores = cpu_oracle_prefill(P, a.cpu_sample_rows)
+        dtps, ddt = cpu_oracle_decode(D, 2)
+        res["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                               "sample": f"{len(rows)} query rows drawn uniformly from the L={L} prefill "
+                                         f"({dt:.1f} s; tokens/s = rows / time, the per-row cost tracks t)",
+                               "decode_tokens_per_s": dtps,
+                               "decode_sample": f"2 of the {D.B} decode sequences ({ddt:.1f} s)"}
+    return res
+
+
+def run_e2e(a, dsa, P, idx, out, ws_p, ws, dev):
+    """Same prefill metric through the public API with pinned host buffers:
+    every step copies the inputs host->device and the output back."""
+    try:
+        host = {n: getattr(P, n).cpu().pin_memory() for n in ("q_I", "q_scale", "w", "k_cache", "k_scale", "q", "kv")}
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    except Exception as e:  # host memory too small to pin
+        return {"value": None, "unit": "tokens/s", "error": f"{type(e).__name__}: {e}"}
+    dev_bufs = {n: getattr(P, n) for n in host}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out.numel() * out.element_size()
+    stream = torch.cuda.current_stream(dev)
+    times = []
+    for s in range(a.warmup + a.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for n, t in host.items():
+            dev_bufs[n].copy_(t, non_blocking=True)
+        dsa.index_topk(P.q_I, P.q_scale, P.w, P.k_cache, P.k_scale, P.topk, idx=idx, workspace=ws_p)
+        dsa.sparse_mla_attn(P.q, P.kv, idx, P.scale, out=out)
+        out_h.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if s >= a.warmup:
+            times.append(e0.elapsed_time(e1))
+    t = max_over_ranks(float(np.mean(times)), ws)
+    return {"value": ws * P.L / (t * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": t, "scope": "prefill (the headline metric)"}
+
+
+# ------------------------------------------------------- reference (oracle)
+
+def run_reference(a, ws, rank):
+    """The float64 oracle on host cores, a bounded sample per step."""
+    cfgP = dict(workloads.CONFIGS["prefill_L131072"])
+    cfgP["L"] = a.prefill_L
+    # inputs drawn on the CPU with the same recipe (a CPU generator stream)
+    P = workloads.make_prefill(cfgP["L"], cfgP["H_I"], cfgP["d_I"], 1, cfgP["topk"], seed=0, device="cpu")
+    # the sample needs only a few query rows of the 128-head queries
+    g = torch.Generator().manual_seed(7)
+    import oracle
+    rows_per_step = max(4, oracle.num_threads())
+    q_rows = torch.randn((rows_per_step * (a.warmup + a.steps), 128, D_QK), generator=g).to(torch.bfloat16)
+    import oracle
+    times = []
+    rng = np.random.default_rng(1)
+    for s in range(a.warmup + a.steps):
+        rows = np.sort(rng.choice(P.L, size=rows_per_step, replace=False))
+        t0 = time.perf_counter()
+        sc = oracle.index_scores(P.q_I, P.q_scale, P.w, P.k_cache, P.k_scale, rows)
+        ix = oracle.topk(sc, rows, P.topk)
+        oracle.sparse_mla(q_rows[s * rows_per_step:(s + 1) * rows_per_step], P.kv, ix, P.scale)
+        dt = time.perf_counter() - t0
+        if s >= a.warmup:
+            times.append(dt)
+    per_row = float(np.mean(times)) / rows_per_step
+    value = 1.0 / per_row
+    cores = min(rows_per_step, oracle.num_threads())
+    sample = f"{rows_per_step} query rows per step drawn uniformly from the L={P.L} prefill"
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": float(np.mean(times)) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"prefill L={P.L} (H_I={P.H_I}, d_I={P.d_I}, topk={P.topk}, Hq=128) rows sampled",
+                       "parallelism": "single"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    a = parse()
+    if a.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        ws = int(os.environ.get("WORLD_SIZE", "1"))
+        if rank != 0:
+            return
+        print(json.dumps(run_reference(a, ws, rank)))
+        return
+    ws, rank, _ = dist_setup(a.gpus)
+    try:
+        res = run_ours(a, ws, rank)
+        if rank == 0:
+            print(json.dumps(res))
+    finally:
+        if ws > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -351,8 +351,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
             const float p0 = (x[2 * c] == -INFINITY) ? 0.f : exp2f(x[2 * c] - m_ref);
             const float p1 = (x[2 * c + 1] == -INFINITY) ? 0.f : exp2f(x[2 * c + 1] - m_ref);
             pk[c] = pack_bf16x2(p0, p1);
-            const __nv_bfloat162 b2 = *reinterpret_cast<__nv_bfloat162*>(&pk[c]);
-            l_sum += __low2float(b2) + __high2float(b2);
+            l_sum += p0 + p1;
           }
           const bool last = (j == nchunk - 1);
           // staging buffer pb is free once the value CTA's MMA consumed its previous message
