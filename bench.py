@@ -312,6 +312,15 @@ def run_ours(a, ws, rank):
 def run_e2e(a, dsa, P, idx, out, ws_p, ws, dev):
     """Same prefill metric through the public API with pinned host buffers:
     every step copies the inputs host->device and the output back."""
+    need = sum(getattr(P, n).numel() * getattr(P, n).element_size()
+               for n in ("q_I", "q_scale", "w", "k_cache", "k_scale", "q", "kv")) + out.numel() * out.element_size()
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except Exception:
+        avail = None
+    if avail is not None and avail < 2 * need:
+        return {"value": None, "unit": "tokens/s", "error": f"host memory: {avail} bytes free, {need} needed pinned"}
     try:
         host = {n: getattr(P, n).cpu().pin_memory() for n in ("q_I", "q_scale", "w", "k_cache", "k_scale", "q", "kv")}
         out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
