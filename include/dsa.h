@@ -136,6 +136,38 @@ dsa_status dsa_sparse_mla_attn_decode(const uint16_t* q, const uint16_t* kv, con
                                       int Hq, int topk, float scale, uint16_t* out, float* lse, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Decode indexer + top-k with no caller workspace and no allocation.
+ *
+ * The pages describe nothing like this call; it exists for callers that
+ * cannot allocate device memory: plugins inside a host framework that owns
+ * every device allocation and gives its extensions no allocator, and
+ * latency-bound serving loops where a cudaMalloc (which may synchronise the
+ * whole device) is not acceptable. It computes exactly what
+ * dsa_index_topk_decode computes (same kernels, same results), but its
+ * scratch (the per-key scores and the selected keys) is a fixed array inside
+ * this library, in the device memory of every GPU that loads the library,
+ * held until the process exits.
+ *
+ * Limits: B * L_max <= DSA_NOALLOC_MAX_SCORES and B * topk <=
+ * DSA_NOALLOC_MAX_KEYS; larger calls return DSA_ERR_UNSUPPORTED (nothing is
+ * enqueued) with the limit in dsa_last_error().
+ * The first call on each device looks up the array's device address (a
+ * runtime query, no allocation); make that first call before any stream
+ * capture. Every call shares the one array: calls whose work overlaps on the
+ * GPU (different streams, or several host threads) race and must be ordered
+ * by the caller. Nothing in the array needs to start at zero: each call
+ * writes every element it later reads. No cudaMalloc, cudaFree or
+ * allocating library routine is called.
+ * Arguments as for dsa_index_topk_decode, without workspace / ws_bytes.
+ * ------------------------------------------------------------------------ */
+#define DSA_NOALLOC_MAX_SCORES (1u << 20) /* 4 MiB of fp32 scores */
+#define DSA_NOALLOC_MAX_KEYS (1u << 16)   /* 512 KiB of selected keys */
+
+dsa_status dsa_index_topk_decode_noalloc(const uint8_t* q_I, const float* q_scale, const float* w,
+                                         const uint8_t* k_cache, const float* k_scale, const int32_t* lens, int B,
+                                         int L_max, int H_I, int d_I, int topk, int32_t* idx, void* stream);
+
+/* ------------------------------------------------------------------------
  * Errors.
  * ------------------------------------------------------------------------ */
 /* Synchronises `stream`, then reads and clears the device error word of the

@@ -57,13 +57,15 @@ def lib() -> ctypes.CDLL:
             L.dsa_index_topk_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P, P, SZ, P]
             L.dsa_index_scores_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, P, P]
             L.dsa_sparse_mla_attn_decode.argtypes = [P, P, P, I, I, I, I, F, P, P, P]
+            L.dsa_index_topk_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P, P]
             L.dsa_get_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_uint)]
             L.dsa_status_string.argtypes = [I]
             L.dsa_status_string.restype = ctypes.c_char_p
             L.dsa_last_error.argtypes = []
             L.dsa_last_error.restype = ctypes.c_char_p
             for name in ("dsa_index_topk", "dsa_index_scores", "dsa_sparse_mla_attn", "dsa_index_topk_decode",
-                         "dsa_index_scores_decode", "dsa_sparse_mla_attn_decode", "dsa_get_device_error"):
+                         "dsa_index_scores_decode", "dsa_sparse_mla_attn_decode", "dsa_get_device_error",
+                         "dsa_index_topk_decode_noalloc"):
                 getattr(L, name).restype = I
             _lib = L
     return _lib
@@ -196,6 +198,22 @@ def index_topk_decode(q_I, q_scale, w, k_cache, k_scale, lens, topk: int, *, idx
     _check(lib().dsa_index_topk_decode(_ptr(q_I), _ptr(q_scale), _ptr(w), _ptr(k_cache), _ptr(k_scale),
                                        _ptr(lens), B, L_max, H_I, d_I, topk, _ptr(idx), _ptr(workspace),
                                        workspace.numel() * workspace.element_size(), _stream(q_I.device)))
+    return idx
+
+
+def index_topk_decode_noalloc(q_I, q_scale, w, k_cache, k_scale, lens, topk: int, *, idx=None):
+    """Decode indexer + top-k whose scratch is a fixed array inside the library
+    (for callers that cannot allocate device memory; limits in include/dsa.h).
+    Same result as index_topk_decode. Calls overlapping on the GPU race on the
+    shared scratch."""
+    q_I, k_cache = _u8(q_I), _u8(k_cache)
+    B, H_I, d_I, L_max = _req_decode(q_I, q_scale, w, k_cache, k_scale, lens)
+    if idx is None:
+        idx = torch.empty((B, topk), dtype=torch.int32, device=q_I.device)
+    _req(idx, "idx", torch.int32, (B, topk))
+    _check(lib().dsa_index_topk_decode_noalloc(_ptr(q_I), _ptr(q_scale), _ptr(w), _ptr(k_cache), _ptr(k_scale),
+                                               _ptr(lens), B, L_max, H_I, d_I, topk, _ptr(idx),
+                                               _stream(q_I.device)))
     return idx
 
 

@@ -386,6 +386,67 @@ dsa_status dsa_sparse_mla_attn_decode(const uint16_t* q, const uint16_t* kv, con
                     static_cast<cudaStream_t>(stream));
 }
 
+// ---- decode indexer + top-k with library-owned scratch ----
+// For callers that cannot allocate device memory (see dsa.h). The scratch
+// lives in this fixed device array: per-key fp32 scores first, then the
+// selected 64-bit keys. Host code must not pass the symbol itself to a
+// kernel (on the host it only names a stand-in); the device address comes
+// from cudaGetSymbolAddress, looked up once per device.
+constexpr size_t kNoAllocScoreBytes = static_cast<size_t>(DSA_NOALLOC_MAX_SCORES) * 4;
+constexpr size_t kNoAllocKeyBytes = static_cast<size_t>(DSA_NOALLOC_MAX_KEYS) * 8;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScoreBytes + kNoAllocKeyBytes];
+
+namespace {
+std::mutex g_noalloc_mu;
+constexpr int kNoAllocMaxDevices = 64;
+void* g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device (set up on the
+// first call per device, with that device current).
+dsa_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(DSA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p) return cuda_fail(e, "cudaGetSymbolAddress(g_noalloc_scratch)");
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return DSA_OK;
+}
+}  // namespace
+
+dsa_status dsa_index_topk_decode_noalloc(const uint8_t* q_I, const float* q_scale, const float* w,
+                                         const uint8_t* k_cache, const float* k_scale, const int32_t* lens, int B,
+                                         int L_max, int H_I, int d_I, int topk, int32_t* idx, void* stream) {
+  dsa_status s = check_decode_args(q_I, q_scale, w, k_cache, k_scale, lens, B, L_max, H_I, d_I);
+  if (s != DSA_OK) return s;
+  if (!idx) return fail(DSA_ERR_INVALID_ARG, "null pointer");
+  if (topk < 1 || topk > DSA_MAX_TOPK) return fail(DSA_ERR_UNSUPPORTED, "topk=%d not in [1, %d]", topk, DSA_MAX_TOPK);
+  if (static_cast<unsigned long long>(B) * L_max > DSA_NOALLOC_MAX_SCORES)
+    return fail(DSA_ERR_UNSUPPORTED, "B*L_max=%lld exceeds the fixed scratch limit of %u scores",
+                static_cast<long long>(B) * L_max, DSA_NOALLOC_MAX_SCORES);
+  if (static_cast<unsigned long long>(B) * topk > DSA_NOALLOC_MAX_KEYS)
+    return fail(DSA_ERR_UNSUPPORTED, "B*topk=%lld exceeds the fixed scratch limit of %u keys",
+                static_cast<long long>(B) * topk, DSA_NOALLOC_MAX_KEYS);
+  void* base = nullptr;
+  s = noalloc_scratch(&base);
+  if (s != DSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* scores = reinterpret_cast<float*>(base);
+  uint64_t* sel = reinterpret_cast<uint64_t*>(reinterpret_cast<char*>(base) + kNoAllocScoreBytes);
+  s = decode_scores(q_I, q_scale, w, k_cache, k_scale, lens, B, L_max, H_I, d_I, scores, st);
+  if (s != DSA_OK) return s;
+  decode_select_kernel<1024><<<B, 1024, 0, st>>>(scores, lens, L_max, topk, sel);
+  s = check_launch("decode_select_kernel");
+  if (s != DSA_OK) return s;
+  return launch_rank_sort(sel, idx, topk, B, st);
+}
+
 dsa_status dsa_get_device_error(void* stream, unsigned int* detail) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   unsigned int h = 0;
