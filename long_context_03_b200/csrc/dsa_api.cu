@@ -97,8 +97,9 @@ dsa_status check_launch(const char* what) {
 // ---- prefill indexer ----
 constexpr int kNetPrefill = 8 * 32;  // epilogue threads of the prefill indexer
 
-int select_maxper(int topk) { return (topk <= 128) ? 2 : 17; }
-int select_cap(int topk) { return select_maxper(topk) * kNetPrefill; }
+// keys per thread per quarter sub-list in a list cut; list capacity = 4 * MQ * 256
+int select_mq(int topk) { return (topk <= 128) ? 1 : 8; }
+int select_cap(int topk) { return 4 * select_mq(topk) * kNetPrefill; }
 
 int rows_per_block(int H_I) { return 2 * (256 / H_I); }
 
@@ -120,7 +121,7 @@ WsPrefill prefill_ws_layout(void* base, int L, int H_I, int topk, int grid) {
   return w;
 }
 
-template <int HI, int DI, bool kSelect, int MAXPER>
+template <int HI, int DI, bool kSelect, int MQ>
 dsa_status launch_prefill(const uint8_t* q_I, const uint8_t* k_cache, const IdxPrefillParams& p, int grid,
                           cudaStream_t st) {
   using C = IdxPrefillCfg<HI, DI>;
@@ -129,20 +130,20 @@ dsa_status launch_prefill(const uint8_t* q_I, const uint8_t* k_cache, const IdxP
   if (s != DSA_OK) return s;
   s = make_map_u8(&tmK, k_cache, DI, static_cast<uint64_t>(p.L), DI, C::BM);
   if (s != DSA_OK) return s;
-  auto kern = indexer_prefill_kernel<HI, DI, kSelect, MAXPER>;
+  auto kern = indexer_prefill_kernel<HI, DI, kSelect, MQ>;
   s = set_smem(kern, C::SMEM_BYTES);
   if (s != DSA_OK) return s;
   kern<<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(tmQ, tmK, p);
   return check_launch("indexer_prefill_kernel");
 }
 
-template <bool kSelect, int MAXPER>
+template <bool kSelect, int MQ>
 dsa_status dispatch_prefill(int H_I, int d_I, const uint8_t* q_I, const uint8_t* k_cache, const IdxPrefillParams& p,
                             int grid, cudaStream_t st) {
-  if (H_I == 64 && d_I == 128) return launch_prefill<64, 128, kSelect, MAXPER>(q_I, k_cache, p, grid, st);
-  if (H_I == 64 && d_I == 64) return launch_prefill<64, 64, kSelect, MAXPER>(q_I, k_cache, p, grid, st);
-  if (H_I == 8 && d_I == 128) return launch_prefill<8, 128, kSelect, MAXPER>(q_I, k_cache, p, grid, st);
-  if (H_I == 8 && d_I == 64) return launch_prefill<8, 64, kSelect, MAXPER>(q_I, k_cache, p, grid, st);
+  if (H_I == 64 && d_I == 128) return launch_prefill<64, 128, kSelect, MQ>(q_I, k_cache, p, grid, st);
+  if (H_I == 64 && d_I == 64) return launch_prefill<64, 64, kSelect, MQ>(q_I, k_cache, p, grid, st);
+  if (H_I == 8 && d_I == 128) return launch_prefill<8, 128, kSelect, MQ>(q_I, k_cache, p, grid, st);
+  if (H_I == 8 && d_I == 64) return launch_prefill<8, 64, kSelect, MQ>(q_I, k_cache, p, grid, st);
   return fail(DSA_ERR_UNSUPPORTED, "H_I=%d d_I=%d not supported", H_I, d_I);
 }
 
@@ -150,10 +151,10 @@ dsa_status launch_rank_sort(const uint64_t* keys, int32_t* idx, int K, int rows,
   if (rows <= 0) return DSA_OK;
   if (K <= 64) rank_sort_kernel<64><<<rows, 256, 0, st>>>(keys, idx, K, rows);
   else if (K <= 128) rank_sort_kernel<128><<<rows, 256, 0, st>>>(keys, idx, K, rows);
-  else if (K <= 256) rank_sort_kernel<256><<<rows, 256, 0, st>>>(keys, idx, K, rows);
-  else if (K <= 512) rank_sort_kernel<512><<<rows, 256, 0, st>>>(keys, idx, K, rows);
-  else if (K <= 1024) rank_sort_kernel<1024><<<rows, 256, 0, st>>>(keys, idx, K, rows);
-  else rank_sort_kernel<2048><<<rows, 256, 0, st>>>(keys, idx, K, rows);
+  else if (K <= 256) rank_sort_reg_kernel<256><<<rows, 32, 0, st>>>(keys, idx, K, rows);
+  else if (K <= 512) rank_sort_reg_kernel<512><<<rows, 64, 0, st>>>(keys, idx, K, rows);
+  else if (K <= 1024) rank_sort_reg_kernel<1024><<<rows, 128, 0, st>>>(keys, idx, K, rows);
+  else rank_sort_reg_kernel<2048><<<rows, 256, 0, st>>>(keys, idx, K, rows);
   return check_launch("rank_sort_kernel");
 }
 
@@ -184,8 +185,9 @@ dsa_status launch_decode_scores(const uint8_t* q_I, const uint8_t* k_cache, int 
 
 dsa_status decode_scores(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
                          const float* k_scale, const int32_t* lens, int B, int L_max, int H_I, int d_I, float* scores,
-                         cudaStream_t st) {
+                         uint32_t* hist, cudaStream_t st) {
   IdxDecodeParams p;
+  p.hist = hist;
   p.q_scale = q_scale;
   p.w = w;
   p.k_scale = k_scale;
@@ -195,6 +197,15 @@ dsa_status decode_scores(const uint8_t* q_I, const float* q_scale, const float* 
   if (H_I == 64 && d_I == 128) return launch_decode_scores<64, 128>(q_I, k_cache, B, p, st);
   if (H_I == 64 && d_I == 64) return launch_decode_scores<64, 64>(q_I, k_cache, B, p, st);
   return fail(DSA_ERR_UNSUPPORTED, "decode: H_I=%d d_I=%d not supported", H_I, d_I);
+}
+
+dsa_status launch_decode_select(const float* scores, const int32_t* lens, int L_max, int topk, const uint32_t* hist,
+                                uint64_t* sel, int B, cudaStream_t st) {
+  const int smem = kDecodeSelBinCap * 8 + (2048 + select_scratch_ints(kDecodeSelThreads)) * 4;
+  dsa_status s = set_smem(decode_select_kernel, smem);
+  if (s != DSA_OK) return s;
+  decode_select_kernel<<<B, kDecodeSelThreads, smem, st>>>(scores, lens, L_max, topk, hist, sel);
+  return check_launch("decode_select_kernel");
 }
 
 dsa_status check_decode_args(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
@@ -294,8 +305,8 @@ dsa_status dsa_index_topk(const uint8_t* q_I, const float* q_scale, const float*
   p.cand = ws.cand;
   p.cap = select_cap(topk);
   p.sel_keys = ws.sel;
-  dsa_status s = (select_maxper(topk) == 2) ? dispatch_prefill<true, 2>(H_I, d_I, q_I, k_cache, p, grid, st)
-                                            : dispatch_prefill<true, 17>(H_I, d_I, q_I, k_cache, p, grid, st);
+  dsa_status s = (select_mq(topk) == 1) ? dispatch_prefill<true, 1>(H_I, d_I, q_I, k_cache, p, grid, st)
+                                        : dispatch_prefill<true, 8>(H_I, d_I, q_I, k_cache, p, grid, st);
   if (s != DSA_OK) return s;
   return launch_rank_sort(ws.sel, idx, topk, L, st);
 }
@@ -342,7 +353,8 @@ dsa_status dsa_sparse_mla_attn(const uint16_t* q, const uint16_t* kv, const int3
 size_t dsa_index_topk_decode_workspace_size(int B, int L_max, int topk) {
   if (B <= 0 || L_max <= 0 || topk <= 0) return 0;
   const size_t scores = (static_cast<size_t>(B) * L_max * 4 + 255) / 256 * 256;
-  return scores + static_cast<size_t>(B) * topk * 8;
+  const size_t keys = (static_cast<size_t>(B) * topk * 8 + 255) / 256 * 256;
+  return scores + keys + static_cast<size_t>(B) * 2048 * 4;
 }
 
 dsa_status dsa_index_topk_decode(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
@@ -356,13 +368,16 @@ dsa_status dsa_index_topk_decode(const uint8_t* q_I, const float* q_scale, const
   if (!workspace || ws_bytes < need) return fail(DSA_ERR_WORKSPACE, "workspace %zu bytes, need %zu", ws_bytes, need);
   if (!aligned16(workspace)) return fail(DSA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  float* scores = reinterpret_cast<float*>(workspace);
-  uint64_t* sel = reinterpret_cast<uint64_t*>(reinterpret_cast<char*>(workspace) +
-                                              (static_cast<size_t>(B) * L_max * 4 + 255) / 256 * 256);
-  s = decode_scores(q_I, q_scale, w, k_cache, k_scale, lens, B, L_max, H_I, d_I, scores, st);
+  char* base = reinterpret_cast<char*>(workspace);
+  float* scores = reinterpret_cast<float*>(base);
+  const size_t off_keys = (static_cast<size_t>(B) * L_max * 4 + 255) / 256 * 256;
+  uint64_t* sel = reinterpret_cast<uint64_t*>(base + off_keys);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(base + off_keys + (static_cast<size_t>(B) * topk * 8 + 255) / 256 * 256);
+  const cudaError_t e = cudaMemsetAsync(hist, 0, static_cast<size_t>(B) * 2048 * 4, st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(histogram)");
+  s = decode_scores(q_I, q_scale, w, k_cache, k_scale, lens, B, L_max, H_I, d_I, scores, hist, st);
   if (s != DSA_OK) return s;
-  decode_select_kernel<1024><<<B, 1024, 0, st>>>(scores, lens, L_max, topk, sel);
-  s = check_launch("decode_select_kernel");
+  s = launch_decode_select(scores, lens, L_max, topk, hist, sel, B, st);
   if (s != DSA_OK) return s;
   return launch_rank_sort(sel, idx, topk, B, st);
 }
@@ -373,7 +388,7 @@ dsa_status dsa_index_scores_decode(const uint8_t* q_I, const float* q_scale, con
   dsa_status s = check_decode_args(q_I, q_scale, w, k_cache, k_scale, lens, B, L_max, H_I, d_I);
   if (s != DSA_OK) return s;
   if (!scores) return fail(DSA_ERR_INVALID_ARG, "null pointer");
-  return decode_scores(q_I, q_scale, w, k_cache, k_scale, lens, B, L_max, H_I, d_I, scores,
+  return decode_scores(q_I, q_scale, w, k_cache, k_scale, lens, B, L_max, H_I, d_I, scores, nullptr,
                        static_cast<cudaStream_t>(stream));
 }
 
@@ -439,10 +454,9 @@ dsa_status dsa_index_topk_decode_noalloc(const uint8_t* q_I, const float* q_scal
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* scores = reinterpret_cast<float*>(base);
   uint64_t* sel = reinterpret_cast<uint64_t*>(reinterpret_cast<char*>(base) + kNoAllocScoreBytes);
-  s = decode_scores(q_I, q_scale, w, k_cache, k_scale, lens, B, L_max, H_I, d_I, scores, st);
+  s = decode_scores(q_I, q_scale, w, k_cache, k_scale, lens, B, L_max, H_I, d_I, scores, nullptr, st);
   if (s != DSA_OK) return s;
-  decode_select_kernel<1024><<<B, 1024, 0, st>>>(scores, lens, L_max, topk, sel);
-  s = check_launch("decode_select_kernel");
+  s = launch_decode_select(scores, lens, L_max, topk, nullptr, sel, B, st);
   if (s != DSA_OK) return s;
   return launch_rank_sort(sel, idx, topk, B, st);
 }

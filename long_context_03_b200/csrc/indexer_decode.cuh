@@ -43,7 +43,8 @@ struct IdxDecodeCfg {
   static constexpr int OFF_K = 0;
   static constexpr int OFF_Q = OFF_K + KST * KTILE_BYTES;
   static constexpr int OFF_W = OFF_Q + ((QBYTES + 1023) / 1024) * 1024;
-  static constexpr int OFF_BAR = OFF_W + HI * 4;
+  static constexpr int OFF_HIST = OFF_W + HI * 4;         // u32 [2048] per-CTA histogram
+  static constexpr int OFF_BAR = OFF_HIST + 2048 * 4;
   static constexpr int NBAR = 1 + 2 * KST + 2 * NACC;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
@@ -57,7 +58,12 @@ struct IdxDecodeParams {
   const int32_t* lens;   // [B]
   int L_max;
   float* scores;         // [B, L_max]; entries s >= lens[b] untouched
+  uint32_t* hist;        // [B, 2048] counts of the top 11 bits of each ranking key, or null
 };
+
+// Bin of a ranking key in the 2048-bin histogram: its top 11 bits (sign,
+// exponent and the top two mantissa bits of the score).
+__device__ __forceinline__ uint32_t key_bin11(uint64_t key) { return static_cast<uint32_t>(key >> 53); }
 
 template <int HI, int DI>
 __global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS)
@@ -101,6 +107,9 @@ __global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS)
     fence_mbar_init();
   }
   for (int i = threadIdx.x; i < HI; i += blockDim.x) w_s[i] = p.w[static_cast<size_t>(b) * HI + i];
+  uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + C::OFF_HIST);
+  if (p.hist)
+    for (int i = threadIdx.x; i < 2048; i += blockDim.x) hist_s[i] = 0;
   if (warp == 1) tmem_alloc(tmem_base_s, C::TMEM_COLS);
   __syncthreads();
   tc_fence_after();
@@ -170,7 +179,19 @@ __global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty + buf);
-      if (s < n) p.scores[static_cast<size_t>(b) * p.L_max + s] = __fmul_rn(__fmul_rn(acc, qs), ks);
+      if (s < n) {
+        const float score = __fmul_rn(__fmul_rn(acc, qs), ks);
+        p.scores[static_cast<size_t>(b) * p.L_max + s] = score;
+        if (p.hist) atomicAdd(hist_s + key_bin11(rank_key(score, static_cast<uint32_t>(s))), 1u);
+      }
+    }
+    if (p.hist) {
+      named_bar_sync(1, 128);
+      const int et = threadIdx.x - 64;
+      for (int i = et; i < 2048; i += 128) {
+        const uint32_t c = hist_s[i];
+        if (c) atomicAdd(p.hist + static_cast<size_t>(b) * 2048 + i, c);
+      }
     }
   }
   __syncthreads();
@@ -181,52 +202,117 @@ __global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS)
 }
 
 // Exact top-k of one sequence's scores (one CTA of kThreads per sequence).
-// Radix select over ranking keys recomputed from (score, s) on every pass;
-// the scores stay in L2 between passes. Writes the k best keys of sequence b
-// (unordered, 0 where lens[b] < k) to sel_keys[b, 0..k).
-template <int kThreads>
-__global__ void __launch_bounds__(kThreads)
+// With the scoring kernel's 2048-bin histogram of ranking keys (top 11 bits),
+// the bin holding the k-th largest key is known before reading any score:
+// one pass writes every key above that bin straight to the output and keeps
+// the bin's own keys in shared memory, where an exact radix select picks the
+// rest. Without a histogram (or if the bin overflows the shared buffer) the
+// kernel counts the histogram itself / falls back to multi-pass selection
+// over global memory. Writes the k best keys of sequence b (unordered, 0
+// where lens[b] < k) to sel_keys[b, 0..k).
+constexpr int kDecodeSelThreads = 1024;
+constexpr int kDecodeSelBinCap = 4096;  // boundary-bin keys kept in shared memory
+
+__global__ void __launch_bounds__(kDecodeSelThreads)
     decode_select_kernel(const float* __restrict__ scores, const int32_t* __restrict__ lens, int L_max, int K,
-                         uint64_t* __restrict__ sel_keys) {
-  __shared__ int hist[256];
-  __shared__ int misc[4];
-  __shared__ unsigned long long mm[2];
+                         const uint32_t* __restrict__ hist_in, uint64_t* __restrict__ sel_keys) {
+  constexpr int NT = kDecodeSelThreads;
+  extern __shared__ __align__(16) uint8_t dsmem[];
+  uint64_t* bin_keys = reinterpret_cast<uint64_t*>(dsmem);                          // [kDecodeSelBinCap]
+  int* hist = reinterpret_cast<int*>(dsmem + kDecodeSelBinCap * 8);                 // [2048]
+  int* scr = hist + 2048;                                                            // select scratch
+  __shared__ int wsum[32];
+  __shared__ int res[4];
+  __shared__ int wpos, bpos;
   const int b = blockIdx.x;
   const int n = lens[b];
   const float* sc = scores + static_cast<size_t>(b) * L_max;
   uint64_t* dst = sel_keys + static_cast<size_t>(b) * K;
   const int tid = threadIdx.x;
   if (n <= K) {
-    for (int i = tid; i < K; i += kThreads) dst[i] = (i < n) ? rank_key(sc[i], static_cast<uint32_t>(i)) : 0ull;
+    for (int i = tid; i < K; i += NT) dst[i] = (i < n) ? rank_key(sc[i], static_cast<uint32_t>(i)) : 0ull;
     return;
   }
-  // common prefix of all keys
-  unsigned long long kmin = ~0ull, kmax = 0ull;
-  for (int i = tid; i < n; i += kThreads) {
-    const uint64_t k = rank_key(sc[i], static_cast<uint32_t>(i));
-    kmin = k < kmin ? k : kmin;
-    kmax = k > kmax ? k : kmax;
+  // 1. the 2048-bin histogram
+  if (hist_in) {
+    for (int i = tid; i < 2048; i += NT) hist[i] = static_cast<int>(hist_in[static_cast<size_t>(b) * 2048 + i]);
+  } else {
+    for (int i = tid; i < 2048; i += NT) hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < n; i += NT) atomicAdd(hist + key_bin11(rank_key(sc[i], static_cast<uint32_t>(i))), 1);
   }
   if (tid == 0) {
-    mm[0] = ~0ull;
-    mm[1] = 0ull;
+    wpos = 0;
+    bpos = 0;
   }
   __syncthreads();
-  atomicMin(&mm[0], kmin);
-  atomicMax(&mm[1], kmax);
-  __syncthreads();
-  const uint64_t diff = mm[0] ^ mm[1];
-  const int hi_bit = diff ? 63 - __clzll(static_cast<long long>(diff)) : 0;
-  int shift = hi_bit & ~7;
-  uint64_t prefix = (shift + 8 >= 64) ? 0ull : (static_cast<uint64_t>(mm[1]) >> (shift + 8)) << (shift + 8);
-  int remaining = K;
-  while (true) {
-    for (int i = tid; i < 256; i += kThreads) hist[i] = 0;
+  // 2. bin of the K-th largest key: descending scan, 2 bins per thread
+  {
+    const int c0 = hist[2047 - 2 * tid], c1 = hist[2046 - 2 * tid];
+    const int tot = c0 + c1;
+    const int l = tid & 31, w = tid >> 5;
+    int incl = tot;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (l >= off) incl += y;
+    }
+    if (l == 31) wsum[w] = incl;
     __syncthreads();
-    for (int i = tid; i < n; i += kThreads) {
+    int wbase = 0;
+    for (int i = 0; i < w; ++i) wbase += wsum[i];
+    const int excl = wbase + incl - tot;
+    if (excl < K && excl + tot >= K) {
+      if (excl + c0 >= K) {
+        res[0] = 2047 - 2 * tid; res[1] = excl; res[2] = c0;
+      } else {
+        res[0] = 2046 - 2 * tid; res[1] = excl + c0; res[2] = c1;
+      }
+    }
+    __syncthreads();
+  }
+  const uint32_t dbin = static_cast<uint32_t>(res[0]);
+  const int above = res[1], inb = res[2];
+  const int need = K - above;  // keys to take from the boundary bin (1..inb)
+  // 3. one pass: keys above the bin go out; the bin's keys are kept
+  const bool fits = inb <= kDecodeSelBinCap;
+  for (int i = tid; i < n; i += NT) {
+    const uint64_t key = rank_key(sc[i], static_cast<uint32_t>(i));
+    const uint32_t bin = key_bin11(key);
+    if (bin > dbin) {
+      dst[atomicAdd(&wpos, 1)] = key;
+    } else if (bin == dbin && fits) {
+      bin_keys[atomicAdd(&bpos, 1)] = key;
+    }
+  }
+  __syncthreads();
+  // 4. exact choice of `need` keys inside the boundary bin
+  if (fits) {
+    uint64_t v[kDecodeSelBinCap / NT];
+#pragma unroll
+    for (int j = 0; j < kDecodeSelBinCap / NT; ++j) {
+      const int i = tid + j * NT;
+      v[j] = (i < inb) ? bin_keys[i] : 0ull;
+    }
+    uint64_t floor = 1ull;
+    if (need < inb) floor = radix_select_floor<NT, kDecodeSelBinCap / NT>(v, need, scr, tid, 1);
+#pragma unroll
+    for (int j = 0; j < kDecodeSelBinCap / NT; ++j)
+      if (v[j] != 0 && v[j] >= floor) dst[atomicAdd(&wpos, 1)] = v[j];
+    return;
+  }
+  // the boundary bin is too large for shared memory: radix select over the
+  // bin's keys in global memory, 8-bit digits below the 11-bit bin, then 5
+  uint64_t prefix = static_cast<uint64_t>(dbin) << 53;
+  int remaining = need;
+  for (int shift = 45; shift >= 0; shift = (shift >= 13) ? shift - 8 : (shift == 5 ? 0 : -1)) {
+    const int width = (shift == 0) ? 5 : 8;
+    for (int i = tid; i < 256; i += NT) hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < n; i += NT) {
       const uint64_t x = rank_key(sc[i], static_cast<uint32_t>(i));
-      if ((shift + 8 >= 64) || ((x >> (shift + 8)) == (prefix >> (shift + 8))))
-        atomicAdd(&hist[(x >> shift) & 255u], 1);
+      if ((x >> (shift + width)) == (prefix >> (shift + width)))
+        atomicAdd(&hist[(x >> shift) & ((1u << width) - 1u)], 1);
     }
     __syncthreads();
     if (tid < 32) {
@@ -248,9 +334,9 @@ __global__ void __launch_bounds__(kThreads)
         int cum = incl - tot;
         for (int i = 0; i < 8; ++i) {
           if (cum + c[i] >= remaining) {
-            misc[0] = 255 - 8 * tid - i;
-            misc[1] = cum;
-            misc[2] = c[i];
+            res[0] = 255 - 8 * tid - i;
+            res[1] = cum;
+            res[2] = c[i];
             break;
           }
           cum += c[i];
@@ -258,18 +344,16 @@ __global__ void __launch_bounds__(kThreads)
       }
     }
     __syncthreads();
-    const int d = misc[0], above = misc[1], inb = misc[2];
-    remaining -= above;
+    const int d = res[0], ab = res[1], ib = res[2];
+    remaining -= ab;
     prefix |= static_cast<uint64_t>(d) << shift;
     __syncthreads();
-    if (inb == remaining || shift == 0) break;
-    shift -= 8;
+    if (ib == remaining) break;
   }
-  if (tid == 0) misc[3] = 0;
-  __syncthreads();
-  for (int i = tid; i < n; i += kThreads) {
+  // keys of the bin that are >= prefix
+  for (int i = tid; i < n; i += NT) {
     const uint64_t x = rank_key(sc[i], static_cast<uint32_t>(i));
-    if (x >= prefix) dst[atomicAdd(&misc[3], 1)] = x;
+    if (key_bin11(x) == dbin && x >= prefix) dst[atomicAdd(&wpos, 1)] = x;
   }
 }
 

@@ -60,9 +60,11 @@ struct IdxPrefillCfg {
   static constexpr int OFF_W = OFF_K + KST * KTILE_BYTES;  // f32 [RB][HI]
   static constexpr int OFF_QS = OFF_W + RB * HI * 4;       // f32 [RB]
   static constexpr int OFF_THR = OFF_QS + RB * 4;          // u64 [RB]
-  static constexpr int OFF_CNT = OFF_THR + RB * 8;         // i32 [RB]
-  static constexpr int OFF_SCR = OFF_CNT + RB * 4;         // i32 [272] select scratch
-  static constexpr int OFF_BAR = (OFF_SCR + 272 * 4 + 7) / 8 * 8;
+  static constexpr int OFF_CNT = OFF_THR + RB * 8;         // i32 [RB][4] sub-list counts
+  static constexpr int OFF_SCR = OFF_CNT + RB * 16;        // i32 select scratch
+  static constexpr int SCR_INTS = (select_scratch_ints(NEPI * 32) > cut_scratch_ints()) ? select_scratch_ints(NEPI * 32)
+                                                                                        : cut_scratch_ints();
+  static constexpr int OFF_BAR = (OFF_SCR + SCR_INTS * 4 + 7) / 8 * 8;
   static constexpr int NBAR = 2 + 2 * KST + 2 * NACC;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;      // tmem base, abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
@@ -87,30 +89,28 @@ struct IdxPrefillParams {
   int row0, nrows;
 };
 
-// sum_j w[j] * max(x_j, 0) over the H_I accumulator columns of one token,
-// j ascending. Shared by both modes so their scores are bit-identical.
+// sum_j w[j] * max(x_j, 0) over the H_I accumulator values of one token
+// (registers loaded from TMEM). Heads are taken in pairs with the packed fp32
+// FMA into four independent accumulator pairs, summed in a fixed order at the
+// end. Shared by both modes so their scores are bit-identical.
 template <int HI>
-__device__ __forceinline__ float relu_weighted_head_sum(uint32_t taddr, const float* __restrict__ w) {
-  float acc = 0.f;
-  if constexpr (HI % 32 == 0) {
+__device__ __forceinline__ float relu_weighted_head_sum(const uint32_t* x, const float* __restrict__ w) {
+  static_assert(HI % 8 == 0, "H_I must be a multiple of 8");
+  const float2* w2 = reinterpret_cast<const float2*>(w);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-    for (int h = 0; h < HI / 32; ++h) {
-      uint32_t r[32];
-      tmem_ld32(taddr + h * 32, r);
+  for (int j = 0; j < HI; j += 8) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) acc = __fmaf_rn(w[h * 32 + j], fmaxf(__uint_as_float(r[j]), 0.f), acc);
+    for (int a = 0; a < 4; ++a) {
+      const float2 xr = make_float2(fmaxf(__uint_as_float(x[j + 2 * a]), 0.f),
+                                    fmaxf(__uint_as_float(x[j + 2 * a + 1]), 0.f));
+      acc[a] = __ffma2_rn(w2[j / 2 + a], xr, acc[a]);
     }
-  } else {
-    static_assert(HI == 8, "H_I must be 8 or a multiple of 32");
-    uint32_t r[8];
-    tmem_ld8(taddr, r);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc = __fmaf_rn(w[j], fmaxf(__uint_as_float(r[j]), 0.f), acc);
   }
-  return acc;
+  return ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
 }
 
-template <int HI, int DI, bool kSelect, int MAXPER>
+template <int HI, int DI, bool kSelect, int MQ>
 __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
     indexer_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                            const IdxPrefillParams p) {
@@ -245,9 +245,15 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
     const int quarter = static_cast<int>(warp & 3);    // TMEM lane quarter this warp may access
     const int half = e / 4;                            // which half of a buffer's tokens
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t lanemask_lt = (1u << lane) - 1u;
     uint32_t af_phase[C::NACC];
     for (int b = 0; b < C::NACC; ++b) af_phase[b] = 0;
+    // Row tl's list is four quarter sub-lists of capq keys; sub-list q only
+    // receives keys from TMEM lane quarter q, so exactly one warp appends to
+    // it and its count needs no atomics.
+    const int capq = p.cap / 4;
     uint64_t* my_cand = p.cand + static_cast<size_t>(blockIdx.x) * C::RB * p.cap;
+    int* pos_s = scr_s + cut_scratch_ints() - 16;  // 9 ints: warp sums of the block scan
 
     for (int j = blockIdx.x; j < nrb; j += G) {
       const int rb = p.rb_end - 1 - j;
@@ -263,58 +269,101 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
         const int t = t0 + i;
         qs_s[i] = (t < p.L) ? p.q_scale[t] : 0.f;
         thr_s[i] = 0ull;
-        cnt_s[i] = 0;
       }
+      for (int i = et; i < 4 * C::RB; i += C::NET) cnt_s[i] = 0;
       named_bar_sync(1, C::NET);
       bool ok = true;
+      float ks_next = 0.f;
+      {
+        const int s0 = quarter * 32 + static_cast<int>(lane);
+        ks_next = (s0 < p.L) ? __ldg(p.k_scale + s0) : 0.f;
+      }
       for (int kt = 0; kt < nkt && ok; ++kt) {
         const int s = kt * C::BM + quarter * 32 + static_cast<int>(lane);
-        const float ks = (s < p.L) ? p.k_scale[s] : 0.f;
+        const float ks = ks_next;
+        if (kt + 1 < nkt) {
+          const int sn = s + C::BM;
+          ks_next = (sn < p.L) ? __ldg(p.k_scale + sn) : 0.f;
+        }
         for (int b = 0; b < C::NACC; ++b) {
           if (!mbar_wait(acc_full + b, af_phase[b], ab, 8)) { ok = false; break; }
           af_phase[b] ^= 1;
           tc_fence_after();
-#pragma unroll 1
-          for (int q = 0; q < C::TOK_PER_WARP; ++q) {
-            const int tt = half * C::TOK_PER_WARP + q;   // token within the buffer
-            const int tl = b * C::TB + tt;               // token within the row block
-            const int t = t0 + tl;
-            const float acc = relu_weighted_head_sum<HI>(tmem + lane_addr + b * C::NCOL + tt * HI, w_s + tl * HI);
-            const float score = __fmul_rn(__fmul_rn(acc, qs_s[tl]), ks);
-            const bool valid = (t < p.L) && (s <= t);
-            if constexpr (kSelect) {
-              const uint64_t key = rank_key(score, static_cast<uint32_t>(s));
-              const bool pred = valid && key > thr_s[tl];
-              const uint32_t m = __ballot_sync(0xffffffffu, pred);
-              if (m) {
-                const int leader = __ffs(m) - 1;
-                int base = 0;
-                if (static_cast<int>(lane) == leader) base = atomicAdd(cnt_s + tl, __popc(m));
-                base = __shfl_sync(0xffffffffu, base, leader);
-                if (pred) my_cand[static_cast<size_t>(tl) * p.cap + base + __popc(m & ((1u << lane) - 1u))] = key;
-              }
-            } else {
-              if (valid && t >= p.row0 && t < p.row0 + p.nrows)
-                p.scores[static_cast<size_t>(t - p.row0) * p.L + s] = score;
-            }
-          }
+          // this warp's tokens are 128 consecutive accumulator columns
+          uint32_t xr[C::TOK_PER_WARP * HI];
+          static_assert(C::TOK_PER_WARP * HI == 128, "one 128-column load per warp and buffer");
+          tmem_ld128(tmem + lane_addr + b * C::NCOL + half * 128, xr);
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(acc_empty + b);
+          if (lane == 0) mbar_arrive(acc_empty + b);  // the tensor core may refill this buffer now
+          // row state first (its loads overlap the arithmetic), every token's
+          // score next (independent chains), then the filter
+          uint64_t thr_r[C::TOK_PER_WARP];
+          int base_r[C::TOK_PER_WARP];
+          if constexpr (kSelect) {
+#pragma unroll
+            for (int q = 0; q < C::TOK_PER_WARP; ++q) {
+              const int tl = b * C::TB + half * C::TOK_PER_WARP + q;
+              thr_r[q] = thr_s[tl];
+              base_r[q] = cnt_s[tl * 4 + quarter];
+            }
+          }
+          float score[C::TOK_PER_WARP];
+#pragma unroll
+          for (int q = 0; q < C::TOK_PER_WARP; ++q) {
+            const int tl = b * C::TB + half * C::TOK_PER_WARP + q;
+            const float acc = relu_weighted_head_sum<HI>(xr + q * HI, w_s + tl * HI);
+            score[q] = __fmul_rn(__fmul_rn(acc, qs_s[tl]), ks);
+          }
+#pragma unroll
+          for (int q = 0; q < C::TOK_PER_WARP; ++q) {
+            const int tl = b * C::TB + half * C::TOK_PER_WARP + q;
+            const int t = t0 + tl;
+            const bool valid = (t < p.L) && (s <= t);
+            if constexpr (kSelect) {
+              int* cnt = cnt_s + tl * 4 + quarter;
+              const int base = base_r[q];
+              const uint64_t key = rank_key(score[q], static_cast<uint32_t>(s));
+              const bool pred = valid && key > thr_r[q];
+              const uint32_t m = __ballot_sync(0xffffffffu, pred);
+              if (pred)
+                my_cand[static_cast<size_t>(tl) * p.cap + static_cast<size_t>(quarter) * capq + base +
+                        __popc(m & lanemask_lt)] = key;
+              __syncwarp();
+              if (lane == 0 && m) *cnt = base + __popc(m);
+            } else {
+              if (valid && t >= p.row0 && t < p.row0 + p.nrows)
+                p.scores[static_cast<size_t>(t - p.row0) * p.L + s] = score[q];
+            }
+          }
         }
         if constexpr (kSelect) {
-          // Cut any list that could overflow on the next tile (at most BM
-          // appends per row per tile).
+          // Cut any list whose sub-list could overflow on the next tile (at
+          // most 32 appends per sub-list and tile): one histogram pass keeps
+          // every key in or above the bin of the k-th largest; if that keeps
+          // too many, an exact select keeps exactly k.
           named_bar_sync(1, C::NET);
           for (int tl = 0; tl < C::RB; ++tl) {
-            const int n = cnt_s[tl];
-            if (n > p.cap - C::BM) {
-              const uint64_t floor =
-                  compact_top_k<C::NET, MAXPER>(my_cand + static_cast<size_t>(tl) * p.cap, n, p.topk, scr_s, et, 1);
-              if (et == 0) {
-                cnt_s[tl] = p.topk;
-                thr_s[tl] = floor - 1;
+            const int* cn = cnt_s + tl * 4;
+            const int nmax = max(max(cn[0], cn[1]), max(cn[2], cn[3]));
+            if (nmax > capq - 32) {
+              uint64_t* row = my_cand + static_cast<size_t>(tl) * p.cap;
+              const int n = cn[0] + cn[1] + cn[2] + cn[3];
+              uint64_t v[4 * MQ];
+              load_sublists<C::NET, MQ>(row, capq, cn, et, v);
+              uint64_t floor = 1ull;  // fewer than topk keys: only rebalance the sub-lists
+              if (n > p.topk) {
+                int above = 0, inb = 0;
+                floor = histogram_cut<C::NET, 4 * MQ>(v, p.topk, scr_s, et, 1, &above, &inb);
+                if (above + inb > p.cap / 2) {
+                  // keys below the boundary bin can go now; exact select on the rest
+#pragma unroll
+                  for (int i = 0; i < 4 * MQ; ++i) v[i] = (v[i] >= floor) ? v[i] : 0ull;
+                  floor = radix_select_floor<C::NET, 4 * MQ>(v, p.topk, scr_s, et, 1);
+                }
               }
+              store_sublists<C::NET, MQ>(row, capq, cnt_s + tl * 4, v, floor, pos_s, et, 1);
+              if (et == 0 && floor - 1 > thr_s[tl]) thr_s[tl] = floor - 1;
               named_bar_sync(1, C::NET);
             }
           }
@@ -322,18 +371,39 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
       }
       if (!ok) break;
       if constexpr (kSelect) {
+        // exact top-k of each row: the histogram pass finds the boundary bin,
+        // a radix select over that bin's keys alone finds the exact cut
         named_bar_sync(1, C::NET);
         for (int tl = 0; tl < C::RB; ++tl) {
           const int t = t0 + tl;
           if (t >= p.L) break;
-          uint64_t* c = my_cand + static_cast<size_t>(tl) * p.cap;
-          int n = cnt_s[tl];
+          const int* cn = cnt_s + tl * 4;
+          const int n = cn[0] + cn[1] + cn[2] + cn[3];
+          uint64_t* row = my_cand + static_cast<size_t>(tl) * p.cap;
+          uint64_t v[4 * MQ];
+          load_sublists<C::NET, MQ>(row, capq, cn, et, v);
+          uint64_t floor = 1ull;  // keep every valid key
           if (n > p.topk) {
-            compact_top_k<C::NET, MAXPER>(c, n, p.topk, scr_s, et, 1);
-            n = p.topk;
+            int above = 0, inb = 0;
+            floor = histogram_cut<C::NET, 4 * MQ>(v, p.topk, scr_s, et, 1, &above, &inb);
+            if (above + inb > p.topk) {
+              // the k-th largest lies in the boundary bin: exact select among keys >= its lower edge
+#pragma unroll
+              for (int i = 0; i < 4 * MQ; ++i) v[i] = (v[i] >= floor) ? v[i] : 0ull;
+              floor = radix_select_floor<C::NET, 4 * MQ>(v, p.topk, scr_s, et, 1);
+            }
           }
+          // write the row's selected keys (unordered) and zero-pad to topk
           uint64_t* dst = p.sel_keys + static_cast<size_t>(t) * p.topk;
-          for (int i = et; i < p.topk; i += C::NET) dst[i] = (i < n) ? c[i] : 0ull;
+          int mine = 0;
+#pragma unroll
+          for (int i = 0; i < 4 * MQ; ++i) mine += (v[i] != 0 && v[i] >= floor) ? 1 : 0;
+          int kept = 0;
+          int pos = block_exclusive_scan<C::NET>(mine, pos_s, et, 1, &kept);
+#pragma unroll
+          for (int i = 0; i < 4 * MQ; ++i)
+            if (v[i] != 0 && v[i] >= floor) dst[pos++] = v[i];
+          for (int i = kept + et; i < p.topk; i += C::NET) dst[i] = 0ull;
         }
       }
       named_bar_sync(1, C::NET);

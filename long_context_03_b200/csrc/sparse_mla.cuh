@@ -47,9 +47,10 @@ struct MlaCfg {
   static constexpr int C_BYTES = NSLAB_QK * SLAB_BYTES;  // 36 KB
   static constexpr int V_BYTES = NSLAB_V * SLAB_BYTES;   // 32 KB
   static constexpr int NCST = 4;              // gather ring depth (score CTA)
-  static constexpr int NVST = 5;              // gather ring depth (value CTA)
+  static constexpr int NVST = 4;              // gather ring depth (value CTA)
   static constexpr int NSB = 4;               // S buffers in TMEM
-  static constexpr int NPB = 2;               // P message buffers
+  static constexpr int NPB = 6;               // P message buffers (hide the cluster round trip)
+  static constexpr int KMAX = 2048;           // largest selection (index row staged in smem)
   static constexpr int P_BYTES = M * NK * 2;  // 8 KB, K-major, 64-byte swizzle
   static constexpr int MSG_ALPHA = P_BYTES;           // f32 [128]
   static constexpr int MSG_CTRL = MSG_ALPHA + M * 4;  // u32 [4]: any_rescale
@@ -71,7 +72,8 @@ struct MlaCfg {
   static constexpr int OFF_RING = 0;          // score CTA: NCST x C_BYTES; value CTA: NVST x V_BYTES
   static constexpr int RING_BYTES = (NCST * C_BYTES > NVST * V_BYTES) ? NCST * C_BYTES : NVST * V_BYTES;
   static constexpr int OFF_MSG = OFF_RING + RING_BYTES;  // NPB x MSG_STRIDE (staging / receive)
-  static constexpr int OFF_BAR = OFF_MSG + NPB * MSG_STRIDE;
+  static constexpr int OFF_IDX = OFF_MSG + NPB * MSG_STRIDE;  // int32 [KMAX]: the token's index row
+  static constexpr int OFF_BAR = OFF_IDX + KMAX * 4;
   // barriers
   static constexpr int B_RING_FULL = 0;                  // [NVST]
   static constexpr int B_RING_EMPTY = B_RING_FULL + NVST;  // [NVST]
@@ -143,12 +145,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // ring slot: slab s of row r at slot + s*SLAB_BYTES + r*128, 16-byte chunk c
 // stored at position c ^ (r & 7). `nslab` slabs (9 = full row, 8 = values).
 __device__ __forceinline__ void gather_chunk(uint32_t slot, const __nv_bfloat16* __restrict__ kv_tok,
-                                             const int32_t* __restrict__ idx_tok, int j, int K, int rows,
-                                             int nslab, int ptid) {
+                                             const int32_t* idx_s, int j, int K, int rows, int nslab, int ptid) {
   // 128 producer threads: 4 per row, each thread takes every 4th 16-byte chunk of its row
   const int r = ptid >> 2;
   const int e = j * MlaCfg::NK + r;
-  int row = (e < K) ? __ldg(idx_tok + e) : -1;
+  int row = (e < K) ? idx_s[e] : -1;
   bool valid = row >= 0;
   if (row >= rows) {
     set_device_error(kErrBadIndex, 0);
@@ -163,6 +164,21 @@ __device__ __forceinline__ void gather_chunk(uint32_t slot, const __nv_bfloat16*
   }
 }
 
+// The producer warps copy a token's index row into shared memory once
+// (named barrier 1 among the 128 producer threads on both sides).
+__device__ __forceinline__ void stage_index_row(int32_t* idx_s, const int32_t* __restrict__ idx_tok, int K,
+                                                int ptid) {
+  named_bar_sync(1, MlaCfg::NPROD * 32);  // everyone is done with the previous row
+  if ((K & 3) == 0 && (reinterpret_cast<uintptr_t>(idx_tok) & 15) == 0) {
+    const int4* src = reinterpret_cast<const int4*>(idx_tok);
+    int4* dst = reinterpret_cast<int4*>(idx_s);
+    for (int i = ptid; i < K / 4; i += MlaCfg::NPROD * 32) dst[i] = __ldg(src + i);
+  } else {
+    for (int i = ptid; i < K; i += MlaCfg::NPROD * 32) idx_s[i] = __ldg(idx_tok + i);
+  }
+  named_bar_sync(1, MlaCfg::NPROD * 32);
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
     sparse_mla_kernel(const MlaParams p) {
   using C = MlaCfg;
@@ -171,6 +187,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   int* abort_s = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
   int* rescale_s = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
+  int32_t* idx_s = reinterpret_cast<int32_t*>(smem + C::OFF_IDX);
   const AbortFlag ab{abort_s};
   const uint32_t rank = cluster_ctarank();
   const uint32_t warp = warp_id();
@@ -227,11 +244,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       uint32_t ph = 1;
       for (int tk = cluster_id; tk < p.T; tk += nclusters) {
         const __nv_bfloat16* kv_tok = p.kv + tk * p.kv_token_stride;
-        const int32_t* idx_tok = p.idx + static_cast<size_t>(tk) * p.K;
+        stage_index_row(idx_s, p.idx + static_cast<size_t>(tk) * p.K, p.K, ptid);
         bool ok = true;
         for (int j = 0; j < nchunk; ++j) {
           if (!mbar_wait(bars + C::B_RING_EMPTY + slot, ph, ab, 31)) { ok = false; break; }
-          gather_chunk(ring + slot * C::C_BYTES, kv_tok, idx_tok, j, p.K, p.rows, C::NSLAB_QK, ptid);
+          gather_chunk(ring + slot * C::C_BYTES, kv_tok, idx_s, j, p.K, p.rows, C::NSLAB_QK, ptid);
           cp_async_mbar_arrive(bars + C::B_RING_FULL + slot);
           if (++slot == C::NCST) { slot = 0; ph ^= 1; }
         }
@@ -319,6 +336,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
         const int32_t* idx_tok = p.idx + static_cast<size_t>(tk) * p.K;
         float m_ref = -INFINITY;
         float l_sum = 0.f;
+        int next_idx = (static_cast<int>(lane) < p.K) ? __ldg(idx_tok + lane) : -1;
         for (int j = 0; j < nchunk; ++j) {
           if (!mbar_wait(bars + C::B_S_FULL + sb, sph, ab, 36)) { ok = false; break; }
           tc_fence_after();
@@ -329,8 +347,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
           if (lane == 0) mbar_arrive(bars + C::B_S_EMPTY + sb);
           if (++sb == C::NSB) { sb = 0; sph ^= 1; }
           // validity of the chunk's 32 entries (same for every head)
-          const int e_l = j * C::NK + static_cast<int>(lane);
-          const int my_idx = (e_l < p.K) ? __ldg(idx_tok + e_l) : -1;
+          const int my_idx = next_idx;
+          {
+            const int e_n = (j + 1) * C::NK + static_cast<int>(lane);
+            next_idx = (e_n < p.K) ? __ldg(idx_tok + e_n) : -1;
+          }
           const uint32_t vmask = __ballot_sync(0xffffffffu, my_idx >= 0 && my_idx < p.rows);
           float x[32];
           float mc = -INFINITY;
@@ -398,11 +419,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       uint32_t ph = 1;
       for (int tk = cluster_id; tk < p.T; tk += nclusters) {
         const __nv_bfloat16* kv_tok = p.kv + tk * p.kv_token_stride;
-        const int32_t* idx_tok = p.idx + static_cast<size_t>(tk) * p.K;
+        stage_index_row(idx_s, p.idx + static_cast<size_t>(tk) * p.K, p.K, ptid);
         bool ok = true;
         for (int j = 0; j < nchunk; ++j) {
           if (!mbar_wait(bars + C::B_RING_EMPTY + slot, ph, ab, 41)) { ok = false; break; }
-          gather_chunk(ring + slot * C::V_BYTES, kv_tok, idx_tok, j, p.K, p.rows, C::NSLAB_V, ptid);
+          gather_chunk(ring + slot * C::V_BYTES, kv_tok, idx_s, j, p.K, p.rows, C::NSLAB_V, ptid);
           cp_async_mbar_arrive(bars + C::B_RING_FULL + slot);
           if (++slot == C::NVST) { slot = 0; ph ^= 1; }
         }
