@@ -101,6 +101,7 @@ dsa_status dsa_index_scores(const uint8_t* q_I, const float* q_scale, const floa
  *   idx      [T, topk] int32       rows of kv (-1 = none)
  *   out      [T, Hq, 512] bf16     output
  *   lse      [T, Hq] f32 or NULL
+ *   scale    softmax scale, finite and > 0 (1/sqrt(576) for the latent row)
  * No workspace.
  * ------------------------------------------------------------------------ */
 dsa_status dsa_sparse_mla_attn(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int T, int L, int Hq,

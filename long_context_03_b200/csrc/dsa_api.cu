@@ -262,7 +262,7 @@ dsa_status check_mla_args(const uint16_t* q, const uint16_t* kv, const int32_t* 
     return fail(DSA_ERR_INVALID_ARG, "q / kv / idx / out not 16-byte aligned");
   if (Hq < 1 || Hq > 128) return fail(DSA_ERR_UNSUPPORTED, "Hq=%d not in [1, 128]", Hq);
   if (topk < 1 || topk > DSA_MAX_TOPK) return fail(DSA_ERR_UNSUPPORTED, "topk=%d not in [1, %d]", topk, DSA_MAX_TOPK);
-  if (!std::isfinite(scale)) return fail(DSA_ERR_INVALID_ARG, "scale is not finite");
+  if (!std::isfinite(scale) || !(scale > 0.f)) return fail(DSA_ERR_INVALID_ARG, "scale must be finite and > 0");
   return DSA_OK;
 }
 

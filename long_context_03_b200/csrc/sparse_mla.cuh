@@ -10,22 +10,27 @@
 //
 // The fp32 output tile of one token (128 heads x 512 values) needs all 512
 // TMEM columns of an SM, so each token runs on a 2-CTA cluster:
-//   CTA 0 (score CTA): Q[t] lives in TMEM (288 columns, bf16 pairs) as the A
-//     operand. Per chunk of 32 selected rows it gathers the rows (cp.async,
-//     128-byte swizzled), runs S = Q C^T (M = 128 heads, N = 32 rows, K = 576),
-//     and its softmax warps (one thread per head) turn S into bf16
-//     probabilities P with a running reference max. The max is only moved
-//     when a chunk exceeds it by more than 2^8, so P <= 256 and the
-//     accumulator rarely needs rescaling. P, the per-head rescale factors and,
-//     after the last chunk, the row sums and maxima go to CTA 1 by a bulk
-//     shared-memory copy across the cluster.
-//   CTA 1 (value CTA): gathers the value part (first 512 values) of the same
-//     rows, rescales O when told to, and runs O += P V (M = 128 heads,
-//     N = 2 x 256 values, K = 32 rows) into its full TMEM. Its MMA commit
-//     signals CTA 0 directly (multicast commit) that the P buffer is free.
-//     After the last chunk it writes u = O / l in bf16 and the log-sum-exp.
-// A cluster is persistent over tokens. Work per chunk is balanced: 2*128*576
-// flops per row for QK^T, 2*128*512 for PV.
+//   CTA 0 (score CTA) keeps Q[t, :, 0:512] in TMEM (256 columns of bf16
+//     pairs, the A operand of a TMEM-sourced MMA) and Q[t, :, 512:576] in
+//     shared memory, and computes S = Q C^T for chunks of 128 selected rows
+//     (M = 128 heads, N = 128 rows: a full-rate tcgen05 shape) into one of two
+//     128-column S buffers. The rows are gathered slab by slab (64 values =
+//     128 bytes of each row, 16 KB per slab tile) through a ring, so the
+//     576-wide chunk never has to be resident at once. Its softmax warps
+//     (one thread per head) turn S into bf16 probabilities P with a running
+//     reference max that only moves when a chunk exceeds it by more than 2^8
+//     (so P <= 256 and the accumulator is rarely rescaled), and ship P, the
+//     per-head rescale factors and, after the last chunk, the row sums and
+//     maxima to CTA 1 with a bulk shared-memory copy across the cluster.
+//   CTA 1 (value CTA) gathers the value part (first 512 values) of the same
+//     rows in 32-row sub-tiles, rescales O when told to, and runs O += P V
+//     (M = 128 heads, N = 2 x 256 values, K = 16 rows per instruction) into
+//     its whole TMEM. Its MMA commit tells CTA 0 directly (multicast commit)
+//     that a P buffer is free. After the last chunk it writes u = O / l in
+//     bf16 and the log-sum-exp.
+// Per 128-row chunk the score CTA issues 36 MMAs of 128x128x16 and the value
+// CTA 16 MMAs of 128x256x16: balanced work, both at the tensor core's full
+// per-instruction rate. A cluster is persistent over tokens.
 //
 // Entries idx < 0 are skipped (probability 0). Entries >= the row bound are
 // also skipped and reported through the device error word.
@@ -38,58 +43,62 @@ namespace dsa {
 struct MlaCfg {
   static constexpr int D = 576;               // QK dims
   static constexpr int DV = 512;              // value dims
-  static constexpr int NK = 32;               // selected rows per chunk
+  static constexpr int NK = 128;              // selected rows per chunk (QK^T N)
   static constexpr int M = 128;               // heads per MMA (rows >= Hq are zero)
-  static constexpr int SLAB = 64;             // bf16 values per 128-byte swizzle row
-  static constexpr int NSLAB_QK = D / SLAB;   // 9
-  static constexpr int NSLAB_V = DV / SLAB;   // 8
-  static constexpr int SLAB_BYTES = NK * 128; // one slab of a chunk: 32 rows x 128 B
-  static constexpr int C_BYTES = NSLAB_QK * SLAB_BYTES;  // 36 KB
-  static constexpr int V_BYTES = NSLAB_V * SLAB_BYTES;   // 32 KB
-  static constexpr int NCST = 4;              // gather ring depth (score CTA)
-  static constexpr int NVST = 4;              // gather ring depth (value CTA)
-  static constexpr int NSB = 4;               // S buffers in TMEM
-  static constexpr int NPB = 6;               // P message buffers (hide the cluster round trip)
+  static constexpr int NSLAB_QK = D / 64;     // 9 slabs of 64 values (128 B)
+  static constexpr int NSLAB_V = DV / 64;     // 8
+  static constexpr int SLAB_TILE = NK * 128;  // one slab of a chunk: 128 rows x 128 B = 16 KB
+  static constexpr int NSST = 8;              // slab-tile ring depth (score CTA)
+  static constexpr int VROWS = 32;            // rows per value sub-tile
+  static constexpr int VSLAB = VROWS * 128;   // one slab of a value sub-tile: 4 KB
+  static constexpr int V_TILE = NSLAB_V * VSLAB;  // 32 KB
+  static constexpr int NVST = 4;              // value sub-tile ring depth (value CTA)
+  static constexpr int NSB = 2;               // S buffers in TMEM
+  static constexpr int NPB = 2;               // P message buffers
   static constexpr int KMAX = 2048;           // largest selection (index row staged in smem)
-  static constexpr int P_BYTES = M * NK * 2;  // 8 KB, K-major, 64-byte swizzle
+  static constexpr int P_BYTES = M * NK * 2;  // 32 KB: two 128-byte-swizzled K slabs of 64 rows
   static constexpr int MSG_ALPHA = P_BYTES;           // f32 [128]
   static constexpr int MSG_CTRL = MSG_ALPHA + M * 4;  // u32 [4]: any_rescale
   static constexpr int MSG_L = MSG_CTRL + 16;         // f32 [128] (last chunk only)
   static constexpr int MSG_M = MSG_L + M * 4;         // f32 [128] (last chunk only)
-  static constexpr int MSG_BYTES_MID = MSG_L;         // 8720
-  static constexpr int MSG_BYTES_LAST = MSG_M + M * 4;  // 9744
+  static constexpr int MSG_BYTES_MID = MSG_L;
+  static constexpr int MSG_BYTES_LAST = MSG_M + M * 4;
   static constexpr int MSG_STRIDE = (MSG_BYTES_LAST + 1023) / 1024 * 1024;
   static constexpr int NPROD = 4;             // producer warps
   static constexpr int W_MMA = 4;
   static constexpr int W_SM0 = 5;             // first softmax / epilogue warp
   static constexpr int NTHREADS = 9 * 32;
-  static constexpr int S_COL = 0;             // S buffers: columns [0, NSB*NK)
-  static constexpr int Q_COL = 128;           // Q: columns [128, 416)
+  static constexpr int S_COL = 0;             // S buffers: columns [0, 256)
+  static constexpr int Q_COL = 256;           // Q dims 0..511: columns [256, 512)
   static constexpr uint32_t IDESC_QK = instr_desc(kFmtBF16, M, NK, false, false);
   static constexpr uint32_t IDESC_PV = instr_desc(kFmtBF16, M, 256, false, true);
-  // shared memory (offsets from a 1024-aligned base); the two CTAs share the
+  // shared memory (offsets from a 1024-aligned base); both CTAs use the same
   // layout so barrier offsets match across the cluster
-  static constexpr int OFF_RING = 0;          // score CTA: NCST x C_BYTES; value CTA: NVST x V_BYTES
-  static constexpr int RING_BYTES = (NCST * C_BYTES > NVST * V_BYTES) ? NCST * C_BYTES : NVST * V_BYTES;
-  static constexpr int OFF_MSG = OFF_RING + RING_BYTES;  // NPB x MSG_STRIDE (staging / receive)
+  static constexpr int OFF_RING = 0;          // score CTA: NSST slab tiles; value CTA: NVST value sub-tiles
+  static constexpr int RING_BYTES = (NSST * SLAB_TILE > NVST * V_TILE) ? NSST * SLAB_TILE : NVST * V_TILE;
+  static constexpr int OFF_QROPE = OFF_RING + RING_BYTES;  // score CTA: Q[:, 512:576] (16 KB)
+  static constexpr int OFF_MSG = OFF_QROPE + M * 128;      // NPB x MSG_STRIDE (staging / receive)
   static constexpr int OFF_IDX = OFF_MSG + NPB * MSG_STRIDE;  // int32 [KMAX]: the token's index row
   static constexpr int OFF_BAR = OFF_IDX + KMAX * 4;
   // barriers
-  static constexpr int B_RING_FULL = 0;                  // [NVST]
-  static constexpr int B_RING_EMPTY = B_RING_FULL + NVST;  // [NVST]
-  static constexpr int B_S_FULL = B_RING_EMPTY + NVST;   // [NSB]  (score CTA)
-  static constexpr int B_S_EMPTY = B_S_FULL + NSB;       // [NSB]  (score CTA)
-  static constexpr int B_Q_READY = B_S_EMPTY + NSB;      // score CTA
-  static constexpr int B_Q_FREE = B_Q_READY + 1;         // score CTA
-  static constexpr int B_P_FREE = B_Q_FREE + 1;          // [NPB] score CTA, arrived by the value CTA's MMA
-  static constexpr int B_P_FULL = B_P_FREE + NPB;        // [NPB] value CTA, completed by the bulk copy
-  static constexpr int B_O_READY = B_P_FULL + NPB;       // [NPB] value CTA: correction done
-  static constexpr int B_PV_DONE = B_O_READY + NPB;      // value CTA: a token's last PV is done
-  static constexpr int B_STAGE = B_PV_DONE + 1;          // score CTA: softmax warps wrote the staging buffer
-  static constexpr int B_QUIESCE = B_STAGE + 1;          // value CTA: all PV issued so far complete
+  static constexpr int NRING = (NSST > NVST) ? NSST : NVST;
+  static constexpr int B_RING_FULL = 0;                     // [NRING]
+  static constexpr int B_RING_EMPTY = B_RING_FULL + NRING;  // [NRING]
+  static constexpr int B_S_FULL = B_RING_EMPTY + NRING;     // [NSB]  (score CTA)
+  static constexpr int B_S_EMPTY = B_S_FULL + NSB;          // [NSB]  (score CTA)
+  static constexpr int B_Q_READY = B_S_EMPTY + NSB;         // score CTA
+  static constexpr int B_Q_FREE = B_Q_READY + 1;            // score CTA
+  static constexpr int B_P_FREE = B_Q_FREE + 1;             // [NPB] score CTA, arrived by the value CTA's MMA
+  static constexpr int B_P_FULL = B_P_FREE + NPB;           // [NPB] value CTA, completed by the bulk copy
+  static constexpr int B_O_READY = B_P_FULL + NPB;          // [NPB] value CTA: correction done
+  static constexpr int B_PV_DONE = B_O_READY + NPB;         // value CTA: a token's last PV is done
+  static constexpr int B_STAGE = B_PV_DONE + 1;             // score CTA: softmax warps wrote the staging buffer
+  static constexpr int B_QUIESCE = B_STAGE + 1;             // value CTA: all PV issued so far complete
   static constexpr int NBAR = B_QUIESCE + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 32;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(KMAX % NK == 0, "chunks tile the largest selection");
 };
 
 struct MlaParams {
@@ -136,31 +145,60 @@ __device__ __forceinline__ void tc_commit_mc(uint64_t* bar, uint16_t mask) {
       : "memory");
 }
 
+// 2^x with the hardware approximation (relative error a few ulp; P is
+// rounded to bf16 afterwards). ex2 of -inf is +0.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Gather rows [j*NK, j*NK+NK) of a token's selection into a 128-byte-swizzled
-// ring slot: slab s of row r at slot + s*SLAB_BYTES + r*128, 16-byte chunk c
-// stored at position c ^ (r & 7). `nslab` slabs (9 = full row, 8 = values).
-__device__ __forceinline__ void gather_chunk(uint32_t slot, const __nv_bfloat16* __restrict__ kv_tok,
-                                             const int32_t* idx_s, int j, int K, int rows, int nslab, int ptid) {
-  // 128 producer threads: 4 per row, each thread takes every 4th 16-byte chunk of its row
-  const int r = ptid >> 2;
-  const int e = j * MlaCfg::NK + r;
+// Row index of selection entry e, or -1 when absent / outside the cache.
+__device__ __forceinline__ int checked_row(const int32_t* idx_s, int e, int K, int rows) {
   int row = (e < K) ? idx_s[e] : -1;
-  bool valid = row >= 0;
   if (row >= rows) {
     set_device_error(kErrBadIndex, 0);
-    valid = false;
+    row = -1;
   }
-  const char* src_row = reinterpret_cast<const char*>(kv_tok + static_cast<long long>(valid ? row : 0) * MlaCfg::D);
-  const int nchunks = nslab * 8;
-  for (int c = (ptid & 3); c < nchunks; c += 4) {
-    const int s = c >> 3, cc = c & 7;
-    const uint32_t dst = slot + s * MlaCfg::SLAB_BYTES + r * 128 + ((cc ^ (r & 7)) << 4);
-    cp_async_16_zfill(dst, src_row + c * 16, valid);
+  return row;
+}
+
+// Score CTA: slab s (values 64s..64s+63) of chunk j's 128 rows into a 16 KB
+// 128-byte-swizzled tile: row r at r*128, 16-byte chunk c at c ^ (r & 7).
+// Eight consecutive threads copy one row's 128 bytes, so each warp-wide copy
+// covers four whole row segments.
+__device__ __forceinline__ void gather_slab_tile(uint32_t tile, const __nv_bfloat16* __restrict__ kv_tok,
+                                                 const int32_t* idx_s, int j, int s, int K, int rows, int ptid) {
+  const int c = ptid & 7;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int r = (ptid >> 3) + 16 * k;
+    const int row = checked_row(idx_s, j * MlaCfg::NK + r, K, rows);
+    const char* src =
+        reinterpret_cast<const char*>(kv_tok + static_cast<long long>(row >= 0 ? row : 0) * MlaCfg::D) + s * 128;
+    cp_async_16_zfill(tile + r * 128 + ((c ^ (r & 7)) << 4), src + c * 16, row >= 0);
+  }
+}
+
+// Value CTA: rows [j*128 + u*32, +32) of the selection, first 512 values, into
+// a 32 KB sub-tile: slab s at s*4096, row r at r*128, chunk c at c ^ (r & 7).
+// Eight consecutive threads copy one (row, slab) segment of 128 bytes.
+__device__ __forceinline__ void gather_value_tile(uint32_t tile, const __nv_bfloat16* __restrict__ kv_tok,
+                                                  const int32_t* idx_s, int j, int u, int K, int rows, int ptid) {
+  const int c = ptid & 7;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const int seg = (ptid >> 3) + 16 * k;  // 0..255 = 32 rows x 8 slabs
+    const int r = seg >> 3, s = seg & 7;
+    const int row = checked_row(idx_s, j * MlaCfg::NK + u * MlaCfg::VROWS + r, K, rows);
+    const char* src =
+        reinterpret_cast<const char*>(kv_tok + static_cast<long long>(row >= 0 ? row : 0) * MlaCfg::D) + s * 128;
+    cp_async_16_zfill(tile + s * MlaCfg::VSLAB + r * 128 + ((c ^ (r & 7)) << 4), src + c * 16, row >= 0);
   }
 }
 
@@ -195,12 +233,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
   const int cluster_id = blockIdx.x >> 1;
   const int nclusters = gridDim.x >> 1;
   const int nchunk = (p.K + C::NK - 1) / C::NK;
+  const int total_msgs = ((p.T - 1 - cluster_id) / nclusters + 1) * nchunk;  // messages this cluster sends
 
   if (threadIdx.x == 0) {
     *abort_s = 0;
     rescale_s[0] = 0;
     rescale_s[1] = 0;
-    for (int i = 0; i < C::NVST; ++i) {
+    for (int i = 0; i < C::NRING; ++i) {
       mbar_init(bars + C::B_RING_FULL + i, C::NPROD * 32);
       mbar_init(bars + C::B_RING_EMPTY + i, 1);
     }
@@ -224,8 +263,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
   __syncthreads();
   // Value CTA: arm the first use of each P receive buffer before the peer can send.
   if (rank == 1 && threadIdx.x == 0) {
-    const int total = ((p.T - 1 - cluster_id) / nclusters + 1) * nchunk;  // messages this cluster receives
-    for (int i = 0; i < C::NPB && i < total; ++i) {
+    for (int i = 0; i < C::NPB && i < total_msgs; ++i) {
       const bool last = ((i % nchunk) == nchunk - 1);
       mbar_arrive_expect_tx(bars + C::B_P_FULL + i, last ? C::MSG_BYTES_LAST : C::MSG_BYTES_MID);
     }
@@ -246,11 +284,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
         const __nv_bfloat16* kv_tok = p.kv + tk * p.kv_token_stride;
         stage_index_row(idx_s, p.idx + static_cast<size_t>(tk) * p.K, p.K, ptid);
         bool ok = true;
-        for (int j = 0; j < nchunk; ++j) {
-          if (!mbar_wait(bars + C::B_RING_EMPTY + slot, ph, ab, 31)) { ok = false; break; }
-          gather_chunk(ring + slot * C::C_BYTES, kv_tok, idx_s, j, p.K, p.rows, C::NSLAB_QK, ptid);
-          cp_async_mbar_arrive(bars + C::B_RING_FULL + slot);
-          if (++slot == C::NCST) { slot = 0; ph ^= 1; }
+        for (int j = 0; j < nchunk && ok; ++j) {
+          for (int s = 0; s < C::NSLAB_QK; ++s) {
+            if (!mbar_wait(bars + C::B_RING_EMPTY + slot, ph, ab, 31)) { ok = false; break; }
+            gather_slab_tile(ring + slot * C::SLAB_TILE, kv_tok, idx_s, j, s, p.K, p.rows, ptid);
+            cp_async_mbar_arrive(bars + C::B_RING_FULL + slot);
+            if (++slot == C::NSST) { slot = 0; ph ^= 1; }
+          }
         }
         if (!ok) break;
       }
@@ -262,26 +302,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
         int sb = 0;
         uint32_t sph = 1;
         uint32_t qph = 0;
+        const uint32_t qrope = smem_u32(smem + C::OFF_QROPE);
         bool ok = true;
         for (int tk = cluster_id; tk < p.T && ok; tk += nclusters) {
           if (!mbar_wait(bars + C::B_Q_READY, qph, ab, 32)) break;
           qph ^= 1;
           tc_fence_after();
-          for (int j = 0; j < nchunk; ++j) {
-            if (!mbar_wait(bars + C::B_RING_FULL + slot, ph, ab, 33)) { ok = false; break; }
+          for (int j = 0; j < nchunk && ok; ++j) {
             if (!mbar_wait(bars + C::B_S_EMPTY + sb, sph, ab, 34)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t cbase = ring + slot * C::C_BYTES;
+            const uint32_t d = tmem + C::S_COL + sb * C::NK;
+            for (int s = 0; s < C::NSLAB_QK; ++s) {
+              if (!mbar_wait(bars + C::B_RING_FULL + slot, ph, ab, 33)) { ok = false; break; }
+              tc_fence_after();
+              const uint32_t tile = ring + slot * C::SLAB_TILE;
 #pragma unroll
-            for (int kk = 0; kk < C::D / 16; ++kk) {
-              const uint32_t baddr = cbase + (kk >> 2) * C::SLAB_BYTES + (kk & 3) * 32;
-              const uint64_t bd = smem_desc(baddr, 16, 1024, kSw128);
-              mma_bf16_ts(tmem + C::S_COL + sb * C::NK, tmem + C::Q_COL + kk * 8, bd, C::IDESC_QK,
-                          kk > 0 ? 1u : 0u);
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t bd = smem_desc(tile + kk * 32, 16, 1024, kSw128);
+                const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+                if (s < C::NSLAB_QK - 1) {
+                  mma_bf16_ts(d, tmem + C::Q_COL + (4 * s + kk) * 8, bd, C::IDESC_QK, acc);
+                } else {
+                  mma_bf16_ss(d, smem_desc(qrope + kk * 32, 16, 1024, kSw128), bd, C::IDESC_QK, acc);
+                }
+              }
+              tc_commit(bars + C::B_RING_EMPTY + slot);
+              if (++slot == C::NSST) { slot = 0; ph ^= 1; }
             }
+            if (!ok) break;
             tc_commit(bars + C::B_S_FULL + sb);
-            tc_commit(bars + C::B_RING_EMPTY + slot);
-            if (++slot == C::NCST) { slot = 0; ph ^= 1; }
             if (++sb == C::NSB) { sb = 0; sph ^= 1; }
           }
           tc_commit(bars + C::B_Q_FREE);
@@ -294,6 +343,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
       const uint32_t peer_msg = map_to_peer(msg, 1);
       const uint32_t peer_pfull = map_to_peer(smem_u32(bars + C::B_P_FULL), 1);
+      uint8_t* qrope_s = smem + C::OFF_QROPE;
       int sb = 0;
       uint32_t sph = 0;
       uint32_t qfree_ph = 1;
@@ -302,14 +352,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       uint32_t stage_ph = 0;
       bool ok = true;
       for (int tk = cluster_id; tk < p.T && ok; tk += nclusters) {
-        // --- load Q[tk] into TMEM once the previous token's QK^T is done ---
+        // --- Q[tk]: values 0..511 to TMEM, 512..575 to shared memory, once
+        //     the previous token's QK^T is done ---
         if (!mbar_wait(bars + C::B_Q_FREE, qfree_ph, ab, 35)) break;
         qfree_ph ^= 1;
         tc_fence_after();
         {
           const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(tk) * p.Hq + h) * C::D);
 #pragma unroll 1
-          for (int cb = 0; cb < C::D / 64; ++cb) {  // 9 blocks of 32 columns (64 values)
+          for (int cb = 0; cb < 8; ++cb) {  // 8 blocks of 32 columns (64 values)
             uint32_t r[32];
 #pragma unroll
             for (int v = 0; v < 8; ++v) {
@@ -322,8 +373,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
             }
             tmem_st32(tmem + lane_addr + C::Q_COL + cb * 32, r);
           }
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint4 x = make_uint4(0, 0, 0, 0);
+            if (h < p.Hq) x = __ldg(qrow + 64 + c);
+            *reinterpret_cast<uint4*>(qrope_s + h * 128 + ((c ^ (h & 7)) << 4)) = x;
+          }
           tmem_st_wait();
         }
+        fence_async_shared();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bars + C::B_Q_READY);
@@ -336,53 +394,88 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
         const int32_t* idx_tok = p.idx + static_cast<size_t>(tk) * p.K;
         float m_ref = -INFINITY;
         float l_sum = 0.f;
-        int next_idx = (static_cast<int>(lane) < p.K) ? __ldg(idx_tok + lane) : -1;
+        int nidx[4];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int e = g * 32 + static_cast<int>(lane);
+          nidx[g] = (e < p.K) ? __ldg(idx_tok + e) : -1;
+        }
         for (int j = 0; j < nchunk; ++j) {
+          // validity of the chunk's 128 entries (same for every head), with
+          // the next chunk's indices already in flight
+          uint32_t vmask[4];
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            vmask[g] = __ballot_sync(0xffffffffu, nidx[g] >= 0 && nidx[g] < p.rows);
+            const int e = (j + 1) * C::NK + g * 32 + static_cast<int>(lane);
+            nidx[g] = (e < p.K) ? __ldg(idx_tok + e) : -1;
+          }
           if (!mbar_wait(bars + C::B_S_FULL + sb, sph, ab, 36)) { ok = false; break; }
           tc_fence_after();
-          uint32_t sr[32];
-          tmem_ld32(tmem + lane_addr + C::S_COL + sb * C::NK, sr);
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bars + C::B_S_EMPTY + sb);
-          if (++sb == C::NSB) { sb = 0; sph ^= 1; }
-          // validity of the chunk's 32 entries (same for every head)
-          const int my_idx = next_idx;
-          {
-            const int e_n = (j + 1) * C::NK + static_cast<int>(lane);
-            next_idx = (e_n < p.K) ? __ldg(idx_tok + e_n) : -1;
-          }
-          const uint32_t vmask = __ballot_sync(0xffffffffu, my_idx >= 0 && my_idx < p.rows);
-          float x[32];
+          const uint32_t s_addr = tmem + lane_addr + C::S_COL + sb * C::NK;
+          // pass 1 over S (32 columns at a time): the chunk's max. Invalid
+          // entries (absent rows, gathered as zeros) are masked to -inf; a
+          // chunk without any is the common case and skips the masking.
+          const bool all_valid = (vmask[0] & vmask[1] & vmask[2] & vmask[3]) == 0xffffffffu;
           float mc = -INFINITY;
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            x[c] = ((vmask >> c) & 1u) ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
-            mc = fmaxf(mc, x[c]);
+          for (int g = 0; g < 4; ++g) {
+            uint32_t sr[32];
+            tmem_ld32(s_addr + g * 32, sr);
+            if (all_valid) {
+#pragma unroll
+              for (int c = 0; c < 32; ++c) mc = fmaxf(mc, __uint_as_float(sr[c]));
+            } else {
+#pragma unroll
+              for (int c = 0; c < 32; ++c)
+                if ((vmask[g] >> c) & 1u) mc = fmaxf(mc, __uint_as_float(sr[c]));
+            }
           }
+          mc = (mc == -INFINITY) ? -INFINITY : mc * p.scale_log2;
           float alpha = 1.f;
           if (mc > -INFINITY && (m_ref == -INFINITY || mc > m_ref + 8.f)) {
             alpha = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - mc);
             m_ref = mc;
             l_sum *= alpha;
           }
-          uint32_t pk[16];
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float p0 = (x[2 * c] == -INFINITY) ? 0.f : exp2f(x[2 * c] - m_ref);
-            const float p1 = (x[2 * c + 1] == -INFINITY) ? 0.f : exp2f(x[2 * c + 1] - m_ref);
-            pk[c] = pack_bf16x2(p0, p1);
-            l_sum += p0 + p1;
-          }
           const bool last = (j == nchunk - 1);
           // staging buffer pb is free once the value CTA's MMA consumed its previous message
           if (!mbar_wait(bars + C::B_P_FREE + pb, pfree_ph, ab, 37)) { ok = false; break; }
           uint8_t* st = smem + C::OFF_MSG + pb * C::MSG_STRIDE;
+          // pass 2: p = 2^(s*scale*log2e - m_ref), packed to bf16 into the
+          // swizzled P rows; eight independent partial row sums
+          const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+          float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int pc = c ^ ((h >> 1) & 3);
-            *reinterpret_cast<uint4*>(st + h * 64 + pc * 16) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          for (int g = 0; g < 4; ++g) {
+            uint32_t sr[32];
+            tmem_ld32(s_addr + g * 32, sr);
+            const uint32_t vm = all_valid ? 0xffffffffu : vmask[g];
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {  // 4 chunks of 8 keys = 16 bytes of the P row
+              uint32_t pk[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int c = c4 * 8 + 2 * i;
+                float p0 = fast_exp2(__fmaf_rn(__uint_as_float(sr[c]), p.scale_log2, neg_m));
+                float p1 = fast_exp2(__fmaf_rn(__uint_as_float(sr[c + 1]), p.scale_log2, neg_m));
+                p0 = ((vm >> c) & 1u) ? p0 : 0.f;
+                p1 = ((vm >> (c + 1)) & 1u) ? p1 : 0.f;
+                pk[i] = pack_bf16x2(p0, p1);
+                part[2 * i] += p0;
+                part[2 * i + 1] += p1;
+              }
+              const int c8 = g * 4 + c4;  // 16-byte chunk index within the 256-byte row
+              const int kslab = c8 >> 3, cc = c8 & 7;
+              *reinterpret_cast<uint4*>(st + kslab * 16384 + h * 128 + ((cc ^ (h & 7)) << 4)) =
+                  make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
           }
+          l_sum += ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bars + C::B_S_EMPTY + sb);
+          if (++sb == C::NSB) { sb = 0; sph ^= 1; }
           reinterpret_cast<float*>(st + C::MSG_ALPHA)[h] = alpha;
           const uint32_t any_rs = __ballot_sync(0xffffffffu, alpha != 1.f);
           if (lane == 0 && any_rs) atomicOr(rescale_s + (pb & 1), 1);
@@ -421,11 +514,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
         const __nv_bfloat16* kv_tok = p.kv + tk * p.kv_token_stride;
         stage_index_row(idx_s, p.idx + static_cast<size_t>(tk) * p.K, p.K, ptid);
         bool ok = true;
-        for (int j = 0; j < nchunk; ++j) {
-          if (!mbar_wait(bars + C::B_RING_EMPTY + slot, ph, ab, 41)) { ok = false; break; }
-          gather_chunk(ring + slot * C::V_BYTES, kv_tok, idx_s, j, p.K, p.rows, C::NSLAB_V, ptid);
-          cp_async_mbar_arrive(bars + C::B_RING_FULL + slot);
-          if (++slot == C::NVST) { slot = 0; ph ^= 1; }
+        for (int j = 0; j < nchunk && ok; ++j) {
+          for (int u = 0; u < C::NK / C::VROWS; ++u) {
+            if (!mbar_wait(bars + C::B_RING_EMPTY + slot, ph, ab, 41)) { ok = false; break; }
+            gather_value_tile(ring + slot * C::V_TILE, kv_tok, idx_s, j, u, p.K, p.rows, ptid);
+            cp_async_mbar_arrive(bars + C::B_RING_FULL + slot);
+            if (++slot == C::NVST) { slot = 0; ph ^= 1; }
+          }
         }
         if (!ok) break;
       }
@@ -437,11 +532,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
         int pb = 0;
         uint32_t pph = 0;
         int use = 0;  // messages consumed, to arm the receive barriers ahead
-        const int total = ((p.T - 1 - cluster_id) / nclusters + 1) * nchunk;
         bool ok = true;
         for (int tk = cluster_id; tk < p.T && ok; tk += nclusters) {
-          for (int j = 0; j < nchunk; ++j) {
-            if (!mbar_wait(bars + C::B_RING_FULL + slot, ph, ab, 42)) { ok = false; break; }
+          for (int j = 0; j < nchunk && ok; ++j) {
             if (!mbar_wait(bars + C::B_P_FULL + pb, pph, ab, 43)) { ok = false; break; }
             const uint32_t any_rs =
                 reinterpret_cast<const volatile uint32_t*>(smem + C::OFF_MSG + pb * C::MSG_STRIDE + C::MSG_CTRL)[0];
@@ -450,28 +543,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
             if (any_rs && j > 0) tc_commit(bars + C::B_QUIESCE);
             if (!mbar_wait(bars + C::B_O_READY + pb, pph, ab, 44)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t vbase = ring + slot * C::V_BYTES;
             const uint32_t pbase = msg + pb * C::MSG_STRIDE;
+            for (int u = 0; u < C::NK / C::VROWS; ++u) {
+              if (!mbar_wait(bars + C::B_RING_FULL + slot, ph, ab, 42)) { ok = false; break; }
+              tc_fence_after();
+              const uint32_t vbase = ring + slot * C::V_TILE;
 #pragma unroll
-            for (int kk = 0; kk < C::NK / 16; ++kk) {
-              const uint64_t ad = smem_desc(pbase + kk * 32, 16, 512, kSw64);
+              for (int kk = 0; kk < C::VROWS / 16; ++kk) {
+                const int ko = u * C::VROWS + kk * 16;  // first key of this k-step within the chunk
+                const uint64_t ad = smem_desc(pbase + (ko >> 6) * 16384 + ((ko & 63) >> 4) * 32, 16, 1024, kSw128);
 #pragma unroll
-              for (int nh = 0; nh < 2; ++nh) {
-                const uint64_t bd = smem_desc(vbase + nh * 4 * C::SLAB_BYTES + kk * 2048, C::SLAB_BYTES, 1024, kSw128);
-                mma_bf16_ss(tmem + nh * 256, ad, bd, C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+                for (int nh = 0; nh < 2; ++nh) {
+                  const uint64_t bd = smem_desc(vbase + nh * 4 * C::VSLAB + kk * 2048, C::VSLAB, 1024, kSw128);
+                  mma_bf16_ss(tmem + nh * 256, ad, bd, C::IDESC_PV, (j > 0 || u > 0 || kk > 0) ? 1u : 0u);
+                }
               }
+              tc_commit(bars + C::B_RING_EMPTY + slot);
+              if (++slot == C::NVST) { slot = 0; ph ^= 1; }
             }
-            tc_commit(bars + C::B_RING_EMPTY + slot);
+            if (!ok) break;
             tc_commit_mc(bars + C::B_P_FREE + pb, 0x1);  // the score CTA's buffer pb is free
             if (j == nchunk - 1) tc_commit(bars + C::B_PV_DONE);
             // re-arm this receive buffer for message use + NPB
             const int nxt = use + C::NPB;
-            if (nxt < total) {
-              const bool last = ((nxt % nchunk) == nchunk - 1);
-              mbar_arrive_expect_tx(bars + C::B_P_FULL + pb, last ? C::MSG_BYTES_LAST : C::MSG_BYTES_MID);
+            if (nxt < total_msgs) {
+              const bool lastm = ((nxt % nchunk) == nchunk - 1);
+              mbar_arrive_expect_tx(bars + C::B_P_FULL + pb, lastm ? C::MSG_BYTES_LAST : C::MSG_BYTES_MID);
             }
             ++use;
-            if (++slot == C::NVST) { slot = 0; ph ^= 1; }
             if (++pb == C::NPB) { pb = 0; pph ^= 1; }
           }
         }
