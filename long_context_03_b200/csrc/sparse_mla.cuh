@@ -168,37 +168,57 @@ __device__ __forceinline__ int checked_row(const int32_t* idx_s, int e, int K, i
   return row;
 }
 
-// Score CTA: slab s (values 64s..64s+63) of chunk j's 128 rows into a 16 KB
-// 128-byte-swizzled tile: row r at r*128, 16-byte chunk c at c ^ (r & 7).
-// Eight consecutive threads copy one row's 128 bytes, so each warp-wide copy
-// covers four whole row segments.
-__device__ __forceinline__ void gather_slab_tile(uint32_t tile, const __nv_bfloat16* __restrict__ kv_tok,
-                                                 const int32_t* idx_s, int j, int s, int K, int rows, int ptid) {
-  const int c = ptid & 7;
+// Score CTA: the 8 rows (r = ptid/8 + 16k) this thread copies for chunk j,
+// as byte pointers to the rows (absent rows point at row 0 and copy zeros).
+struct ChunkRows {
+  const char* src[8];
+  uint32_t valid;  // bit k: row k present
+};
+__device__ __forceinline__ ChunkRows chunk_rows(const __nv_bfloat16* __restrict__ kv_tok, const int32_t* idx_s, int j,
+                                                int K, int rows, int ptid) {
+  ChunkRows cr;
+  cr.valid = 0;
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
     const int r = (ptid >> 3) + 16 * k;
     const int row = checked_row(idx_s, j * MlaCfg::NK + r, K, rows);
-    const char* src =
-        reinterpret_cast<const char*>(kv_tok + static_cast<long long>(row >= 0 ? row : 0) * MlaCfg::D) + s * 128;
-    cp_async_16_zfill(tile + r * 128 + ((c ^ (r & 7)) << 4), src + c * 16, row >= 0);
+    cr.src[k] = reinterpret_cast<const char*>(kv_tok + static_cast<long long>(row >= 0 ? row : 0) * MlaCfg::D) +
+                (ptid & 7) * 16;
+    cr.valid |= (row >= 0 ? 1u : 0u) << k;
+  }
+  return cr;
+}
+// Slab s (values 64s..64s+63) of the chunk's 128 rows into a 16 KB
+// 128-byte-swizzled tile: row r at r*128, 16-byte chunk c at c ^ (r & 7).
+// Eight consecutive threads copy one row's 128 bytes, so each warp-wide copy
+// covers four whole row segments.
+__device__ __forceinline__ void gather_slab_tile(uint32_t tile, const ChunkRows& cr, int s, int ptid) {
+  const int c = ptid & 7;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int r = (ptid >> 3) + 16 * k;
+    cp_async_16_zfill(tile + r * 128 + ((c ^ (r & 7)) << 4), cr.src[k] + s * 128, (cr.valid >> k) & 1u);
   }
 }
 
 // Value CTA: rows [j*128 + u*32, +32) of the selection, first 512 values, into
 // a 32 KB sub-tile: slab s at s*4096, row r at r*128, chunk c at c ^ (r & 7).
-// Eight consecutive threads copy one (row, slab) segment of 128 bytes.
+// Eight consecutive threads copy one (row, slab) segment of 128 bytes; each
+// group of eight handles rows g and g+16 across all eight slabs, so a thread
+// looks up two row indices per sub-tile.
 __device__ __forceinline__ void gather_value_tile(uint32_t tile, const __nv_bfloat16* __restrict__ kv_tok,
                                                   const int32_t* idx_s, int j, int u, int K, int rows, int ptid) {
   const int c = ptid & 7;
+  const int g = ptid >> 3;  // 0..15
 #pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    const int seg = (ptid >> 3) + 16 * k;  // 0..255 = 32 rows x 8 slabs
-    const int r = seg >> 3, s = seg & 7;
+  for (int half = 0; half < 2; ++half) {
+    const int r = g + 16 * half;
     const int row = checked_row(idx_s, j * MlaCfg::NK + u * MlaCfg::VROWS + r, K, rows);
     const char* src =
-        reinterpret_cast<const char*>(kv_tok + static_cast<long long>(row >= 0 ? row : 0) * MlaCfg::D) + s * 128;
-    cp_async_16_zfill(tile + s * MlaCfg::VSLAB + r * 128 + ((c ^ (r & 7)) << 4), src + c * 16, row >= 0);
+        reinterpret_cast<const char*>(kv_tok + static_cast<long long>(row >= 0 ? row : 0) * MlaCfg::D) + c * 16;
+#pragma unroll
+    for (int sl = 0; sl < 8; ++sl)
+      cp_async_16_zfill(tile + sl * MlaCfg::VSLAB + r * 128 + ((c ^ (r & 7)) << 4), src + sl * 128, row >= 0);
   }
 }
 
@@ -285,9 +305,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
         stage_index_row(idx_s, p.idx + static_cast<size_t>(tk) * p.K, p.K, ptid);
         bool ok = true;
         for (int j = 0; j < nchunk && ok; ++j) {
+          const ChunkRows cr = chunk_rows(kv_tok, idx_s, j, p.K, p.rows, ptid);
           for (int s = 0; s < C::NSLAB_QK; ++s) {
             if (!mbar_wait(bars + C::B_RING_EMPTY + slot, ph, ab, 31)) { ok = false; break; }
-            gather_slab_tile(ring + slot * C::SLAB_TILE, kv_tok, idx_s, j, s, p.K, p.rows, ptid);
+            gather_slab_tile(ring + slot * C::SLAB_TILE, cr, s, ptid);
             cp_async_mbar_arrive(bars + C::B_RING_FULL + slot);
             if (++slot == C::NSST) { slot = 0; ph ^= 1; }
           }
