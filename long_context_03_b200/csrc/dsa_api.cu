@@ -95,10 +95,10 @@ dsa_status check_launch(const char* what) {
 }
 
 // ---- prefill indexer ----
-constexpr int kNetPrefill = 8 * 32;  // epilogue threads of the prefill indexer
+constexpr int kNetPrefill = 16 * 32;  // epilogue threads of the prefill indexer
 
 // keys per thread per quarter sub-list in a list cut; list capacity = 4 * MQ * 256
-int select_mq(int topk) { return (topk <= 128) ? 1 : 8; }
+int select_mq(int topk) { return (topk <= 128) ? 1 : 4; }
 int select_cap(int topk) { return 4 * select_mq(topk) * kNetPrefill; }
 
 int rows_per_block(int H_I) { return 2 * (256 / H_I); }
@@ -306,7 +306,7 @@ dsa_status dsa_index_topk(const uint8_t* q_I, const float* q_scale, const float*
   p.cap = select_cap(topk);
   p.sel_keys = ws.sel;
   dsa_status s = (select_mq(topk) == 1) ? dispatch_prefill<true, 1>(H_I, d_I, q_I, k_cache, p, grid, st)
-                                        : dispatch_prefill<true, 8>(H_I, d_I, q_I, k_cache, p, grid, st);
+                                        : dispatch_prefill<true, 4>(H_I, d_I, q_I, k_cache, p, grid, st);
   if (s != DSA_OK) return s;
   return launch_rank_sort(ws.sel, idx, topk, L, st);
 }

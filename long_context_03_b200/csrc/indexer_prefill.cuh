@@ -45,10 +45,11 @@ struct IdxPrefillCfg {
   static constexpr int KST = 4;                // key-tile ring depth
   static constexpr int QBUF_BYTES = NCOL * DI; // one Q half: 256 (token, head) rows x d_I bytes
   static constexpr int KTILE_BYTES = BM * DI;
-  static constexpr int NEPI = 8;               // epilogue warps (2 per TMEM lane quarter)
+  static constexpr int NEPI = 16;              // epilogue warps (4 per TMEM lane quarter)
   static constexpr int NTHREADS = (2 + NEPI) * 32;
   static constexpr int NET = NEPI * 32;        // epilogue threads
-  static constexpr int TOK_PER_WARP = TB / 2;  // tokens of a buffer per epilogue warp
+  static constexpr int TOK_PER_WARP = TB / 4;  // tokens of a buffer per epilogue warp (64 columns)
+  static constexpr int CHECK_EVERY = 4;        // key tiles between list-capacity checks
   static constexpr SwizzleMode SW = (DI == 128) ? kSw128 : kSw64;
   static constexpr uint32_t SBO = 8 * DI;      // bytes between 8-row core groups
   static constexpr uint32_t IDESC = instr_desc(kFmtE4M3, 128, NCOL, false, false);
@@ -70,7 +71,8 @@ struct IdxPrefillCfg {
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
 
   static_assert(HI * TB == NCOL, "heads must divide 256");
-  static_assert(TB % 2 == 0, "two epilogue warps per lane quarter split a buffer's tokens");
+  static_assert(TB % 4 == 0, "four epilogue warps per lane quarter split a buffer's tokens");
+  static_assert(TOK_PER_WARP * HI == 64, "one 64-column slice per warp and buffer");
 };
 
 struct IdxPrefillParams {
@@ -93,6 +95,24 @@ struct IdxPrefillParams {
 // (registers loaded from TMEM). Heads are taken in pairs with the packed fp32
 // FMA into four independent accumulator pairs, summed in a fixed order at the
 // end. Shared by both modes so their scores are bit-identical.
+template <int HI>
+__device__ __forceinline__ void relu_weighted_acc(float2 (&acc)[4], const uint32_t* x, const float* __restrict__ w) {
+  static_assert(HI % 8 == 0, "a multiple of 8 heads");
+  const float2* w2 = reinterpret_cast<const float2*>(w);
+#pragma unroll
+  for (int j = 0; j < HI; j += 8) {
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const float2 xr = make_float2(fmaxf(__uint_as_float(x[j + 2 * a]), 0.f),
+                                    fmaxf(__uint_as_float(x[j + 2 * a + 1]), 0.f));
+      acc[a] = __ffma2_rn(w2[j / 2 + a], xr, acc[a]);
+    }
+  }
+}
+__device__ __forceinline__ float relu_weighted_finish(const float2 (&acc)[4]) {
+  return ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+}
+
 template <int HI>
 __device__ __forceinline__ float relu_weighted_head_sum(const uint32_t* x, const float* __restrict__ w) {
   static_assert(HI % 8 == 0, "H_I must be a multiple of 8");
@@ -243,7 +263,7 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
     const int e = static_cast<int>(warp) - 2;          // 0..NEPI-1
     const int et = e * 32 + static_cast<int>(lane);    // 0..NET-1
     const int quarter = static_cast<int>(warp & 3);    // TMEM lane quarter this warp may access
-    const int half = e / 4;                            // which half of a buffer's tokens
+    const int half = e / 4;                            // which quarter of a buffer's tokens
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t lanemask_lt = (1u << lane) - 1u;
     uint32_t af_phase[C::NACC];
@@ -290,12 +310,13 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
           af_phase[b] ^= 1;
           tc_fence_after();
           // this warp's tokens are 128 consecutive accumulator columns
-          uint32_t xr[C::TOK_PER_WARP * HI];
-          static_assert(C::TOK_PER_WARP * HI == 128, "one 128-column load per warp and buffer");
-          tmem_ld128(tmem + lane_addr + b * C::NCOL + half * 128, xr);
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(acc_empty + b);  // the tensor core may refill this buffer now
+          // this warp's 64 columns in two halves: the second half loads while
+          // the first is reduced
+          const uint32_t cbase = tmem + lane_addr + b * C::NCOL + half * 64;
+          uint32_t xa[32], xb[32];
+          tmem_ld32_nowait(cbase, xa);
+          tmem_ld_wait_fence(xa);
+          tmem_ld32_nowait(cbase + 32, xb);
           // row state first (its loads overlap the arithmetic), every token's
           // score next (independent chains), then the filter
           uint64_t thr_r[C::TOK_PER_WARP];
@@ -309,11 +330,33 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
             }
           }
           float score[C::TOK_PER_WARP];
+          {
+            // columns [0,32) then [32,64) of the slice; a token spans HI columns
+            constexpr int TPH = (HI >= 32) ? 1 : 32 / HI;  // tokens per 32-column half
+            float2 acc[C::TOK_PER_WARP][4];
 #pragma unroll
-          for (int q = 0; q < C::TOK_PER_WARP; ++q) {
-            const int tl = b * C::TB + half * C::TOK_PER_WARP + q;
-            const float acc = relu_weighted_head_sum<HI>(xr + q * HI, w_s + tl * HI);
-            score[q] = __fmul_rn(__fmul_rn(acc, qs_s[tl]), ks);
+            for (int q = 0; q < C::TOK_PER_WARP; ++q)
+#pragma unroll
+              for (int a = 0; a < 4; ++a) acc[q][a] = make_float2(0.f, 0.f);
+            const int tl0 = b * C::TB + half * C::TOK_PER_WARP;
+            if constexpr (HI >= 32) {
+              relu_weighted_acc<32>(acc[0], xa, w_s + tl0 * HI);
+              tmem_ld_wait_fence(xb);
+              relu_weighted_acc<32>(acc[0], xb, w_s + tl0 * HI + 32);
+            } else {
+#pragma unroll
+              for (int q = 0; q < TPH; ++q) relu_weighted_acc<HI>(acc[q], xa + q * HI, w_s + (tl0 + q) * HI);
+              tmem_ld_wait_fence(xb);
+#pragma unroll
+              for (int q = 0; q < TPH; ++q)
+                relu_weighted_acc<HI>(acc[TPH + q], xb + q * HI, w_s + (tl0 + TPH + q) * HI);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty + b);  // the tensor core may refill this buffer now
+#pragma unroll
+            for (int q = 0; q < C::TOK_PER_WARP; ++q)
+              score[q] = __fmul_rn(__fmul_rn(relu_weighted_finish(acc[q]), qs_s[tl0 + q]), ks);
           }
 #pragma unroll
           for (int q = 0; q < C::TOK_PER_WARP; ++q) {
@@ -321,16 +364,21 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
             const int t = t0 + tl;
             const bool valid = (t < p.L) && (s <= t);
             if constexpr (kSelect) {
-              int* cnt = cnt_s + tl * 4 + quarter;
-              const int base = base_r[q];
-              const uint64_t key = rank_key(score[q], static_cast<uint32_t>(s));
-              const bool pred = valid && key > thr_r[q];
-              const uint32_t m = __ballot_sync(0xffffffffu, pred);
-              if (pred)
-                my_cand[static_cast<size_t>(tl) * p.cap + static_cast<size_t>(quarter) * capq + base +
-                        __popc(m & lanemask_lt)] = key;
-              __syncwarp();
-              if (lane == 0 && m) *cnt = base + __popc(m);
+              // a key can only pass if its score reaches the threshold's score
+              const uint32_t sk = float_order_key(score[q]);
+              const bool maybe = valid && sk >= static_cast<uint32_t>(thr_r[q] >> 32);
+              if (__any_sync(0xffffffffu, maybe)) {
+                int* cnt = cnt_s + tl * 4 + quarter;
+                const int base = base_r[q];
+                const uint64_t key = (static_cast<uint64_t>(sk) << 32) | static_cast<uint64_t>(~static_cast<uint32_t>(s));
+                const bool pred = maybe && key > thr_r[q];
+                const uint32_t m = __ballot_sync(0xffffffffu, pred);
+                if (pred)
+                  my_cand[static_cast<size_t>(tl) * p.cap + static_cast<size_t>(quarter) * capq + base +
+                          __popc(m & lanemask_lt)] = key;
+                __syncwarp();
+                if (lane == 0 && m) *cnt = base + __popc(m);
+              }
             } else {
               if (valid && t >= p.row0 && t < p.row0 + p.nrows)
                 p.scores[static_cast<size_t>(t - p.row0) * p.L + s] = score[q];
@@ -338,15 +386,17 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
           }
         }
         if constexpr (kSelect) {
-          // Cut any list whose sub-list could overflow on the next tile (at
-          // most 32 appends per sub-list and tile): one histogram pass keeps
-          // every key in or above the bin of the k-th largest; if that keeps
-          // too many, an exact select keeps exactly k.
+          // Every CHECK_EVERY tiles, cut any list whose sub-list could
+          // overflow before the next check (at most 32 appends per sub-list
+          // and tile): one histogram pass keeps every key in or above the bin
+          // of the k-th largest; if that keeps too many, an exact select
+          // keeps exactly k.
+          if ((kt % C::CHECK_EVERY) != C::CHECK_EVERY - 1) continue;
           named_bar_sync(1, C::NET);
           for (int tl = 0; tl < C::RB; ++tl) {
             const int* cn = cnt_s + tl * 4;
             const int nmax = max(max(cn[0], cn[1]), max(cn[2], cn[3]));
-            if (nmax > capq - 32) {
+            if (nmax > capq - 32 * C::CHECK_EVERY) {
               uint64_t* row = my_cand + static_cast<size_t>(tl) * p.cap;
               const int n = cn[0] + cn[1] + cn[2] + cn[3];
               uint64_t v[4 * MQ];

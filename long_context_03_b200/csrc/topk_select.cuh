@@ -181,7 +181,7 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int* wsum, int et, ui
 // ---------------------------------------------------------------------------
 // Scratch layout (ints) for the cut below: [0, 2048) histogram, then 8 warp
 // sums, then small fields.
-__host__ __device__ constexpr int cut_scratch_ints() { return 2048 + 64; }
+__host__ __device__ constexpr int cut_scratch_ints() { return 2048 + 64; }  // wsum needs NT/32 <= 16 ints
 
 // Count of each 11-bit digit of the valid keys (from the highest bit where the
 // keys differ), then find the digit bin holding the K-th largest key.
@@ -191,7 +191,8 @@ template <int NT, int M>
 __device__ __forceinline__ uint64_t histogram_cut(const uint64_t (&v)[M], int K, int* scratch, int et,
                                                   uint32_t bar_id, int* above_out, int* inb_out) {
   constexpr int NW = NT / 32;
-  static_assert(NT == 256, "the 2048-bin scan assumes 256 threads");
+  static_assert(NT == 256 || NT == 512, "the 2048-bin scan takes 256 or 512 threads");
+  constexpr int BPT = 2048 / NT;  // bins per thread
   int* hist = scratch;
   int* wsum = scratch + 2048;
   unsigned long long* mm = reinterpret_cast<unsigned long long*>(scratch + 2048 + 16);
@@ -232,12 +233,12 @@ __device__ __forceinline__ uint64_t histogram_cut(const uint64_t (&v)[M], int K,
   for (int j = 0; j < M; ++j)
     if (v[j] != 0) atomicAdd(&hist[(v[j] >> shift) & 2047u], 1);
   named_bar_sync(bar_id, NT);
-  // descending scan: thread et owns bins 2047-8et .. 2040-8et
-  int c[8];
+  // descending scan: thread et owns bins 2047-BPT*et .. 2048-BPT*(et+1)
+  int c[BPT];
   int tot = 0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    c[i] = hist[2047 - 8 * et - i];
+  for (int i = 0; i < BPT; ++i) {
+    c[i] = hist[2047 - BPT * et - i];
     tot += c[i];
   }
   const int l = et & 31, w = et >> 5;
@@ -256,9 +257,9 @@ __device__ __forceinline__ uint64_t histogram_cut(const uint64_t (&v)[M], int K,
   if (excl < K && excl + tot >= K) {
     int cum = excl;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < BPT; ++i) {
       if (cum + c[i] >= K) {
-        res[0] = 2047 - 8 * et - i;
+        res[0] = 2047 - BPT * et - i;
         res[1] = cum;
         res[2] = c[i];
         break;
