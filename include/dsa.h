@@ -94,7 +94,9 @@ dsa_status dsa_index_scores(const uint8_t* q_I, const float* q_scale, const floa
  *   z_s = scale * q[t,h,:] . kv[s,:]          for s in idx[t,:], s >= 0
  *   out[t,h,:] = sum_s softmax(z)_s * kv[s, 0:512]   (bf16 out, fp32 math)
  *   lse[t,h] = log(sum_s exp(z_s))            (natural log; -inf if no entry)
- * All heads share each selected row. Entries < 0 are skipped.
+ * All heads share each selected row. Entries < 0 are skipped; an entry >= L
+ * is skipped too and reported as DSA_ERR_BAD_INDEX by dsa_get_device_error.
+ * T = 0 is a no-op that launches nothing (q, idx, out may then be NULL).
  *
  *   q        [T, Hq, 576] bf16
  *   kv       [L, 576] bf16         latent cache rows

@@ -256,8 +256,8 @@ dsa_status launch_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
 
 dsa_status check_mla_args(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int T, int L, int Hq, int topk,
                           float scale, const uint16_t* out) {
-  if (!q || !kv || !idx || !out) return fail(DSA_ERR_INVALID_ARG, "null pointer");
   if (T < 0 || L <= 0) return fail(DSA_ERR_INVALID_ARG, "T=%d L=%d", T, L);
+  if (!kv || (T > 0 && (!q || !idx || !out))) return fail(DSA_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(q) || !aligned16(kv) || !aligned16(out) || !aligned16(idx))
     return fail(DSA_ERR_INVALID_ARG, "q / kv / idx / out not 16-byte aligned");
   if (Hq < 1 || Hq > 128) return fail(DSA_ERR_UNSUPPORTED, "Hq=%d not in [1, 128]", Hq);

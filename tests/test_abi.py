@@ -54,3 +54,10 @@ def test_misaligned_arrays_are_rejected(lib):
 def test_status_strings(lib):
     assert lib.dsa_status_string(0) == b"ok"
     assert lib.dsa_status_string(-5) == b"workspace too small"
+
+
+def test_empty_attention_batch_needs_no_pointers(lib):
+    # T = 0 returns before any CUDA call, so this runs without a GPU
+    kv = ctypes.c_void_p(256)
+    assert lib.dsa_sparse_mla_attn(None, kv, None, 0, 4, 16, 8, ctypes.c_float(0.1), None, None, None) == 0
+    assert lib.dsa_sparse_mla_attn(None, None, None, 0, 4, 16, 8, ctypes.c_float(0.1), None, None, None) == -1
