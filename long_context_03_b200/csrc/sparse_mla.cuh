@@ -317,25 +317,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       }
       asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp == C::W_MMA) {
-      if (lane == 0) {
-        int slot = 0;
-        uint32_t ph = 0;
-        int sb = 0;
-        uint32_t sph = 1;
-        uint32_t qph = 0;
-        const uint32_t qrope = smem_u32(smem + C::OFF_QROPE);
-        bool ok = true;
-        for (int tk = cluster_id; tk < p.T && ok; tk += nclusters) {
-          if (!mbar_wait(bars + C::B_Q_READY, qph, ab, 32)) break;
-          qph ^= 1;
+      // The whole warp runs the loop and waits converged; one elected lane
+      // issues each slab's MMAs together with every commit that covers them.
+      int slot = 0;
+      uint32_t ph = 0;
+      int sb = 0;
+      uint32_t sph = 1;
+      uint32_t qph = 0;
+      const uint32_t qrope = smem_u32(smem + C::OFF_QROPE);
+      bool ok = true;
+      for (int tk = cluster_id; tk < p.T && ok; tk += nclusters) {
+        if (!mbar_wait_warp(bars + C::B_Q_READY, qph, ab, 32)) break;
+        qph ^= 1;
+        tc_fence_after();
+        for (int j = 0; j < nchunk && ok; ++j) {
+          if (!mbar_wait_warp(bars + C::B_S_EMPTY + sb, sph, ab, 34)) { ok = false; break; }
           tc_fence_after();
-          for (int j = 0; j < nchunk && ok; ++j) {
-            if (!mbar_wait(bars + C::B_S_EMPTY + sb, sph, ab, 34)) { ok = false; break; }
+          const uint32_t d = tmem + C::S_COL + sb * C::NK;
+          for (int s = 0; s < C::NSLAB_QK; ++s) {
+            if (!mbar_wait_warp(bars + C::B_RING_FULL + slot, ph, ab, 33)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t d = tmem + C::S_COL + sb * C::NK;
-            for (int s = 0; s < C::NSLAB_QK; ++s) {
-              if (!mbar_wait(bars + C::B_RING_FULL + slot, ph, ab, 33)) { ok = false; break; }
-              tc_fence_after();
+            if (elect_one()) {
               const uint32_t tile = ring + slot * C::SLAB_TILE;
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
@@ -348,13 +350,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
                 }
               }
               tc_commit(bars + C::B_RING_EMPTY + slot);
-              if (++slot == C::NSST) { slot = 0; ph ^= 1; }
+              if (s == C::NSLAB_QK - 1) {
+                tc_commit(bars + C::B_S_FULL + sb);
+                if (j == nchunk - 1) tc_commit(bars + C::B_Q_FREE);
+              }
             }
-            if (!ok) break;
-            tc_commit(bars + C::B_S_FULL + sb);
-            if (++sb == C::NSB) { sb = 0; sph ^= 1; }
+            __syncwarp();
+            if (++slot == C::NSST) { slot = 0; ph ^= 1; }
           }
-          tc_commit(bars + C::B_Q_FREE);
+          if (!ok) break;
+          if (++sb == C::NSB) { sb = 0; sph ^= 1; }
         }
       }
     } else {
@@ -547,27 +552,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       }
       asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp == C::W_MMA) {
-      if (lane == 0) {
-        int slot = 0;
-        uint32_t ph = 0;
-        int pb = 0;
-        uint32_t pph = 0;
-        int use = 0;  // messages consumed, to arm the receive barriers ahead
-        bool ok = true;
-        for (int tk = cluster_id; tk < p.T && ok; tk += nclusters) {
-          for (int j = 0; j < nchunk && ok; ++j) {
-            if (!mbar_wait(bars + C::B_P_FULL + pb, pph, ab, 43)) { ok = false; break; }
-            const uint32_t any_rs =
-                reinterpret_cast<const volatile uint32_t*>(smem + C::OFF_MSG + pb * C::MSG_STRIDE + C::MSG_CTRL)[0];
-            // A rescale needs O quiescent: commit everything issued so far to
-            // QUIESCE; the correction warps wait on it, rescale, then signal O_READY.
-            if (any_rs && j > 0) tc_commit(bars + C::B_QUIESCE);
-            if (!mbar_wait(bars + C::B_O_READY + pb, pph, ab, 44)) { ok = false; break; }
+      // whole warp waits converged; one elected lane issues and commits
+      int slot = 0;
+      uint32_t ph = 0;
+      int pb = 0;
+      uint32_t pph = 0;
+      int use = 0;  // messages consumed, to arm the receive barriers ahead
+      bool ok = true;
+      for (int tk = cluster_id; tk < p.T && ok; tk += nclusters) {
+        for (int j = 0; j < nchunk && ok; ++j) {
+          if (!mbar_wait_warp(bars + C::B_P_FULL + pb, pph, ab, 43)) { ok = false; break; }
+          const uint32_t any_rs =
+              reinterpret_cast<const volatile uint32_t*>(smem + C::OFF_MSG + pb * C::MSG_STRIDE + C::MSG_CTRL)[0];
+          // A rescale needs O quiescent: commit everything issued so far to
+          // QUIESCE; the correction warps wait on it, rescale, then signal O_READY.
+          if (any_rs && j > 0) {
+            if (elect_one()) tc_commit(bars + C::B_QUIESCE);
+            __syncwarp();
+          }
+          if (!mbar_wait_warp(bars + C::B_O_READY + pb, pph, ab, 44)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t pbase = msg + pb * C::MSG_STRIDE;
+          for (int u = 0; u < C::NK / C::VROWS; ++u) {
+            if (!mbar_wait_warp(bars + C::B_RING_FULL + slot, ph, ab, 42)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t pbase = msg + pb * C::MSG_STRIDE;
-            for (int u = 0; u < C::NK / C::VROWS; ++u) {
-              if (!mbar_wait(bars + C::B_RING_FULL + slot, ph, ab, 42)) { ok = false; break; }
-              tc_fence_after();
+            if (elect_one()) {
               const uint32_t vbase = ring + slot * C::V_TILE;
 #pragma unroll
               for (int kk = 0; kk < C::VROWS / 16; ++kk) {
@@ -580,20 +589,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
                 }
               }
               tc_commit(bars + C::B_RING_EMPTY + slot);
-              if (++slot == C::NVST) { slot = 0; ph ^= 1; }
+              if (u == C::NK / C::VROWS - 1) {
+                tc_commit_mc(bars + C::B_P_FREE + pb, 0x1);  // the score CTA's buffer pb is free
+                if (j == nchunk - 1) tc_commit(bars + C::B_PV_DONE);
+                // re-arm this receive buffer for message use + NPB
+                const int nxt = use + C::NPB;
+                if (nxt < total_msgs) {
+                  const bool lastm = ((nxt % nchunk) == nchunk - 1);
+                  mbar_arrive_expect_tx(bars + C::B_P_FULL + pb, lastm ? C::MSG_BYTES_LAST : C::MSG_BYTES_MID);
+                }
+              }
             }
-            if (!ok) break;
-            tc_commit_mc(bars + C::B_P_FREE + pb, 0x1);  // the score CTA's buffer pb is free
-            if (j == nchunk - 1) tc_commit(bars + C::B_PV_DONE);
-            // re-arm this receive buffer for message use + NPB
-            const int nxt = use + C::NPB;
-            if (nxt < total_msgs) {
-              const bool lastm = ((nxt % nchunk) == nchunk - 1);
-              mbar_arrive_expect_tx(bars + C::B_P_FULL + pb, lastm ? C::MSG_BYTES_LAST : C::MSG_BYTES_MID);
-            }
-            ++use;
-            if (++pb == C::NPB) { pb = 0; pph ^= 1; }
+            __syncwarp();
+            if (++slot == C::NVST) { slot = 0; ph ^= 1; }
           }
+          if (!ok) break;
+          ++use;
+          if (++pb == C::NPB) { pb = 0; pph ^= 1; }
         }
       }
     } else {
