@@ -131,15 +131,16 @@ __global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS)
         mbar_wait(k_empty + kt % C::KST, (kt / C::KST) & 1, ab, 12);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      bool ok = mbar_wait(q_full, 0, ab, 13);
-      const uint32_t q_addr = smem_u32(q_s);
-      for (int kt = 0; kt < nkt && ok; ++kt) {
-        const int slot = kt % C::KST;
-        const int buf = kt % C::NACC;
-        if (!mbar_wait(k_full + slot, (kt / C::KST) & 1, ab, 14)) break;
-        if (!mbar_wait(acc_empty + buf, ((kt / C::NACC) & 1) ^ 1, ab, 15)) break;
-        tc_fence_after();
+    // the warp waits converged; one elected lane issues and commits
+    bool ok = mbar_wait_warp(q_full, 0, ab, 13);
+    const uint32_t q_addr = smem_u32(q_s);
+    for (int kt = 0; kt < nkt && ok; ++kt) {
+      const int slot = kt % C::KST;
+      const int buf = kt % C::NACC;
+      if (!mbar_wait_warp(k_full + slot, (kt / C::KST) & 1, ab, 14)) break;
+      if (!mbar_wait_warp(acc_empty + buf, ((kt / C::NACC) & 1) ^ 1, ab, 15)) break;
+      tc_fence_after();
+      if (elect_one()) {
         const uint32_t a_addr = smem_u32(k_s + slot * C::KTILE_BYTES);
 #pragma unroll
         for (int kk = 0; kk < C::KSTEPS; ++kk) {
@@ -150,6 +151,7 @@ __global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS)
         tc_commit(acc_full + buf);
         tc_commit(k_empty + slot);
       }
+      __syncwarp();
     }
   } else {
     const int quarter = static_cast<int>(warp & 3);

@@ -217,8 +217,8 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
       if (!ab.raised()) mbar_wait(q_empty, qe_phase, ab, 4);
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
+    // ---------------- MMA issuer: the warp waits converged, one elected lane issues ----------------
+    {
       uint32_t qf_phase = 0;
       int kslot = 0;
       uint32_t kf_phase = 0;
@@ -231,30 +231,36 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
         const int t0 = rb * C::RB;
         const int tlast = min(t0 + C::RB, p.L) - 1;
         const int nkt = tlast / C::BM + 1;
-        if (!mbar_wait(q_full, qf_phase, ab, 5)) break;
+        if (!mbar_wait_warp(q_full, qf_phase, ab, 5)) break;
         qf_phase ^= 1;
         bool ok = true;
         for (int kt = 0; kt < nkt && ok; ++kt) {
-          if (!mbar_wait(k_full + kslot, kf_phase, ab, 6)) { ok = false; break; }
+          if (!mbar_wait_warp(k_full + kslot, kf_phase, ab, 6)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = k_base + kslot * C::KTILE_BYTES;
           for (int b = 0; b < C::NACC; ++b) {
-            if (!mbar_wait(acc_empty + b, ae_phase[b], ab, 7)) { ok = false; break; }
+            if (!mbar_wait_warp(acc_empty + b, ae_phase[b], ab, 7)) { ok = false; break; }
             ae_phase[b] ^= 1;
             tc_fence_after();
-            const uint32_t b_addr = q_base + b * C::QBUF_BYTES;
+            if (elect_one()) {
+              const uint32_t b_addr = q_base + b * C::QBUF_BYTES;
 #pragma unroll
-            for (int kk = 0; kk < C::KSTEPS; ++kk) {
-              const uint64_t ad = smem_desc(a_addr + kk * 32, 16, C::SBO, C::SW);
-              const uint64_t bd = smem_desc(b_addr + kk * 32, 16, C::SBO, C::SW);
-              mma_f8(tmem + b * C::NCOL, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
+              for (int kk = 0; kk < C::KSTEPS; ++kk) {
+                const uint64_t ad = smem_desc(a_addr + kk * 32, 16, C::SBO, C::SW);
+                const uint64_t bd = smem_desc(b_addr + kk * 32, 16, C::SBO, C::SW);
+                mma_f8(tmem + b * C::NCOL, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
+              }
+              tc_commit(acc_full + b);
+              if (b == C::NACC - 1) {
+                tc_commit(k_empty + kslot);
+                if (kt == nkt - 1) tc_commit(q_empty);
+              }
             }
-            tc_commit(acc_full + b);
+            __syncwarp();
           }
-          tc_commit(k_empty + kslot);
+          if (!ok) break;
           if (++kslot == C::KST) { kslot = 0; kf_phase ^= 1; }
         }
-        tc_commit(q_empty);
         if (!ok) break;
       }
     }

@@ -79,7 +79,8 @@ struct MlaCfg {
   static constexpr int OFF_QROPE = OFF_RING + RING_BYTES;  // score CTA: Q[:, 512:576] (16 KB)
   static constexpr int OFF_MSG = OFF_QROPE + M * 128;      // NPB x MSG_STRIDE (staging / receive)
   static constexpr int OFF_IDX = OFF_MSG + NPB * MSG_STRIDE;  // int32 [KMAX]: the token's index row
-  static constexpr int OFF_BAR = OFF_IDX + KMAX * 4;
+  static constexpr int OFF_VMASK = OFF_IDX + KMAX * 4;       // score CTA: u32 [2][KMAX/32] validity bits per token
+  static constexpr int OFF_BAR = OFF_VMASK + 2 * (KMAX / 32) * 4;
   // barriers
   static constexpr int NRING = (NSST > NVST) ? NSST : NVST;
   static constexpr int B_RING_FULL = 0;                     // [NRING]
@@ -94,7 +95,9 @@ struct MlaCfg {
   static constexpr int B_PV_DONE = B_O_READY + NPB;         // value CTA: a token's last PV is done
   static constexpr int B_STAGE = B_PV_DONE + 1;             // score CTA: softmax warps wrote the staging buffer
   static constexpr int B_QUIESCE = B_STAGE + 1;             // value CTA: all PV issued so far complete
-  static constexpr int NBAR = B_QUIESCE + 1;
+  static constexpr int B_MASK_FULL = B_QUIESCE + 1;         // [2] score CTA: producers wrote a token's masks
+  static constexpr int B_MASK_FREE = B_MASK_FULL + 2;       // [2] score CTA: softmax is done with them
+  static constexpr int NBAR = B_MASK_FREE + 2;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 32;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -166,6 +169,15 @@ __device__ __forceinline__ int checked_row(const int32_t* idx_s, int e, int K, i
     row = -1;
   }
   return row;
+}
+
+// Slab order within chunk j: the RoPE slab (8, multiplied from shared memory)
+// comes last in even chunks and first in odd ones, so consecutive chunks' RoPE
+// MMAs run back to back. Every switch between the TMEM-A and shared-memory-A
+// MMA forms drains the tensor pipe (measured on B200: ~740 cycles), so this
+// halves the switches.
+__device__ __forceinline__ int slab_at(int j, int i) {
+  return (j & 1) ? (i == 0 ? MlaCfg::NSLAB_QK - 1 : i - 1) : i;
 }
 
 // Score CTA: the 8 rows (r = ptid/8 + 16k) this thread copies for chunk j,
@@ -246,6 +258,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
   int* abort_s = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
   int* rescale_s = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
   int32_t* idx_s = reinterpret_cast<int32_t*>(smem + C::OFF_IDX);
+  uint32_t* vmask_s = reinterpret_cast<uint32_t*>(smem + C::OFF_VMASK);
   const AbortFlag ab{abort_s};
   const uint32_t rank = cluster_ctarank();
   const uint32_t warp = warp_id();
@@ -277,6 +290,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
     mbar_init(bars + C::B_PV_DONE, 1);
     mbar_init(bars + C::B_STAGE, 4);
     mbar_init(bars + C::B_QUIESCE, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bars + C::B_MASK_FULL + i, C::NPROD);
+      mbar_init(bars + C::B_MASK_FREE + i, 4);
+    }
     fence_mbar_init();
   }
   if (warp == C::W_MMA) tmem_alloc(tmem_base_s, 512);
@@ -300,15 +317,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       const int ptid = threadIdx.x;
       int slot = 0;
       uint32_t ph = 1;
-      for (int tk = cluster_id; tk < p.T; tk += nclusters) {
+      int n = 0;  // tokens done by this cluster
+      for (int tk = cluster_id; tk < p.T; tk += nclusters, ++n) {
         const __nv_bfloat16* kv_tok = p.kv + tk * p.kv_token_stride;
+        // the softmax warps are done with this mask buffer (two tokens back)
+        const int mb = n & 1;
+        if (!mbar_wait(bars + C::B_MASK_FREE + mb, ((n >> 1) & 1) ^ 1, ab, 30)) break;
         stage_index_row(idx_s, p.idx + static_cast<size_t>(tk) * p.K, p.K, ptid);
+        // validity bits of every selection entry, 32 per word (entry e -> word e/32)
+        for (int wd = static_cast<int>(warp); wd < nchunk * (C::NK / 32); wd += C::NPROD) {
+          const int e = wd * 32 + static_cast<int>(lane);
+          const int row = (e < p.K) ? idx_s[e] : -1;
+          const uint32_t m = __ballot_sync(0xffffffffu, row >= 0 && row < p.rows);
+          if (lane == 0) vmask_s[mb * (C::KMAX / 32) + wd] = m;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + C::B_MASK_FULL + mb);
         bool ok = true;
         for (int j = 0; j < nchunk && ok; ++j) {
           const ChunkRows cr = chunk_rows(kv_tok, idx_s, j, p.K, p.rows, ptid);
-          for (int s = 0; s < C::NSLAB_QK; ++s) {
+          for (int i = 0; i < C::NSLAB_QK; ++i) {
             if (!mbar_wait(bars + C::B_RING_EMPTY + slot, ph, ab, 31)) { ok = false; break; }
-            gather_slab_tile(ring + slot * C::SLAB_TILE, cr, s, ptid);
+            gather_slab_tile(ring + slot * C::SLAB_TILE, cr, slab_at(j, i), ptid);
             cp_async_mbar_arrive(bars + C::B_RING_FULL + slot);
             if (++slot == C::NSST) { slot = 0; ph ^= 1; }
           }
@@ -334,15 +364,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
           if (!mbar_wait_warp(bars + C::B_S_EMPTY + sb, sph, ab, 34)) { ok = false; break; }
           tc_fence_after();
           const uint32_t d = tmem + C::S_COL + sb * C::NK;
-          for (int s = 0; s < C::NSLAB_QK; ++s) {
+          for (int i = 0; i < C::NSLAB_QK; ++i) {
             if (!mbar_wait_warp(bars + C::B_RING_FULL + slot, ph, ab, 33)) { ok = false; break; }
             tc_fence_after();
             if (elect_one()) {
+              const int s = slab_at(j, i);
               const uint32_t tile = ring + slot * C::SLAB_TILE;
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
                 const uint64_t bd = smem_desc(tile + kk * 32, 16, 1024, kSw128);
-                const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+                const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
                 if (s < C::NSLAB_QK - 1) {
                   mma_bf16_ts(d, tmem + C::Q_COL + (4 * s + kk) * 8, bd, C::IDESC_QK, acc);
                 } else {
@@ -350,7 +381,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
                 }
               }
               tc_commit(bars + C::B_RING_EMPTY + slot);
-              if (s == C::NSLAB_QK - 1) {
+              if (i == C::NSLAB_QK - 1) {
                 tc_commit(bars + C::B_S_FULL + sb);
                 if (j == nchunk - 1) tc_commit(bars + C::B_Q_FREE);
               }
@@ -377,33 +408,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       uint32_t pfree_ph = 1;
       uint32_t stage_ph = 0;
       bool ok = true;
-      for (int tk = cluster_id; tk < p.T && ok; tk += nclusters) {
+      int n = 0;  // tokens done by this cluster
+      for (int tk = cluster_id; tk < p.T && ok; tk += nclusters, ++n) {
         // --- Q[tk]: values 0..511 to TMEM, 512..575 to shared memory, once
         //     the previous token's QK^T is done ---
         if (!mbar_wait(bars + C::B_Q_FREE, qfree_ph, ab, 35)) break;
         qfree_ph ^= 1;
         tc_fence_after();
         {
+          // the head's 1152-byte row in 9 blocks of 64 values (blocks 0..7 to
+          // TMEM as 32 columns each, block 8 to shared memory), loaded three
+          // blocks at a time so each round trip has 24 loads in flight
           const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(tk) * p.Hq + h) * C::D);
-#pragma unroll 1
-          for (int cb = 0; cb < 8; ++cb) {  // 8 blocks of 32 columns (64 values)
-            uint32_t r[32];
 #pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              uint4 x = make_uint4(0, 0, 0, 0);
-              if (h < p.Hq) x = __ldg(qrow + cb * 8 + v);
-              r[4 * v + 0] = x.x;
-              r[4 * v + 1] = x.y;
-              r[4 * v + 2] = x.z;
-              r[4 * v + 3] = x.w;
+          for (int rnd = 0; rnd < 3; ++rnd) {
+            uint4 x[24];
+#pragma unroll
+            for (int i = 0; i < 24; ++i) x[i] = (h < p.Hq) ? __ldg(qrow + rnd * 24 + i) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int bb = 0; bb < 3; ++bb) {
+              const int cb = rnd * 3 + bb;
+              if (cb < 8) {
+                uint32_t r[32];
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                  r[4 * v + 0] = x[bb * 8 + v].x;
+                  r[4 * v + 1] = x[bb * 8 + v].y;
+                  r[4 * v + 2] = x[bb * 8 + v].z;
+                  r[4 * v + 3] = x[bb * 8 + v].w;
+                }
+                tmem_st32(tmem + lane_addr + C::Q_COL + cb * 32, r);
+              } else {
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                  *reinterpret_cast<uint4*>(qrope_s + h * 128 + ((c ^ (h & 7)) << 4)) = x[bb * 8 + c];
+              }
             }
-            tmem_st32(tmem + lane_addr + C::Q_COL + cb * 32, r);
-          }
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint4 x = make_uint4(0, 0, 0, 0);
-            if (h < p.Hq) x = __ldg(qrow + 64 + c);
-            *reinterpret_cast<uint4*>(qrope_s + h * 128 + ((c ^ (h & 7)) << 4)) = x;
           }
           tmem_st_wait();
         }
@@ -417,25 +457,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
           const uint32_t qbytes = static_cast<uint32_t>(p.Hq) * C::D * 2;
           asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(nq), "r"(qbytes) : "memory");
         }
-        const int32_t* idx_tok = p.idx + static_cast<size_t>(tk) * p.K;
         float m_ref = -INFINITY;
         float l_sum = 0.f;
-        int nidx[4];
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int e = g * 32 + static_cast<int>(lane);
-          nidx[g] = (e < p.K) ? __ldg(idx_tok + e) : -1;
-        }
+        // validity bits of this token's selection, staged by the producer warps
+        const int mb = n & 1;
+        if (!mbar_wait(bars + C::B_MASK_FULL + mb, (n >> 1) & 1, ab, 39)) break;
+        const uint4* vm_tok = reinterpret_cast<const uint4*>(vmask_s + mb * (C::KMAX / 32));
         for (int j = 0; j < nchunk; ++j) {
-          // validity of the chunk's 128 entries (same for every head), with
-          // the next chunk's indices already in flight
-          uint32_t vmask[4];
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            vmask[g] = __ballot_sync(0xffffffffu, nidx[g] >= 0 && nidx[g] < p.rows);
-            const int e = (j + 1) * C::NK + g * 32 + static_cast<int>(lane);
-            nidx[g] = (e < p.K) ? __ldg(idx_tok + e) : -1;
-          }
+          // validity of the chunk's 128 entries (the same for every head)
+          const uint4 vm4 = vm_tok[j];
+          const uint32_t vmask[4] = {vm4.x, vm4.y, vm4.z, vm4.w};
           if (!mbar_wait(bars + C::B_S_FULL + sb, sph, ab, 36)) { ok = false; break; }
           tc_fence_after();
           const uint32_t s_addr = tmem + lane_addr + C::S_COL + sb * C::NK;
@@ -528,6 +559,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
           if (++pb == C::NPB) { pb = 0; pfree_ph ^= 1; }
           if (!ok) break;
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + C::B_MASK_FREE + mb);
       }
     }
   } else {
