@@ -70,13 +70,26 @@ typedef enum {
  *                                   dsa_index_topk_workspace_size(L, H_I, d_I, topk)
  *                                   bytes; its contents are not kept between calls.
  * The L x L score matrix is never formed: scores are streamed into per-row
- * candidate lists bounded by the workspace size.
+ * candidate lists bounded by the workspace size. Long rows first score a
+ * stratified sample of 8 key tiles and start their threshold at a sampled
+ * score expected to admit ~2.5 * topk keys; a row that ends with fewer than
+ * topk admitted keys is recomputed without the sample within the same call,
+ * so the result never depends on the sample.
  * ------------------------------------------------------------------------ */
 size_t dsa_index_topk_workspace_size(int L, int H_I, int d_I, int topk);
 
 dsa_status dsa_index_topk(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
                           const float* k_scale, int L, int H_I, int d_I, int topk, int32_t* idx, void* workspace,
                           size_t ws_bytes, void* stream);
+
+/* Test hook: after dsa_index_topk returned with this workspace (and the same
+ * L, H_I, d_I, topk), the number of row blocks of 8 tokens whose sampled
+ * starting threshold proved too high and that were therefore recomputed with
+ * plain streaming (the result is the same either way). Synchronises `stream`
+ * and copies one int to *count. No counterpart in the pages: it only exposes
+ * how often this implementation's shortcut had to be undone. */
+dsa_status dsa_index_topk_rerun_count(const void* workspace, int L, int H_I, int d_I, int topk, int* count,
+                                      void* stream);
 
 /* Test hook: the same kernel's fp32 scores for query rows [row0, row0+nrows),
  * written to scores[nrows, L] (row r is query t = row0 + r; entries s > t are

@@ -51,6 +51,7 @@ def lib() -> ctypes.CDLL:
             L.dsa_index_topk_workspace_size.restype = SZ
             L.dsa_index_topk.argtypes = [P, P, P, P, P, I, I, I, I, P, P, SZ, P]
             L.dsa_index_scores.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P]
+            L.dsa_index_topk_rerun_count.argtypes = [P, I, I, I, I, ctypes.POINTER(I), P]
             L.dsa_sparse_mla_attn.argtypes = [P, P, P, I, I, I, I, F, P, P, P]
             L.dsa_index_topk_decode_workspace_size.argtypes = [I, I, I]
             L.dsa_index_topk_decode_workspace_size.restype = SZ
@@ -63,7 +64,7 @@ def lib() -> ctypes.CDLL:
             L.dsa_status_string.restype = ctypes.c_char_p
             L.dsa_last_error.argtypes = []
             L.dsa_last_error.restype = ctypes.c_char_p
-            for name in ("dsa_index_topk", "dsa_index_scores", "dsa_sparse_mla_attn", "dsa_index_topk_decode",
+            for name in ("dsa_index_topk", "dsa_index_topk_rerun_count", "dsa_index_scores", "dsa_sparse_mla_attn", "dsa_index_topk_decode",
                          "dsa_index_scores_decode", "dsa_sparse_mla_attn_decode", "dsa_get_device_error",
                          "dsa_index_topk_decode_noalloc"):
                 getattr(L, name).restype = I
@@ -124,6 +125,15 @@ def index_topk(q_I, q_scale, w, k_cache, k_scale, topk: int, *, idx=None, worksp
                                 topk, _ptr(idx), _ptr(workspace), workspace.numel() * workspace.element_size(),
                                 _stream(q_I.device)))
     return idx
+
+
+def index_topk_rerun_count(workspace, L: int, H_I: int, d_I: int, topk: int) -> int:
+    """Test hook: row blocks the last index_topk call with this workspace recomputed
+    because their sampled starting threshold was too high (synchronises)."""
+    n = ctypes.c_int(0)
+    _check(lib().dsa_index_topk_rerun_count(_ptr(workspace), L, H_I, d_I, topk, ctypes.byref(n),
+                                            _stream(workspace.device)))
+    return int(n.value)
 
 
 def index_scores(q_I, q_scale, w, k_cache, k_scale, row0: int = 0, nrows: Optional[int] = None,

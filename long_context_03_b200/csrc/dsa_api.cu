@@ -108,18 +108,26 @@ bool prefill_shape_ok(int H_I, int d_I) { return (H_I == 8 || H_I == 64) && (d_I
 struct WsPrefill {
   uint64_t* cand;
   uint64_t* sel;
+  int* redo;  // [0]: count, [4 ..]: row blocks to re-run
   size_t bytes;
 };
 
 WsPrefill prefill_ws_layout(void* base, int L, int H_I, int topk, int grid) {
   WsPrefill w;
+  const int nrb = (L + rows_per_block(H_I) - 1) / rows_per_block(H_I);
   const size_t cand_bytes = static_cast<size_t>(grid) * rows_per_block(H_I) * select_cap(topk) * 8;
   const size_t sel_bytes = static_cast<size_t>(L) * topk * 8;
+  const size_t redo_bytes = (static_cast<size_t>(nrb) + 4) * 4;
   w.cand = reinterpret_cast<uint64_t*>(base);
   w.sel = reinterpret_cast<uint64_t*>(reinterpret_cast<char*>(base) + cand_bytes);
-  w.bytes = cand_bytes + sel_bytes;
+  w.redo = reinterpret_cast<int*>(reinterpret_cast<char*>(base) + cand_bytes + sel_bytes);
+  w.bytes = cand_bytes + sel_bytes + redo_bytes;
   return w;
 }
+
+// Rows at least this long start from a sampled threshold (twice the list
+// capacity: shorter rows rarely cut their lists anyway).
+int spec_min_row(int topk) { return 2 * select_cap(topk) > 4096 ? 2 * select_cap(topk) : 4096; }
 
 template <int HI, int DI, bool kSelect, int MQ>
 dsa_status launch_prefill(const uint8_t* q_I, const uint8_t* k_cache, const IdxPrefillParams& p, int grid,
@@ -305,10 +313,42 @@ dsa_status dsa_index_topk(const uint8_t* q_I, const float* q_scale, const float*
   p.cand = ws.cand;
   p.cap = select_cap(topk);
   p.sel_keys = ws.sel;
+  p.spec_min_t = spec_min_row(topk);
+  p.redo_count = ws.redo;
+  p.redo_list = ws.redo + 4;
+  const cudaError_t me = cudaMemsetAsync(ws.redo, 0, sizeof(int), st);
+  if (me != cudaSuccess) return cuda_fail(me, "cudaMemsetAsync");
   dsa_status s = (select_mq(topk) == 1) ? dispatch_prefill<true, 1>(H_I, d_I, q_I, k_cache, p, grid, st)
-                                        : dispatch_prefill<true, 4>(H_I, d_I, q_I, k_cache, p, grid, st);
+                             : dispatch_prefill<true, 4>(H_I, d_I, q_I, k_cache, p, grid, st);
+  if (s != DSA_OK) return s;
+  // Row blocks whose sampled start proved too high run again with plain
+  // streaming; the count is read on the device, so an empty list costs one
+  // short launch and no host synchronisation.
+  IdxPrefillParams r = p;
+  r.spec_min_t = 0;
+  r.rb_list = ws.redo + 4;
+  r.list_count = ws.redo;
+  r.redo_count = nullptr;
+  r.redo_list = nullptr;
+  s = (select_mq(topk) == 1) ? dispatch_prefill<true, 1>(H_I, d_I, q_I, k_cache, r, grid, st)
+                             : dispatch_prefill<true, 4>(H_I, d_I, q_I, k_cache, r, grid, st);
   if (s != DSA_OK) return s;
   return launch_rank_sort(ws.sel, idx, topk, L, st);
+}
+
+dsa_status dsa_index_topk_rerun_count(const void* workspace, int L, int H_I, int d_I, int topk, int* count,
+                                     void* stream) {
+  if (!workspace || !count) return fail(DSA_ERR_INVALID_ARG, "null pointer");
+  if (L <= 0 || !prefill_shape_ok(H_I, d_I)) return fail(DSA_ERR_INVALID_ARG, "L=%d H_I=%d d_I=%d", L, H_I, d_I);
+  const int rb = rows_per_block(H_I);
+  const int nrb = (L + rb - 1) / rb;
+  const int grid = nrb < num_sms() ? nrb : num_sms();
+  const WsPrefill ws = prefill_ws_layout(const_cast<void*>(workspace), L, H_I, topk, grid);
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  e = cudaMemcpy(count, ws.redo, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy");
+  return DSA_OK;
 }
 
 dsa_status dsa_index_scores(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,

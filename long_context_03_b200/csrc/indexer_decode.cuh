@@ -76,8 +76,10 @@ __global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS)
   if (s0 >= n) return;  // whole CTA, before any barrier or TMEM allocation
   const int nkt = min(C::NKT, (n - s0 + C::BM - 1) / C::BM);
 
+  // 1024-byte aligned base, derived from the shared array by an offset so
+  // the compiler keeps every access in the shared address space
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* k_s = smem + C::OFF_K;
   uint8_t* q_s = smem + C::OFF_Q;
   float* w_s = reinterpret_cast<float*>(smem + C::OFF_W);

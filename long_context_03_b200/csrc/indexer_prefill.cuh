@@ -50,6 +50,7 @@ struct IdxPrefillCfg {
   static constexpr int NET = NEPI * 32;        // epilogue threads
   static constexpr int TOK_PER_WARP = TB / 4;  // tokens of a buffer per epilogue warp (64 columns)
   static constexpr int CHECK_EVERY = 4;        // key tiles between list-capacity checks
+  static constexpr int NSAMPLE = 8;            // key tiles scored first to set a row's starting threshold
   static constexpr SwizzleMode SW = (DI == 128) ? kSw128 : kSw64;
   static constexpr uint32_t SBO = 8 * DI;      // bytes between 8-row core groups
   static constexpr uint32_t IDESC = instr_desc(kFmtE4M3, 128, NCOL, false, false);
@@ -86,48 +87,61 @@ struct IdxPrefillParams {
   uint64_t* cand;        // [gridDim.x][RB][cap] candidate lists
   int cap;
   uint64_t* sel_keys;    // [L][topk] exact top-k keys per row, unordered, 0-padded
+  // Sampled starting thresholds: row blocks with t0 >= spec_min_t (0: never)
+  // first score NSAMPLE evenly spread key tiles and start from the sample's
+  // r-th largest score (r ~ 2.5 * topk * sampled keys / (t+1)). A row that
+  // ends with fewer than topk keys at or above that start is re-run: its row
+  // block index goes to redo_list[atomicAdd(redo_count, 1)].
+  int spec_min_t;
+  int* redo_count;
+  int* redo_list;
+  // Re-run mode: when rb_list is set, process row blocks rb_list[0 .. *list_count)
+  // (plain streaming, no sampling) instead of [rb_begin, rb_end).
+  const int* rb_list;
+  const int* list_count;
   // score mode (test hook)
   float* scores;         // [nrows][L]; rows t in [row0, row0 + nrows)
   int row0, nrows;
 };
 
 // sum_j w[j] * max(x_j, 0) over the H_I accumulator values of one token
-// (registers loaded from TMEM). Heads are taken in pairs with the packed fp32
-// FMA into four independent accumulator pairs, summed in a fixed order at the
-// end. Shared by both modes so their scores are bit-identical.
+// (registers loaded from TMEM), into eight independent partial sums (head j
+// goes to sum j % 8) added in a fixed order at the end. Scalar FMAs: the
+// packed two-lane form needs its operands in aligned register pairs, which
+// cost a register move per ReLU output. Shared by both modes so their scores
+// are bit-identical.
 template <int HI>
-__device__ __forceinline__ void relu_weighted_acc(float2 (&acc)[4], const uint32_t* x, const float* __restrict__ w) {
+__device__ __forceinline__ void relu_weighted_acc(float (&acc)[8], const uint32_t* x, const float* __restrict__ w) {
   static_assert(HI % 8 == 0, "a multiple of 8 heads");
-  const float2* w2 = reinterpret_cast<const float2*>(w);
 #pragma unroll
   for (int j = 0; j < HI; j += 8) {
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      const float2 xr = make_float2(fmaxf(__uint_as_float(x[j + 2 * a]), 0.f),
-                                    fmaxf(__uint_as_float(x[j + 2 * a + 1]), 0.f));
-      acc[a] = __ffma2_rn(w2[j / 2 + a], xr, acc[a]);
-    }
+    for (int a = 0; a < 8; ++a) acc[a] = __fmaf_rn(w[j + a], fmaxf(__uint_as_float(x[j + a]), 0.f), acc[a]);
   }
 }
-__device__ __forceinline__ float relu_weighted_finish(const float2 (&acc)[4]) {
-  return ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+__device__ __forceinline__ float relu_weighted_finish(const float (&acc)[8]) {
+  return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 }
 
-template <int HI>
-__device__ __forceinline__ float relu_weighted_head_sum(const uint32_t* x, const float* __restrict__ w) {
-  static_assert(HI % 8 == 0, "H_I must be a multiple of 8");
-  const float2* w2 = reinterpret_cast<const float2*>(w);
-  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-  for (int j = 0; j < HI; j += 8) {
-#pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      const float2 xr = make_float2(fmaxf(__uint_as_float(x[j + 2 * a]), 0.f),
-                                    fmaxf(__uint_as_float(x[j + 2 * a + 1]), 0.f));
-      acc[a] = __ffma2_rn(w2[j / 2 + a], xr, acc[a]);
-    }
-  }
-  return ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+// Key tile of step i of a row block's sequence: with sampling, steps
+// 0..NSAMPLE-1 are tiles at the middles of NSAMPLE equal strata of the
+// block's nkt tiles, then every tile 0..nkt-1 follows in order.
+template <int NS>
+__device__ __forceinline__ int tile_at(int i, int nkt, bool spec) {
+  if (!spec) return i;
+  if (i < NS) return ((2 * i + 1) * nkt) / (2 * NS);
+  return i - NS;
+}
+// Rank r of the sampled key whose score starts a row's threshold: about 2.5
+// times the row's share of topk among the sampled keys, so that the expected
+// count of keys at or above it is ~2.5 * topk; at least 1, at most n.
+__device__ __forceinline__ int sample_rank(int topk, int sampled_keys, int t, int n) {
+  const long long num = 5ll * topk * sampled_keys;
+  const long long den = 2ll * (t + 1);
+  long long r = (num + den - 1) / den;
+  if (r > n) r = n;
+  if (r < 1) r = 1;
+  return static_cast<int>(r);
 }
 
 template <int HI, int DI, bool kSelect, int MQ>
@@ -135,8 +149,10 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
     indexer_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                            const IdxPrefillParams p) {
   using C = IdxPrefillCfg<HI, DI>;
+  // 1024-byte aligned base, derived from the shared array by an offset so
+  // the compiler keeps every access in the shared address space
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* q_s = smem + C::OFF_Q;
   uint8_t* k_s = smem + C::OFF_K;
   float* w_s = reinterpret_cast<float*>(smem + C::OFF_W);
@@ -179,8 +195,14 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_base_s;
 
-  const int nrb = p.rb_end - p.rb_begin;
+  const bool list_mode = p.rb_list != nullptr;
+  const int nrb = list_mode ? *p.list_count : (p.rb_end - p.rb_begin);
   const int G = gridDim.x;
+  // row block of step j and whether it samples first (the same on every role)
+  auto block_of = [&](int j) { return list_mode ? p.rb_list[j] : p.rb_end - 1 - j; };
+  auto samples = [&](int t0, int nkt) {
+    return kSelect && !list_mode && p.spec_min_t > 0 && t0 >= p.spec_min_t && nkt >= 4 * C::NSAMPLE;
+  };
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -189,20 +211,22 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
       int kslot = 0;
       uint32_t ke_phase = 1;
       for (int j = blockIdx.x; j < nrb; j += G) {
-        const int rb = p.rb_end - 1 - j;
+        const int rb = block_of(j);
         const int t0 = rb * C::RB;
         const int tlast = min(t0 + C::RB, p.L) - 1;
         const int nkt = tlast / C::BM + 1;
+        const bool spec = samples(t0, nkt);
+        const int nsteps = nkt + (spec ? C::NSAMPLE : 0);
         if (!mbar_wait(q_empty, qe_phase, ab, 1)) break;
         qe_phase ^= 1;
         mbar_arrive_expect_tx(q_full, C::NACC * C::QBUF_BYTES);
         for (int b = 0; b < C::NACC; ++b)
           tma_load_2d(q_s + b * C::QBUF_BYTES, &tmQ, q_full, 0, (t0 + b * C::TB) * HI);
         bool ok = true;
-        for (int kt = 0; kt < nkt; ++kt) {
+        for (int i = 0; i < nsteps; ++i) {
           if (!mbar_wait(k_empty + kslot, ke_phase, ab, 2)) { ok = false; break; }
           mbar_arrive_expect_tx(k_full + kslot, C::KTILE_BYTES);
-          tma_load_2d(k_s + kslot * C::KTILE_BYTES, &tmK, k_full + kslot, 0, kt * C::BM);
+          tma_load_2d(k_s + kslot * C::KTILE_BYTES, &tmK, k_full + kslot, 0, tile_at<C::NSAMPLE>(i, nkt, spec) * C::BM);
           if (++kslot == C::KST) { kslot = 0; ke_phase ^= 1; }
         }
         if (!ok) break;
@@ -227,14 +251,15 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
       const uint32_t q_base = smem_u32(q_s);
       const uint32_t k_base = smem_u32(k_s);
       for (int j = blockIdx.x; j < nrb; j += G) {
-        const int rb = p.rb_end - 1 - j;
+        const int rb = block_of(j);
         const int t0 = rb * C::RB;
         const int tlast = min(t0 + C::RB, p.L) - 1;
         const int nkt = tlast / C::BM + 1;
+        const int nsteps = nkt + (samples(t0, nkt) ? C::NSAMPLE : 0);
         if (!mbar_wait_warp(q_full, qf_phase, ab, 5)) break;
         qf_phase ^= 1;
         bool ok = true;
-        for (int kt = 0; kt < nkt && ok; ++kt) {
+        for (int kt = 0; kt < nsteps && ok; ++kt) {
           if (!mbar_wait_warp(k_full + kslot, kf_phase, ab, 6)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = k_base + kslot * C::KTILE_BYTES;
@@ -253,7 +278,7 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
               tc_commit(acc_full + b);
               if (b == C::NACC - 1) {
                 tc_commit(k_empty + kslot);
-                if (kt == nkt - 1) tc_commit(q_empty);
+                if (kt == nsteps - 1) tc_commit(q_empty);
               }
             }
             __syncwarp();
@@ -282,10 +307,12 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
     int* pos_s = scr_s + cut_scratch_ints() - 16;  // 9 ints: warp sums of the block scan
 
     for (int j = blockIdx.x; j < nrb; j += G) {
-      const int rb = p.rb_end - 1 - j;
+      const int rb = block_of(j);
       const int t0 = rb * C::RB;
       const int tlast = min(t0 + C::RB, p.L) - 1;
       const int nkt = tlast / C::BM + 1;
+      const bool spec = samples(t0, nkt);
+      const int nsteps = nkt + (spec ? C::NSAMPLE : 0);
       // per-row-block state
       for (int i = et; i < C::RB * HI; i += C::NET) {
         const int t = t0 + i / HI;
@@ -301,14 +328,15 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
       bool ok = true;
       float ks_next = 0.f;
       {
-        const int s0 = quarter * 32 + static_cast<int>(lane);
+        const int s0 = tile_at<C::NSAMPLE>(0, nkt, spec) * C::BM + quarter * 32 + static_cast<int>(lane);
         ks_next = (s0 < p.L) ? __ldg(p.k_scale + s0) : 0.f;
       }
-      for (int kt = 0; kt < nkt && ok; ++kt) {
+      for (int i = 0; i < nsteps && ok; ++i) {
+        const int kt = tile_at<C::NSAMPLE>(i, nkt, spec);
         const int s = kt * C::BM + quarter * 32 + static_cast<int>(lane);
         const float ks = ks_next;
-        if (kt + 1 < nkt) {
-          const int sn = s + C::BM;
+        if (i + 1 < nsteps) {
+          const int sn = tile_at<C::NSAMPLE>(i + 1, nkt, spec) * C::BM + quarter * 32 + static_cast<int>(lane);
           ks_next = (sn < p.L) ? __ldg(p.k_scale + sn) : 0.f;
         }
         for (int b = 0; b < C::NACC; ++b) {
@@ -339,11 +367,11 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
           {
             // columns [0,32) then [32,64) of the slice; a token spans HI columns
             constexpr int TPH = (HI >= 32) ? 1 : 32 / HI;  // tokens per 32-column half
-            float2 acc[C::TOK_PER_WARP][4];
+            float acc[C::TOK_PER_WARP][8];
 #pragma unroll
             for (int q = 0; q < C::TOK_PER_WARP; ++q)
 #pragma unroll
-              for (int a = 0; a < 4; ++a) acc[q][a] = make_float2(0.f, 0.f);
+              for (int a = 0; a < 8; ++a) acc[q][a] = 0.f;
             const int tl0 = b * C::TB + half * C::TOK_PER_WARP;
             if constexpr (HI >= 32) {
               relu_weighted_acc<32>(acc[0], xa, w_s + tl0 * HI);
@@ -397,7 +425,40 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
           // and tile): one histogram pass keeps every key in or above the bin
           // of the k-th largest; if that keeps too many, an exact select
           // keeps exactly k.
-          if ((kt % C::CHECK_EVERY) != C::CHECK_EVERY - 1) continue;
+          if (spec && i == C::NSAMPLE - 1) {
+            // End of the sample: each row's threshold starts at the score of
+            // its r-th largest sampled key (keys scoring at least that pass;
+            // index bits cleared so equal scores are kept), and the list is
+            // emptied: the sampled tiles come round again in order.
+            named_bar_sync(1, C::NET);
+            for (int tl = 0; tl < C::RB; ++tl) {
+              const int t = t0 + tl;
+              if (t >= p.L) break;
+              const int* cn = cnt_s + tl * 4;
+              const int n = cn[0] + cn[1] + cn[2] + cn[3];
+              if (n == 0) continue;
+              const int r = sample_rank(p.topk, C::NSAMPLE * C::BM, t, n);
+              uint64_t* row = my_cand + static_cast<size_t>(tl) * p.cap;
+              uint64_t v[4 * MQ];
+              load_sublists<C::NET, MQ>(row, capq, cn, et, v);
+              int above = 0, inb = 0;
+              uint64_t floor = histogram_cut<C::NET, 4 * MQ>(v, r, scr_s, et, 1, &above, &inb);
+              if (above + inb > r) {
+#pragma unroll
+                for (int q = 0; q < 4 * MQ; ++q) v[q] = (v[q] >= floor) ? v[q] : 0ull;
+                floor = radix_select_floor<C::NET, 4 * MQ>(v, r, scr_s, et, 1);
+              }
+              if (et == 0) {
+                const uint64_t hi = floor >> 32;
+                thr_s[tl] = (hi == 0) ? 0ull : (hi << 32) - 1;
+              }
+              named_bar_sync(1, C::NET);
+            }
+            if (et < 4 * C::RB) cnt_s[et] = 0;
+            named_bar_sync(1, C::NET);
+            continue;
+          }
+          if ((i % C::CHECK_EVERY) != C::CHECK_EVERY - 1) continue;
           named_bar_sync(1, C::NET);
           for (int tl = 0; tl < C::RB; ++tl) {
             const int* cn = cnt_s + tl * 4;
@@ -430,11 +491,14 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
         // exact top-k of each row: the histogram pass finds the boundary bin,
         // a radix select over that bin's keys alone finds the exact cut
         named_bar_sync(1, C::NET);
+        bool redo = false;
         for (int tl = 0; tl < C::RB; ++tl) {
           const int t = t0 + tl;
           if (t >= p.L) break;
           const int* cn = cnt_s + tl * 4;
           const int n = cn[0] + cn[1] + cn[2] + cn[3];
+          // a sampled start above the row's k-th largest score left too few keys
+          if (spec && n < min(p.topk, t + 1)) redo = true;
           uint64_t* row = my_cand + static_cast<size_t>(tl) * p.cap;
           uint64_t v[4 * MQ];
           load_sublists<C::NET, MQ>(row, capq, cn, et, v);
@@ -461,6 +525,7 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
             if (v[i] != 0 && v[i] >= floor) dst[pos++] = v[i];
           for (int i = kept + et; i < p.topk; i += C::NET) dst[i] = 0ull;
         }
+        if (redo && et == 0) p.redo_list[atomicAdd(p.redo_count, 1)] = rb;
       }
       named_bar_sync(1, C::NET);
     }
