@@ -186,8 +186,9 @@ dsa_status launch_decode_scores(const uint8_t* q_I, const uint8_t* k_cache, int 
   auto kern = indexer_decode_kernel<HI, DI>;
   s = set_smem(kern, C::SMEM_BYTES);
   if (s != DSA_OK) return s;
-  dim3 grid((p.L_max + C::CHUNK - 1) / C::CHUNK, B);
-  kern<<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(tmQ, tmK, p);
+  const int items = ((p.L_max + C::CHUNK - 1) / C::CHUNK) * B;
+  const int slots = 2 * num_sms();  // two persistent CTAs per SM (shared memory)
+  kern<<<items < slots ? items : slots, C::NTHREADS, C::SMEM_BYTES, st>>>(tmQ, tmK, p);
   return check_launch("indexer_decode_kernel");
 }
 
@@ -201,6 +202,7 @@ dsa_status decode_scores(const uint8_t* q_I, const float* q_scale, const float* 
   p.k_scale = k_scale;
   p.lens = lens;
   p.L_max = L_max;
+  p.B = B;
   p.scores = scores;
   if (H_I == 64 && d_I == 128) return launch_decode_scores<64, 128>(q_I, k_cache, B, p, st);
   if (H_I == 64 && d_I == 64) return launch_decode_scores<64, 64>(q_I, k_cache, B, p, st);

@@ -8,12 +8,13 @@
 // (b) Decoding) is the regime here: one query per sequence, so the work is a
 // single pass over the key cache and HBM bandwidth is the bound.
 //
-// Scoring kernel: a CTA takes 1024 keys of one sequence, streams its 8 key
-// tiles through a 4-stage TMA ring, multiplies each against the sequence's
-// [H_I x d_I] query on the tensor core (M = 128 keys, N = H_I heads) and the
-// epilogue reduces the heads per key, writing one fp32 score per key to the
-// scores buffer. Several CTAs share an SM so enough loads are in flight to
-// cover HBM latency.
+// Scoring kernel: persistent CTAs (two per SM) walk contiguous ranges of
+// (sequence, 1024-key chunk) items. For each item the query is loaded once,
+// its 8 key tiles stream through a 4-stage TMA ring, each tile is multiplied
+// against the [H_I x d_I] query on the tensor core (M = 128 keys, N = H_I
+// heads) and the epilogue reduces the heads per key, writing one fp32 score
+// per key and counting its 11-bit bin in a shared histogram that is added to
+// the sequence's global histogram when the CTA moves to another sequence.
 //
 // Selection kernel: one CTA per sequence runs an exact radix select over the
 // 64-bit ranking keys (score, then lower index) of its scores and writes the
@@ -42,10 +43,11 @@ struct IdxDecodeCfg {
   static constexpr int TMEM_COLS = 128;        // 2 x HI (<= 128) rounded to a power of two >= 32
   static constexpr int OFF_K = 0;
   static constexpr int OFF_Q = OFF_K + KST * KTILE_BYTES;
-  static constexpr int OFF_W = OFF_Q + ((QBYTES + 1023) / 1024) * 1024;
+  static constexpr int QPAD = ((QBYTES + 1023) / 1024) * 1024;
+  static constexpr int OFF_W = OFF_Q + 2 * QPAD;  // two query buffers: the next item's loads early
   static constexpr int OFF_HIST = OFF_W + HI * 4;         // u32 [2048] per-CTA histogram
   static constexpr int OFF_BAR = OFF_HIST + 2048 * 4;
-  static constexpr int NBAR = 1 + 2 * KST + 2 * NACC;
+  static constexpr int NBAR = 4 + 2 * KST + 2 * NACC;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static_assert(HI % 16 == 0 && HI <= 64, "decode indexer: H_I must be 16, 32, 48 or 64");
@@ -57,6 +59,7 @@ struct IdxDecodeParams {
   const float* k_scale;  // [B, L_max]
   const int32_t* lens;   // [B]
   int L_max;
+  int B;
   float* scores;         // [B, L_max]; entries s >= lens[b] untouched
   uint32_t* hist;        // [B, 2048] counts of the top 11 bits of each ranking key, or null
 };
@@ -70,11 +73,15 @@ __global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS)
     indexer_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const IdxDecodeParams p) {
   using C = IdxDecodeCfg<HI, DI>;
-  const int b = blockIdx.y;
-  const int s0 = blockIdx.x * C::CHUNK;
-  const int n = p.lens[b];
-  if (s0 >= n) return;  // whole CTA, before any barrier or TMEM allocation
-  const int nkt = min(C::NKT, (n - s0 + C::BM - 1) / C::BM);
+  // Persistent: work item i is chunk i % nch of sequence i / nch; each CTA
+  // takes a contiguous range of items (so its sequence rarely changes) and
+  // keeps its barriers, TMEM and ring phases from one item to the next.
+  const int nch = (p.L_max + C::CHUNK - 1) / C::CHUNK;
+  const int total = p.B * nch;
+  const int per = (total + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
+  const int it0 = static_cast<int>(blockIdx.x) * per;
+  const int it1 = min(total, it0 + per);
+  if (it0 >= it1) return;  // whole CTA, before any barrier or TMEM allocation
 
   // 1024-byte aligned base, derived from the shared array by an offset so
   // the compiler keeps every access in the shared address space
@@ -83,12 +90,14 @@ __global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS)
   uint8_t* k_s = smem + C::OFF_K;
   uint8_t* q_s = smem + C::OFF_Q;
   float* w_s = reinterpret_cast<float*>(smem + C::OFF_W);
+  uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + C::OFF_HIST);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;
-  uint64_t* k_empty = bars + 1 + C::KST;
-  uint64_t* acc_full = bars + 1 + 2 * C::KST;
-  uint64_t* acc_empty = bars + 1 + 2 * C::KST + C::NACC;
+  uint64_t* q_full = bars;      // [2]
+  uint64_t* q_empty = bars + 2;  // [2]
+  uint64_t* k_full = bars + 4;
+  uint64_t* k_empty = bars + 4 + C::KST;
+  uint64_t* acc_full = bars + 4 + 2 * C::KST;
+  uint64_t* acc_empty = bars + 4 + 2 * C::KST + C::NACC;
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   int* abort_s = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
   const AbortFlag ab{abort_s};
@@ -97,7 +106,10 @@ __global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS)
 
   if (threadIdx.x == 0) {
     *abort_s = 0;
-    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(q_full + i, 1);
+      mbar_init(q_empty + i, 1);
+    }
     for (int i = 0; i < C::KST; ++i) {
       mbar_init(k_full + i, 1);
       mbar_init(k_empty + i, 1);
@@ -108,94 +120,151 @@ __global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS)
     }
     fence_mbar_init();
   }
-  for (int i = threadIdx.x; i < HI; i += blockDim.x) w_s[i] = p.w[static_cast<size_t>(b) * HI + i];
-  uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + C::OFF_HIST);
   if (p.hist)
     for (int i = threadIdx.x; i < 2048; i += blockDim.x) hist_s[i] = 0;
   if (warp == 1) tmem_alloc(tmem_base_s, C::TMEM_COLS);
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_base_s;
-  const size_t row0 = static_cast<size_t>(b) * p.L_max + s0;  // first key row of this CTA
+
+  // sequence, first key, key tiles and length of item `it`; false when the
+  // chunk starts past the sequence's length (the same answer on every role)
+  auto item = [&](int it, int& b, int& s0, int& nkt, int& n) {
+    b = it / nch;
+    s0 = (it % nch) * C::CHUNK;
+    n = min(p.lens[b], p.L_max);
+    if (s0 >= n) return false;
+    nkt = min(C::NKT, (n - s0 + C::BM - 1) / C::BM);
+    return true;
+  };
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, C::QBYTES);
-      tma_load_2d(q_s, &tmQ, q_full, 0, b * HI);
-      for (int kt = 0; kt < nkt; ++kt) {
-        const int slot = kt % C::KST;
-        if (!mbar_wait(k_empty + slot, ((kt / C::KST) & 1) ^ 1, ab, 11)) break;
-        mbar_arrive_expect_tx(k_full + slot, C::KTILE_BYTES);
-        tma_load_2d(k_s + slot * C::KTILE_BYTES, &tmK, k_full + slot, 0, static_cast<int>(row0) + kt * C::BM);
+      int g = 0;   // key tiles issued so far (ring position and phase)
+      int qn = 0;  // query loads issued so far
+      for (int it = it0; it < it1; ++it) {
+        int b, s0, nkt, n;
+        if (!item(it, b, s0, nkt, n)) continue;
+        // query buffer qn & 1: the MMA has finished with the item two back
+        const int qb = qn & 1;
+        if (!mbar_wait(q_empty + qb, ((qn >> 1) & 1) ^ 1, ab, 10)) break;
+        mbar_arrive_expect_tx(q_full + qb, C::QBYTES);
+        tma_load_2d(q_s + qb * C::QPAD, &tmQ, q_full + qb, 0, b * HI);
+        ++qn;
+        const int row0 = b * p.L_max + s0;  // B * L_max < 2^31 (checked on the host)
+        bool ok = true;
+        for (int kt = 0; kt < nkt; ++kt, ++g) {
+          const int slot = g % C::KST;
+          if (!mbar_wait(k_empty + slot, ((g / C::KST) & 1) ^ 1, ab, 11)) { ok = false; break; }
+          mbar_arrive_expect_tx(k_full + slot, C::KTILE_BYTES);
+          tma_load_2d(k_s + slot * C::KTILE_BYTES, &tmK, k_full + slot, 0, row0 + kt * C::BM);
+        }
+        if (!ok) break;
       }
       // wait until the MMA has consumed every issued tile (copies landed)
-      for (int kt = max(0, nkt - C::KST); kt < nkt && !ab.raised(); ++kt)
-        mbar_wait(k_empty + kt % C::KST, (kt / C::KST) & 1, ab, 12);
+      for (int gg = max(0, g - C::KST); gg < g && !ab.raised(); ++gg)
+        mbar_wait(k_empty + gg % C::KST, (gg / C::KST) & 1, ab, 12);
     }
   } else if (warp == 1) {
     // the warp waits converged; one elected lane issues and commits
-    bool ok = mbar_wait_warp(q_full, 0, ab, 13);
-    const uint32_t q_addr = smem_u32(q_s);
-    for (int kt = 0; kt < nkt && ok; ++kt) {
-      const int slot = kt % C::KST;
-      const int buf = kt % C::NACC;
-      if (!mbar_wait_warp(k_full + slot, (kt / C::KST) & 1, ab, 14)) break;
-      if (!mbar_wait_warp(acc_empty + buf, ((kt / C::NACC) & 1) ^ 1, ab, 15)) break;
-      tc_fence_after();
-      if (elect_one()) {
-        const uint32_t a_addr = smem_u32(k_s + slot * C::KTILE_BYTES);
+    int g = 0;
+    int qn = 0;
+    bool ok = true;
+    for (int it = it0; it < it1 && ok; ++it) {
+      int b, s0, nkt, n;
+      if (!item(it, b, s0, nkt, n)) continue;
+      const int qb = qn & 1;
+      if (!mbar_wait_warp(q_full + qb, (qn >> 1) & 1, ab, 13)) break;
+      ++qn;
+      const uint32_t q_addr = smem_u32(q_s + qb * C::QPAD);
+      for (int kt = 0; kt < nkt; ++kt, ++g) {
+        const int slot = g % C::KST;
+        const int buf = g % C::NACC;
+        if (!mbar_wait_warp(k_full + slot, (g / C::KST) & 1, ab, 14)) { ok = false; break; }
+        if (!mbar_wait_warp(acc_empty + buf, ((g / C::NACC) & 1) ^ 1, ab, 15)) { ok = false; break; }
+        tc_fence_after();
+        if (elect_one()) {
+          const uint32_t a_addr = smem_u32(k_s + slot * C::KTILE_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < C::KSTEPS; ++kk) {
-          const uint64_t ad = smem_desc(a_addr + kk * 32, 16, C::SBO, C::SW);
-          const uint64_t bd = smem_desc(q_addr + kk * 32, 16, C::SBO, C::SW);
-          mma_f8(tmem + buf * HI, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < C::KSTEPS; ++kk) {
+            const uint64_t ad = smem_desc(a_addr + kk * 32, 16, C::SBO, C::SW);
+            const uint64_t bd = smem_desc(q_addr + kk * 32, 16, C::SBO, C::SW);
+            mma_f8(tmem + buf * HI, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(acc_full + buf);
+          tc_commit(k_empty + slot);
+          if (kt == nkt - 1) tc_commit(q_empty + qb);  // this item's query buffer may be reused
         }
-        tc_commit(acc_full + buf);
-        tc_commit(k_empty + slot);
+        __syncwarp();
       }
-      __syncwarp();
     }
   } else {
     const int quarter = static_cast<int>(warp & 3);
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    const float qs = p.q_scale[b];
-    for (int kt = 0; kt < nkt; ++kt) {
-      const int buf = kt % C::NACC;
-      const int s = s0 + kt * C::BM + quarter * 32 + static_cast<int>(lane);
-      const float ks = (s < n) ? p.k_scale[static_cast<size_t>(b) * p.L_max + s] : 0.f;
-      if (!mbar_wait(acc_full + buf, (kt / C::NACC) & 1, ab, 16)) break;
-      tc_fence_after();
-      float acc = 0.f;
-      if constexpr (HI % 32 == 0) {
-#pragma unroll
-        for (int h = 0; h < HI / 32; ++h) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_addr + buf * HI + h * 32, r);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) acc = __fmaf_rn(w_s[h * 32 + j], fmaxf(__uint_as_float(r[j]), 0.f), acc);
-        }
-      } else {
-        uint32_t r[16];
-        tmem_ld16(tmem + lane_addr + buf * HI, r);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) acc = __fmaf_rn(w_s[j], fmaxf(__uint_as_float(r[j]), 0.f), acc);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty + buf);
-      if (s < n) {
-        const float score = __fmul_rn(__fmul_rn(acc, qs), ks);
-        p.scores[static_cast<size_t>(b) * p.L_max + s] = score;
-        if (p.hist) atomicAdd(hist_s + key_bin11(rank_key(score, static_cast<uint32_t>(s))), 1u);
-      }
-    }
-    if (p.hist) {
-      named_bar_sync(1, 128);
-      const int et = threadIdx.x - 64;
+    const int et = static_cast<int>(threadIdx.x) - 64;  // 0..127
+    // add this CTA's counts of sequence bq to the global histogram, zeroing them
+    auto flush_hist = [&](int bq) {
       for (int i = et; i < 2048; i += 128) {
         const uint32_t c = hist_s[i];
-        if (c) atomicAdd(p.hist + static_cast<size_t>(b) * 2048 + i, c);
+        if (c) {
+          atomicAdd(p.hist + static_cast<size_t>(bq) * 2048 + i, c);
+          hist_s[i] = 0;
+        }
       }
+    };
+    int g = 0;
+    int cur_b = -1;
+    bool ok = true;
+    for (int it = it0; it < it1 && ok; ++it) {
+      int b, s0, nkt, n;
+      if (!item(it, b, s0, nkt, n)) continue;
+      if (b != cur_b) {
+        named_bar_sync(1, 128);  // the previous sequence's weights and counts are done with
+        if (p.hist && cur_b >= 0) flush_hist(cur_b);
+        for (int i = et; i < HI; i += 128) w_s[i] = p.w[static_cast<size_t>(b) * HI + i];
+        named_bar_sync(1, 128);
+        cur_b = b;
+      }
+      const float qs = p.q_scale[b];
+      for (int kt = 0; kt < nkt; ++kt, ++g) {
+        const int buf = g % C::NACC;
+        const int s = s0 + kt * C::BM + quarter * 32 + static_cast<int>(lane);
+        const float ks = (s < n) ? p.k_scale[static_cast<size_t>(b) * p.L_max + s] : 0.f;
+        if (!mbar_wait(acc_full + buf, (g / C::NACC) & 1, ab, 16)) { ok = false; break; }
+        tc_fence_after();
+        // eight independent partial sums (head j to sum j % 8), added in a
+        // fixed order: a single running sum would be a 64-deep dependent chain
+        float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if constexpr (HI % 32 == 0) {
+#pragma unroll
+          for (int h = 0; h < HI / 32; ++h) {
+            uint32_t r[32];
+            tmem_ld32(tmem + lane_addr + buf * HI + h * 32, r);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              part[j & 7] = __fmaf_rn(w_s[h * 32 + j], fmaxf(__uint_as_float(r[j]), 0.f), part[j & 7]);
+          }
+        } else {
+          uint32_t r[16];
+          tmem_ld16(tmem + lane_addr + buf * HI, r);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            part[j & 7] = __fmaf_rn(w_s[j], fmaxf(__uint_as_float(r[j]), 0.f), part[j & 7]);
+        }
+        const float acc = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty + buf);
+        if (s < n) {
+          const float score = __fmul_rn(__fmul_rn(acc, qs), ks);
+          p.scores[static_cast<size_t>(b) * p.L_max + s] = score;
+          if (p.hist) atomicAdd(hist_s + key_bin11(rank_key(score, static_cast<uint32_t>(s))), 1u);
+        }
+      }
+    }
+    if (p.hist && cur_b >= 0) {
+      named_bar_sync(1, 128);
+      flush_hist(cur_b);
     }
   }
   __syncthreads();
@@ -215,7 +284,7 @@ __global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS)
 // over global memory. Writes the k best keys of sequence b (unordered, 0
 // where lens[b] < k) to sel_keys[b, 0..k).
 constexpr int kDecodeSelThreads = 1024;
-constexpr int kDecodeSelBinCap = 4096;  // boundary-bin keys kept in shared memory
+constexpr int kDecodeSelBinCap = 16384;  // boundary-bin keys kept in shared memory (128 KB)
 
 __global__ void __launch_bounds__(kDecodeSelThreads)
     decode_select_kernel(const float* __restrict__ scores, const int32_t* __restrict__ lens, int L_max, int K,
@@ -229,7 +298,7 @@ __global__ void __launch_bounds__(kDecodeSelThreads)
   __shared__ int res[4];
   __shared__ int wpos, bpos;
   const int b = blockIdx.x;
-  const int n = lens[b];
+  const int n = min(lens[b], L_max);
   const float* sc = scores + static_cast<size_t>(b) * L_max;
   uint64_t* dst = sel_keys + static_cast<size_t>(b) * K;
   const int tid = threadIdx.x;
@@ -280,14 +349,28 @@ __global__ void __launch_bounds__(kDecodeSelThreads)
   const int need = K - above;  // keys to take from the boundary bin (1..inb)
   // 3. one pass: keys above the bin go out; the bin's keys are kept
   const bool fits = inb <= kDecodeSelBinCap;
-  for (int i = tid; i < n; i += NT) {
-    const uint64_t key = rank_key(sc[i], static_cast<uint32_t>(i));
+  // (warp-aggregated appends: one shared atomic per warp and destination)
+  const uint32_t lane = tid & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  const int nround = (n + NT - 1) / NT;  // same trip count on every lane
+#pragma unroll 4
+  for (int rd = 0; rd < nround; ++rd) {
+    const int i = rd * NT + tid;
+    const uint64_t key = (i < n) ? rank_key(sc[i], static_cast<uint32_t>(i)) : 0ull;
     const uint32_t bin = key_bin11(key);
-    if (bin > dbin) {
-      dst[atomicAdd(&wpos, 1)] = key;
-    } else if (bin == dbin && fits) {
-      bin_keys[atomicAdd(&bpos, 1)] = key;
+    const bool hi = (i < n) && bin > dbin;
+    const bool eq = (i < n) && bin == dbin && fits;
+    const uint32_t mh = __ballot_sync(0xffffffffu, hi);
+    const uint32_t me = __ballot_sync(0xffffffffu, eq);
+    int bh = 0, be = 0;
+    if (lane == 0) {
+      if (mh) bh = atomicAdd(&wpos, __popc(mh));
+      if (me) be = atomicAdd(&bpos, __popc(me));
     }
+    bh = __shfl_sync(0xffffffffu, bh, 0);
+    be = __shfl_sync(0xffffffffu, be, 0);
+    if (hi) dst[bh + __popc(mh & lt)] = key;
+    if (eq) bin_keys[be + __popc(me & lt)] = key;
   }
   __syncthreads();
   // 4. exact choice of `need` keys inside the boundary bin
