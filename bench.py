@@ -39,6 +39,20 @@ if ROOT not in sys.path:
 import workloads  # noqa: E402
 
 METRIC = "DSA prefill tokens/s @128K & decode tok/s, % of FP8/BF16/HBM roofline"
+
+# DRAM bytes (read + write) per timed unit of the default workload, from one
+# single-pass ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of
+# this benchmark on B200. Valid only for the kernels they were taken on: set
+# an entry to None when its kernels change. Units: the prefill indexer entry
+# covers its main pass, re-run pass and rank sort; decode entries cover one
+# decode batch.
+MEASURED_TRAFFIC = {
+    "prefill_indexer": 1.699e9 + 5.262e9 + 7.1e4 + 2.148e9 + 1.041e9,
+    "prefill_attention": 75.06e9 + 17.18e9,
+    "decode_step": 0.554e9 + 0.014e9 + 0.017e9 + 0.001e9 + 0.161e9,
+    "decode_indexer": 0.554e9 + 0.014e9 + 0.017e9 + 0.001e9,
+}
+DEFAULT_SIZES = (131072, 64, 65536)  # prefill L, decode B, decode L the traffic was measured on
 D_QK, D_V = 576, 512
 
 
@@ -293,6 +307,9 @@ def run_ours(a, ws, rank):
         "decode_indexer": {"bound": "hbm", "achieved": dec_idx_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                            "frac": dec_idx_gbs / pk["hbm_gbs"], "traffic": None},
     }
+    if (L, D.B, D.L) == DEFAULT_SIZES:
+        for key, val in MEASURED_TRAFFIC.items():
+            rl[key]["traffic"] = val
     dom = "prefill_indexer" if t_idx >= t_attn else "prefill_attention"
     res = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": a.steps, "warmup": a.warmup,
@@ -306,7 +323,7 @@ def run_ours(a, ws, rank):
         "roofline": dict(rl[dom], kernel=dom),
         "roofline_all": rl,
         "peaks": {"source": pk["source"], "fp8": "2 x bf16_tflops_sustained"},
-        "gpu_launches": 7 * a.steps,
+        "gpu_launches": 8 * a.steps,  # prefill: indexer (main + re-run), rank sort, attention; decode: scores, select, rank sort, attention
         "clocks": clocks,
         "wall_s_timed": t_wall,
     }

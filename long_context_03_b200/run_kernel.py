@@ -1,0 +1,77 @@
+"""Run one hot-path call repeatedly on seeded synthetic inputs, for profiling a
+single kernel (e.g. under ncu with -k and -s/-c) without the rest of the
+benchmark's allocations.
+
+    python -m long_context_03_b200.run_kernel indexer --L 65536
+    python -m long_context_03_b200.run_kernel attention --L 16384
+    python -m long_context_03_b200.run_kernel decode --B 64 --L 65536
+
+Prints the CUDA-event time of the last call. Inputs come from the seeded
+generators of the benchmark (`workloads`); the indexer case uses a single
+query head for the attention inputs, which the indexer never reads.
+"""
+from __future__ import annotations
+
+import argparse
+import os
+import sys
+
+import torch
+
+_ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if _ROOT not in sys.path:
+    sys.path.insert(0, _ROOT)
+
+import long_context_03_b200 as dsa  # noqa: E402
+import workloads  # noqa: E402
+
+
+def _time(fn, repeat):
+    for _ in range(repeat - 1):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    fn()
+    e1.record()
+    torch.cuda.synchronize()
+    dsa.check_device_error()
+    return e0.elapsed_time(e1)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("op", choices=["indexer", "attention", "decode"])
+    ap.add_argument("--L", type=int, default=65536)
+    ap.add_argument("--B", type=int, default=64)
+    ap.add_argument("--topk", type=int, default=2048)
+    ap.add_argument("--repeat", type=int, default=3)
+    a = ap.parse_args(argv)
+    dev = torch.device("cuda", 0)
+    if a.op == "indexer":
+        P = workloads.make_prefill(a.L, 64, 128, 1, a.topk, seed=0, device=dev)
+        ws = torch.empty(dsa.index_topk_workspace_size(a.L, 64, 128, a.topk), dtype=torch.uint8, device=dev)
+        idx = torch.empty((a.L, a.topk), dtype=torch.int32, device=dev)
+        ms = _time(lambda: dsa.index_topk(P.q_I, P.q_scale, P.w, P.k_cache, P.k_scale, a.topk, idx=idx,
+                                          workspace=ws), a.repeat)
+    elif a.op == "attention":
+        P = workloads.make_prefill(a.L, 64, 128, 128, a.topk, seed=0, device=dev)
+        idx = dsa.index_topk(P.q_I, P.q_scale, P.w, P.k_cache, P.k_scale, a.topk)
+        out = torch.empty((a.L, 128, 512), dtype=torch.bfloat16, device=dev)
+        ms = _time(lambda: dsa.sparse_mla_attn(P.q, P.kv, idx, P.scale, out=out), a.repeat)
+    else:
+        D = workloads.make_decode(a.B, a.L, 64, 128, 128, a.topk, seed=0, device=dev)
+        ws = torch.empty(dsa.index_topk_decode_workspace_size(a.B, a.L, a.topk), dtype=torch.uint8, device=dev)
+        idx = torch.empty((a.B, a.topk), dtype=torch.int32, device=dev)
+        out = torch.empty((a.B, 128, 512), dtype=torch.bfloat16, device=dev)
+
+        def step():
+            dsa.index_topk_decode(D.q_I, D.q_scale, D.w, D.k_cache, D.k_scale, D.lens, a.topk, idx=idx, workspace=ws)
+            dsa.sparse_mla_attn_decode(D.q, D.kv, idx, D.scale, out=out)
+
+        ms = _time(step, a.repeat)
+    print(f"{a.op} L={a.L} B={a.B} topk={a.topk}: {ms:.3f} ms (last of {a.repeat} calls)")
+
+
+if __name__ == "__main__":
+    main()

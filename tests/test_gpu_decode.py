@@ -42,3 +42,24 @@ def test_decode_path(dsa, d_I):
         ok, mx, rl = attn_close(out[b:b + 1], ref_o)
         assert ok, (b, mx, rl)
         np.testing.assert_allclose(lse[b].cpu().numpy(), ref_l[0], rtol=1e-4, atol=1e-4)
+
+
+def test_decode_selection_with_all_scores_tied(dsa):
+    # one 11-bit bin holds every key: 40000 keys overflow the on-chip bin
+    # buffer (global multi-pass path), 10000 keys fit it; ties go to the
+    # lower index, so the answer is 0..k-1 in order
+    B, L, k = 3, 40000, 2048
+    lens = [40000, 10000, 3000]
+    inp = workloads.make_decode(B, L, 64, 128, 16, k, seed=41, lens=lens)
+    inp.k_cache[:] = inp.k_cache[:, :1]
+    inp.k_scale[:] = inp.k_scale[:, :1]
+    d = inp.to("cuda")
+    sc = dsa.index_scores_decode(d.q_I, d.q_scale, d.w, d.k_cache, d.k_scale, d.lens).cpu().numpy()
+    idx = dsa.index_topk_decode(d.q_I, d.q_scale, d.w, d.k_cache, d.k_scale, d.lens, k)
+    dsa.check_device_error()
+    idx = idx.cpu().numpy()
+    for b in range(B):
+        n = lens[b]
+        assert np.all(sc[b, :n] == sc[b, 0])
+        assert np.array_equal(idx[b], np.arange(k, dtype=np.int32))
+        assert np.array_equal(idx[b], cpu_topk_of(sc[b:b + 1, :n], [n - 1], k)[0])
