@@ -169,6 +169,9 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
   uint64_t* acc_empty = bars + 2 + 2 * C::KST + C::NACC;
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   int* abort_s = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
+  // bit tl: a sub-list of row tl may overflow before the next check (set by
+  // the appending warp, read at the capacity checks)
+  int* cutmask_s = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
   const AbortFlag ab{abort_s};
 
   const uint32_t warp = warp_id();
@@ -324,6 +327,7 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
         thr_s[i] = 0ull;
       }
       for (int i = et; i < 4 * C::RB; i += C::NET) cnt_s[i] = 0;
+      if (et == 0) *cutmask_s = 0;
       named_bar_sync(1, C::NET);
       bool ok = true;
       float ks_next = 0.f;
@@ -411,7 +415,10 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
                   my_cand[static_cast<size_t>(tl) * p.cap + static_cast<size_t>(quarter) * capq + base +
                           __popc(m & lanemask_lt)] = key;
                 __syncwarp();
-                if (lane == 0 && m) *cnt = base + __popc(m);
+                if (lane == 0 && m) {
+                  *cnt = base + __popc(m);
+                  if (base + __popc(m) > capq - 32 * C::CHECK_EVERY) atomicOr(cutmask_s, 1 << tl);
+                }
               }
             } else {
               if (valid && t >= p.row0 && t < p.row0 + p.nrows)
@@ -455,15 +462,17 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
               named_bar_sync(1, C::NET);
             }
             if (et < 4 * C::RB) cnt_s[et] = 0;
+            if (et == 0) *cutmask_s = 0;
             named_bar_sync(1, C::NET);
             continue;
           }
           if ((i % C::CHECK_EVERY) != C::CHECK_EVERY - 1) continue;
           named_bar_sync(1, C::NET);
+          const uint32_t cmask = static_cast<uint32_t>(*cutmask_s);
+          if (cmask == 0) continue;
           for (int tl = 0; tl < C::RB; ++tl) {
             const int* cn = cnt_s + tl * 4;
-            const int nmax = max(max(cn[0], cn[1]), max(cn[2], cn[3]));
-            if (nmax > capq - 32 * C::CHECK_EVERY) {
+            if ((cmask >> tl) & 1u) {
               uint64_t* row = my_cand + static_cast<size_t>(tl) * p.cap;
               const int n = cn[0] + cn[1] + cn[2] + cn[3];
               uint64_t v[4 * MQ];
@@ -484,6 +493,9 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
               named_bar_sync(1, C::NET);
             }
           }
+          // every flagged row was cut; all threads read the mask before the cuts' barriers
+          if (et == 0) *cutmask_s = 0;
+          named_bar_sync(1, C::NET);
         }
       }
       if (!ok) break;
