@@ -10,14 +10,16 @@
 //
 // The fp32 output tile of one token (128 heads x 512 values) needs all 512
 // TMEM columns of an SM, so each token runs on a 2-CTA cluster:
-//   CTA 0 (score CTA) keeps Q[t, :, 0:512] in TMEM (256 columns of bf16
-//     pairs, the A operand of a TMEM-sourced MMA) and Q[t, :, 512:576] in
-//     shared memory, and computes S = Q C^T for chunks of 128 selected rows
-//     (M = 128 heads, N = 128 rows: a full-rate tcgen05 shape) into one of two
-//     128-column S buffers. The rows are gathered slab by slab (64 values =
-//     128 bytes of each row, 16 KB per slab tile) through a ring, so the
-//     576-wide chunk never has to be resident at once. Its softmax warps
-//     (one thread per head) turn S into bf16 probabilities P with a running
+//   CTA 0 (score CTA) keeps all of Q[t] in TMEM (288 columns of bf16 pairs,
+//     the A operand of TMEM-sourced MMAs) and computes S = Q C^T for chunks
+//     of 128 selected rows (M = 128 heads, N = 128 rows: a full-rate tcgen05
+//     shape) into a single 128-column S buffer. The rows are gathered slab by
+//     slab (64 values = 128 bytes of each row, 16 KB per slab tile) through a
+//     ring, so the 576-wide chunk never has to be resident at once. Its
+//     softmax warps (one thread per head) copy their 128 scores of the chunk
+//     into registers and hand the S buffer back at once, so the next chunk's
+//     QK^T overlaps this chunk's softmax with one buffer. They turn S into
+//     bf16 probabilities P with a running
 //     reference max that only moves when a chunk exceeds it by more than 2^8
 //     (so P <= 256 and the accumulator is rarely rescaled), and ship P, the
 //     per-head rescale factors and, after the last chunk, the row sums and
@@ -53,7 +55,7 @@ struct MlaCfg {
   static constexpr int VSLAB = VROWS * 128;   // one slab of a value sub-tile: 4 KB
   static constexpr int V_TILE = NSLAB_V * VSLAB;  // 32 KB
   static constexpr int NVST = 4;              // value sub-tile ring depth (value CTA)
-  static constexpr int NSB = 2;               // S buffers in TMEM
+  static constexpr int NSB = 1;               // S buffer in TMEM (the softmax copies it to registers at once)
   static constexpr int NPB = 2;               // P message buffers
   static constexpr int KMAX = 2048;           // largest selection (index row staged in smem)
   static constexpr int P_BYTES = M * NK * 2;  // 32 KB: two 128-byte-swizzled K slabs of 64 rows
@@ -68,16 +70,15 @@ struct MlaCfg {
   static constexpr int W_MMA = 4;
   static constexpr int W_SM0 = 5;             // first softmax / epilogue warp
   static constexpr int NTHREADS = 9 * 32;
-  static constexpr int S_COL = 0;             // S buffers: columns [0, 256)
-  static constexpr int Q_COL = 256;           // Q dims 0..511: columns [256, 512)
+  static constexpr int Q_COL = 0;             // Q dims 0..575: columns [0, 288)
+  static constexpr int S_COL = 288;           // S: columns [288, 416)
   static constexpr uint32_t IDESC_QK = instr_desc(kFmtBF16, M, NK, false, false);
   static constexpr uint32_t IDESC_PV = instr_desc(kFmtBF16, M, 256, false, true);
   // shared memory (offsets from a 1024-aligned base); both CTAs use the same
   // layout so barrier offsets match across the cluster
   static constexpr int OFF_RING = 0;          // score CTA: NSST slab tiles; value CTA: NVST value sub-tiles
   static constexpr int RING_BYTES = (NSST * SLAB_TILE > NVST * V_TILE) ? NSST * SLAB_TILE : NVST * V_TILE;
-  static constexpr int OFF_QROPE = OFF_RING + RING_BYTES;  // score CTA: Q[:, 512:576] (16 KB)
-  static constexpr int OFF_MSG = OFF_QROPE + M * 128;      // NPB x MSG_STRIDE (staging / receive)
+  static constexpr int OFF_MSG = OFF_RING + RING_BYTES;    // NPB x MSG_STRIDE (staging / receive)
   static constexpr int OFF_IDX = OFF_MSG + NPB * MSG_STRIDE;  // int32 [KMAX]: the token's index row
   static constexpr int OFF_VMASK = OFF_IDX + KMAX * 4;       // score CTA: u32 [2][KMAX/32] validity bits per token
   static constexpr int OFF_BAR = OFF_VMASK + 2 * (KMAX / 32) * 4;
@@ -169,15 +170,6 @@ __device__ __forceinline__ int checked_row(const int32_t* idx_s, int e, int K, i
     row = -1;
   }
   return row;
-}
-
-// Slab order within chunk j: the RoPE slab (8, multiplied from shared memory)
-// comes last in even chunks and first in odd ones, so consecutive chunks' RoPE
-// MMAs run back to back. Every switch between the TMEM-A and shared-memory-A
-// MMA forms drains the tensor pipe (measured on B200: ~740 cycles), so this
-// halves the switches.
-__device__ __forceinline__ int slab_at(int j, int i) {
-  return (j & 1) ? (i == 0 ? MlaCfg::NSLAB_QK - 1 : i - 1) : i;
 }
 
 // Score CTA: the 8 rows (r = ptid/8 + 16k) this thread copies for chunk j,
@@ -338,7 +330,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
           const ChunkRows cr = chunk_rows(kv_tok, idx_s, j, p.K, p.rows, ptid);
           for (int i = 0; i < C::NSLAB_QK; ++i) {
             if (!mbar_wait(bars + C::B_RING_EMPTY + slot, ph, ab, 31)) { ok = false; break; }
-            gather_slab_tile(ring + slot * C::SLAB_TILE, cr, slab_at(j, i), ptid);
+            gather_slab_tile(ring + slot * C::SLAB_TILE, cr, i, ptid);
             cp_async_mbar_arrive(bars + C::B_RING_FULL + slot);
             if (++slot == C::NSST) { slot = 0; ph ^= 1; }
           }
@@ -351,38 +343,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       // issues each slab's MMAs together with every commit that covers them.
       int slot = 0;
       uint32_t ph = 0;
-      int sb = 0;
       uint32_t sph = 1;
       uint32_t qph = 0;
-      const uint32_t qrope = smem_u32(smem + C::OFF_QROPE);
       bool ok = true;
       for (int tk = cluster_id; tk < p.T && ok; tk += nclusters) {
         if (!mbar_wait_warp(bars + C::B_Q_READY, qph, ab, 32)) break;
         qph ^= 1;
         tc_fence_after();
         for (int j = 0; j < nchunk && ok; ++j) {
-          if (!mbar_wait_warp(bars + C::B_S_EMPTY + sb, sph, ab, 34)) { ok = false; break; }
+          if (!mbar_wait_warp(bars + C::B_S_EMPTY, sph, ab, 34)) { ok = false; break; }
+          sph ^= 1;
           tc_fence_after();
-          const uint32_t d = tmem + C::S_COL + sb * C::NK;
+          const uint32_t d = tmem + C::S_COL;
           for (int i = 0; i < C::NSLAB_QK; ++i) {
             if (!mbar_wait_warp(bars + C::B_RING_FULL + slot, ph, ab, 33)) { ok = false; break; }
             tc_fence_after();
             if (elect_one()) {
-              const int s = slab_at(j, i);
               const uint32_t tile = ring + slot * C::SLAB_TILE;
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
                 const uint64_t bd = smem_desc(tile + kk * 32, 16, 1024, kSw128);
-                const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-                if (s < C::NSLAB_QK - 1) {
-                  mma_bf16_ts(d, tmem + C::Q_COL + (4 * s + kk) * 8, bd, C::IDESC_QK, acc);
-                } else {
-                  mma_bf16_ss(d, smem_desc(qrope + kk * 32, 16, 1024, kSw128), bd, C::IDESC_QK, acc);
-                }
+                mma_bf16_ts(d, tmem + C::Q_COL + (4 * i + kk) * 8, bd, C::IDESC_QK, (i > 0 || kk > 0) ? 1u : 0u);
               }
               tc_commit(bars + C::B_RING_EMPTY + slot);
               if (i == C::NSLAB_QK - 1) {
-                tc_commit(bars + C::B_S_FULL + sb);
+                tc_commit(bars + C::B_S_FULL);
                 if (j == nchunk - 1) tc_commit(bars + C::B_Q_FREE);
               }
             }
@@ -390,7 +375,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
             if (++slot == C::NSST) { slot = 0; ph ^= 1; }
           }
           if (!ok) break;
-          if (++sb == C::NSB) { sb = 0; sph ^= 1; }
         }
       }
     } else {
@@ -400,8 +384,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
       const uint32_t peer_msg = map_to_peer(msg, 1);
       const uint32_t peer_pfull = map_to_peer(smem_u32(bars + C::B_P_FULL), 1);
-      uint8_t* qrope_s = smem + C::OFF_QROPE;
-      int sb = 0;
       uint32_t sph = 0;
       uint32_t qfree_ph = 1;
       int pb = 0;
@@ -416,9 +398,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
         qfree_ph ^= 1;
         tc_fence_after();
         {
-          // the head's 1152-byte row in 9 blocks of 64 values (blocks 0..7 to
-          // TMEM as 32 columns each, block 8 to shared memory), loaded three
-          // blocks at a time so each round trip has 24 loads in flight
+          // the head's 1152-byte row in 9 blocks of 64 values, each to 32 TMEM
+          // columns, loaded three blocks at a time so each round trip has 24
+          // loads in flight
           const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(tk) * p.Hq + h) * C::D);
 #pragma unroll
           for (int rnd = 0; rnd < 3; ++rnd) {
@@ -428,21 +410,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
 #pragma unroll
             for (int bb = 0; bb < 3; ++bb) {
               const int cb = rnd * 3 + bb;
-              if (cb < 8) {
-                uint32_t r[32];
+              uint32_t r[32];
 #pragma unroll
-                for (int v = 0; v < 8; ++v) {
-                  r[4 * v + 0] = x[bb * 8 + v].x;
-                  r[4 * v + 1] = x[bb * 8 + v].y;
-                  r[4 * v + 2] = x[bb * 8 + v].z;
-                  r[4 * v + 3] = x[bb * 8 + v].w;
-                }
-                tmem_st32(tmem + lane_addr + C::Q_COL + cb * 32, r);
-              } else {
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                  *reinterpret_cast<uint4*>(qrope_s + h * 128 + ((c ^ (h & 7)) << 4)) = x[bb * 8 + c];
+              for (int v = 0; v < 8; ++v) {
+                r[4 * v + 0] = x[bb * 8 + v].x;
+                r[4 * v + 1] = x[bb * 8 + v].y;
+                r[4 * v + 2] = x[bb * 8 + v].z;
+                r[4 * v + 3] = x[bb * 8 + v].w;
               }
+              tmem_st32(tmem + lane_addr + C::Q_COL + cb * 32, r);
             }
           }
           tmem_st_wait();
@@ -467,25 +443,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
           // validity of the chunk's 128 entries (the same for every head)
           const uint4 vm4 = vm_tok[j];
           const uint32_t vmask[4] = {vm4.x, vm4.y, vm4.z, vm4.w};
-          if (!mbar_wait(bars + C::B_S_FULL + sb, sph, ab, 36)) { ok = false; break; }
+          if (!mbar_wait(bars + C::B_S_FULL, sph, ab, 36)) { ok = false; break; }
+          sph ^= 1;
           tc_fence_after();
-          const uint32_t s_addr = tmem + lane_addr + C::S_COL + sb * C::NK;
-          // pass 1 over S (32 columns at a time): the chunk's max. Invalid
-          // entries (absent rows, gathered as zeros) are masked to -inf; a
-          // chunk without any is the common case and skips the masking.
+          // this head's 128 scores of the chunk into registers; the S buffer
+          // goes back to the tensor core at once, so the next chunk's QK^T
+          // overlaps this chunk's softmax with a single S buffer in TMEM
+          const uint32_t s_addr = tmem + lane_addr + C::S_COL;
+          uint32_t sr[4][32];
+#pragma unroll
+          for (int g = 0; g < 4; ++g) tmem_ld32_nowait(s_addr + g * 32, sr[g]);
+#pragma unroll
+          for (int g = 0; g < 4; ++g) tmem_ld_wait_fence(sr[g]);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bars + C::B_S_EMPTY);
+          // pass 1: the chunk's max. Invalid entries (absent rows, gathered
+          // as zeros) are masked to -inf; a chunk without any is the common
+          // case and skips the masking.
           const bool all_valid = (vmask[0] & vmask[1] & vmask[2] & vmask[3]) == 0xffffffffu;
           float mc = -INFINITY;
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
-            uint32_t sr[32];
-            tmem_ld32(s_addr + g * 32, sr);
             if (all_valid) {
 #pragma unroll
-              for (int c = 0; c < 32; ++c) mc = fmaxf(mc, __uint_as_float(sr[c]));
+              for (int c = 0; c < 32; ++c) mc = fmaxf(mc, __uint_as_float(sr[g][c]));
             } else {
 #pragma unroll
               for (int c = 0; c < 32; ++c)
-                if ((vmask[g] >> c) & 1u) mc = fmaxf(mc, __uint_as_float(sr[c]));
+                if ((vmask[g] >> c) & 1u) mc = fmaxf(mc, __uint_as_float(sr[g][c]));
             }
           }
           mc = (mc == -INFINITY) ? -INFINITY : mc * p.scale_log2;
@@ -505,8 +491,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
           float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
-            uint32_t sr[32];
-            tmem_ld32(s_addr + g * 32, sr);
             const uint32_t vm = all_valid ? 0xffffffffu : vmask[g];
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4) {  // 4 chunks of 8 keys = 16 bytes of the P row
@@ -514,8 +498,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
                 const int c = c4 * 8 + 2 * i;
-                float p0 = fast_exp2(__fmaf_rn(__uint_as_float(sr[c]), p.scale_log2, neg_m));
-                float p1 = fast_exp2(__fmaf_rn(__uint_as_float(sr[c + 1]), p.scale_log2, neg_m));
+                float p0 = fast_exp2(__fmaf_rn(__uint_as_float(sr[g][c]), p.scale_log2, neg_m));
+                float p1 = fast_exp2(__fmaf_rn(__uint_as_float(sr[g][c + 1]), p.scale_log2, neg_m));
                 p0 = ((vm >> c) & 1u) ? p0 : 0.f;
                 p1 = ((vm >> (c + 1)) & 1u) ? p1 : 0.f;
                 pk[i] = pack_bf16x2(p0, p1);
@@ -529,10 +513,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
             }
           }
           l_sum += ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bars + C::B_S_EMPTY + sb);
-          if (++sb == C::NSB) { sb = 0; sph ^= 1; }
           reinterpret_cast<float*>(st + C::MSG_ALPHA)[h] = alpha;
           const uint32_t any_rs = __ballot_sync(0xffffffffu, alpha != 1.f);
           if (lane == 0 && any_rs) atomicOr(rescale_s + (pb & 1), 1);
