@@ -349,28 +349,54 @@ __global__ void __launch_bounds__(kDecodeSelThreads)
   const int need = K - above;  // keys to take from the boundary bin (1..inb)
   // 3. one pass: keys above the bin go out; the bin's keys are kept
   const bool fits = inb <= kDecodeSelBinCap;
-  // (warp-aggregated appends: one shared atomic per warp and destination)
-  const uint32_t lane = tid & 31;
-  const uint32_t lt = (1u << lane) - 1u;
-  const int nround = (n + NT - 1) / NT;  // same trip count on every lane
-#pragma unroll 4
+  // Each thread takes 4 consecutive keys per round (one 16-byte load when
+  // the rows are 16-byte aligned); a warp scan of the per-thread counts
+  // gives every thread its write positions, one shared atomic per warp and
+  // destination.
+  const int lane = tid & 31;
+  const bool vec = ((L_max & 3) == 0) && ((reinterpret_cast<uintptr_t>(scores) & 15) == 0);
+  const int nround = (n + 4 * NT - 1) / (4 * NT);  // same trip count on every lane
   for (int rd = 0; rd < nround; ++rd) {
-    const int i = rd * NT + tid;
-    const uint64_t key = (i < n) ? rank_key(sc[i], static_cast<uint32_t>(i)) : 0ull;
-    const uint32_t bin = key_bin11(key);
-    const bool hi = (i < n) && bin > dbin;
-    const bool eq = (i < n) && bin == dbin && fits;
-    const uint32_t mh = __ballot_sync(0xffffffffu, hi);
-    const uint32_t me = __ballot_sync(0xffffffffu, eq);
-    int bh = 0, be = 0;
-    if (lane == 0) {
-      if (mh) bh = atomicAdd(&wpos, __popc(mh));
-      if (me) be = atomicAdd(&bpos, __popc(me));
+    const int i0 = 4 * (rd * NT + tid);
+    float f[4];
+    if (vec && i0 + 3 < n) {
+      const float4 x = *reinterpret_cast<const float4*>(sc + i0);
+      f[0] = x.x; f[1] = x.y; f[2] = x.z; f[3] = x.w;
+    } else {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) f[u] = (i0 + u < n) ? sc[i0 + u] : 0.f;
     }
-    bh = __shfl_sync(0xffffffffu, bh, 0);
-    be = __shfl_sync(0xffffffffu, be, 0);
-    if (hi) dst[bh + __popc(mh & lt)] = key;
-    if (eq) bin_keys[be + __popc(me & lt)] = key;
+    uint64_t key[4];
+    uint32_t hi = 0, eq = 0;  // bit u: key u goes out / is kept for the bin
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      key[u] = rank_key(f[u], static_cast<uint32_t>(i0 + u));
+      const uint32_t bin = key_bin11(key[u]);
+      const bool in = i0 + u < n;
+      hi |= (in && bin > dbin) ? (1u << u) : 0u;
+      eq |= (in && bin == dbin && fits) ? (1u << u) : 0u;
+    }
+    // counts packed as (eq << 16) | hi; inclusive warp scan
+    const int mine = __popc(hi) | (__popc(eq) << 16);
+    int incl = mine;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    int base = 0;
+    if (lane == 31 && incl != 0) {
+      const int th = incl & 0xffff, te = incl >> 16;
+      base = (th ? atomicAdd(&wpos, th) : 0) | ((te ? atomicAdd(&bpos, te) : 0) << 16);
+    }
+    base = __shfl_sync(0xffffffffu, base, 31);
+    int ph = (base & 0xffff) + ((incl - mine) & 0xffff);
+    int pe = (base >> 16) + ((incl - mine) >> 16);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if ((hi >> u) & 1u) dst[ph++] = key[u];
+      if ((eq >> u) & 1u) bin_keys[pe++] = key[u];
+    }
   }
   __syncthreads();
   // 4. exact choice of `need` keys inside the boundary bin
