@@ -82,6 +82,24 @@ dsa_status dsa_index_topk(const uint8_t* q_I, const float* q_scale, const float*
                           const float* k_scale, int L, int H_I, int d_I, int topk, int32_t* idx, void* workspace,
                           size_t ws_bytes, void* stream);
 
+/* Chunked prefill: the same selection for a chunk of Tq new query tokens at
+ * positions q0 .. q0+Tq-1 against a key cache of L >= q0 + Tq tokens (the
+ * cache already holds the chunk's own keys; query r sees keys s <= q0 + r).
+ * Row r of the result equals row q0 + r of dsa_index_topk over the first
+ * q0 + Tq tokens.
+ *
+ *   q_I      [Tq, H_I, d_I] e4m3      q_scale [Tq]   w [Tq, H_I]
+ *   k_cache  [L, d_I] e4m3            k_scale [L]
+ *   idx      [Tq, topk] int32         output (key positions, -1 padded)
+ *   workspace, ws_bytes               at least dsa_index_topk_workspace_size(Tq, H_I, d_I, topk)
+ * Errors: DSA_ERR_INVALID_ARG unless q0 >= 0, Tq >= 1 and q0 + Tq <= L;
+ * otherwise as dsa_index_topk. A serving step of the method (the pages'
+ * prefill and decoding cost figure covers the two extremes, Tq = L and
+ * Tq = 1); the selection rule is unchanged. */
+dsa_status dsa_index_topk_chunk(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
+                                const float* k_scale, int q0, int Tq, int L, int H_I, int d_I, int topk, int32_t* idx,
+                                void* workspace, size_t ws_bytes, void* stream);
+
 /* Test hook: after dsa_index_topk returned with this workspace (and the same
  * L, H_I, d_I, topk), the number of row blocks of 8 tokens whose sampled
  * starting threshold proved too high and that were therefore recomputed with

@@ -52,6 +52,7 @@ def lib() -> ctypes.CDLL:
             L.dsa_index_topk.argtypes = [P, P, P, P, P, I, I, I, I, P, P, SZ, P]
             L.dsa_index_scores.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P]
             L.dsa_index_topk_rerun_count.argtypes = [P, I, I, I, I, ctypes.POINTER(I), P]
+            L.dsa_index_topk_chunk.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P, SZ, P]
             L.dsa_sparse_mla_attn.argtypes = [P, P, P, I, I, I, I, F, P, P, P]
             L.dsa_index_topk_decode_workspace_size.argtypes = [I, I, I]
             L.dsa_index_topk_decode_workspace_size.restype = SZ
@@ -64,7 +65,7 @@ def lib() -> ctypes.CDLL:
             L.dsa_status_string.restype = ctypes.c_char_p
             L.dsa_last_error.argtypes = []
             L.dsa_last_error.restype = ctypes.c_char_p
-            for name in ("dsa_index_topk", "dsa_index_topk_rerun_count", "dsa_index_scores", "dsa_sparse_mla_attn", "dsa_index_topk_decode",
+            for name in ("dsa_index_topk", "dsa_index_topk_rerun_count", "dsa_index_topk_chunk", "dsa_index_scores", "dsa_sparse_mla_attn", "dsa_index_topk_decode",
                          "dsa_index_scores_decode", "dsa_sparse_mla_attn_decode", "dsa_get_device_error",
                          "dsa_index_topk_decode_noalloc"):
                 getattr(L, name).restype = I
@@ -124,6 +125,29 @@ def index_topk(q_I, q_scale, w, k_cache, k_scale, topk: int, *, idx=None, worksp
     _check(lib().dsa_index_topk(_ptr(q_I), _ptr(q_scale), _ptr(w), _ptr(k_cache), _ptr(k_scale), L, H_I, d_I,
                                 topk, _ptr(idx), _ptr(workspace), workspace.numel() * workspace.element_size(),
                                 _stream(q_I.device)))
+    return idx
+
+
+def index_topk_chunk(q_I, q_scale, w, k_cache, k_scale, q0: int, topk: int, *, idx=None, workspace=None):
+    """Chunked prefill: queries q_I [Tq, H_I, d_I] at positions q0..q0+Tq-1 against
+    k_cache [L, d_I] (L >= q0 + Tq); idx [Tq, topk] int32 (ranked key positions, -1 padded)."""
+    q_I, k_cache = _u8(q_I), _u8(k_cache)
+    Tq, H_I, d_I = q_I.shape
+    L = k_cache.shape[0]
+    _req(q_I, "q_I", torch.uint8)
+    _req(q_scale, "q_scale", torch.float32, (Tq,))
+    _req(w, "w", torch.float32, (Tq, H_I))
+    _req(k_cache, "k_cache", torch.uint8, (L, d_I))
+    _req(k_scale, "k_scale", torch.float32, (L,))
+    if idx is None:
+        idx = torch.empty((Tq, topk), dtype=torch.int32, device=q_I.device)
+    _req(idx, "idx", torch.int32, (Tq, topk))
+    need = index_topk_workspace_size(Tq, H_I, d_I, topk)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q_I.device)
+    _check(lib().dsa_index_topk_chunk(_ptr(q_I), _ptr(q_scale), _ptr(w), _ptr(k_cache), _ptr(k_scale), q0, Tq, L,
+                                      H_I, d_I, topk, _ptr(idx), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _stream(q_I.device)))
     return idx
 
 

@@ -134,7 +134,7 @@ dsa_status launch_prefill(const uint8_t* q_I, const uint8_t* k_cache, const IdxP
                           cudaStream_t st) {
   using C = IdxPrefillCfg<HI, DI>;
   CUtensorMap tmQ, tmK;
-  dsa_status s = make_map_u8(&tmQ, q_I, DI, static_cast<uint64_t>(p.L) * HI, DI, C::NCOL);
+  dsa_status s = make_map_u8(&tmQ, q_I, DI, static_cast<uint64_t>(p.Tq) * HI, DI, C::NCOL);
   if (s != DSA_OK) return s;
   s = make_map_u8(&tmK, k_cache, DI, static_cast<uint64_t>(p.L), DI, C::BM);
   if (s != DSA_OK) return s;
@@ -287,28 +287,31 @@ size_t dsa_index_topk_workspace_size(int L, int H_I, int d_I, int topk) {
   return prefill_ws_layout(nullptr, L, H_I, topk, grid).bytes;
 }
 
-dsa_status dsa_index_topk(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
-                          const float* k_scale, int L, int H_I, int d_I, int topk, int32_t* idx, void* workspace,
-                          size_t ws_bytes, void* stream) {
+// Queries r = 0..Tq-1 at positions q0 + r against keys 0..L-1 (q0 + Tq <= L).
+static dsa_status index_topk_impl(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
+                           const float* k_scale, int q0, int Tq, int L, int H_I, int d_I, int topk, int32_t* idx,
+                           void* workspace, size_t ws_bytes, cudaStream_t st) {
   if (!q_I || !q_scale || !w || !k_cache || !k_scale || !idx) return fail(DSA_ERR_INVALID_ARG, "null pointer");
-  if (L <= 0) return fail(DSA_ERR_INVALID_ARG, "L=%d", L);
+  if (L <= 0 || Tq <= 0 || q0 < 0 || static_cast<long long>(q0) + Tq > L)
+    return fail(DSA_ERR_INVALID_ARG, "q0=%d Tq=%d L=%d (need q0 >= 0, Tq >= 1, q0 + Tq <= L)", q0, Tq, L);
   if (!prefill_shape_ok(H_I, d_I)) return fail(DSA_ERR_UNSUPPORTED, "H_I=%d d_I=%d not supported", H_I, d_I);
   if (topk < 1 || topk > DSA_MAX_TOPK) return fail(DSA_ERR_UNSUPPORTED, "topk=%d not in [1, %d]", topk, DSA_MAX_TOPK);
-  if (static_cast<long long>(L) * H_I >= (1ll << 31)) return fail(DSA_ERR_UNSUPPORTED, "L*H_I too large");
+  if (static_cast<long long>(Tq) * H_I >= (1ll << 31)) return fail(DSA_ERR_UNSUPPORTED, "Tq*H_I too large");
   if (!aligned16(q_I) || !aligned16(k_cache)) return fail(DSA_ERR_INVALID_ARG, "q_I / k_cache not 16-byte aligned");
   const int rb = rows_per_block(H_I);
-  const int nrb = (L + rb - 1) / rb;
+  const int nrb = (Tq + rb - 1) / rb;
   const int grid = nrb < num_sms() ? nrb : num_sms();
-  const WsPrefill ws = prefill_ws_layout(workspace, L, H_I, topk, grid);
+  const WsPrefill ws = prefill_ws_layout(workspace, Tq, H_I, topk, grid);
   if (!workspace || ws_bytes < ws.bytes)
     return fail(DSA_ERR_WORKSPACE, "workspace %zu bytes, need %zu", ws_bytes, ws.bytes);
   if (!aligned16(workspace)) return fail(DSA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   IdxPrefillParams p = {};
   p.q_scale = q_scale;
   p.w = w;
   p.k_scale = k_scale;
   p.L = L;
+  p.q0 = q0;
+  p.Tq = Tq;
   p.topk = topk;
   p.rb_begin = 0;
   p.rb_end = nrb;
@@ -321,7 +324,7 @@ dsa_status dsa_index_topk(const uint8_t* q_I, const float* q_scale, const float*
   const cudaError_t me = cudaMemsetAsync(ws.redo, 0, sizeof(int), st);
   if (me != cudaSuccess) return cuda_fail(me, "cudaMemsetAsync");
   dsa_status s = (select_mq(topk) == 1) ? dispatch_prefill<true, 1>(H_I, d_I, q_I, k_cache, p, grid, st)
-                             : dispatch_prefill<true, 4>(H_I, d_I, q_I, k_cache, p, grid, st);
+                                        : dispatch_prefill<true, 4>(H_I, d_I, q_I, k_cache, p, grid, st);
   if (s != DSA_OK) return s;
   // Row blocks whose sampled start proved too high run again with plain
   // streaming; the count is read on the device, so an empty list costs one
@@ -335,7 +338,21 @@ dsa_status dsa_index_topk(const uint8_t* q_I, const float* q_scale, const float*
   s = (select_mq(topk) == 1) ? dispatch_prefill<true, 1>(H_I, d_I, q_I, k_cache, r, grid, st)
                              : dispatch_prefill<true, 4>(H_I, d_I, q_I, k_cache, r, grid, st);
   if (s != DSA_OK) return s;
-  return launch_rank_sort(ws.sel, idx, topk, L, st);
+  return launch_rank_sort(ws.sel, idx, topk, Tq, st);
+}
+
+dsa_status dsa_index_topk(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
+                          const float* k_scale, int L, int H_I, int d_I, int topk, int32_t* idx, void* workspace,
+                          size_t ws_bytes, void* stream) {
+  return index_topk_impl(q_I, q_scale, w, k_cache, k_scale, 0, L, L, H_I, d_I, topk, idx, workspace, ws_bytes,
+                         static_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_index_topk_chunk(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
+                                const float* k_scale, int q0, int Tq, int L, int H_I, int d_I, int topk, int32_t* idx,
+                                void* workspace, size_t ws_bytes, void* stream) {
+  return index_topk_impl(q_I, q_scale, w, k_cache, k_scale, q0, Tq, L, H_I, d_I, topk, idx, workspace, ws_bytes,
+                         static_cast<cudaStream_t>(stream));
 }
 
 dsa_status dsa_index_topk_rerun_count(const void* workspace, int L, int H_I, int d_I, int topk, int* count,
@@ -373,6 +390,8 @@ dsa_status dsa_index_scores(const uint8_t* q_I, const float* q_scale, const floa
   p.w = w;
   p.k_scale = k_scale;
   p.L = L;
+  p.q0 = 0;
+  p.Tq = L;
   p.topk = 1;
   p.rb_begin = row0 / rb;
   p.rb_end = (row0 + nrows + rb - 1) / rb;

@@ -80,9 +80,10 @@ struct IdxPrefillParams {
   const float* q_scale;  // [L]
   const float* w;        // [L, HI]
   const float* k_scale;  // [L]
-  int L;
+  int L;                 // keys in the cache (positions 0..L-1)
+  int q0, Tq;            // query row r sits at position q0 + r, r < Tq (q0 + Tq <= L)
   int topk;
-  int rb_begin, rb_end;  // row blocks [rb_begin, rb_end) of RB tokens
+  int rb_begin, rb_end;  // row blocks [rb_begin, rb_end) of RB query rows
   // selection mode
   uint64_t* cand;        // [gridDim.x][RB][cap] candidate lists
   int cap;
@@ -215,8 +216,9 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
       uint32_t ke_phase = 1;
       for (int j = blockIdx.x; j < nrb; j += G) {
         const int rb = block_of(j);
-        const int t0 = rb * C::RB;
-        const int tlast = min(t0 + C::RB, p.L) - 1;
+        const int r0 = rb * C::RB;
+        const int t0 = p.q0 + r0;
+        const int tlast = p.q0 + min(r0 + C::RB, p.Tq) - 1;
         const int nkt = tlast / C::BM + 1;
         const bool spec = samples(t0, nkt);
         const int nsteps = nkt + (spec ? C::NSAMPLE : 0);
@@ -224,7 +226,7 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
         qe_phase ^= 1;
         mbar_arrive_expect_tx(q_full, C::NACC * C::QBUF_BYTES);
         for (int b = 0; b < C::NACC; ++b)
-          tma_load_2d(q_s + b * C::QBUF_BYTES, &tmQ, q_full, 0, (t0 + b * C::TB) * HI);
+          tma_load_2d(q_s + b * C::QBUF_BYTES, &tmQ, q_full, 0, (r0 + b * C::TB) * HI);
         bool ok = true;
         for (int i = 0; i < nsteps; ++i) {
           if (!mbar_wait(k_empty + kslot, ke_phase, ab, 2)) { ok = false; break; }
@@ -255,8 +257,9 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
       const uint32_t k_base = smem_u32(k_s);
       for (int j = blockIdx.x; j < nrb; j += G) {
         const int rb = block_of(j);
-        const int t0 = rb * C::RB;
-        const int tlast = min(t0 + C::RB, p.L) - 1;
+        const int r0 = rb * C::RB;
+        const int t0 = p.q0 + r0;
+        const int tlast = p.q0 + min(r0 + C::RB, p.Tq) - 1;
         const int nkt = tlast / C::BM + 1;
         const int nsteps = nkt + (samples(t0, nkt) ? C::NSAMPLE : 0);
         if (!mbar_wait_warp(q_full, qf_phase, ab, 5)) break;
@@ -311,19 +314,20 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
 
     for (int j = blockIdx.x; j < nrb; j += G) {
       const int rb = block_of(j);
-      const int t0 = rb * C::RB;
-      const int tlast = min(t0 + C::RB, p.L) - 1;
+      const int r0 = rb * C::RB;
+      const int t0 = p.q0 + r0;  // position of the block's first query row
+      const int tlast = p.q0 + min(r0 + C::RB, p.Tq) - 1;
       const int nkt = tlast / C::BM + 1;
       const bool spec = samples(t0, nkt);
       const int nsteps = nkt + (spec ? C::NSAMPLE : 0);
       // per-row-block state
       for (int i = et; i < C::RB * HI; i += C::NET) {
-        const int t = t0 + i / HI;
-        w_s[i] = (t < p.L) ? p.w[static_cast<size_t>(t) * HI + (i % HI)] : 0.f;
+        const int r = r0 + i / HI;
+        w_s[i] = (r < p.Tq) ? p.w[static_cast<size_t>(r) * HI + (i % HI)] : 0.f;
       }
       for (int i = et; i < C::RB; i += C::NET) {
-        const int t = t0 + i;
-        qs_s[i] = (t < p.L) ? p.q_scale[t] : 0.f;
+        const int r = r0 + i;
+        qs_s[i] = (r < p.Tq) ? p.q_scale[r] : 0.f;
         thr_s[i] = 0ull;
       }
       for (int i = et; i < 4 * C::RB; i += C::NET) cnt_s[i] = 0;
@@ -400,7 +404,7 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
           for (int q = 0; q < C::TOK_PER_WARP; ++q) {
             const int tl = b * C::TB + half * C::TOK_PER_WARP + q;
             const int t = t0 + tl;
-            const bool valid = (t < p.L) && (s <= t);
+            const bool valid = (r0 + tl < p.Tq) && (s <= t);
             if constexpr (kSelect) {
               // a key can only pass if its score reaches the threshold's score
               const uint32_t sk = float_order_key(score[q]);
@@ -440,7 +444,7 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
             named_bar_sync(1, C::NET);
             for (int tl = 0; tl < C::RB; ++tl) {
               const int t = t0 + tl;
-              if (t >= p.L) break;
+              if (r0 + tl >= p.Tq) break;
               const int* cn = cnt_s + tl * 4;
               const int n = cn[0] + cn[1] + cn[2] + cn[3];
               if (n == 0) continue;
@@ -506,7 +510,7 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
         bool redo = false;
         for (int tl = 0; tl < C::RB; ++tl) {
           const int t = t0 + tl;
-          if (t >= p.L) break;
+          if (r0 + tl >= p.Tq) break;
           const int* cn = cnt_s + tl * 4;
           const int n = cn[0] + cn[1] + cn[2] + cn[3];
           // a sampled start above the row's k-th largest score left too few keys
@@ -526,7 +530,7 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
             }
           }
           // write the row's selected keys (unordered) and zero-pad to topk
-          uint64_t* dst = p.sel_keys + static_cast<size_t>(t) * p.topk;
+          uint64_t* dst = p.sel_keys + static_cast<size_t>(r0 + tl) * p.topk;  // row r0 + tl of the output
           int mine = 0;
 #pragma unroll
           for (int i = 0; i < 4 * MQ; ++i) mine += (v[i] != 0 && v[i] >= floor) ? 1 : 0;

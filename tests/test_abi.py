@@ -61,3 +61,12 @@ def test_empty_attention_batch_needs_no_pointers(lib):
     kv = ctypes.c_void_p(256)
     assert lib.dsa_sparse_mla_attn(None, kv, None, 0, 4, 16, 8, ctypes.c_float(0.1), None, None, None) == 0
     assert lib.dsa_sparse_mla_attn(None, None, None, 0, 4, 16, 8, ctypes.c_float(0.1), None, None, None) == -1
+
+
+def test_chunk_entry_rejects_bad_offsets(lib):
+    p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    # q0 + Tq > L
+    assert lib.dsa_index_topk_chunk(p, p, p, p, p, 100, 50, 120, 64, 128, 8, p, p, 1 << 30, None) == -1
+    # Tq = 0, negative q0
+    assert lib.dsa_index_topk_chunk(p, p, p, p, p, 0, 0, 120, 64, 128, 8, p, p, 1 << 30, None) == -1
+    assert lib.dsa_index_topk_chunk(p, p, p, p, p, -1, 8, 120, 64, 128, 8, p, p, 1 << 30, None) == -1
