@@ -100,6 +100,26 @@ dsa_status dsa_index_topk_chunk(const uint8_t* q_I, const float* q_scale, const 
                                 const float* k_scale, int q0, int Tq, int L, int H_I, int d_I, int topk, int32_t* idx,
                                 void* workspace, size_t ws_bytes, void* stream);
 
+/* Packed batch of sequences (cu_seqlens form): sequence b owns query rows
+ * [cu_q[b], cu_q[b+1]) of q_I / q_scale / w and keys [cu_k[b], cu_k[b+1]) of
+ * k_cache / k_scale; its queries sit at positions q_pos0[b] .. q_pos0[b] +
+ * (cu_q[b+1] - cu_q[b]) - 1 of its own cache (q_pos0 NULL: the queries are the
+ * last tokens of each cache). Row i of idx [cu_q[nseq], topk] is the selection
+ * of query row i, as key positions local to its sequence (0 = the sequence's
+ * first key), -1 padded. Each sequence's rows equal what dsa_index_topk_chunk
+ * gives for that sequence alone. cu_q, cu_k, q_pos0 are HOST arrays (the
+ * call builds a longest-first row-block table from them and copies it into
+ * the workspace); everything else is device memory.
+ * Errors: DSA_ERR_INVALID_ARG unless cu_q[0] = cu_k[0] = 0, the offsets do
+ * not decrease, and every sequence has q_pos0 >= 0 and q_pos0 + queries <=
+ * keys; otherwise as dsa_index_topk. Serving layout of the same selection
+ * rule; no counterpart step in the pages. */
+size_t dsa_index_topk_varlen_workspace_size(int total_q, int nseq, int H_I, int d_I, int topk);
+dsa_status dsa_index_topk_varlen(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
+                                 const float* k_scale, const int32_t* cu_q, const int32_t* cu_k,
+                                 const int32_t* q_pos0, int nseq, int H_I, int d_I, int topk, int32_t* idx,
+                                 void* workspace, size_t ws_bytes, void* stream);
+
 /* Test hook: after dsa_index_topk returned with this workspace (and the same
  * L, H_I, d_I, topk), the number of row blocks of 8 tokens whose sampled
  * starting threshold proved too high and that were therefore recomputed with

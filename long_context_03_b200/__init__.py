@@ -53,6 +53,9 @@ def lib() -> ctypes.CDLL:
             L.dsa_index_scores.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P]
             L.dsa_index_topk_rerun_count.argtypes = [P, I, I, I, I, ctypes.POINTER(I), P]
             L.dsa_index_topk_chunk.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P, SZ, P]
+            L.dsa_index_topk_varlen_workspace_size.argtypes = [I, I, I, I, I]
+            L.dsa_index_topk_varlen_workspace_size.restype = SZ
+            L.dsa_index_topk_varlen.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, P, P, SZ, P]
             L.dsa_sparse_mla_attn.argtypes = [P, P, P, I, I, I, I, F, P, P, P]
             L.dsa_index_topk_decode_workspace_size.argtypes = [I, I, I]
             L.dsa_index_topk_decode_workspace_size.restype = SZ
@@ -65,7 +68,8 @@ def lib() -> ctypes.CDLL:
             L.dsa_status_string.restype = ctypes.c_char_p
             L.dsa_last_error.argtypes = []
             L.dsa_last_error.restype = ctypes.c_char_p
-            for name in ("dsa_index_topk", "dsa_index_topk_rerun_count", "dsa_index_topk_chunk", "dsa_index_scores", "dsa_sparse_mla_attn", "dsa_index_topk_decode",
+            for name in ("dsa_index_topk", "dsa_index_topk_rerun_count", "dsa_index_topk_chunk",
+                         "dsa_index_topk_varlen", "dsa_index_scores", "dsa_sparse_mla_attn", "dsa_index_topk_decode",
                          "dsa_index_scores_decode", "dsa_sparse_mla_attn_decode", "dsa_get_device_error",
                          "dsa_index_topk_decode_noalloc"):
                 getattr(L, name).restype = I
@@ -148,6 +152,41 @@ def index_topk_chunk(q_I, q_scale, w, k_cache, k_scale, q0: int, topk: int, *, i
     _check(lib().dsa_index_topk_chunk(_ptr(q_I), _ptr(q_scale), _ptr(w), _ptr(k_cache), _ptr(k_scale), q0, Tq, L,
                                       H_I, d_I, topk, _ptr(idx), _ptr(workspace),
                                       workspace.numel() * workspace.element_size(), _stream(q_I.device)))
+    return idx
+
+
+def index_topk_varlen(q_I, q_scale, w, k_cache, k_scale, cu_q, cu_k, topk: int, *, q_pos0=None, idx=None,
+                      workspace=None):
+    """Packed batch: sequence b owns query rows cu_q[b]:cu_q[b+1] and keys cu_k[b]:cu_k[b+1]
+    (host integer sequences); its queries sit at positions q_pos0[b].. of its cache (default: the
+    last tokens). idx [total_q, topk] int32 of key positions local to each sequence."""
+    q_I, k_cache = _u8(q_I), _u8(k_cache)
+    total_q, H_I, d_I = q_I.shape
+    total_k = k_cache.shape[0]
+    cu_q = [int(x) for x in cu_q]
+    cu_k = [int(x) for x in cu_k]
+    nseq = len(cu_q) - 1
+    if len(cu_k) != nseq + 1 or cu_q[-1] != total_q or cu_k[-1] != total_k:
+        raise ValueError("cu_q / cu_k do not match the packed tensors")
+    _req(q_I, "q_I", torch.uint8)
+    _req(q_scale, "q_scale", torch.float32, (total_q,))
+    _req(w, "w", torch.float32, (total_q, H_I))
+    _req(k_cache, "k_cache", torch.uint8, (total_k, d_I))
+    _req(k_scale, "k_scale", torch.float32, (total_k,))
+    if idx is None:
+        idx = torch.empty((total_q, topk), dtype=torch.int32, device=q_I.device)
+    _req(idx, "idx", torch.int32, (total_q, topk))
+    need = int(lib().dsa_index_topk_varlen_workspace_size(total_q, nseq, H_I, d_I, topk))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q_I.device)
+    IA = ctypes.c_int32 * (nseq + 1)
+    cq, ck = IA(*cu_q), IA(*cu_k)
+    qp = None if q_pos0 is None else (ctypes.c_int32 * nseq)(*[int(x) for x in q_pos0])
+    _check(lib().dsa_index_topk_varlen(_ptr(q_I), _ptr(q_scale), _ptr(w), _ptr(k_cache), _ptr(k_scale),
+                                       ctypes.cast(cq, ctypes.c_void_p), ctypes.cast(ck, ctypes.c_void_p),
+                                       None if qp is None else ctypes.cast(qp, ctypes.c_void_p), nseq, H_I, d_I,
+                                       topk, _ptr(idx), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _stream(q_I.device)))
     return idx
 
 

@@ -6,6 +6,8 @@
 
 #include <cmath>
 #include <cstdarg>
+#include <algorithm>
+#include <vector>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -353,6 +355,137 @@ dsa_status dsa_index_topk_chunk(const uint8_t* q_I, const float* q_scale, const 
                                 void* workspace, size_t ws_bytes, void* stream) {
   return index_topk_impl(q_I, q_scale, w, k_cache, k_scale, q0, Tq, L, H_I, d_I, topk, idx, workspace, ws_bytes,
                          static_cast<cudaStream_t>(stream));
+}
+
+// ---- packed batch of sequences (cu_seqlens) ----
+// Workspace: candidate lists and selected keys as for total_q rows, then the
+// re-run list and the row-block table (upper bound on the block count).
+struct WsVarlen {
+  WsPrefill base;
+  int* redo;
+  int* table;  // blk_seq[nb_max], blk_lrb[nb_max], cuq[nseq+1], cuk[nseq+1], q0[nseq]
+  size_t bytes;
+};
+static int varlen_max_blocks(int total_q, int nseq, int H_I) { return total_q / rows_per_block(H_I) + nseq + 1; }
+static WsVarlen varlen_ws_layout(void* base, int total_q, int nseq, int H_I, int topk, int grid) {
+  WsVarlen w;
+  const size_t cand_bytes = static_cast<size_t>(grid) * rows_per_block(H_I) * select_cap(topk) * 8;
+  const size_t sel_bytes = static_cast<size_t>(total_q) * topk * 8;
+  const int nbm = varlen_max_blocks(total_q, nseq, H_I);
+  const size_t redo_bytes = (static_cast<size_t>(nbm) + 4) * 4;
+  const size_t table_bytes = (2 * static_cast<size_t>(nbm) + 3 * static_cast<size_t>(nseq) + 2) * 4;
+  char* c = reinterpret_cast<char*>(base);
+  w.base.cand = reinterpret_cast<uint64_t*>(c);
+  w.base.sel = reinterpret_cast<uint64_t*>(c + cand_bytes);
+  w.redo = reinterpret_cast<int*>(c + cand_bytes + sel_bytes);
+  w.table = reinterpret_cast<int*>(c + cand_bytes + sel_bytes + redo_bytes);
+  w.bytes = cand_bytes + sel_bytes + redo_bytes + table_bytes;
+  return w;
+}
+
+size_t dsa_index_topk_varlen_workspace_size(int total_q, int nseq, int H_I, int d_I, int topk) {
+  if (total_q <= 0 || nseq <= 0 || topk <= 0 || !prefill_shape_ok(H_I, d_I)) return 0;
+  const int nbm = varlen_max_blocks(total_q, nseq, H_I);
+  const int grid = nbm < num_sms() ? nbm : num_sms();
+  return varlen_ws_layout(nullptr, total_q, nseq, H_I, topk, grid).bytes;
+}
+
+dsa_status dsa_index_topk_varlen(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
+                                 const float* k_scale, const int32_t* cu_q, const int32_t* cu_k,
+                                 const int32_t* q_pos0, int nseq, int H_I, int d_I, int topk, int32_t* idx,
+                                 void* workspace, size_t ws_bytes, void* stream) {
+  if (!q_I || !q_scale || !w || !k_cache || !k_scale || !idx || !cu_q || !cu_k)
+    return fail(DSA_ERR_INVALID_ARG, "null pointer");
+  if (nseq <= 0) return fail(DSA_ERR_INVALID_ARG, "nseq=%d", nseq);
+  if (!prefill_shape_ok(H_I, d_I)) return fail(DSA_ERR_UNSUPPORTED, "H_I=%d d_I=%d not supported", H_I, d_I);
+  if (topk < 1 || topk > DSA_MAX_TOPK) return fail(DSA_ERR_UNSUPPORTED, "topk=%d not in [1, %d]", topk, DSA_MAX_TOPK);
+  if (cu_q[0] != 0 || cu_k[0] != 0) return fail(DSA_ERR_INVALID_ARG, "cu_q[0] and cu_k[0] must be 0");
+  const int RB = rows_per_block(H_I);
+  std::vector<int> q0(nseq);
+  std::vector<long long> order;  // (-(last position) << 32 | block): longest first
+  for (int b = 0; b < nseq; ++b) {
+    const int tq = cu_q[b + 1] - cu_q[b], lk = cu_k[b + 1] - cu_k[b];
+    q0[b] = q_pos0 ? q_pos0[b] : lk - tq;
+    if (tq < 0 || lk < 0 || q0[b] < 0 || static_cast<long long>(q0[b]) + tq > lk)
+      return fail(DSA_ERR_INVALID_ARG, "sequence %d: %d queries at position %d, %d keys", b, tq, q0[b], lk);
+  }
+  const int total_q = cu_q[nseq], total_k = cu_k[nseq];
+  if (total_q <= 0 || total_k <= 0) return fail(DSA_ERR_INVALID_ARG, "total_q=%d total_k=%d", total_q, total_k);
+  if (static_cast<long long>(total_q) * H_I >= (1ll << 31)) return fail(DSA_ERR_UNSUPPORTED, "total_q*H_I too large");
+  if (!aligned16(q_I) || !aligned16(k_cache)) return fail(DSA_ERR_INVALID_ARG, "q_I / k_cache not 16-byte aligned");
+  std::vector<int> bseq, blrb;
+  {
+    std::vector<std::pair<long long, int>> keyed;  // (last position, block) to sort longest first
+    std::vector<std::pair<int, int>> blocks;
+    for (int b = 0; b < nseq; ++b) {
+      const int tq = cu_q[b + 1] - cu_q[b];
+      for (int l = 0; l * RB < tq; ++l) {
+        keyed.push_back({static_cast<long long>(q0[b]) + std::min((l + 1) * RB, tq), static_cast<int>(blocks.size())});
+        blocks.push_back({b, l});
+      }
+    }
+    std::stable_sort(keyed.begin(), keyed.end(), [](const auto& a, const auto& c) { return a.first > c.first; });
+    for (const auto& k : keyed) {
+      bseq.push_back(blocks[k.second].first);
+      blrb.push_back(blocks[k.second].second);
+    }
+  }
+  const int nblk = static_cast<int>(bseq.size());
+  const int nbm = varlen_max_blocks(total_q, nseq, H_I);
+  const int grid = nbm < num_sms() ? nbm : num_sms();
+  const WsVarlen ws = varlen_ws_layout(workspace, total_q, nseq, H_I, topk, grid);
+  if (!workspace || ws_bytes < ws.bytes)
+    return fail(DSA_ERR_WORKSPACE, "workspace %zu bytes, need %zu", ws_bytes, ws.bytes);
+  if (!aligned16(workspace)) return fail(DSA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+  // the table to the device (staged from this host buffer before the call returns)
+  std::vector<int> host(2 * static_cast<size_t>(nbm) + 3 * static_cast<size_t>(nseq) + 2, 0);
+  std::copy(bseq.begin(), bseq.end(), host.begin());
+  std::copy(blrb.begin(), blrb.end(), host.begin() + nbm);
+  for (int b = 0; b <= nseq; ++b) {
+    host[2 * nbm + b] = cu_q[b];
+    host[2 * nbm + nseq + 1 + b] = cu_k[b];
+  }
+  for (int b = 0; b < nseq; ++b) host[2 * nbm + 2 * (nseq + 1) + b] = q0[b];
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(ws.table, host.data(), host.size() * 4, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync(row-block table)");
+  e = cudaMemsetAsync(ws.redo, 0, sizeof(int), st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  IdxPrefillParams p = {};
+  p.q_scale = q_scale;
+  p.w = w;
+  p.k_scale = k_scale;
+  p.L = total_k;
+  p.q0 = 0;
+  p.Tq = total_q;
+  p.topk = topk;
+  p.rb_begin = 0;
+  p.rb_end = nblk;
+  p.cand = ws.base.cand;
+  p.cap = select_cap(topk);
+  p.sel_keys = ws.base.sel;
+  p.spec_min_t = spec_min_row(topk);
+  p.redo_count = ws.redo;
+  p.redo_list = ws.redo + 4;
+  p.blk_seq = ws.table;
+  p.blk_lrb = ws.table + nbm;
+  p.seq_cuq = ws.table + 2 * nbm;
+  p.seq_cuk = ws.table + 2 * nbm + nseq + 1;
+  p.seq_q0 = ws.table + 2 * nbm + 2 * (nseq + 1);
+  const int g = nblk < grid ? nblk : grid;
+  dsa_status s = (select_mq(topk) == 1) ? dispatch_prefill<true, 1>(H_I, d_I, q_I, k_cache, p, g, st)
+                                        : dispatch_prefill<true, 4>(H_I, d_I, q_I, k_cache, p, g, st);
+  if (s != DSA_OK) return s;
+  IdxPrefillParams r = p;
+  r.spec_min_t = 0;
+  r.rb_list = ws.redo + 4;
+  r.list_count = ws.redo;
+  r.redo_count = nullptr;
+  r.redo_list = nullptr;
+  s = (select_mq(topk) == 1) ? dispatch_prefill<true, 1>(H_I, d_I, q_I, k_cache, r, g, st)
+                             : dispatch_prefill<true, 4>(H_I, d_I, q_I, k_cache, r, g, st);
+  if (s != DSA_OK) return s;
+  return launch_rank_sort(ws.base.sel, idx, topk, total_q, st);
 }
 
 dsa_status dsa_index_topk_rerun_count(const void* workspace, int L, int H_I, int d_I, int topk, int* count,

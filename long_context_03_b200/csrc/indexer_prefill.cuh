@@ -100,6 +100,15 @@ struct IdxPrefillParams {
   // (plain streaming, no sampling) instead of [rb_begin, rb_end).
   const int* rb_list;
   const int* list_count;
+  // Packed batch: when blk_seq is set, row block id covers local block
+  // blk_lrb[id] of sequence blk_seq[id]; sequence b owns query rows
+  // [seq_cuq[b], seq_cuq[b+1]) at positions from seq_q0[b] and keys
+  // [seq_cuk[b], seq_cuk[b+1]) (local positions 0..). Ids are in longest-first order.
+  const int* blk_seq;
+  const int* blk_lrb;
+  const int* seq_cuq;
+  const int* seq_cuk;
+  const int* seq_q0;
   // score mode (test hook)
   float* scores;         // [nrows][L]; rows t in [row0, row0 + nrows)
   int row0, nrows;
@@ -203,7 +212,30 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
   const int nrb = list_mode ? *p.list_count : (p.rb_end - p.rb_begin);
   const int G = gridDim.x;
   // row block of step j and whether it samples first (the same on every role)
-  auto block_of = [&](int j) { return list_mode ? p.rb_list[j] : p.rb_end - 1 - j; };
+  auto block_of = [&](int j) { return list_mode ? p.rb_list[j] : (p.blk_seq ? j : p.rb_end - 1 - j); };
+  // where row block `id` lives: first query row, end of its sequence's rows,
+  // position of its first row, its sequence's key count and first key row
+  struct Blk {
+    int r0, rend, t0, L, kbase;
+  };
+  auto blk = [&](int id) {
+    Blk k;
+    if (p.blk_seq) {
+      const int sq = p.blk_seq[id], lrb = p.blk_lrb[id];
+      k.r0 = p.seq_cuq[sq] + lrb * C::RB;
+      k.rend = p.seq_cuq[sq + 1];
+      k.t0 = p.seq_q0[sq] + lrb * C::RB;
+      k.kbase = p.seq_cuk[sq];
+      k.L = p.seq_cuk[sq + 1] - k.kbase;
+    } else {
+      k.r0 = id * C::RB;
+      k.rend = p.Tq;
+      k.t0 = p.q0 + k.r0;
+      k.kbase = 0;
+      k.L = p.L;
+    }
+    return k;
+  };
   auto samples = [&](int t0, int nkt) {
     return kSelect && !list_mode && p.spec_min_t > 0 && t0 >= p.spec_min_t && nkt >= 4 * C::NSAMPLE;
   };
@@ -215,10 +247,10 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
       int kslot = 0;
       uint32_t ke_phase = 1;
       for (int j = blockIdx.x; j < nrb; j += G) {
-        const int rb = block_of(j);
-        const int r0 = rb * C::RB;
-        const int t0 = p.q0 + r0;
-        const int tlast = p.q0 + min(r0 + C::RB, p.Tq) - 1;
+        const Blk bk = blk(block_of(j));
+        const int r0 = bk.r0;
+        const int t0 = bk.t0;
+        const int tlast = t0 + min(C::RB, bk.rend - r0) - 1;
         const int nkt = tlast / C::BM + 1;
         const bool spec = samples(t0, nkt);
         const int nsteps = nkt + (spec ? C::NSAMPLE : 0);
@@ -231,7 +263,8 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
         for (int i = 0; i < nsteps; ++i) {
           if (!mbar_wait(k_empty + kslot, ke_phase, ab, 2)) { ok = false; break; }
           mbar_arrive_expect_tx(k_full + kslot, C::KTILE_BYTES);
-          tma_load_2d(k_s + kslot * C::KTILE_BYTES, &tmK, k_full + kslot, 0, tile_at<C::NSAMPLE>(i, nkt, spec) * C::BM);
+          tma_load_2d(k_s + kslot * C::KTILE_BYTES, &tmK, k_full + kslot, 0,
+                      bk.kbase + tile_at<C::NSAMPLE>(i, nkt, spec) * C::BM);
           if (++kslot == C::KST) { kslot = 0; ke_phase ^= 1; }
         }
         if (!ok) break;
@@ -256,10 +289,9 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
       const uint32_t q_base = smem_u32(q_s);
       const uint32_t k_base = smem_u32(k_s);
       for (int j = blockIdx.x; j < nrb; j += G) {
-        const int rb = block_of(j);
-        const int r0 = rb * C::RB;
-        const int t0 = p.q0 + r0;
-        const int tlast = p.q0 + min(r0 + C::RB, p.Tq) - 1;
+        const Blk bk = blk(block_of(j));
+        const int t0 = bk.t0;
+        const int tlast = t0 + min(C::RB, bk.rend - bk.r0) - 1;
         const int nkt = tlast / C::BM + 1;
         const int nsteps = nkt + (samples(t0, nkt) ? C::NSAMPLE : 0);
         if (!mbar_wait_warp(q_full, qf_phase, ab, 5)) break;
@@ -314,20 +346,21 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
 
     for (int j = blockIdx.x; j < nrb; j += G) {
       const int rb = block_of(j);
-      const int r0 = rb * C::RB;
-      const int t0 = p.q0 + r0;  // position of the block's first query row
-      const int tlast = p.q0 + min(r0 + C::RB, p.Tq) - 1;
+      const Blk bk = blk(rb);
+      const int r0 = bk.r0;
+      const int t0 = bk.t0;  // position of the block's first query row
+      const int tlast = t0 + min(C::RB, bk.rend - r0) - 1;
       const int nkt = tlast / C::BM + 1;
       const bool spec = samples(t0, nkt);
       const int nsteps = nkt + (spec ? C::NSAMPLE : 0);
       // per-row-block state
       for (int i = et; i < C::RB * HI; i += C::NET) {
         const int r = r0 + i / HI;
-        w_s[i] = (r < p.Tq) ? p.w[static_cast<size_t>(r) * HI + (i % HI)] : 0.f;
+        w_s[i] = (r < bk.rend) ? p.w[static_cast<size_t>(r) * HI + (i % HI)] : 0.f;
       }
       for (int i = et; i < C::RB; i += C::NET) {
         const int r = r0 + i;
-        qs_s[i] = (r < p.Tq) ? p.q_scale[r] : 0.f;
+        qs_s[i] = (r < bk.rend) ? p.q_scale[r] : 0.f;
         thr_s[i] = 0ull;
       }
       for (int i = et; i < 4 * C::RB; i += C::NET) cnt_s[i] = 0;
@@ -337,7 +370,7 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
       float ks_next = 0.f;
       {
         const int s0 = tile_at<C::NSAMPLE>(0, nkt, spec) * C::BM + quarter * 32 + static_cast<int>(lane);
-        ks_next = (s0 < p.L) ? __ldg(p.k_scale + s0) : 0.f;
+        ks_next = (s0 < bk.L) ? __ldg(p.k_scale + bk.kbase + s0) : 0.f;
       }
       for (int i = 0; i < nsteps && ok; ++i) {
         const int kt = tile_at<C::NSAMPLE>(i, nkt, spec);
@@ -345,7 +378,7 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
         const float ks = ks_next;
         if (i + 1 < nsteps) {
           const int sn = tile_at<C::NSAMPLE>(i + 1, nkt, spec) * C::BM + quarter * 32 + static_cast<int>(lane);
-          ks_next = (sn < p.L) ? __ldg(p.k_scale + sn) : 0.f;
+          ks_next = (sn < bk.L) ? __ldg(p.k_scale + bk.kbase + sn) : 0.f;
         }
         for (int b = 0; b < C::NACC; ++b) {
           if (!mbar_wait(acc_full + b, af_phase[b], ab, 8)) { ok = false; break; }
@@ -404,7 +437,7 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
           for (int q = 0; q < C::TOK_PER_WARP; ++q) {
             const int tl = b * C::TB + half * C::TOK_PER_WARP + q;
             const int t = t0 + tl;
-            const bool valid = (r0 + tl < p.Tq) && (s <= t);
+            const bool valid = (r0 + tl < bk.rend) && (s <= t);
             if constexpr (kSelect) {
               // a key can only pass if its score reaches the threshold's score
               const uint32_t sk = float_order_key(score[q]);
@@ -444,7 +477,7 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
             named_bar_sync(1, C::NET);
             for (int tl = 0; tl < C::RB; ++tl) {
               const int t = t0 + tl;
-              if (r0 + tl >= p.Tq) break;
+              if (r0 + tl >= bk.rend) break;
               const int* cn = cnt_s + tl * 4;
               const int n = cn[0] + cn[1] + cn[2] + cn[3];
               if (n == 0) continue;
@@ -510,7 +543,7 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
         bool redo = false;
         for (int tl = 0; tl < C::RB; ++tl) {
           const int t = t0 + tl;
-          if (r0 + tl >= p.Tq) break;
+          if (r0 + tl >= bk.rend) break;
           const int* cn = cnt_s + tl * 4;
           const int n = cn[0] + cn[1] + cn[2] + cn[3];
           // a sampled start above the row's k-th largest score left too few keys

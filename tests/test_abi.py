@@ -70,3 +70,17 @@ def test_chunk_entry_rejects_bad_offsets(lib):
     # Tq = 0, negative q0
     assert lib.dsa_index_topk_chunk(p, p, p, p, p, 0, 0, 120, 64, 128, 8, p, p, 1 << 30, None) == -1
     assert lib.dsa_index_topk_chunk(p, p, p, p, p, -1, 8, 120, 64, 128, 8, p, p, 1 << 30, None) == -1
+
+
+def test_varlen_entry_validates_offsets_on_the_host(lib):
+    p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    IA = ctypes.c_int32 * 3
+    bad_first = IA(1, 5, 9)
+    ok_q, ok_k = IA(0, 4, 8), IA(0, 10, 20)
+    too_many_q = IA(0, 12, 16)  # 12 queries against 10 keys
+    call = lambda cq, ck: lib.dsa_index_topk_varlen(p, p, p, p, p, ctypes.cast(cq, ctypes.c_void_p),
+                                                    ctypes.cast(ck, ctypes.c_void_p), None, 2, 64, 128, 8, p, p,
+                                                    1 << 40, None)
+    assert call(bad_first, ok_k) == -1
+    assert call(too_many_q, ok_k) == -1
+    assert lib.dsa_index_topk_varlen_workspace_size(8, 2, 64, 128, 8) > 0
