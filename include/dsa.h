@@ -157,6 +157,18 @@ dsa_status dsa_index_scores(const uint8_t* q_I, const float* q_scale, const floa
  *   scale    softmax scale, finite and > 0 (1/sqrt(576) for the latent row)
  * No workspace.
  * ------------------------------------------------------------------------ */
+/* Short-sequence dense fallback: when a sequence has at most DSA_MAX_TOPK
+ * tokens every causal key is selected anyway, so the indexer can be skipped
+ * and token t (position q0 + t) attends to kv rows 0..q0+t directly, with the
+ * same arithmetic as dsa_sparse_mla_attn over the selection {0..q0+t}
+ * (causal MQA over the latent rows: the short-input mode of
+ * "DeepSeek-V3.2-Exp解析" section 一.1, where the selection covers
+ * everything). q [T, Hq, 576], kv [L, 576] (L <= DSA_MAX_TOPK, q0 + T <= L),
+ * out [T, Hq, 512], lse [T, Hq] or NULL. Errors: DSA_ERR_UNSUPPORTED for
+ * L > DSA_MAX_TOPK, otherwise as dsa_sparse_mla_attn. */
+dsa_status dsa_dense_mla_attn_causal(const uint16_t* q, const uint16_t* kv, int T, int L, int q0, int Hq, float scale,
+                                     uint16_t* out, float* lse, void* stream);
+
 dsa_status dsa_sparse_mla_attn(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int T, int L, int Hq,
                                int topk, float scale, uint16_t* out, float* lse, void* stream);
 

@@ -57,6 +57,7 @@ def lib() -> ctypes.CDLL:
             L.dsa_index_topk_varlen_workspace_size.restype = SZ
             L.dsa_index_topk_varlen.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, P, P, SZ, P]
             L.dsa_sparse_mla_attn.argtypes = [P, P, P, I, I, I, I, F, P, P, P]
+            L.dsa_dense_mla_attn_causal.argtypes = [P, P, I, I, I, I, F, P, P, P]
             L.dsa_index_topk_decode_workspace_size.argtypes = [I, I, I]
             L.dsa_index_topk_decode_workspace_size.restype = SZ
             L.dsa_index_topk_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P, P, SZ, P]
@@ -69,7 +70,7 @@ def lib() -> ctypes.CDLL:
             L.dsa_last_error.argtypes = []
             L.dsa_last_error.restype = ctypes.c_char_p
             for name in ("dsa_index_topk", "dsa_index_topk_rerun_count", "dsa_index_topk_chunk",
-                         "dsa_index_topk_varlen", "dsa_index_scores", "dsa_sparse_mla_attn", "dsa_index_topk_decode",
+                         "dsa_index_topk_varlen", "dsa_dense_mla_attn_causal", "dsa_index_scores", "dsa_sparse_mla_attn", "dsa_index_topk_decode",
                          "dsa_index_scores_decode", "dsa_sparse_mla_attn_decode", "dsa_get_device_error",
                          "dsa_index_topk_decode_noalloc"):
                 getattr(L, name).restype = I
@@ -237,6 +238,25 @@ def sparse_mla_attn(q, kv, idx, scale: float, *, out=None, lse=None, want_lse: b
         _req(lse, "lse", torch.float32, (T, Hq))
     _check(lib().dsa_sparse_mla_attn(_ptr(q), _ptr(kv), _ptr(idx), T, L, Hq, topk, float(scale), _ptr(out),
                                      _ptr(lse), _stream(q.device)))
+    return out, lse
+
+
+def dense_mla_attn_causal(q, kv, scale: float, *, q0: int = 0, out=None, lse=None, want_lse: bool = False):
+    """Short sequences (L <= 2048): token t at position q0 + t attends to kv rows 0..q0+t, no indexer.
+    q [T, Hq, 576], kv [L, 576] -> out [T, Hq, 512] bf16 (and lse [T, Hq] f32)."""
+    T, Hq, D = q.shape
+    L = kv.shape[0]
+    _req(q, "q", torch.bfloat16, (T, Hq, D_QK))
+    _req(kv, "kv", torch.bfloat16, (L, D_QK))
+    if out is None:
+        out = torch.empty((T, Hq, D_V), dtype=torch.bfloat16, device=q.device)
+    _req(out, "out", torch.bfloat16, (T, Hq, D_V))
+    if lse is None and want_lse:
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _req(lse, "lse", torch.float32, (T, Hq))
+    _check(lib().dsa_dense_mla_attn_causal(_ptr(q), _ptr(kv), T, L, q0, Hq, float(scale), _ptr(out), _ptr(lse),
+                                           _stream(q.device)))
     return out, lse
 
 

@@ -233,7 +233,7 @@ dsa_status check_decode_args(const uint8_t* q_I, const float* q_scale, const flo
 
 // ---- attention ----
 dsa_status launch_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int T, int rows, long long kv_stride,
-                      int Hq, int topk, float scale, uint16_t* out, float* lse, cudaStream_t st) {
+                      int Hq, int topk, float scale, uint16_t* out, float* lse, cudaStream_t st, int causal_q0 = 0) {
   MlaParams p;
   p.q = reinterpret_cast<const __nv_bfloat16*>(q);
   p.kv = reinterpret_cast<const __nv_bfloat16*>(kv);
@@ -245,6 +245,7 @@ dsa_status launch_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
   p.T = T;
   p.Hq = Hq;
   p.K = topk;
+  p.causal_q0 = causal_q0;
   p.scale_log2 = scale * 1.4426950408889634f;
   dsa_status s = set_smem(sparse_mla_kernel, MlaCfg::SMEM_BYTES);
   if (s != DSA_OK) return s;
@@ -534,6 +535,21 @@ dsa_status dsa_index_scores(const uint8_t* q_I, const float* q_scale, const floa
   const int nrb = p.rb_end - p.rb_begin;
   const int grid = nrb < num_sms() ? nrb : num_sms();
   return dispatch_prefill<false, 1>(H_I, d_I, q_I, k_cache, p, grid, st);
+}
+
+dsa_status dsa_dense_mla_attn_causal(const uint16_t* q, const uint16_t* kv, int T, int L, int q0, int Hq, float scale,
+                                     uint16_t* out, float* lse, void* stream) {
+  if (T < 0 || L <= 0 || q0 < 0 || static_cast<long long>(q0) + T > L)
+    return fail(DSA_ERR_INVALID_ARG, "T=%d L=%d q0=%d (need q0 + T <= L)", T, L, q0);
+  if (L > DSA_MAX_TOPK)
+    return fail(DSA_ERR_UNSUPPORTED, "dense causal attention covers L <= %d (longer sequences take the selection)",
+                DSA_MAX_TOPK);
+  if (!kv || (T > 0 && (!q || !out))) return fail(DSA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(kv) || !aligned16(out)) return fail(DSA_ERR_INVALID_ARG, "q / kv / out not 16-byte aligned");
+  if (Hq < 1 || Hq > 128) return fail(DSA_ERR_UNSUPPORTED, "Hq=%d not in [1, 128]", Hq);
+  if (!std::isfinite(scale) || !(scale > 0.f)) return fail(DSA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (T == 0) return DSA_OK;
+  return launch_mla(q, kv, nullptr, T, L, 0, Hq, L, scale, out, lse, static_cast<cudaStream_t>(stream), q0);
 }
 
 dsa_status dsa_sparse_mla_attn(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int T, int L, int Hq,

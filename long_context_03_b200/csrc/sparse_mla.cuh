@@ -108,12 +108,13 @@ struct MlaCfg {
 struct MlaParams {
   const __nv_bfloat16* q;    // [T, Hq, 576]
   const __nv_bfloat16* kv;   // latent rows; token i reads kv + i*kv_token_stride
-  const int32_t* idx;        // [T, K]
+  const int32_t* idx;        // [T, K], or null: dense causal, token i takes rows 0..causal_q0 + i
   __nv_bfloat16* out;        // [T, Hq, 512]
   float* lse;                // [T, Hq] or null
   long long kv_token_stride; // elements between consecutive tokens' caches (0: one shared cache)
   int rows;                  // valid row bound of a token's cache
   int T, Hq, K;
+  int causal_q0;             // position of token 0 when idx is null
   float scale_log2;          // softmax scale * log2(e)
 };
 
@@ -227,11 +228,14 @@ __device__ __forceinline__ void gather_value_tile(uint32_t tile, const __nv_bflo
 }
 
 // The producer warps copy a token's index row into shared memory once
-// (named barrier 1 among the 128 producer threads on both sides).
-__device__ __forceinline__ void stage_index_row(int32_t* idx_s, const int32_t* __restrict__ idx_tok, int K,
-                                                int ptid) {
+// (named barrier 1 among the 128 producer threads on both sides). Without
+// an index row (dense causal mode) entry e is row e for e <= pos, else absent.
+__device__ __forceinline__ void stage_index_row(int32_t* idx_s, const int32_t* __restrict__ idx_tok, int K, int ptid,
+                                                int pos) {
   named_bar_sync(1, MlaCfg::NPROD * 32);  // everyone is done with the previous row
-  if ((K & 3) == 0 && (reinterpret_cast<uintptr_t>(idx_tok) & 15) == 0) {
+  if (idx_tok == nullptr) {
+    for (int i = ptid; i < K; i += MlaCfg::NPROD * 32) idx_s[i] = (i <= pos) ? i : -1;
+  } else if ((K & 3) == 0 && (reinterpret_cast<uintptr_t>(idx_tok) & 15) == 0) {
     const int4* src = reinterpret_cast<const int4*>(idx_tok);
     int4* dst = reinterpret_cast<int4*>(idx_s);
     for (int i = ptid; i < K / 4; i += MlaCfg::NPROD * 32) dst[i] = __ldg(src + i);
@@ -315,7 +319,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
         // the softmax warps are done with this mask buffer (two tokens back)
         const int mb = n & 1;
         if (!mbar_wait(bars + C::B_MASK_FREE + mb, ((n >> 1) & 1) ^ 1, ab, 30)) break;
-        stage_index_row(idx_s, p.idx + static_cast<size_t>(tk) * p.K, p.K, ptid);
+        stage_index_row(idx_s, p.idx ? p.idx + static_cast<size_t>(tk) * p.K : nullptr, p.K, ptid, p.causal_q0 + tk);
         // validity bits of every selection entry, 32 per word (entry e -> word e/32)
         for (int wd = static_cast<int>(warp); wd < nchunk * (C::NK / 32); wd += C::NPROD) {
           const int e = wd * 32 + static_cast<int>(lane);
@@ -551,7 +555,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       uint32_t ph = 1;
       for (int tk = cluster_id; tk < p.T; tk += nclusters) {
         const __nv_bfloat16* kv_tok = p.kv + tk * p.kv_token_stride;
-        stage_index_row(idx_s, p.idx + static_cast<size_t>(tk) * p.K, p.K, ptid);
+        stage_index_row(idx_s, p.idx ? p.idx + static_cast<size_t>(tk) * p.K : nullptr, p.K, ptid, p.causal_q0 + tk);
         bool ok = true;
         for (int j = 0; j < nchunk && ok; ++j) {
           for (int u = 0; u < C::NK / C::VROWS; ++u) {

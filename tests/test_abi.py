@@ -84,3 +84,11 @@ def test_varlen_entry_validates_offsets_on_the_host(lib):
     assert call(bad_first, ok_k) == -1
     assert call(too_many_q, ok_k) == -1
     assert lib.dsa_index_topk_varlen_workspace_size(8, 2, 64, 128, 8) > 0
+
+
+def test_dense_fallback_limits(lib):
+    p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    f = ctypes.c_float(0.1)
+    assert lib.dsa_dense_mla_attn_causal(p, p, 4, 4096, 0, 16, f, p, None, None) == -2  # L > 2048
+    assert lib.dsa_dense_mla_attn_causal(p, p, 10, 100, 95, 16, f, p, None, None) == -1  # q0 + T > L
+    assert lib.dsa_dense_mla_attn_causal(None, p, 0, 100, 0, 16, f, None, None, None) == 0  # empty batch
