@@ -54,6 +54,10 @@ def _load():
             lib.oracle_topk.restype = None
             lib.oracle_sparse_mla.argtypes = [P, P, P, i32, i64, i32, i32, i32, f64, P, P]
             lib.oracle_sparse_mla.restype = None
+            lib.oracle_double_to_e4m3.argtypes = [f64]
+            lib.oracle_double_to_e4m3.restype = ctypes.c_uint8
+            lib.oracle_quantize_e4m3.argtypes = [P, i64, i64, P, P]
+            lib.oracle_quantize_e4m3.restype = None
             lib.oracle_num_threads.argtypes = []
             lib.oracle_num_threads.restype = i32
             _lib = lib
@@ -102,6 +106,21 @@ def bf16_to_f64(bits) -> np.ndarray:
         b = b.view(np.uint16)
     lut = np.array([lib.oracle_bf16_to_double(c) for c in range(65536)], dtype=np.float64)
     return lut[b]
+
+
+def double_to_e4m3(x: float) -> int:
+    """E4M3 code of x: nearest representable value, ties to even, saturating to +-448."""
+    return int(_load().oracle_double_to_e4m3(float(x)))
+
+
+def quantize_e4m3(x) -> tuple:
+    """Per-row quantiser: x [n, d] fp32 -> (codes uint8 [n, d], scale fp32 [n]), scale = absmax/448."""
+    xf = np.ascontiguousarray(_np(x, np.float32))
+    n, d = xf.shape
+    codes = np.empty((n, d), dtype=np.uint8)
+    scale = np.empty(n, dtype=np.float32)
+    _load().oracle_quantize_e4m3(_ptr(xf), n, d, _ptr(codes), _ptr(scale))
+    return codes, scale
 
 
 def index_scores(q_I, q_scale, w, k_cache, k_scale, rows, *, query_rows=None) -> np.ndarray:

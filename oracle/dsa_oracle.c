@@ -27,6 +27,11 @@
  *
  * The causal bound is s <= t (a token scores itself), and rows with fewer than
  * k candidates select all of them.
+ *
+ * For quantising newly appended tokens on the device ("Lightning Indexer 的计算
+ * 过程", step 2 <2>, FP8 量化): per row, scale = absmax/448 in fp32 (1 for an
+ * all-zero row) and codes = E4M3(x/scale) by round-to-nearest-even with
+ * saturation to +-448 (oracle_double_to_e4m3, oracle_quantize_e4m3).
  */
 #include <math.h>
 #include <stdint.h>
@@ -64,6 +69,63 @@ double oracle_bf16_to_double(uint16_t b) {
  *   rows    [nrows] causal position t of each query (each < S)
  *   out     [nrows, S] f64: I[t,s] for s <= t, -INFINITY for s > t.
  */
+/* E4M3 encoding of a finite value by the plain definition: round to the
+ * nearest representable value, ties to the even code, saturating to +-448.
+ * The representable magnitudes are m * 2^-9 (m = 0..7, subnormal) and
+ * (1 + m/8) * 2^e (e = -6..8, m = 0..7, at most 448 = 1.75 * 2^8). NaN maps to
+ * the NaN code 0x7F (sign kept). */
+uint8_t oracle_double_to_e4m3(double x) {
+    uint8_t sign = (x < 0.0 || (x == 0.0 && signbit(x))) ? 0x80 : 0x00;
+    if (isnan(x)) return (uint8_t)(sign | 0x7F);
+    double a = fabs(x);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+    /* candidates on the grid of the binade of a (or the subnormal grid) */
+    double step;
+    if (a < ldexp(1.0, -6)) {
+        step = ldexp(1.0, -9);
+    } else {
+        int e;
+        frexp(a, &e); /* a = f * 2^e, f in [0.5, 1): binade [2^(e-1), 2^e) */
+        step = ldexp(1.0, e - 1 - 3);
+    }
+    double q = a / step; /* exact: step is a power of two */
+    double lo = floor(q);
+    double frac = q - lo;
+    double n = lo;
+    if (frac > 0.5 || (frac == 0.5 && fmod(lo, 2.0) != 0.0)) n = lo + 1.0;
+    double v = n * step; /* the rounded magnitude (may be the next binade's first value) */
+    if (v > 448.0) v = 448.0;
+    /* encode v exactly */
+    if (v < ldexp(1.0, -6)) return (uint8_t)(sign | (uint8_t)(v / ldexp(1.0, -9)));
+    int e;
+    double f = frexp(v, &e); /* v = f * 2^e, f in [0.5, 1) */
+    int m = (int)((f * 2.0 - 1.0) * 8.0);
+    int ef = e - 1 + 7;
+    return (uint8_t)(sign | (uint8_t)(ef << 3) | (uint8_t)m);
+}
+
+/* Per-row FP8 quantiser for newly appended keys / queries: scale = absmax/448
+ * (1 for an all-zero row) in fp32, codes = e4m3(fp32(x / scale)) clamped to
+ * +-448. The division is the float32 one the quantised caches are defined
+ * with; the encoding is oracle_double_to_e4m3. */
+void oracle_quantize_e4m3(const float *x, int64_t n, int64_t d, uint8_t *codes, float *scale) {
+    for (int64_t r = 0; r < n; ++r) {
+        float amax = 0.0f;
+        for (int64_t i = 0; i < d; ++i) {
+            float v = fabsf(x[r * d + i]);
+            if (v > amax) amax = v;
+        }
+        float sc = (amax > 0.0f) ? amax / 448.0f : 1.0f;
+        scale[r] = sc;
+        for (int64_t i = 0; i < d; ++i) {
+            float y = x[r * d + i] / sc;
+            if (y > 448.0f) y = 448.0f;
+            if (y < -448.0f) y = -448.0f;
+            codes[r * d + i] = oracle_double_to_e4m3((double)y);
+        }
+    }
+}
+
 void oracle_index_scores(const uint8_t *q8, const float *q_scale, const float *w,
                          const uint8_t *k8, const float *k_scale, int64_t S, int H, int D,
                          const int64_t *rows, int64_t nrows, double *out) {

@@ -255,3 +255,46 @@ def test_decode_matches_last_prefill_row():
     sc2 = oracle.index_scores(q8, qs, w, dec.k_cache[b], dec.k_scale[b], [699])
     assert np.array_equal(sc, sc2[0])
     assert np.array_equal(ix, oracle.topk(sc2, [699], 256)[0])
+
+
+# ---------------------------------------------------------------- FP8 encoder
+
+def _finite_codes():
+    return [c for c in range(256) if (c & 0x7F) != 0x7F]
+
+
+def test_e4m3_encoder_round_trips_every_finite_code():
+    for c in _finite_codes():
+        assert oracle.double_to_e4m3(oracle.e4m3_to_f64(np.array([c], np.uint8))[0]) == c, c
+
+
+def test_e4m3_encoder_ties_go_to_the_even_code():
+    vals = oracle.e4m3_to_f64(np.arange(0x7F, dtype=np.uint8))  # 0 .. 448, increasing
+    for c in range(0x7E):
+        lo, hi = vals[c], vals[c + 1]
+        mid = (lo + hi) / 2
+        even = c if c % 2 == 0 else c + 1
+        assert oracle.double_to_e4m3(mid) == even, c
+        assert oracle.double_to_e4m3(-mid) == even | 0x80, c
+        assert oracle.double_to_e4m3(np.nextafter(mid, 0)) == c
+        assert oracle.double_to_e4m3(np.nextafter(mid, 1e9)) == c + 1
+    assert oracle.double_to_e4m3(1e6) == 0x7E and oracle.double_to_e4m3(-1e6) == 0xFE  # saturation
+
+
+def test_e4m3_encoder_matches_torch_conversion():
+    g = torch.Generator().manual_seed(3)
+    x = torch.cat([torch.randn(20000, generator=g) * s for s in (1e-4, 1e-2, 1.0, 30.0, 300.0)])
+    x = x.clamp(-448, 448)
+    ref = x.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.double_to_e4m3(float(v)) for v in x.tolist()], dtype=np.uint8)
+    assert np.array_equal(got, ref)
+
+
+def test_row_quantiser_matches_the_input_recipe():
+    g = torch.Generator().manual_seed(4)
+    x = torch.randn((64, 128), generator=g) * torch.logspace(-3, 2, 64)[:, None]
+    x[5] = 0.0  # an all-zero row takes scale 1
+    codes, scale = oracle.quantize_e4m3(x)
+    ref_codes, ref_scale = workloads.quantize_e4m3_per_token(x)
+    assert np.array_equal(scale, ref_scale.numpy())
+    assert np.array_equal(codes, ref_codes.numpy())
