@@ -47,10 +47,10 @@ METRIC = "DSA prefill tokens/s @128K & decode tok/s, % of FP8/BF16/HBM roofline"
 # covers its main pass, re-run pass and rank sort; decode entries cover one
 # decode batch.
 MEASURED_TRAFFIC = {
-    "prefill_indexer": 1.7048e9 + 5.1869e9 + 1e5 + 2.1496e9 + 1.0413e9,
-    "prefill_attention": 75.1601e9 + 17.1764e9,
-    "decode_step": 0.5543e9 + 0.0143e9 + 0.0174e9 + 0.0011e9 + 0.1611e9 + 0.0004e9,
-    "decode_indexer": 0.5543e9 + 0.0143e9 + 0.0174e9 + 0.0011e9,
+    "prefill_indexer": 1.6947e9 + 5.2533e9 + 0.0001e9 + 2.1494e9 + 1.0408e9,
+    "prefill_attention": 75.2040e9 + 17.1771e9,
+    "decode_step": 0.5543e9 + 0.0140e9 + 0.0173e9 + 0.0011e9 + 0.1610e9 + 0.0002e9,
+    "decode_indexer": 0.5543e9 + 0.0140e9 + 0.0173e9 + 0.0011e9,
 }
 DEFAULT_SIZES = (131072, 64, 65536)  # prefill L, decode B, decode L the traffic was measured on
 D_QK, D_V = 576, 512

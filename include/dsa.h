@@ -157,6 +157,14 @@ dsa_status dsa_index_scores(const uint8_t* q_I, const float* q_scale, const floa
  *   scale    softmax scale, finite and > 0 (1/sqrt(576) for the latent row)
  * No workspace.
  * ------------------------------------------------------------------------ */
+/* FP8 quantiser for newly appended tokens (indexer keys or queries): for each
+ * of n rows of d fp32 values, scale[r] = absmax/448 (1 for an all-zero row)
+ * and codes[r, i] = E4M3(x[r, i] / scale[r]), nearest with ties to even,
+ * saturating to +-448 ("Lightning Indexer 的计算过程", step 2 <2>, FP8 量化).
+ * Bit-identical to that definition evaluated in fp32. x [n, d] f32, codes
+ * [n, d] e4m3 bytes, scale [n] f32, all device memory. n = 0 is a no-op. */
+dsa_status dsa_quantize_e4m3_rows(const float* x, int n, int d, uint8_t* codes, float* scale, void* stream);
+
 /* Short-sequence dense fallback: when a sequence has at most DSA_MAX_TOPK
  * tokens every causal key is selected anyway, so the indexer can be skipped
  * and token t (position q0 + t) attends to kv rows 0..q0+t directly, with the

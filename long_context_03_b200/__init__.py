@@ -58,6 +58,7 @@ def lib() -> ctypes.CDLL:
             L.dsa_index_topk_varlen.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, P, P, SZ, P]
             L.dsa_sparse_mla_attn.argtypes = [P, P, P, I, I, I, I, F, P, P, P]
             L.dsa_dense_mla_attn_causal.argtypes = [P, P, I, I, I, I, F, P, P, P]
+            L.dsa_quantize_e4m3_rows.argtypes = [P, I, I, P, P, P]
             L.dsa_index_topk_decode_workspace_size.argtypes = [I, I, I]
             L.dsa_index_topk_decode_workspace_size.restype = SZ
             L.dsa_index_topk_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P, P, SZ, P]
@@ -70,7 +71,8 @@ def lib() -> ctypes.CDLL:
             L.dsa_last_error.argtypes = []
             L.dsa_last_error.restype = ctypes.c_char_p
             for name in ("dsa_index_topk", "dsa_index_topk_rerun_count", "dsa_index_topk_chunk",
-                         "dsa_index_topk_varlen", "dsa_dense_mla_attn_causal", "dsa_index_scores", "dsa_sparse_mla_attn", "dsa_index_topk_decode",
+                         "dsa_index_topk_varlen", "dsa_dense_mla_attn_causal", "dsa_quantize_e4m3_rows",
+                         "dsa_index_scores", "dsa_sparse_mla_attn", "dsa_index_topk_decode",
                          "dsa_index_scores_decode", "dsa_sparse_mla_attn_decode", "dsa_get_device_error",
                          "dsa_index_topk_decode_noalloc"):
                 getattr(L, name).restype = I
@@ -239,6 +241,20 @@ def sparse_mla_attn(q, kv, idx, scale: float, *, out=None, lse=None, want_lse: b
     _check(lib().dsa_sparse_mla_attn(_ptr(q), _ptr(kv), _ptr(idx), T, L, Hq, topk, float(scale), _ptr(out),
                                      _ptr(lse), _stream(q.device)))
     return out, lse
+
+
+def quantize_e4m3_rows(x, *, codes=None, scale=None):
+    """x [n, d] f32 (device) -> (codes uint8 [n, d], scale f32 [n]): per-row absmax/448 scale, E4M3 RNE codes."""
+    n, d = x.shape
+    _req(x, "x", torch.float32, (n, d))
+    if codes is None:
+        codes = torch.empty((n, d), dtype=torch.uint8, device=x.device)
+    if scale is None:
+        scale = torch.empty((n,), dtype=torch.float32, device=x.device)
+    _req(codes, "codes", torch.uint8, (n, d))
+    _req(scale, "scale", torch.float32, (n,))
+    _check(lib().dsa_quantize_e4m3_rows(_ptr(x), n, d, _ptr(codes), _ptr(scale), _stream(x.device)))
+    return codes, scale
 
 
 def dense_mla_attn_causal(q, kv, scale: float, *, q0: int = 0, out=None, lse=None, want_lse: bool = False):

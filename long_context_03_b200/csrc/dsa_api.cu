@@ -17,6 +17,7 @@
 #include "indexer_decode.cuh"
 #include "indexer_prefill.cuh"
 #include "sparse_mla.cuh"
+#include "quantize.cuh"
 #include "topk_select.cuh"
 
 using namespace dsa;
@@ -535,6 +536,15 @@ dsa_status dsa_index_scores(const uint8_t* q_I, const float* q_scale, const floa
   const int nrb = p.rb_end - p.rb_begin;
   const int grid = nrb < num_sms() ? nrb : num_sms();
   return dispatch_prefill<false, 1>(H_I, d_I, q_I, k_cache, p, grid, st);
+}
+
+dsa_status dsa_quantize_e4m3_rows(const float* x, int n, int d, uint8_t* codes, float* scale, void* stream) {
+  if (n < 0 || d <= 0) return fail(DSA_ERR_INVALID_ARG, "n=%d d=%d", n, d);
+  if (n == 0) return DSA_OK;
+  if (!x || !codes || !scale) return fail(DSA_ERR_INVALID_ARG, "null pointer");
+  const int grid = n < 8 * num_sms() ? n : 8 * num_sms();
+  quantize_e4m3_rows_kernel<<<grid, kQuantThreads, 0, static_cast<cudaStream_t>(stream)>>>(x, n, d, codes, scale);
+  return check_launch("quantize_e4m3_rows_kernel");
 }
 
 dsa_status dsa_dense_mla_attn_causal(const uint16_t* q, const uint16_t* kv, int T, int L, int q0, int Hq, float scale,

@@ -92,3 +92,10 @@ def test_dense_fallback_limits(lib):
     assert lib.dsa_dense_mla_attn_causal(p, p, 4, 4096, 0, 16, f, p, None, None) == -2  # L > 2048
     assert lib.dsa_dense_mla_attn_causal(p, p, 10, 100, 95, 16, f, p, None, None) == -1  # q0 + T > L
     assert lib.dsa_dense_mla_attn_causal(None, p, 0, 100, 0, 16, f, None, None, None) == 0  # empty batch
+
+
+def test_quantiser_argument_checks(lib):
+    p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    assert lib.dsa_quantize_e4m3_rows(None, 0, 128, None, None, None) == 0  # nothing to do
+    assert lib.dsa_quantize_e4m3_rows(p, 4, 0, p, p, None) == -1
+    assert lib.dsa_quantize_e4m3_rows(None, 4, 128, p, p, None) == -1
