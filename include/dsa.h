@@ -157,6 +157,21 @@ dsa_status dsa_index_scores(const uint8_t* q_I, const float* q_scale, const floa
  *   scale    softmax scale, finite and > 0 (1/sqrt(576) for the latent row)
  * No workspace.
  * ------------------------------------------------------------------------ */
+/* Sparse MQA attention over a paged latent cache: kv_pool [pool_rows, 576]
+ * holds pages of page_size rows (a power of two, 16..4096); logical row r of
+ * token t is physical row block_table[t * bt_stride + r / page_size] *
+ * page_size + r % page_size (bt_stride 0: every token uses the first table
+ * row, as the tokens of one prefill do; bt_stride = max_blocks: one table row
+ * per token, as in decode). idx [T, topk] holds logical rows < rows, with
+ * rows <= max_blocks * page_size. Same results as dsa_sparse_mla_attn over
+ * the contiguous cache; a page entry outside the pool skips its rows and is
+ * reported as DSA_ERR_BAD_INDEX by dsa_get_device_error. Serving layout, no
+ * counterpart step in the pages. */
+dsa_status dsa_sparse_mla_attn_paged(const uint16_t* q, const uint16_t* kv_pool, const int32_t* block_table,
+                                     const int32_t* idx, int T, int rows, int pool_rows, int bt_stride,
+                                     int max_blocks, int page_size, int Hq, int topk, float scale, uint16_t* out,
+                                     float* lse, void* stream);
+
 /* FP8 quantiser for newly appended tokens (indexer keys or queries): for each
  * of n rows of d fp32 values, scale[r] = absmax/448 (1 for an all-zero row)
  * and codes[r, i] = E4M3(x[r, i] / scale[r]), nearest with ties to even,

@@ -59,6 +59,7 @@ def lib() -> ctypes.CDLL:
             L.dsa_sparse_mla_attn.argtypes = [P, P, P, I, I, I, I, F, P, P, P]
             L.dsa_dense_mla_attn_causal.argtypes = [P, P, I, I, I, I, F, P, P, P]
             L.dsa_quantize_e4m3_rows.argtypes = [P, I, I, P, P, P]
+            L.dsa_sparse_mla_attn_paged.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, F, P, P, P]
             L.dsa_index_topk_decode_workspace_size.argtypes = [I, I, I]
             L.dsa_index_topk_decode_workspace_size.restype = SZ
             L.dsa_index_topk_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P, P, SZ, P]
@@ -72,6 +73,7 @@ def lib() -> ctypes.CDLL:
             L.dsa_last_error.restype = ctypes.c_char_p
             for name in ("dsa_index_topk", "dsa_index_topk_rerun_count", "dsa_index_topk_chunk",
                          "dsa_index_topk_varlen", "dsa_dense_mla_attn_causal", "dsa_quantize_e4m3_rows",
+                         "dsa_sparse_mla_attn_paged",
                          "dsa_index_scores", "dsa_sparse_mla_attn", "dsa_index_topk_decode",
                          "dsa_index_scores_decode", "dsa_sparse_mla_attn_decode", "dsa_get_device_error",
                          "dsa_index_topk_decode_noalloc"):
@@ -240,6 +242,34 @@ def sparse_mla_attn(q, kv, idx, scale: float, *, out=None, lse=None, want_lse: b
         _req(lse, "lse", torch.float32, (T, Hq))
     _check(lib().dsa_sparse_mla_attn(_ptr(q), _ptr(kv), _ptr(idx), T, L, Hq, topk, float(scale), _ptr(out),
                                      _ptr(lse), _stream(q.device)))
+    return out, lse
+
+
+def sparse_mla_attn_paged(q, kv_pool, block_table, idx, rows: int, scale: float, *, page_size: int = 64,
+                          out=None, lse=None, want_lse: bool = False):
+    """Attention over a paged latent cache. block_table [T, max_blocks] (one table row per token)
+    or [1, max_blocks] (shared by all tokens); idx holds logical rows < rows."""
+    T, Hq, D = q.shape
+    pool_rows = kv_pool.shape[0]
+    topk = idx.shape[1]
+    nbt, max_blocks = block_table.shape
+    _req(q, "q", torch.bfloat16, (T, Hq, D_QK))
+    _req(kv_pool, "kv_pool", torch.bfloat16, (pool_rows, D_QK))
+    _req(block_table, "block_table", torch.int32, (nbt, max_blocks))
+    _req(idx, "idx", torch.int32, (T, topk))
+    if nbt not in (1, T):
+        raise ValueError("block_table needs one row per token or a single shared row")
+    bt_stride = 0 if nbt == 1 else max_blocks
+    if out is None:
+        out = torch.empty((T, Hq, D_V), dtype=torch.bfloat16, device=q.device)
+    _req(out, "out", torch.bfloat16, (T, Hq, D_V))
+    if lse is None and want_lse:
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _req(lse, "lse", torch.float32, (T, Hq))
+    _check(lib().dsa_sparse_mla_attn_paged(_ptr(q), _ptr(kv_pool), _ptr(block_table), _ptr(idx), T, rows, pool_rows,
+                                           bt_stride, max_blocks, page_size, Hq, topk, float(scale), _ptr(out),
+                                           _ptr(lse), _stream(q.device)))
     return out, lse
 
 

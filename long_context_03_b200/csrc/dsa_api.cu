@@ -233,8 +233,13 @@ dsa_status check_decode_args(const uint8_t* q_I, const float* q_scale, const flo
 }
 
 // ---- attention ----
+struct MlaPaging {
+  const int32_t* block_table = nullptr;
+  int bt_stride = 0, page_shift = 0, pool_rows = 0;
+};
 dsa_status launch_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int T, int rows, long long kv_stride,
-                      int Hq, int topk, float scale, uint16_t* out, float* lse, cudaStream_t st, int causal_q0 = 0) {
+                      int Hq, int topk, float scale, uint16_t* out, float* lse, cudaStream_t st, int causal_q0 = 0,
+                      MlaPaging pg = MlaPaging()) {
   MlaParams p;
   p.q = reinterpret_cast<const __nv_bfloat16*>(q);
   p.kv = reinterpret_cast<const __nv_bfloat16*>(kv);
@@ -247,24 +252,29 @@ dsa_status launch_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
   p.Hq = Hq;
   p.K = topk;
   p.causal_q0 = causal_q0;
+  p.block_table = pg.block_table;
+  p.bt_stride = pg.bt_stride;
+  p.page_shift = pg.page_shift;
+  p.pool_rows = pg.pool_rows;
   p.scale_log2 = scale * 1.4426950408889634f;
-  dsa_status s = set_smem(sparse_mla_kernel, MlaCfg::SMEM_BYTES);
+  auto kern = pg.block_table ? sparse_mla_kernel<true> : sparse_mla_kernel<false>;
+  dsa_status s = set_smem(kern, MlaCfg::SMEM_BYTES);
   if (s != DSA_OK) return s;
-  static int max_clusters = 0;
+  static int max_clusters = 0;  // the same for both instances (same resources)
   if (max_clusters == 0) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * 512, 1, 1);
     cfg.blockDim = dim3(MlaCfg::NTHREADS, 1, 1);
     cfg.dynamicSmemBytes = MlaCfg::SMEM_BYTES;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, sparse_mla_kernel, &cfg) != cudaSuccess || n <= 0) {
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
       cudaGetLastError();
       n = num_sms() / 2;
     }
     max_clusters = n;
   }
   const int nclusters = T < max_clusters ? T : max_clusters;
-  sparse_mla_kernel<<<2 * nclusters, MlaCfg::NTHREADS, MlaCfg::SMEM_BYTES, st>>>(p);
+  kern<<<2 * nclusters, MlaCfg::NTHREADS, MlaCfg::SMEM_BYTES, st>>>(p);
   return check_launch("sparse_mla_kernel");
 }
 
@@ -536,6 +546,28 @@ dsa_status dsa_index_scores(const uint8_t* q_I, const float* q_scale, const floa
   const int nrb = p.rb_end - p.rb_begin;
   const int grid = nrb < num_sms() ? nrb : num_sms();
   return dispatch_prefill<false, 1>(H_I, d_I, q_I, k_cache, p, grid, st);
+}
+
+dsa_status dsa_sparse_mla_attn_paged(const uint16_t* q, const uint16_t* kv_pool, const int32_t* block_table,
+                                     const int32_t* idx, int T, int rows, int pool_rows, int bt_stride,
+                                     int max_blocks, int page_size, int Hq, int topk, float scale, uint16_t* out,
+                                     float* lse, void* stream) {
+  dsa_status s = check_mla_args(q, kv_pool, idx, T, rows, Hq, topk, scale, out);
+  if (s != DSA_OK) return s;
+  if (!block_table && T > 0) return fail(DSA_ERR_INVALID_ARG, "null pointer");
+  if (page_size < 16 || page_size > 4096 || (page_size & (page_size - 1)) != 0)
+    return fail(DSA_ERR_UNSUPPORTED, "page_size=%d (a power of two in [16, 4096])", page_size);
+  if (pool_rows <= 0 || bt_stride < 0 || max_blocks <= 0 ||
+      static_cast<long long>(max_blocks) * page_size < rows)
+    return fail(DSA_ERR_INVALID_ARG, "pool_rows=%d bt_stride=%d max_blocks=%d page_size=%d rows=%d", pool_rows,
+                bt_stride, max_blocks, page_size, rows);
+  if (T == 0) return DSA_OK;
+  MlaPaging pg;
+  pg.block_table = block_table;
+  pg.bt_stride = bt_stride;
+  pg.page_shift = __builtin_ctz(static_cast<unsigned>(page_size));
+  pg.pool_rows = pool_rows;
+  return launch_mla(q, kv_pool, idx, T, rows, 0, Hq, topk, scale, out, lse, static_cast<cudaStream_t>(stream), 0, pg);
 }
 
 dsa_status dsa_quantize_e4m3_rows(const float* x, int n, int d, uint8_t* codes, float* scale, void* stream) {

@@ -115,6 +115,11 @@ struct MlaParams {
   int rows;                  // valid row bound of a token's cache
   int T, Hq, K;
   int causal_q0;             // position of token 0 when idx is null
+  // Paged latent cache: when block_table is set, logical row r of token i is
+  // physical row block_table[i * bt_stride + (r >> page_shift)] * page + (r & (page - 1))
+  // of kv (a pool of pool_rows rows); bt_stride 0 shares one table row.
+  const int32_t* block_table;
+  int bt_stride, page_shift, pool_rows;
   float scale_log2;          // softmax scale * log2(e)
 };
 
@@ -175,11 +180,27 @@ __device__ __forceinline__ int checked_row(const int32_t* idx_s, int e, int K, i
 
 // Score CTA: the 8 rows (r = ptid/8 + 16k) this thread copies for chunk j,
 // as byte pointers to the rows (absent rows point at row 0 and copy zeros).
+// Paged cache: address of the latent row a token's (checked) logical row
+// points to through the token's page table; null when the row is absent or
+// the page leads outside the pool (reported as a bad index).
+__device__ __forceinline__ const char* paged_row(const MlaParams& p, int tk, int row) {
+  if (row < 0) return nullptr;
+  const int page = p.block_table[static_cast<long long>(tk) * p.bt_stride + (row >> p.page_shift)];
+  const long long phys = (static_cast<long long>(page) << p.page_shift) + (row & ((1 << p.page_shift) - 1));
+  if (page < 0 || phys >= p.pool_rows) {
+    set_device_error(kErrBadIndex, 1);
+    return nullptr;
+  }
+  return reinterpret_cast<const char*>(p.kv + phys * MlaCfg::D);
+}
+
 struct ChunkRows {
   const char* src[8];
   uint32_t valid;  // bit k: row k present
 };
-__device__ __forceinline__ ChunkRows chunk_rows(const __nv_bfloat16* __restrict__ kv_tok, const int32_t* idx_s, int j,
+template <bool kPaged>
+__device__ __forceinline__ ChunkRows chunk_rows(const MlaParams& p, const __nv_bfloat16* __restrict__ kv_tok, int tk,
+                                                const int32_t* idx_s, int j,
                                                 int K, int rows, int ptid) {
   ChunkRows cr;
   cr.valid = 0;
@@ -187,9 +208,16 @@ __device__ __forceinline__ ChunkRows chunk_rows(const __nv_bfloat16* __restrict_
   for (int k = 0; k < 8; ++k) {
     const int r = (ptid >> 3) + 16 * k;
     const int row = checked_row(idx_s, j * MlaCfg::NK + r, K, rows);
-    cr.src[k] = reinterpret_cast<const char*>(kv_tok + static_cast<long long>(row >= 0 ? row : 0) * MlaCfg::D) +
-                (ptid & 7) * 16;
-    cr.valid |= (row >= 0 ? 1u : 0u) << k;
+    if constexpr (kPaged) {
+      const char* src = paged_row(p, tk, row);
+      // absent rows copy zeros (source size 0); any valid address serves
+      cr.src[k] = (src ? src : reinterpret_cast<const char*>(p.kv)) + (ptid & 7) * 16;
+      cr.valid |= (src ? 1u : 0u) << k;
+    } else {
+      cr.src[k] = reinterpret_cast<const char*>(kv_tok + static_cast<long long>(row >= 0 ? row : 0) * MlaCfg::D) +
+                  (ptid & 7) * 16;
+      cr.valid |= (row >= 0 ? 1u : 0u) << k;
+    }
   }
   return cr;
 }
@@ -211,7 +239,9 @@ __device__ __forceinline__ void gather_slab_tile(uint32_t tile, const ChunkRows&
 // Eight consecutive threads copy one (row, slab) segment of 128 bytes; each
 // group of eight handles rows g and g+16 across all eight slabs, so a thread
 // looks up two row indices per sub-tile.
-__device__ __forceinline__ void gather_value_tile(uint32_t tile, const __nv_bfloat16* __restrict__ kv_tok,
+template <bool kPaged>
+__device__ __forceinline__ void gather_value_tile(uint32_t tile, const MlaParams& p,
+                                                  const __nv_bfloat16* __restrict__ kv_tok, int tk,
                                                   const int32_t* idx_s, int j, int u, int K, int rows, int ptid) {
   const int c = ptid & 7;
   const int g = ptid >> 3;  // 0..15
@@ -219,11 +249,19 @@ __device__ __forceinline__ void gather_value_tile(uint32_t tile, const __nv_bflo
   for (int half = 0; half < 2; ++half) {
     const int r = g + 16 * half;
     const int row = checked_row(idx_s, j * MlaCfg::NK + u * MlaCfg::VROWS + r, K, rows);
-    const char* src =
-        reinterpret_cast<const char*>(kv_tok + static_cast<long long>(row >= 0 ? row : 0) * MlaCfg::D) + c * 16;
+    const char* src;
+    bool present;
+    if constexpr (kPaged) {
+      const char* rp = paged_row(p, tk, row);
+      present = rp != nullptr;
+      src = (rp ? rp : reinterpret_cast<const char*>(p.kv)) + c * 16;
+    } else {
+      present = row >= 0;
+      src = reinterpret_cast<const char*>(kv_tok + static_cast<long long>(row >= 0 ? row : 0) * MlaCfg::D) + c * 16;
+    }
 #pragma unroll
     for (int sl = 0; sl < 8; ++sl)
-      cp_async_16_zfill(tile + sl * MlaCfg::VSLAB + r * 128 + ((c ^ (r & 7)) << 4), src + sl * 128, row >= 0);
+      cp_async_16_zfill(tile + sl * MlaCfg::VSLAB + r * 128 + ((c ^ (r & 7)) << 4), src + sl * 128, present);
   }
 }
 
@@ -245,6 +283,7 @@ __device__ __forceinline__ void stage_index_row(int32_t* idx_s, const int32_t* _
   named_bar_sync(1, MlaCfg::NPROD * 32);
 }
 
+template <bool kPaged>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
     sparse_mla_kernel(const MlaParams p) {
   using C = MlaCfg;
@@ -324,14 +363,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
         for (int wd = static_cast<int>(warp); wd < nchunk * (C::NK / 32); wd += C::NPROD) {
           const int e = wd * 32 + static_cast<int>(lane);
           const int row = (e < p.K) ? idx_s[e] : -1;
-          const uint32_t m = __ballot_sync(0xffffffffu, row >= 0 && row < p.rows);
+          bool present = row >= 0 && row < p.rows;
+          if (kPaged && present) {  // paged: the page must lie inside the pool
+            const int page = p.block_table[static_cast<long long>(tk) * p.bt_stride + (row >> p.page_shift)];
+            present = page >= 0 && (static_cast<long long>(page) << p.page_shift) +
+                                           (row & ((1 << p.page_shift) - 1)) < p.pool_rows;
+          }
+          const uint32_t m = __ballot_sync(0xffffffffu, present);
           if (lane == 0) vmask_s[mb * (C::KMAX / 32) + wd] = m;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(bars + C::B_MASK_FULL + mb);
         bool ok = true;
         for (int j = 0; j < nchunk && ok; ++j) {
-          const ChunkRows cr = chunk_rows(kv_tok, idx_s, j, p.K, p.rows, ptid);
+          const ChunkRows cr = chunk_rows<kPaged>(p, kv_tok, tk, idx_s, j, p.K, p.rows, ptid);
           for (int i = 0; i < C::NSLAB_QK; ++i) {
             if (!mbar_wait(bars + C::B_RING_EMPTY + slot, ph, ab, 31)) { ok = false; break; }
             gather_slab_tile(ring + slot * C::SLAB_TILE, cr, i, ptid);
@@ -560,7 +605,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
         for (int j = 0; j < nchunk && ok; ++j) {
           for (int u = 0; u < C::NK / C::VROWS; ++u) {
             if (!mbar_wait(bars + C::B_RING_EMPTY + slot, ph, ab, 41)) { ok = false; break; }
-            gather_value_tile(ring + slot * C::V_TILE, kv_tok, idx_s, j, u, p.K, p.rows, ptid);
+            gather_value_tile<kPaged>(ring + slot * C::V_TILE, p, kv_tok, tk, idx_s, j, u, p.K, p.rows, ptid);
             cp_async_mbar_arrive(bars + C::B_RING_FULL + slot);
             if (++slot == C::NVST) { slot = 0; ph ^= 1; }
           }

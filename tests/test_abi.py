@@ -99,3 +99,11 @@ def test_quantiser_argument_checks(lib):
     assert lib.dsa_quantize_e4m3_rows(None, 0, 128, None, None, None) == 0  # nothing to do
     assert lib.dsa_quantize_e4m3_rows(p, 4, 0, p, p, None) == -1
     assert lib.dsa_quantize_e4m3_rows(None, 4, 128, p, p, None) == -1
+
+
+def test_paged_attention_argument_checks(lib):
+    p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    f = ctypes.c_float(0.1)
+    # page size not a power of two; table too small for the rows
+    assert lib.dsa_sparse_mla_attn_paged(p, p, p, p, 2, 1000, 4096, 16, 16, 48, 16, 8, f, p, None, None) == -2
+    assert lib.dsa_sparse_mla_attn_paged(p, p, p, p, 2, 1000, 4096, 15, 15, 64, 16, 8, f, p, None, None) == -1
