@@ -214,6 +214,23 @@ dsa_status dsa_index_topk_decode(const uint8_t* q_I, const float* q_scale, const
                                  const float* k_scale, const int32_t* lens, int B, int L_max, int H_I, int d_I,
                                  int topk, int32_t* idx, void* workspace, size_t ws_bytes, void* stream);
 
+/* Decode indexer + top-k over a paged FP8 key cache. k_pool [pool_rows, d_I]
+ * e4m3 and k_scale_pool [pool_rows] f32 hold pages of page_size rows (a power
+ * of two, 16..4096; pool_rows a multiple of it); key s of sequence b is pool
+ * row block_table[b * max_blocks + s / page_size] * page_size + s % page_size
+ * (block_table [B, max_blocks] int32, device). Entries for pages at or past
+ * lens[b] are never read. Equivalent to dsa_index_topk_decode with L_max =
+ * max_blocks * page_size over the gathered contiguous cache: same scores bit
+ * for bit, same idx. Workspace: dsa_index_topk_decode_workspace_size(B,
+ * max_blocks * page_size, topk). A page entry outside [0, pool_rows /
+ * page_size) for a key below lens[b] gives that page's keys zero codes and
+ * zero scale (score 0) and is reported as DSA_ERR_BAD_INDEX by
+ * dsa_get_device_error. Serving layout, no counterpart step in the pages. */
+dsa_status dsa_index_topk_decode_paged(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_pool,
+                                       const float* k_scale_pool, const int32_t* block_table, const int32_t* lens,
+                                       int B, int max_blocks, int page_size, int pool_rows, int H_I, int d_I, int topk,
+                                       int32_t* idx, void* workspace, size_t ws_bytes, void* stream);
+
 /* Test hook: decode scores[B, L_max] f32 (entries s >= lens[b] untouched). */
 dsa_status dsa_index_scores_decode(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
                                    const float* k_scale, const int32_t* lens, int B, int L_max, int H_I, int d_I,

@@ -63,6 +63,7 @@ def lib() -> ctypes.CDLL:
             L.dsa_index_topk_decode_workspace_size.argtypes = [I, I, I]
             L.dsa_index_topk_decode_workspace_size.restype = SZ
             L.dsa_index_topk_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P, P, SZ, P]
+            L.dsa_index_topk_decode_paged.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, SZ, P]
             L.dsa_index_scores_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, P, P]
             L.dsa_sparse_mla_attn_decode.argtypes = [P, P, P, I, I, I, I, F, P, P, P]
             L.dsa_index_topk_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P, P]
@@ -76,7 +77,7 @@ def lib() -> ctypes.CDLL:
                          "dsa_sparse_mla_attn_paged",
                          "dsa_index_scores", "dsa_sparse_mla_attn", "dsa_index_topk_decode",
                          "dsa_index_scores_decode", "dsa_sparse_mla_attn_decode", "dsa_get_device_error",
-                         "dsa_index_topk_decode_noalloc"):
+                         "dsa_index_topk_decode_noalloc", "dsa_index_topk_decode_paged"):
                 getattr(L, name).restype = I
             _lib = L
     return _lib
@@ -337,6 +338,36 @@ def index_topk_decode(q_I, q_scale, w, k_cache, k_scale, lens, topk: int, *, idx
     _check(lib().dsa_index_topk_decode(_ptr(q_I), _ptr(q_scale), _ptr(w), _ptr(k_cache), _ptr(k_scale),
                                        _ptr(lens), B, L_max, H_I, d_I, topk, _ptr(idx), _ptr(workspace),
                                        workspace.numel() * workspace.element_size(), _stream(q_I.device)))
+    return idx
+
+
+def index_topk_decode_paged(q_I, q_scale, w, k_pool, k_scale_pool, block_table, lens, topk: int, *,
+                            page_size: int = 64, idx=None, workspace=None):
+    """Decode indexer + top-k over a paged FP8 key cache: k_pool [pool_rows, d_I] e4m3 and
+    k_scale_pool [pool_rows] f32 in pages of page_size rows, block_table [B, max_blocks] int32
+    (page of key s of sequence b: block_table[b, s // page_size]). Same idx as index_topk_decode
+    over the gathered contiguous cache with L_max = max_blocks * page_size."""
+    q_I, k_pool = _u8(q_I), _u8(k_pool)
+    B, H_I, d_I = q_I.shape
+    pool_rows = k_pool.shape[0]
+    max_blocks = block_table.shape[1]
+    _req(q_I, "q_I", torch.uint8)
+    _req(q_scale, "q_scale", torch.float32, (B,))
+    _req(w, "w", torch.float32, (B, H_I))
+    _req(k_pool, "k_pool", torch.uint8, (pool_rows, d_I))
+    _req(k_scale_pool, "k_scale_pool", torch.float32, (pool_rows,))
+    _req(block_table, "block_table", torch.int32, (B, max_blocks))
+    _req(lens, "lens", torch.int32, (B,))
+    if idx is None:
+        idx = torch.empty((B, topk), dtype=torch.int32, device=q_I.device)
+    _req(idx, "idx", torch.int32, (B, topk))
+    need = index_topk_decode_workspace_size(B, max_blocks * page_size, topk)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q_I.device)
+    _check(lib().dsa_index_topk_decode_paged(_ptr(q_I), _ptr(q_scale), _ptr(w), _ptr(k_pool), _ptr(k_scale_pool),
+                                             _ptr(block_table), _ptr(lens), B, max_blocks, page_size, pool_rows,
+                                             H_I, d_I, topk, _ptr(idx), _ptr(workspace),
+                                             workspace.numel() * workspace.element_size(), _stream(q_I.device)))
     return idx
 
 

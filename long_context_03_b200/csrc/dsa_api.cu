@@ -181,12 +181,20 @@ template <int HI, int DI>
 dsa_status launch_decode_scores(const uint8_t* q_I, const uint8_t* k_cache, int B, const IdxDecodeParams& p,
                                 cudaStream_t st) {
   using C = IdxDecodeCfg<HI, DI>;
+  const bool paged = p.block_table != nullptr;
   CUtensorMap tmQ, tmK;
   dsa_status s = make_map_u8(&tmQ, q_I, DI, static_cast<uint64_t>(B) * HI, DI, HI);
   if (s != DSA_OK) return s;
-  s = make_map_u8(&tmK, k_cache, DI, static_cast<uint64_t>(B) * p.L_max, DI, C::BM);
+  if (paged) {
+    // the pool's rows, loaded one page (at most one tile) per box
+    const int page = 1 << p.page_shift;
+    s = make_map_u8(&tmK, k_cache, DI, static_cast<uint64_t>(p.pool_pages) * page, DI,
+                    static_cast<uint32_t>(page < C::BM ? page : C::BM));
+  } else {
+    s = make_map_u8(&tmK, k_cache, DI, static_cast<uint64_t>(B) * p.L_max, DI, C::BM);
+  }
   if (s != DSA_OK) return s;
-  auto kern = indexer_decode_kernel<HI, DI>;
+  auto kern = paged ? indexer_decode_kernel<HI, DI, true> : indexer_decode_kernel<HI, DI, false>;
   s = set_smem(kern, C::SMEM_BYTES);
   if (s != DSA_OK) return s;
   const int items = ((p.L_max + C::CHUNK - 1) / C::CHUNK) * B;
@@ -195,10 +203,19 @@ dsa_status launch_decode_scores(const uint8_t* q_I, const uint8_t* k_cache, int 
   return check_launch("indexer_decode_kernel");
 }
 
+struct KeyPaging {
+  const int32_t* block_table = nullptr;
+  int bt_stride = 0, page_shift = 0, pool_pages = 0;
+};
+
 dsa_status decode_scores(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
                          const float* k_scale, const int32_t* lens, int B, int L_max, int H_I, int d_I, float* scores,
-                         uint32_t* hist, cudaStream_t st) {
+                         uint32_t* hist, cudaStream_t st, KeyPaging pg = KeyPaging()) {
   IdxDecodeParams p;
+  p.block_table = pg.block_table;
+  p.bt_stride = pg.bt_stride;
+  p.page_shift = pg.page_shift;
+  p.pool_pages = pg.pool_pages;
   p.hist = hist;
   p.q_scale = q_scale;
   p.w = w;
@@ -628,6 +645,46 @@ dsa_status dsa_index_topk_decode(const uint8_t* q_I, const float* q_scale, const
   const cudaError_t e = cudaMemsetAsync(hist, 0, static_cast<size_t>(B) * 2048 * 4, st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(histogram)");
   s = decode_scores(q_I, q_scale, w, k_cache, k_scale, lens, B, L_max, H_I, d_I, scores, hist, st);
+  if (s != DSA_OK) return s;
+  s = launch_decode_select(scores, lens, L_max, topk, hist, sel, B, st);
+  if (s != DSA_OK) return s;
+  return launch_rank_sort(sel, idx, topk, B, st);
+}
+
+dsa_status dsa_index_topk_decode_paged(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_pool,
+                                       const float* k_scale_pool, const int32_t* block_table, const int32_t* lens,
+                                       int B, int max_blocks, int page_size, int pool_rows, int H_I, int d_I, int topk,
+                                       int32_t* idx, void* workspace, size_t ws_bytes, void* stream) {
+  if (!block_table) return fail(DSA_ERR_INVALID_ARG, "null pointer");
+  if (page_size < 16 || page_size > 4096 || (page_size & (page_size - 1)))
+    return fail(DSA_ERR_INVALID_ARG, "page_size=%d must be a power of two in [16, 4096]", page_size);
+  if (max_blocks <= 0 || pool_rows <= 0 || pool_rows % page_size)
+    return fail(DSA_ERR_INVALID_ARG, "max_blocks=%d pool_rows=%d (a positive multiple of page_size)", max_blocks,
+                pool_rows);
+  if (static_cast<long long>(max_blocks) * page_size >= (1ll << 31))
+    return fail(DSA_ERR_UNSUPPORTED, "max_blocks*page_size too large");
+  const int L_max = max_blocks * page_size;
+  dsa_status s = check_decode_args(q_I, q_scale, w, k_pool, k_scale_pool, lens, B, L_max, H_I, d_I);
+  if (s != DSA_OK) return s;
+  if (!idx) return fail(DSA_ERR_INVALID_ARG, "null pointer");
+  if (topk < 1 || topk > DSA_MAX_TOPK) return fail(DSA_ERR_UNSUPPORTED, "topk=%d not in [1, %d]", topk, DSA_MAX_TOPK);
+  const size_t need = dsa_index_topk_decode_workspace_size(B, L_max, topk);
+  if (!workspace || ws_bytes < need) return fail(DSA_ERR_WORKSPACE, "workspace %zu bytes, need %zu", ws_bytes, need);
+  if (!aligned16(workspace)) return fail(DSA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* base = reinterpret_cast<char*>(workspace);
+  float* scores = reinterpret_cast<float*>(base);
+  const size_t off_keys = (static_cast<size_t>(B) * L_max * 4 + 255) / 256 * 256;
+  uint64_t* sel = reinterpret_cast<uint64_t*>(base + off_keys);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(base + off_keys + (static_cast<size_t>(B) * topk * 8 + 255) / 256 * 256);
+  const cudaError_t e = cudaMemsetAsync(hist, 0, static_cast<size_t>(B) * 2048 * 4, st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(histogram)");
+  KeyPaging pg;
+  pg.block_table = block_table;
+  pg.bt_stride = max_blocks;
+  pg.page_shift = __builtin_ctz(static_cast<unsigned>(page_size));
+  pg.pool_pages = pool_rows / page_size;
+  s = decode_scores(q_I, q_scale, w, k_pool, k_scale_pool, lens, B, L_max, H_I, d_I, scores, hist, st, pg);
   if (s != DSA_OK) return s;
   s = launch_decode_select(scores, lens, L_max, topk, hist, sel, B, st);
   if (s != DSA_OK) return s;

@@ -22,7 +22,7 @@ __device__ unsigned int g_device_error = 0;
 
 enum DeviceErr : unsigned int {
   kErrTimeout = 1u,       // an mbarrier wait ran past its bound
-  kErrBadIndex = 2u,      // an attention index outside [0, L) (skipped)
+  kErrBadIndex = 2u,      // an index or page-table entry outside its cache (skipped)
 };
 
 __device__ __forceinline__ void set_device_error(unsigned int code, unsigned int where) {

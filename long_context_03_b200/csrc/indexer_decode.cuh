@@ -49,7 +49,9 @@ struct IdxDecodeCfg {
   static constexpr int OFF_BAR = OFF_HIST + 2048 * 4;
   static constexpr int NBAR = 4 + 2 * KST + 2 * NACC;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr int MAX_ITEM_PAGES = CHUNK / 16;  // pages one item touches at the smallest page size
+  static constexpr int OFF_PG = OFF_MISC + 16;       // i32 [MAX_ITEM_PAGES]: paged producer's staged pages
+  static constexpr int SMEM_BYTES = OFF_PG + MAX_ITEM_PAGES * 4 + 1024;
   static_assert(HI % 16 == 0 && HI <= 64, "decode indexer: H_I must be 16, 32, 48 or 64");
 };
 
@@ -62,13 +64,26 @@ struct IdxDecodeParams {
   int B;
   float* scores;         // [B, L_max]; entries s >= lens[b] untouched
   uint32_t* hist;        // [B, 2048] counts of the top 11 bits of each ranking key, or null
+  // paged key cache (paged instance only): key s of sequence b is pool row
+  // block_table[b * bt_stride + (s >> page_shift)] * page + (s & (page - 1));
+  // k_scale is then indexed by pool row; the pool holds pool_pages pages
+  const int32_t* block_table;
+  int bt_stride, page_shift, pool_pages;
 };
+
+// Pool row of key s of sequence b in a paged cache, or -1 when its page entry
+// lies outside the pool.
+__device__ __forceinline__ int paged_key_row(const IdxDecodeParams& p, int b, int s) {
+  const int page = p.block_table[static_cast<long long>(b) * p.bt_stride + (s >> p.page_shift)];
+  if (page < 0 || page >= p.pool_pages) return -1;
+  return (page << p.page_shift) + (s & ((1 << p.page_shift) - 1));
+}
 
 // Bin of a ranking key in the 2048-bin histogram: its top 11 bits (sign,
 // exponent and the top two mantissa bits of the score).
 __device__ __forceinline__ uint32_t key_bin11(uint64_t key) { return static_cast<uint32_t>(key >> 53); }
 
-template <int HI, int DI>
+template <int HI, int DI, bool kPaged>
 __global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS)
     indexer_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const IdxDecodeParams p) {
@@ -139,7 +154,62 @@ __global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS)
   };
 
   if (warp == 0) {
-    if (lane == 0) {
+    if constexpr (kPaged) {
+      // Paged producer: the whole warp first stages the pool row of the first
+      // key of every page the item touches (one round trip for all of them),
+      // then lane 0 issues the boxes: R = min(page, BM) rows per box. A box past
+      // the sequence or behind a bad page entry starts outside the pool and
+      // lands as zeros (its bytes still count).
+      int* pg_s = reinterpret_cast<int*>(smem + C::OFF_PG);
+      const int shift = p.page_shift;
+      const int R = min(1 << shift, C::BM);
+      const int oob = p.pool_pages << shift;
+      int g = 0;   // key tiles issued so far (ring position and phase)
+      int qn = 0;  // query loads issued so far
+      bool ok = true;
+      for (int it = it0; it < it1 && ok; ++it) {
+        int b, s0, nkt, n;
+        if (!item(it, b, s0, nkt, n)) continue;
+        const int fp = s0 >> shift;                                     // first page of the item
+        const int npg = ((min(s0 + nkt * C::BM, n) - 1) >> shift) - fp + 1;  // <= MAX_ITEM_PAGES
+        __syncwarp();  // lane 0 is done with the previous item's entries
+        for (int j = static_cast<int>(lane); j < npg; j += 32) {
+          const int page = p.block_table[static_cast<long long>(b) * p.bt_stride + fp + j];
+          const bool bad = page < 0 || page >= p.pool_pages;
+          if (bad) set_device_error(kErrBadIndex, 2);
+          pg_s[j] = bad ? -1 : (page << shift);
+        }
+        __syncwarp();
+        if (lane == 0) {
+          const int qb = qn & 1;
+          if (!mbar_wait(q_empty + qb, ((qn >> 1) & 1) ^ 1, ab, 10)) ok = false;
+          if (ok) {
+            mbar_arrive_expect_tx(q_full + qb, C::QBYTES);
+            tma_load_2d(q_s + qb * C::QPAD, &tmQ, q_full + qb, 0, b * HI);
+            ++qn;
+          }
+          for (int kt = 0; kt < nkt && ok; ++kt, ++g) {
+            const int slot = g % C::KST;
+            if (!mbar_wait(k_empty + slot, ((g / C::KST) & 1) ^ 1, ab, 11)) { ok = false; break; }
+            mbar_arrive_expect_tx(k_full + slot, C::KTILE_BYTES);
+            for (int i = 0; i < C::BM; i += R) {
+              const int sk = s0 + kt * C::BM + i;
+              int prow = oob;
+              if (sk < n) {
+                const int base = pg_s[(sk >> shift) - fp];
+                if (base >= 0) prow = base + (sk & ((1 << shift) - 1));
+              }
+              tma_load_2d(k_s + slot * C::KTILE_BYTES + i * DI, &tmK, k_full + slot, 0, prow);
+            }
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      }
+      // wait until the MMA has consumed every issued tile (copies landed)
+      if (lane == 0)
+        for (int gg = max(0, g - C::KST); gg < g && !ab.raised(); ++gg)
+          mbar_wait(k_empty + gg % C::KST, (gg / C::KST) & 1, ab, 12);
+    } else if (lane == 0) {
       int g = 0;   // key tiles issued so far (ring position and phase)
       int qn = 0;  // query loads issued so far
       for (int it = it0; it < it1; ++it) {
@@ -229,7 +299,13 @@ __global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS)
       for (int kt = 0; kt < nkt; ++kt, ++g) {
         const int buf = g % C::NACC;
         const int s = s0 + kt * C::BM + quarter * 32 + static_cast<int>(lane);
-        const float ks = (s < n) ? p.k_scale[static_cast<size_t>(b) * p.L_max + s] : 0.f;
+        float ks = 0.f;
+        if constexpr (kPaged) {
+          const int r = (s < n) ? paged_key_row(p, b, s) : -1;
+          if (r >= 0) ks = p.k_scale[r];
+        } else {
+          if (s < n) ks = p.k_scale[static_cast<size_t>(b) * p.L_max + s];
+        }
         if (!mbar_wait(acc_full + buf, (g / C::NACC) & 1, ab, 16)) { ok = false; break; }
         tc_fence_after();
         // eight independent partial sums (head j to sum j % 8), added in a

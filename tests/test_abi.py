@@ -107,3 +107,19 @@ def test_paged_attention_argument_checks(lib):
     # page size not a power of two; table too small for the rows
     assert lib.dsa_sparse_mla_attn_paged(p, p, p, p, 2, 1000, 4096, 16, 16, 48, 16, 8, f, p, None, None) == -2
     assert lib.dsa_sparse_mla_attn_paged(p, p, p, p, 2, 1000, 4096, 15, 15, 64, 16, 8, f, p, None, None) == -1
+
+
+def test_paged_decode_indexer_argument_checks(lib):
+    p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    # (q_I, q_scale, w, k_pool, k_scale_pool, table, lens, B, max_blocks, page, pool_rows, H_I, d_I, topk,
+    #  idx, workspace, ws_bytes, stream)
+    assert lib.dsa_index_topk_decode_paged(p, p, p, p, p, None, p, 2, 8, 64, 1024, 64, 128, 16, p, p, 1 << 30,
+                                           None) == -1  # no table
+    assert lib.dsa_index_topk_decode_paged(p, p, p, p, p, p, p, 2, 8, 48, 1024, 64, 128, 16, p, p, 1 << 30,
+                                           None) == -1  # page not a power of two
+    assert lib.dsa_index_topk_decode_paged(p, p, p, p, p, p, p, 2, 8, 64, 1000, 64, 128, 16, p, p, 1 << 30,
+                                           None) == -1  # pool not whole pages
+    assert lib.dsa_index_topk_decode_paged(p, p, p, p, p, p, p, 2, 8, 64, 1024, 64, 128, 16, p, None, 0,
+                                           None) == -5  # no workspace
+    assert lib.dsa_index_topk_decode_paged(p, p, p, p, p, p, p, 2, 8, 64, 1024, 32, 128, 16, p, p, 1 << 30,
+                                           None) == -2  # H_I outside the supported set

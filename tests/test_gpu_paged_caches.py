@@ -1,0 +1,158 @@
+"""Paged caches equal the contiguous ones bit for bit.
+
+Attention over a paged latent cache gathers the same rows in the same order
+as over the contiguous cache, for per-token tables (decode) and one shared
+table (prefill); a page entry outside the pool skips its rows and is
+reported. The decode indexer over a paged FP8 key cache computes the same
+scores (same codes, same scales, same arithmetic), so its top-k equals the
+contiguous call's exactly; a bad page entry is reported."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dsa():
+    import long_context_03_b200 as m
+    m.lib()
+    return m
+
+
+def _page(kv_rows, page, gen):
+    """Scatter [n, 576] rows into a shuffled pool of pages; return (pool, table [n_pages])."""
+    n = kv_rows.shape[0]
+    npg = (n + page - 1) // page
+    perm = torch.randperm(npg + 3, generator=gen)[:npg]  # a few spare pages in the pool
+    pool = torch.zeros(((npg + 3) * page, 576), dtype=torch.bfloat16, device=kv_rows.device)
+    for i in range(npg):
+        rows = kv_rows[i * page:(i + 1) * page]
+        pool[perm[i] * page:perm[i] * page + rows.shape[0]] = rows
+    return pool, perm.to(torch.int32)
+
+
+def test_decode_tables_match_contiguous(dsa):
+    B, L, page = 6, 5000, 64
+    D = workloads.make_decode(B, L, 64, 128, 128, 2048, seed=31, lens=[5000, 4999, 1, 2048, 2049, 3333], device="cuda")
+    idx = dsa.index_topk_decode(D.q_I, D.q_scale, D.w, D.k_cache, D.k_scale, D.lens, 2048)
+    ref, ref_lse = dsa.sparse_mla_attn_decode(D.q, D.kv, idx, D.scale, want_lse=True)
+    gen = torch.Generator().manual_seed(5)
+    pools, tables = [], []
+    base = 0
+    for b in range(B):
+        pool, table = _page(D.kv[b], page, gen)
+        pools.append(pool)
+        tables.append(table + base)
+        base += pool.shape[0] // page
+    pool = torch.cat(pools)
+    table = torch.stack(tables).cuda()
+    out, lse = dsa.sparse_mla_attn_paged(D.q, pool, table, idx, L, D.scale, page_size=page, want_lse=True)
+    dsa.check_device_error()
+    assert torch.equal(out, ref) and torch.equal(lse, ref_lse)
+
+
+def test_prefill_shared_table_and_bad_page(dsa):
+    P = workloads.make_config("tiny_L512", device="cuda")
+    idx = dsa.index_topk(P.q_I, P.q_scale, P.w, P.k_cache, P.k_scale, P.topk)
+    ref, _ = dsa.sparse_mla_attn(P.q, P.kv, idx, P.scale)
+    pool, table = _page(P.kv, 16, torch.Generator().manual_seed(6))
+    table = table.cuda()[None]
+    out, _ = dsa.sparse_mla_attn_paged(P.q, pool, table, idx, P.L, P.scale, page_size=16)
+    dsa.check_device_error()
+    assert torch.equal(out, ref)
+    # page 3 (rows 48..63) leads outside the pool: those rows are skipped and reported
+    bad = table.clone()
+    bad[0, 3] = 10 ** 6
+    out_bad, _ = dsa.sparse_mla_attn_paged(P.q, pool, bad, idx, P.L, P.scale, page_size=16)
+    st, _ = dsa.device_error()
+    assert st == -6  # DSA_ERR_BAD_INDEX
+    idx_skip = idx.clone()
+    idx_skip[(idx_skip >= 48) & (idx_skip < 64)] = -1
+    ref_skip, _ = dsa.sparse_mla_attn(P.q, P.kv, idx_skip, P.scale)
+    assert torch.equal(out_bad, ref_skip)
+
+
+def _page_keys(k_cache, k_scale, lens, page, gen, spare=5):
+    """Scatter every sequence's key pages into one shuffled pool.
+
+    Returns (k_pool [pool_rows, d], ks_pool [pool_rows], table [B, max_blocks]);
+    table entries of pages past a sequence's length are -1 (never read)."""
+    B, L, d = k_cache.shape
+    max_blocks = (L + page - 1) // page
+    Lp = max_blocks * page
+    kc = torch.zeros((B, Lp, d), dtype=torch.uint8, device=k_cache.device)
+    kc[:, :L] = k_cache.view(torch.uint8)
+    ks = torch.zeros((B, Lp), dtype=torch.float32, device=k_cache.device)
+    ks[:, :L] = k_scale
+    used = [(int(n) + page - 1) // page for n in lens.tolist()]
+    total = sum(used)
+    perm = torch.randperm(total + spare, generator=gen)[:total].to(k_cache.device)
+    k_pool = torch.zeros(((total + spare) * page, d), dtype=torch.uint8, device=k_cache.device)
+    ks_pool = torch.full(((total + spare) * page,), 7.0, dtype=torch.float32, device=k_cache.device)
+    table = torch.full((B, max_blocks), -1, dtype=torch.int32)
+    i = 0
+    for b in range(B):
+        dst = perm[i:i + used[b]]
+        rows = (dst[:, None] * page + torch.arange(page, device=k_cache.device)[None]).reshape(-1)
+        k_pool[rows] = kc[b, :used[b] * page].reshape(-1, d)
+        ks_pool[rows] = ks[b, :used[b] * page].reshape(-1)
+        table[b, :used[b]] = dst.cpu().to(torch.int32)
+        i += used[b]
+    return k_pool, ks_pool, table.to(k_cache.device)
+
+
+@pytest.mark.parametrize("page", [16, 64, 128, 256])
+def test_decode_indexer_paged_keys_match_contiguous(dsa, page):
+    B, L = 6, 5000
+    D = workloads.make_decode(B, L, 64, 128, 128, 2048, seed=41, lens=[5000, 4999, 1, 2048, 2049, 3333],
+                              device="cuda")
+    ref = dsa.index_topk_decode(D.q_I, D.q_scale, D.w, D.k_cache, D.k_scale, D.lens, 2048)
+    k_pool, ks_pool, table = _page_keys(D.k_cache, D.k_scale, D.lens, page, torch.Generator().manual_seed(page))
+    idx = dsa.index_topk_decode_paged(D.q_I, D.q_scale, D.w, k_pool, ks_pool, table, D.lens, 2048, page_size=page)
+    dsa.check_device_error()
+    assert torch.equal(idx, ref)
+
+
+def test_paged_decode_step_matches_contiguous(dsa):
+    """A whole decode step (indexer + attention) with both caches paged, at 64K."""
+    B, L, page = 16, 65536, 64
+    lens = [65536, 65535, 40000, 2049, 1, 30001, 65472, 12345, 65536, 777, 50000, 64, 65, 2048, 33333, 60000]
+    D = workloads.make_decode(B, L, 64, 128, 128, 2048, seed=43, lens=lens, device="cuda")
+    ref_idx = dsa.index_topk_decode(D.q_I, D.q_scale, D.w, D.k_cache, D.k_scale, D.lens, 2048)
+    ref_out, ref_lse = dsa.sparse_mla_attn_decode(D.q, D.kv, ref_idx, D.scale, want_lse=True)
+    gen = torch.Generator().manual_seed(9)
+    k_pool, ks_pool, table = _page_keys(D.k_cache, D.k_scale, D.lens, page, gen)
+    # the latent rows use the same page numbers as the keys (one page table per sequence)
+    kv_pool = torch.zeros((k_pool.shape[0], 576), dtype=torch.bfloat16, device="cuda")
+    for b in range(B):
+        n = (lens[b] + page - 1) // page
+        rows = (table[b, :n].long()[:, None] * page + torch.arange(page, device="cuda")[None]).reshape(-1)
+        src = torch.zeros((n * page, 576), dtype=torch.bfloat16, device="cuda")
+        m = min(n * page, L)
+        src[:m] = D.kv[b, :m]
+        kv_pool[rows] = src
+    idx = dsa.index_topk_decode_paged(D.q_I, D.q_scale, D.w, k_pool, ks_pool, table, D.lens, 2048, page_size=page)
+    out, lse = dsa.sparse_mla_attn_paged(D.q, kv_pool, table, idx, L, D.scale, page_size=page, want_lse=True)
+    dsa.check_device_error()
+    assert torch.equal(idx, ref_idx)
+    assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
+
+
+def test_decode_indexer_bad_page_is_reported(dsa):
+    B, L, page = 2, 3000, 64
+    D = workloads.make_decode(B, L, 64, 128, 128, 2048, seed=47, lens=[3000, 2500], device="cuda")
+    k_pool, ks_pool, table = _page_keys(D.k_cache, D.k_scale, D.lens, page, torch.Generator().manual_seed(3))
+    dsa.check_device_error()
+    bad = table.clone()
+    bad[1, 5] = 10 ** 6
+    dsa.index_topk_decode_paged(D.q_I, D.q_scale, D.w, k_pool, ks_pool, bad, D.lens, 2048, page_size=page)
+    st, _ = dsa.device_error()
+    assert st == -6  # DSA_ERR_BAD_INDEX
+    # the good sequence is unaffected
+    ref = dsa.index_topk_decode(D.q_I, D.q_scale, D.w, D.k_cache, D.k_scale, D.lens, 2048)
+    idx = dsa.index_topk_decode_paged(D.q_I, D.q_scale, D.w, k_pool, ks_pool, bad, D.lens, 2048, page_size=page)
+    dsa.device_error()
+    assert torch.equal(idx[0], ref[0])
