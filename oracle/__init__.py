@@ -211,3 +211,54 @@ def decode_seqs(inp, seqs):
         out, lse = sparse_mla(_bf16_bits(inp.q[b:b + 1]), inp.kv[b, :n], ix[None], inp.scale)
         res.append((sc, ix, out[0], lse[0]))
     return res
+
+
+# ---------------------------------------------------------------------------
+# Rotary position encoding of newly appended indexer queries / keys, before
+# their FP8 quantisation ("Lightning Indexer 的计算过程", step 2 <1>: the first
+# rope_head_dim = 64 dimensions of each query head and of the key are split
+# off, rotated by the token's position and joined back to the rest; step 2
+# <2>: the result is quantised to FP8 with a scale). The pages do not spell
+# the rotation out; this is the rotary encoding as its authors define it
+# (RoFormer): dimension pairs are rotated by pos * theta_i with
+# theta_i = base^(-2i / rope_dim), i < rope_dim / 2. Which dimensions form a
+# pair is a convention the pages leave open: consecutive dimensions
+# (2i, 2i+1) when `interleaved`, else (i, i + rope_dim/2).
+# ---------------------------------------------------------------------------
+
+def rope(x, pos, *, rope_dim: int = 64, base: float = 10000.0, interleaved: bool = True) -> np.ndarray:
+    """Rotate the first rope_dim dimensions of every head of x by its row's position.
+
+    x [n, H, d] or [n, d] (one head), pos [n] integer positions; returns float64
+    of x's shape. Dimensions >= rope_dim are returned unchanged.
+    """
+    xv = np.asarray(_np(x), dtype=np.float64)
+    squeeze = xv.ndim == 2
+    if squeeze:
+        xv = xv[:, None, :]
+    n, H, d = xv.shape
+    if rope_dim % 2 or rope_dim > d:
+        raise ValueError(f"rope_dim={rope_dim} must be even and <= d={d}")
+    p = np.asarray(_np(pos), dtype=np.int64).reshape(n)
+    half = rope_dim // 2
+    out = xv.copy()
+    for i in range(half):
+        theta = base ** (-2.0 * i / rope_dim)
+        ang = p.astype(np.float64) * theta  # exact product of an integer and a double, rounded once
+        c, s = np.cos(ang)[:, None], np.sin(ang)[:, None]
+        a_dim, b_dim = (2 * i, 2 * i + 1) if interleaved else (i, i + half)
+        a, b = xv[:, :, a_dim], xv[:, :, b_dim]
+        out[:, :, a_dim] = a * c - b * s
+        out[:, :, b_dim] = a * s + b * c
+    return out[:, 0, :] if squeeze else out
+
+
+def rope_quantize_e4m3(x, pos, *, rope_dim: int = 64, base: float = 10000.0, interleaved: bool = True) -> tuple:
+    """RoPE, then the per-row FP8 quantiser: x [n, H, d] or [n, d] fp32 ->
+    (codes uint8 of x's shape, scale fp32 [n]). The rotated row is rounded to
+    fp32 (the quantiser's input precision) and quantised with one scale over
+    all of the row's H * d values."""
+    r = rope(x, pos, rope_dim=rope_dim, base=base, interleaved=interleaved)
+    shape = r.shape
+    codes, scale = quantize_e4m3(r.reshape(shape[0], -1).astype(np.float32))
+    return codes.reshape(shape), scale

@@ -298,3 +298,98 @@ def test_row_quantiser_matches_the_input_recipe():
     ref_codes, ref_scale = workloads.quantize_e4m3_per_token(x)
     assert np.array_equal(scale, ref_scale.numpy())
     assert np.array_equal(codes, ref_codes.numpy())
+
+
+# --- rotary position encoding of appended tokens ---------------------------
+
+def _rope_inputs(n=5, H=3, d=128, seed=3):
+    rng = np.random.default_rng(seed)
+    return rng.standard_normal((n, H, d)), rng.integers(0, 131072, size=n)
+
+
+def test_rope_position_zero_is_the_identity():
+    x, _ = _rope_inputs()
+    assert np.array_equal(oracle.rope(x, np.zeros(len(x), dtype=np.int64)), x)
+
+
+def test_rope_first_pair_turns_by_the_position_in_radians():
+    # theta_0 = base^0 = 1: the unit vector (1, 0) at position p becomes (cos p, sin p)
+    x = np.zeros((4, 128))
+    x[:, 0] = 1.0
+    pos = np.array([1, 2, 7, 100000])
+    r = oracle.rope(x, pos)
+    assert np.allclose(r[:, 0], [math.cos(p) for p in pos], rtol=0, atol=1e-12)
+    assert np.allclose(r[:, 1], [math.sin(p) for p in pos], rtol=0, atol=1e-12)  # counter-clockwise
+
+
+def test_rope_equals_complex_multiplication():
+    # each pair as the complex number a + ib, multiplied by exp(i * p * theta_i)
+    x, pos = _rope_inputs()
+    r = oracle.rope(x, pos)
+    z = x[..., 0:64:2] + 1j * x[..., 1:64:2]
+    rz = r[..., 0:64:2] + 1j * r[..., 1:64:2]
+    # the frequencies, recovered from a rotation at position 1 of the vector (1, 0)
+    e = np.zeros((1, 128))
+    e[0, 0:64:2] = 1.0
+    r1 = oracle.rope(e, [1])[0]
+    theta = np.arctan2(r1[1:64:2], r1[0:64:2])
+    want = z * np.exp(1j * pos[:, None, None] * theta[None, None, :])
+    assert np.abs(rz - want).max() < 1e-9
+    assert np.array_equal(r[..., 64:], x[..., 64:])  # the rest of each head is untouched
+
+
+def test_rope_frequencies_fall_geometrically_from_one_to_nearly_one_over_base():
+    e = np.zeros((1, 64))
+    e[0, 0::2] = 1.0
+    r1 = oracle.rope(e, [1], rope_dim=64, base=10000.0)[0]
+    theta = np.arctan2(r1[1::2], r1[0::2])
+    assert theta[0] == pytest.approx(1.0, abs=1e-15)
+    ratios = theta[1:] / theta[:-1]
+    assert np.allclose(ratios, 10000.0 ** (-1 / 32), rtol=1e-12)  # 32 pairs span base^(-31/32)
+    assert theta[-1] == pytest.approx(10000.0 ** (-31 / 32), rel=1e-12)
+
+
+def test_rope_scores_depend_on_the_relative_position_only():
+    rng = np.random.default_rng(5)
+    q, k = rng.standard_normal((1, 128)), rng.standard_normal((1, 128))
+    for m, n in [(5, 2), (1000, 10), (70000, 69999)]:
+        base_dot = float(oracle.rope(q, [m])[0] @ oracle.rope(k, [n])[0])
+        for c in (1, 333, 40000):
+            shifted = float(oracle.rope(q, [m + c])[0] @ oracle.rope(k, [n + c])[0])
+            assert shifted == pytest.approx(base_dot, rel=1e-9, abs=1e-9)
+
+
+def test_rope_rotations_compose_and_keep_pair_norms():
+    x, _ = _rope_inputs(n=3)
+    a, b = np.array([3, 500, 60000]), np.array([4, 12345, 7])
+    twice = oracle.rope(oracle.rope(x, a), b)
+    once = oracle.rope(x, a + b)
+    assert np.abs(twice - once).max() < 1e-9
+    norms = x[..., 0:64:2] ** 2 + x[..., 1:64:2] ** 2
+    rn = once[..., 0:64:2] ** 2 + once[..., 1:64:2] ** 2
+    assert np.allclose(rn, norms, rtol=1e-12)
+
+
+def test_rope_pair_layouts_are_one_permutation_apart():
+    # split-half pairs (i, i+32) are consecutive pairs after moving dim i to 2i and i+32 to 2i+1
+    x, pos = _rope_inputs()
+    perm = np.arange(128)
+    perm[0:64:2], perm[1:64:2] = np.arange(32), np.arange(32, 64)
+    inter = oracle.rope(x[..., perm], pos, interleaved=True)
+    half = oracle.rope(x, pos, interleaved=False)
+    assert np.abs(inter - half[..., perm]).max() < 1e-12
+
+
+def test_rope_quantiser_at_position_zero_is_the_plain_quantiser():
+    x, _ = _rope_inputs(n=4, H=2)
+    x32 = x.astype(np.float32)
+    codes, scale = oracle.rope_quantize_e4m3(x32, np.zeros(4, dtype=np.int64))
+    c0, s0 = oracle.quantize_e4m3(x32.reshape(4, -1))
+    assert np.array_equal(codes.reshape(4, -1), c0) and np.array_equal(scale, s0)
+    # and the codes stay within half a step of the rotated row (torch's decoder)
+    pos = np.array([1, 99, 4096, 131071])
+    codes, scale = oracle.rope_quantize_e4m3(x32, pos)
+    deq = _torch_dequant(codes.reshape(4, -1), scale)
+    ref = oracle.rope(x32, pos).reshape(4, -1)
+    step = np.where(np.abs(ref) >= 2.0 ** -6 * scale[:, None], np.abs(ref) / 8, 2.0 ** -9 * scale[:, None])
+    assert np.all(np.abs(deq - ref) <= 0.5 * step * 1.0001 + 1e-7 * np.abs(ref))
