@@ -115,7 +115,7 @@ struct MlaParams {
   int rows;                  // valid row bound of a token's cache
   int T, Hq, K;
   int causal_q0;             // position of token 0 when idx is null
-  // Paged latent cache: when block_table is set, logical row r of token i is
+  // Paged latent cache (the kernel's paged instance): logical row r of token i is
   // physical row block_table[i * bt_stride + (r >> page_shift)] * page + (r & (page - 1))
   // of kv (a pool of pool_rows rows); bt_stride 0 shares one table row.
   const int32_t* block_table;

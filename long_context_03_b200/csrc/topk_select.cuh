@@ -370,7 +370,6 @@ template <int P>
 __global__ void __launch_bounds__(P / 8) rank_sort_reg_kernel(const uint64_t* __restrict__ keys,
                                                                int32_t* __restrict__ idx, int K, int rows) {
   static_assert(P >= 256 && P <= 2048, "8 keys per thread, at least one warp");
-  constexpr int NT = P / 8;
   __shared__ uint64_t sm[P];
   const int r = blockIdx.x;
   if (r >= rows) return;
