@@ -95,3 +95,6 @@ def test_reference_arm_prints_one_contract_line():
         assert key in d, key
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["value"] > 0
+    # the same workload description as the GPU arm's line, so the two lines compare
+    import bench
+    assert d["config"] == bench.workload_config(bench.parse(["--prefill-L", "1024"]), 1)
