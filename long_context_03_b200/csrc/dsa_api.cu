@@ -784,7 +784,7 @@ dsa_status dsa_get_device_error(void* stream, unsigned int* detail) {
   if (e != cudaSuccess) return cuda_fail(e, "dsa_get_device_error (clear)");
   const unsigned int code = h & 0xFFu;
   if (code == kErrTimeout) return fail(DSA_ERR_TIMEOUT, "a kernel gave up waiting (site %u)", h >> 8);
-  return fail(DSA_ERR_BAD_INDEX, "an attention index was outside its cache (site %u)", h >> 8);
+  return fail(DSA_ERR_BAD_INDEX, "an index or page-table entry was outside its cache (site %u)", h >> 8);
 }
 
 const char* dsa_status_string(dsa_status s) {
