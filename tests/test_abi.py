@@ -135,3 +135,26 @@ def test_rope_quantiser_argument_checks(lib):
                                            None) == -1  # base
     assert lib.dsa_rope_quantize_e4m3_rows(None, p, 4, 64, 128, 64, b, 1, p, p, None, None) == -1  # null x
     assert lib.dsa_rope_quantize_e4m3_rows(None, None, 0, 64, 128, 64, b, 1, None, None, None, None) == 0  # empty
+
+
+def _declared_arity():
+    """Number of parameters of every function declared in include/dsa.h."""
+    src = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for name, args in re.findall(r"\b(dsa_[a-z_0-9]+)\s*\(([^)]*)\)\s*;", src):
+        args = args.strip()
+        out[name] = 0 if args in ("", "void") else args.count(",") + 1
+    return out
+
+
+def test_binding_declares_every_entry_with_its_arity(lib):
+    # the ctypes binding sets argtypes for each ABI call, with as many arguments as the header
+    import long_context_03_b200 as m
+    L = m.lib()
+    arity = _declared_arity()
+    assert len(arity) >= 20
+    for name, n in arity.items():
+        fn = getattr(L, name)
+        assert fn.argtypes is not None, name
+        assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
