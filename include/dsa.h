@@ -180,6 +180,22 @@ dsa_status dsa_sparse_mla_attn_paged(const uint16_t* q, const uint16_t* kv_pool,
  * [n, d] e4m3 bytes, scale [n] f32, all device memory. n = 0 is a no-op. */
 dsa_status dsa_quantize_e4m3_rows(const float* x, int n, int d, uint8_t* codes, float* scale, void* stream);
 
+/* RoPE + FP8 quantiser for newly appended indexer queries or keys
+ * ("Lightning Indexer 的计算过程", step 2 <1> then <2>). Row r of x [n, heads,
+ * d] f32 (device) has the first rope_dim dimensions of every head rotated by
+ * position pos[r] (pos [n] int32, device): pair i < rope_dim/2 turns by
+ * pos[r] * base^(-2i / rope_dim) radians, (a, b) -> (a cos - b sin, a sin +
+ * b cos), the pairs being dimensions (2i, 2i+1) when interleaved != 0, else
+ * (i, i + rope_dim/2); the other dimensions pass through. The rotation is
+ * evaluated in float64 and rounded once to fp32; the fp32 row is then
+ * quantised exactly as by dsa_quantize_e4m3_rows with one scale over its
+ * heads * d values. codes [n, heads * d] e4m3, scale [n] f32, rotated
+ * [n, heads * d] f32 or NULL (receives the fp32 rotated rows). rope_dim even,
+ * 2 <= rope_dim <= min(d, 128); base finite and > 0. n = 0 is a no-op. */
+dsa_status dsa_rope_quantize_e4m3_rows(const float* x, const int32_t* pos, int n, int heads, int d, int rope_dim,
+                                       double base, int interleaved, uint8_t* codes, float* scale, float* rotated,
+                                       void* stream);
+
 /* Short-sequence dense fallback: when a sequence has at most DSA_MAX_TOPK
  * tokens every causal key is selected anyway, so the indexer can be skipped
  * and token t (position q0 + t) attends to kv rows 0..q0+t directly, with the

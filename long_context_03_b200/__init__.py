@@ -59,6 +59,7 @@ def lib() -> ctypes.CDLL:
             L.dsa_sparse_mla_attn.argtypes = [P, P, P, I, I, I, I, F, P, P, P]
             L.dsa_dense_mla_attn_causal.argtypes = [P, P, I, I, I, I, F, P, P, P]
             L.dsa_quantize_e4m3_rows.argtypes = [P, I, I, P, P, P]
+            L.dsa_rope_quantize_e4m3_rows.argtypes = [P, P, I, I, I, I, ctypes.c_double, I, P, P, P, P]
             L.dsa_sparse_mla_attn_paged.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, F, P, P, P]
             L.dsa_index_topk_decode_workspace_size.argtypes = [I, I, I]
             L.dsa_index_topk_decode_workspace_size.restype = SZ
@@ -74,6 +75,7 @@ def lib() -> ctypes.CDLL:
             L.dsa_last_error.restype = ctypes.c_char_p
             for name in ("dsa_index_topk", "dsa_index_topk_rerun_count", "dsa_index_topk_chunk",
                          "dsa_index_topk_varlen", "dsa_dense_mla_attn_causal", "dsa_quantize_e4m3_rows",
+                         "dsa_rope_quantize_e4m3_rows",
                          "dsa_sparse_mla_attn_paged",
                          "dsa_index_scores", "dsa_sparse_mla_attn", "dsa_index_topk_decode",
                          "dsa_index_scores_decode", "dsa_sparse_mla_attn_decode", "dsa_get_device_error",
@@ -286,6 +288,30 @@ def quantize_e4m3_rows(x, *, codes=None, scale=None):
     _req(scale, "scale", torch.float32, (n,))
     _check(lib().dsa_quantize_e4m3_rows(_ptr(x), n, d, _ptr(codes), _ptr(scale), _stream(x.device)))
     return codes, scale
+
+
+def rope_quantize_e4m3_rows(x, pos, *, rope_dim: int = 64, base: float = 10000.0, interleaved: bool = True,
+                            codes=None, scale=None, want_rotated: bool = False):
+    """RoPE on the first rope_dim dims of each head, then the per-row E4M3 quantiser.
+
+    x [n, heads, d] (or [n, d]) f32, pos [n] int32 positions (device) -> (codes uint8 of x's shape,
+    scale f32 [n], rotated f32 of x's shape or None)."""
+    squeeze = x.dim() == 2
+    n = x.shape[0]
+    heads, d = (1, x.shape[1]) if squeeze else (x.shape[1], x.shape[2])
+    _req(x, "x", torch.float32, tuple(x.shape))
+    _req(pos, "pos", torch.int32, (n,))
+    if codes is None:
+        codes = torch.empty(tuple(x.shape), dtype=torch.uint8, device=x.device)
+    if scale is None:
+        scale = torch.empty((n,), dtype=torch.float32, device=x.device)
+    _req(codes, "codes", torch.uint8, tuple(x.shape))
+    _req(scale, "scale", torch.float32, (n,))
+    rotated = torch.empty(tuple(x.shape), dtype=torch.float32, device=x.device) if want_rotated else None
+    _check(lib().dsa_rope_quantize_e4m3_rows(_ptr(x), _ptr(pos), n, heads, d, rope_dim, float(base),
+                                             1 if interleaved else 0, _ptr(codes), _ptr(scale),
+                                             _ptr(rotated) if rotated is not None else None, _stream(x.device)))
+    return codes, scale, rotated
 
 
 def dense_mla_attn_causal(q, kv, scale: float, *, q0: int = 0, out=None, lse=None, want_lse: bool = False):

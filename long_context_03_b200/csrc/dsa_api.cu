@@ -596,6 +596,22 @@ dsa_status dsa_quantize_e4m3_rows(const float* x, int n, int d, uint8_t* codes, 
   return check_launch("quantize_e4m3_rows_kernel");
 }
 
+dsa_status dsa_rope_quantize_e4m3_rows(const float* x, const int32_t* pos, int n, int heads, int d, int rope_dim,
+                                       double base, int interleaved, uint8_t* codes, float* scale, float* rotated,
+                                       void* stream) {
+  if (n < 0 || heads <= 0 || d <= 0) return fail(DSA_ERR_INVALID_ARG, "n=%d heads=%d d=%d", n, heads, d);
+  if (static_cast<long long>(heads) * d >= (1ll << 31)) return fail(DSA_ERR_UNSUPPORTED, "heads*d too large");
+  if (rope_dim < 2 || (rope_dim & 1) || rope_dim > d || rope_dim > 2 * kRopeMaxHalf)
+    return fail(DSA_ERR_UNSUPPORTED, "rope_dim=%d must be even, in [2, min(d, %d)]", rope_dim, 2 * kRopeMaxHalf);
+  if (!std::isfinite(base) || !(base > 0.0)) return fail(DSA_ERR_INVALID_ARG, "base must be finite and > 0");
+  if (n == 0) return DSA_OK;
+  if (!x || !pos || !codes || !scale) return fail(DSA_ERR_INVALID_ARG, "null pointer");
+  const int grid = n < 8 * num_sms() ? n : 8 * num_sms();
+  rope_quantize_e4m3_rows_kernel<<<grid, kQuantThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      x, pos, n, heads, d, rope_dim, base, interleaved, codes, scale, rotated);
+  return check_launch("rope_quantize_e4m3_rows_kernel");
+}
+
 dsa_status dsa_dense_mla_attn_causal(const uint16_t* q, const uint16_t* kv, int T, int L, int q0, int Hq, float scale,
                                      uint16_t* out, float* lse, void* stream) {
   if (T < 0 || L <= 0 || q0 < 0 || static_cast<long long>(q0) + T > L)

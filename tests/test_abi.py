@@ -123,3 +123,15 @@ def test_paged_decode_indexer_argument_checks(lib):
                                            None) == -5  # no workspace
     assert lib.dsa_index_topk_decode_paged(p, p, p, p, p, p, p, 2, 8, 64, 1024, 32, 128, 16, p, p, 1 << 30,
                                            None) == -2  # H_I outside the supported set
+
+
+def test_rope_quantiser_argument_checks(lib):
+    p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    b = ctypes.c_double(10000.0)
+    # (x, pos, n, heads, d, rope_dim, base, interleaved, codes, scale, rotated, stream)
+    assert lib.dsa_rope_quantize_e4m3_rows(p, p, 4, 64, 128, 63, b, 1, p, p, None, None) == -2  # odd
+    assert lib.dsa_rope_quantize_e4m3_rows(p, p, 4, 64, 128, 256, b, 1, p, p, None, None) == -2  # > d
+    assert lib.dsa_rope_quantize_e4m3_rows(p, p, 4, 64, 128, 64, ctypes.c_double(-1.0), 1, p, p, None,
+                                           None) == -1  # base
+    assert lib.dsa_rope_quantize_e4m3_rows(None, p, 4, 64, 128, 64, b, 1, p, p, None, None) == -1  # null x
+    assert lib.dsa_rope_quantize_e4m3_rows(None, None, 0, 64, 128, 64, b, 1, None, None, None, None) == 0  # empty
