@@ -132,16 +132,23 @@ WsPrefill prefill_ws_layout(void* base, int L, int H_I, int topk, int grid) {
 // capacity: shorter rows rarely cut their lists anyway).
 int spec_min_row(int topk) { return 2 * select_cap(topk) > 4096 ? 2 * select_cap(topk) : 4096; }
 
-template <int HI, int DI, bool kSelect, int MQ>
+template <int HI, int DI, bool kSelect, int MQ, bool kPaged = false>
 dsa_status launch_prefill(const uint8_t* q_I, const uint8_t* k_cache, const IdxPrefillParams& p, int grid,
                           cudaStream_t st) {
   using C = IdxPrefillCfg<HI, DI>;
   CUtensorMap tmQ, tmK;
   dsa_status s = make_map_u8(&tmQ, q_I, DI, static_cast<uint64_t>(p.Tq) * HI, DI, C::NCOL);
   if (s != DSA_OK) return s;
-  s = make_map_u8(&tmK, k_cache, DI, static_cast<uint64_t>(p.L), DI, C::BM);
+  if (kPaged) {
+    // the pool's rows, one page (at most one key tile) per box
+    const int page = 1 << p.page_shift;
+    s = make_map_u8(&tmK, k_cache, DI, static_cast<uint64_t>(p.pool_pages) * page, DI,
+                    static_cast<uint32_t>(page < C::BM ? page : C::BM));
+  } else {
+    s = make_map_u8(&tmK, k_cache, DI, static_cast<uint64_t>(p.L), DI, C::BM);
+  }
   if (s != DSA_OK) return s;
-  auto kern = indexer_prefill_kernel<HI, DI, kSelect, MQ>;
+  auto kern = indexer_prefill_kernel<HI, DI, kSelect, MQ, kPaged>;
   s = set_smem(kern, C::SMEM_BYTES);
   if (s != DSA_OK) return s;
   kern<<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(tmQ, tmK, p);
@@ -151,6 +158,13 @@ dsa_status launch_prefill(const uint8_t* q_I, const uint8_t* k_cache, const IdxP
 template <bool kSelect, int MQ>
 dsa_status dispatch_prefill(int H_I, int d_I, const uint8_t* q_I, const uint8_t* k_cache, const IdxPrefillParams& p,
                             int grid, cudaStream_t st) {
+  if constexpr (kSelect) {
+    if (p.block_table) {  // paged key cache: the H_I = 64 shapes
+      if (H_I == 64 && d_I == 128) return launch_prefill<64, 128, true, MQ, true>(q_I, k_cache, p, grid, st);
+      if (H_I == 64 && d_I == 64) return launch_prefill<64, 64, true, MQ, true>(q_I, k_cache, p, grid, st);
+      return fail(DSA_ERR_UNSUPPORTED, "paged keys: H_I=%d d_I=%d not supported", H_I, d_I);
+    }
+  }
   if (H_I == 64 && d_I == 128) return launch_prefill<64, 128, kSelect, MQ>(q_I, k_cache, p, grid, st);
   if (H_I == 64 && d_I == 64) return launch_prefill<64, 64, kSelect, MQ>(q_I, k_cache, p, grid, st);
   if (H_I == 8 && d_I == 128) return launch_prefill<8, 128, kSelect, MQ>(q_I, k_cache, p, grid, st);
@@ -319,9 +333,15 @@ size_t dsa_index_topk_workspace_size(int L, int H_I, int d_I, int topk) {
 }
 
 // Queries r = 0..Tq-1 at positions q0 + r against keys 0..L-1 (q0 + Tq <= L).
+struct PrefillKeyPaging {
+  const int32_t* block_table = nullptr;
+  int page_shift = 0, pool_pages = 0;
+};
+
 static dsa_status index_topk_impl(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
                            const float* k_scale, int q0, int Tq, int L, int H_I, int d_I, int topk, int32_t* idx,
-                           void* workspace, size_t ws_bytes, cudaStream_t st) {
+                           void* workspace, size_t ws_bytes, cudaStream_t st,
+                           PrefillKeyPaging pg = PrefillKeyPaging()) {
   if (!q_I || !q_scale || !w || !k_cache || !k_scale || !idx) return fail(DSA_ERR_INVALID_ARG, "null pointer");
   if (L <= 0 || Tq <= 0 || q0 < 0 || static_cast<long long>(q0) + Tq > L)
     return fail(DSA_ERR_INVALID_ARG, "q0=%d Tq=%d L=%d (need q0 >= 0, Tq >= 1, q0 + Tq <= L)", q0, Tq, L);
@@ -352,6 +372,9 @@ static dsa_status index_topk_impl(const uint8_t* q_I, const float* q_scale, cons
   p.spec_min_t = spec_min_row(topk);
   p.redo_count = ws.redo;
   p.redo_list = ws.redo + 4;
+  p.block_table = pg.block_table;
+  p.page_shift = pg.page_shift;
+  p.pool_pages = pg.pool_pages;
   const cudaError_t me = cudaMemsetAsync(ws.redo, 0, sizeof(int), st);
   if (me != cudaSuccess) return cuda_fail(me, "cudaMemsetAsync");
   dsa_status s = (select_mq(topk) == 1) ? dispatch_prefill<true, 1>(H_I, d_I, q_I, k_cache, p, grid, st)
@@ -384,6 +407,26 @@ dsa_status dsa_index_topk_chunk(const uint8_t* q_I, const float* q_scale, const 
                                 void* workspace, size_t ws_bytes, void* stream) {
   return index_topk_impl(q_I, q_scale, w, k_cache, k_scale, q0, Tq, L, H_I, d_I, topk, idx, workspace, ws_bytes,
                          static_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_index_topk_chunk_paged(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_pool,
+                                      const float* k_scale_pool, const int32_t* block_table, int max_blocks,
+                                      int page_size, int pool_rows, int q0, int Tq, int L, int H_I, int d_I, int topk,
+                                      int32_t* idx, void* workspace, size_t ws_bytes, void* stream) {
+  if (!block_table) return fail(DSA_ERR_INVALID_ARG, "null pointer");
+  if (page_size < 16 || page_size > 4096 || (page_size & (page_size - 1)))
+    return fail(DSA_ERR_INVALID_ARG, "page_size=%d must be a power of two in [16, 4096]", page_size);
+  if (pool_rows <= 0 || pool_rows % page_size)
+    return fail(DSA_ERR_INVALID_ARG, "pool_rows=%d (a positive multiple of page_size)", pool_rows);
+  if (max_blocks <= 0 || static_cast<long long>(max_blocks) * page_size < L)
+    return fail(DSA_ERR_INVALID_ARG, "max_blocks=%d pages of %d rows do not cover L=%d", max_blocks, page_size, L);
+  if (H_I != 64) return fail(DSA_ERR_UNSUPPORTED, "paged keys: H_I=%d not supported", H_I);
+  PrefillKeyPaging pg;
+  pg.block_table = block_table;
+  pg.page_shift = __builtin_ctz(static_cast<unsigned>(page_size));
+  pg.pool_pages = pool_rows / page_size;
+  return index_topk_impl(q_I, q_scale, w, k_pool, k_scale_pool, q0, Tq, L, H_I, d_I, topk, idx, workspace, ws_bytes,
+                         static_cast<cudaStream_t>(stream), pg);
 }
 
 // ---- packed batch of sequences (cu_seqlens) ----

@@ -112,6 +112,11 @@ struct IdxPrefillParams {
   // score mode (test hook)
   float* scores;         // [nrows][L]; rows t in [row0, row0 + nrows)
   int row0, nrows;
+  // Paged key cache (the kernel's paged instance, one sequence): key s is pool
+  // row block_table[s >> page_shift] * page + (s & (page - 1)) of the FP8 keys
+  // and of k_scale; the pool holds pool_pages pages.
+  const int32_t* block_table;
+  int page_shift, pool_pages;
 };
 
 // sum_j w[j] * max(x_j, 0) over the H_I accumulator values of one token
@@ -154,7 +159,22 @@ __device__ __forceinline__ int sample_rank(int topk, int sampled_keys, int t, in
   return static_cast<int>(r);
 }
 
-template <int HI, int DI, bool kSelect, int MQ>
+// Paged key cache: the page-table entry of key s (-1 past the cache), and the
+// pool row a box starting at key s reads (the pool's end, which TMA fills
+// with zeros, past the cache or behind a bad entry).
+__device__ __forceinline__ int prefill_page_entry(const IdxPrefillParams& p, int s, int L) {
+  return (s < L) ? __ldg(p.block_table + (s >> p.page_shift)) : -1;
+}
+__device__ __forceinline__ int prefill_pool_row(const IdxPrefillParams& p, int s, int L, int page) {
+  if (s >= L) return p.pool_pages << p.page_shift;
+  if (page < 0 || page >= p.pool_pages) {
+    set_device_error(kErrBadIndex, 3);
+    return p.pool_pages << p.page_shift;
+  }
+  return (page << p.page_shift) + (s & ((1 << p.page_shift) - 1));
+}
+
+template <int HI, int DI, bool kSelect, int MQ, bool kPaged = false>
 __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
     indexer_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                            const IdxPrefillParams p) {
@@ -260,11 +280,41 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
         for (int b = 0; b < C::NACC; ++b)
           tma_load_2d(q_s + b * C::QBUF_BYTES, &tmQ, q_full, 0, (r0 + b * C::TB) * HI);
         bool ok = true;
+        // paged: one box of R = min(page, BM) rows per page of the tile; the
+        // next tile's page entries load before the wait for this tile's slot
+        constexpr int MAXB = C::BM / 16;
+        [[maybe_unused]] const int R = kPaged ? min(1 << p.page_shift, C::BM) : C::BM;
+        [[maybe_unused]] int nxt[MAXB];
+        if constexpr (kPaged) {
+#pragma unroll
+          for (int q = 0; q < MAXB; ++q)
+            nxt[q] = (q * R < C::BM) ? prefill_page_entry(p, tile_at<C::NSAMPLE>(0, nkt, spec) * C::BM + q * R, bk.L)
+                                     : -1;
+        }
         for (int i = 0; i < nsteps; ++i) {
+          [[maybe_unused]] int cur[MAXB];
+          if constexpr (kPaged) {
+#pragma unroll
+            for (int q = 0; q < MAXB; ++q) cur[q] = nxt[q];
+            if (i + 1 < nsteps) {
+              const int sn = tile_at<C::NSAMPLE>(i + 1, nkt, spec) * C::BM;
+#pragma unroll
+              for (int q = 0; q < MAXB; ++q) nxt[q] = (q * R < C::BM) ? prefill_page_entry(p, sn + q * R, bk.L) : -1;
+            }
+          }
           if (!mbar_wait(k_empty + kslot, ke_phase, ab, 2)) { ok = false; break; }
           mbar_arrive_expect_tx(k_full + kslot, C::KTILE_BYTES);
-          tma_load_2d(k_s + kslot * C::KTILE_BYTES, &tmK, k_full + kslot, 0,
-                      bk.kbase + tile_at<C::NSAMPLE>(i, nkt, spec) * C::BM);
+          if constexpr (kPaged) {
+            const int sc = tile_at<C::NSAMPLE>(i, nkt, spec) * C::BM;
+#pragma unroll
+            for (int q = 0; q < MAXB; ++q)
+              if (q * R < C::BM)
+                tma_load_2d(k_s + kslot * C::KTILE_BYTES + q * R * DI, &tmK, k_full + kslot, 0,
+                            prefill_pool_row(p, sc + q * R, bk.L, cur[q]));
+          } else {
+            tma_load_2d(k_s + kslot * C::KTILE_BYTES, &tmK, k_full + kslot, 0,
+                        bk.kbase + tile_at<C::NSAMPLE>(i, nkt, spec) * C::BM);
+          }
           if (++kslot == C::KST) { kslot = 0; ke_phase ^= 1; }
         }
         if (!ok) break;
@@ -368,9 +418,20 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
       named_bar_sync(1, C::NET);
       bool ok = true;
       float ks_next = 0.f;
+      // paged: page entry of the key two steps ahead, its scale one step ahead
+      // (no dependent load waits inside a step)
+      [[maybe_unused]] int pg_next = -1;
       {
         const int s0 = tile_at<C::NSAMPLE>(0, nkt, spec) * C::BM + quarter * 32 + static_cast<int>(lane);
-        ks_next = (s0 < bk.L) ? __ldg(p.k_scale + bk.kbase + s0) : 0.f;
+        if constexpr (kPaged) {
+          const int r = prefill_pool_row(p, s0, bk.L, prefill_page_entry(p, s0, bk.L));
+          ks_next = (s0 < bk.L && r < (p.pool_pages << p.page_shift)) ? __ldg(p.k_scale + r) : 0.f;
+          if (1 < nsteps)
+            pg_next = prefill_page_entry(
+                p, tile_at<C::NSAMPLE>(1, nkt, spec) * C::BM + quarter * 32 + static_cast<int>(lane), bk.L);
+        } else {
+          ks_next = (s0 < bk.L) ? __ldg(p.k_scale + bk.kbase + s0) : 0.f;
+        }
       }
       for (int i = 0; i < nsteps && ok; ++i) {
         const int kt = tile_at<C::NSAMPLE>(i, nkt, spec);
@@ -378,7 +439,15 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
         const float ks = ks_next;
         if (i + 1 < nsteps) {
           const int sn = tile_at<C::NSAMPLE>(i + 1, nkt, spec) * C::BM + quarter * 32 + static_cast<int>(lane);
-          ks_next = (sn < bk.L) ? __ldg(p.k_scale + bk.kbase + sn) : 0.f;
+          if constexpr (kPaged) {
+            const int r = prefill_pool_row(p, sn, bk.L, pg_next);
+            ks_next = (sn < bk.L && r < (p.pool_pages << p.page_shift)) ? __ldg(p.k_scale + r) : 0.f;
+            if (i + 2 < nsteps)
+              pg_next = prefill_page_entry(
+                  p, tile_at<C::NSAMPLE>(i + 2, nkt, spec) * C::BM + quarter * 32 + static_cast<int>(lane), bk.L);
+          } else {
+            ks_next = (sn < bk.L) ? __ldg(p.k_scale + bk.kbase + sn) : 0.f;
+          }
         }
         for (int b = 0; b < C::NACC; ++b) {
           if (!mbar_wait(acc_full + b, af_phase[b], ab, 8)) { ok = false; break; }
