@@ -70,6 +70,7 @@ def lib() -> ctypes.CDLL:
             L.dsa_sparse_mla_attn_decode.argtypes = [P, P, P, I, I, I, I, F, P, P, P]
             L.dsa_index_topk_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P, P]
             L.dsa_get_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_uint)]
+            L.dsa_selftest_wait_timeout.argtypes = [P]
             L.dsa_status_string.argtypes = [I]
             L.dsa_status_string.restype = ctypes.c_char_p
             L.dsa_last_error.argtypes = []
@@ -81,7 +82,8 @@ def lib() -> ctypes.CDLL:
                          "dsa_sparse_mla_attn_paged",
                          "dsa_index_scores", "dsa_sparse_mla_attn", "dsa_index_topk_decode",
                          "dsa_index_scores_decode", "dsa_sparse_mla_attn_decode", "dsa_get_device_error",
-                         "dsa_index_topk_decode_noalloc", "dsa_index_topk_decode_paged"):
+                         "dsa_index_topk_decode_noalloc", "dsa_index_topk_decode_paged",
+                         "dsa_selftest_wait_timeout"):
                 getattr(L, name).restype = I
             _lib = L
     return _lib
@@ -480,6 +482,12 @@ def device_error(device=None) -> Tuple[int, int]:
     detail = ctypes.c_uint(0)
     st = lib().dsa_get_device_error(_stream(device), ctypes.byref(detail))
     return int(st), int(detail.value)
+
+
+def selftest_wait_timeout(device=None):
+    """Enqueue the failure-path self-test: a kernel whose bounded wait runs out
+    (~1 s) and records DSA_ERR_TIMEOUT; read it with device_error()."""
+    _check(lib().dsa_selftest_wait_timeout(_stream(device)))
 
 
 def check_device_error(device=None):

@@ -189,6 +189,26 @@ __global__ void fill_f32_kernel(float* p, size_t n, float v) {
     p[i] = v;
 }
 
+// ---- failure-path self-test ----
+// One CTA waits, with the library's bounded wait, on an mbarrier that no
+// thread arrives on: the wait gives up after its bound (~2^31 cycles), records
+// a timeout with site kSelftestSite in the device error word and the kernel
+// returns, leaving the context usable.
+constexpr unsigned int kSelftestSite = 99;
+__global__ void selftest_wait_timeout_kernel() {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const AbortFlag ab{&abort_flag};
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, ab, kSelftestSite);
+  __syncthreads();
+}
+
 // ---- decode ----
 
 template <int HI, int DI>
@@ -843,7 +863,12 @@ dsa_status dsa_get_device_error(void* stream, unsigned int* detail) {
   if (e != cudaSuccess) return cuda_fail(e, "dsa_get_device_error (clear)");
   const unsigned int code = h & 0xFFu;
   if (code == kErrTimeout) return fail(DSA_ERR_TIMEOUT, "a kernel gave up waiting (site %u)", h >> 8);
-  return fail(DSA_ERR_BAD_INDEX, "an attention index was outside its cache (site %u)", h >> 8);
+  return fail(DSA_ERR_BAD_INDEX, "an index or page-table entry was outside its cache (site %u)", h >> 8);
+}
+
+dsa_status dsa_selftest_wait_timeout(void* stream) {
+  selftest_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+  return check_launch("selftest_wait_timeout_kernel");
 }
 
 const char* dsa_status_string(dsa_status s) {

@@ -150,3 +150,8 @@ def test_paged_prefill_chunk_argument_checks(lib):
     assert lib.dsa_index_topk_chunk_paged(*short_table) == -1
     heads8 = list(args); heads8[12] = 8
     assert lib.dsa_index_topk_chunk_paged(*heads8) == -2
+
+
+def test_error_strings_cover_every_status(lib):
+    for st in (0, -1, -2, -3, -4, -5, -6):
+        assert lib.dsa_status_string(st) not in (None, b"unknown status")
