@@ -43,7 +43,7 @@ typedef enum {
   DSA_ERR_CUDA = -3,        /* a CUDA call or launch failed (see dsa_last_error) */
   DSA_ERR_TIMEOUT = -4,     /* reported by dsa_get_device_error: a kernel gave up on a wait */
   DSA_ERR_WORKSPACE = -5,   /* workspace null or smaller than the *_workspace_size() result */
-  DSA_ERR_BAD_INDEX = -6    /* reported by dsa_get_device_error: an index outside its cache */
+  DSA_ERR_BAD_INDEX = -6    /* reported by dsa_get_device_error: an index or page entry outside its cache */
 } dsa_status;
 
 /* Latent row geometry of the MLA cache (576 = 512 latent + 64 RoPE values). */
