@@ -113,6 +113,18 @@ def _req(t: torch.Tensor, name: str, dtype, shape=None):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
 
 
+def _ws(workspace, need: int, device) -> torch.Tensor:
+    """The caller's workspace (a contiguous CUDA tensor on the inputs' device; the
+    library checks its size and alignment) or a new one of `need` bytes."""
+    if workspace is None:
+        return torch.empty(max(need, 16), dtype=torch.uint8, device=device)
+    if not isinstance(workspace, torch.Tensor) or not workspace.is_cuda or workspace.device != device:
+        raise ValueError(f"workspace must be a CUDA tensor on {device}")
+    if not workspace.is_contiguous():
+        raise ValueError("workspace must be contiguous")
+    return workspace
+
+
 def _u8(t: torch.Tensor) -> torch.Tensor:
     return t.view(torch.uint8) if t.dtype == torch.float8_e4m3fn else t
 
@@ -136,8 +148,7 @@ def index_topk(q_I, q_scale, w, k_cache, k_scale, topk: int, *, idx=None, worksp
         idx = torch.empty((L, topk), dtype=torch.int32, device=q_I.device)
     _req(idx, "idx", torch.int32, (L, topk))
     need = index_topk_workspace_size(L, H_I, d_I, topk)
-    if workspace is None:
-        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q_I.device)
+    workspace = _ws(workspace, need, q_I.device)
     _check(lib().dsa_index_topk(_ptr(q_I), _ptr(q_scale), _ptr(w), _ptr(k_cache), _ptr(k_scale), L, H_I, d_I,
                                 topk, _ptr(idx), _ptr(workspace), workspace.numel() * workspace.element_size(),
                                 _stream(q_I.device)))
@@ -159,8 +170,7 @@ def index_topk_chunk(q_I, q_scale, w, k_cache, k_scale, q0: int, topk: int, *, i
         idx = torch.empty((Tq, topk), dtype=torch.int32, device=q_I.device)
     _req(idx, "idx", torch.int32, (Tq, topk))
     need = index_topk_workspace_size(Tq, H_I, d_I, topk)
-    if workspace is None:
-        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q_I.device)
+    workspace = _ws(workspace, need, q_I.device)
     _check(lib().dsa_index_topk_chunk(_ptr(q_I), _ptr(q_scale), _ptr(w), _ptr(k_cache), _ptr(k_scale), q0, Tq, L,
                                       H_I, d_I, topk, _ptr(idx), _ptr(workspace),
                                       workspace.numel() * workspace.element_size(), _stream(q_I.device)))
@@ -217,8 +227,7 @@ def index_topk_varlen(q_I, q_scale, w, k_cache, k_scale, cu_q, cu_k, topk: int, 
         idx = torch.empty((total_q, topk), dtype=torch.int32, device=q_I.device)
     _req(idx, "idx", torch.int32, (total_q, topk))
     need = int(lib().dsa_index_topk_varlen_workspace_size(total_q, nseq, H_I, d_I, topk))
-    if workspace is None:
-        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q_I.device)
+    workspace = _ws(workspace, need, q_I.device)
     IA = ctypes.c_int32 * (nseq + 1)
     cq, ck = IA(*cu_q), IA(*cu_k)
     qp = None if q_pos0 is None else (ctypes.c_int32 * nseq)(*[int(x) for x in q_pos0])
@@ -234,6 +243,8 @@ def index_topk_rerun_count(workspace, L: int, H_I: int, d_I: int, topk: int) -> 
     """Test hook: row blocks the last index_topk call with this workspace recomputed
     because their sampled starting threshold was too high (synchronises)."""
     n = ctypes.c_int(0)
+    if not isinstance(workspace, torch.Tensor) or not workspace.is_cuda:
+        raise ValueError("workspace must be a CUDA tensor")
     _check(lib().dsa_index_topk_rerun_count(_ptr(workspace), L, H_I, d_I, topk, ctypes.byref(n),
                                             _stream(workspace.device)))
     return int(n.value)
@@ -391,8 +402,7 @@ def index_topk_decode(q_I, q_scale, w, k_cache, k_scale, lens, topk: int, *, idx
         idx = torch.empty((B, topk), dtype=torch.int32, device=q_I.device)
     _req(idx, "idx", torch.int32, (B, topk))
     need = index_topk_decode_workspace_size(B, L_max, topk)
-    if workspace is None:
-        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q_I.device)
+    workspace = _ws(workspace, need, q_I.device)
     _check(lib().dsa_index_topk_decode(_ptr(q_I), _ptr(q_scale), _ptr(w), _ptr(k_cache), _ptr(k_scale),
                                        _ptr(lens), B, L_max, H_I, d_I, topk, _ptr(idx), _ptr(workspace),
                                        workspace.numel() * workspace.element_size(), _stream(q_I.device)))
@@ -420,8 +430,7 @@ def index_topk_decode_paged(q_I, q_scale, w, k_pool, k_scale_pool, block_table, 
         idx = torch.empty((B, topk), dtype=torch.int32, device=q_I.device)
     _req(idx, "idx", torch.int32, (B, topk))
     need = index_topk_decode_workspace_size(B, max_blocks * page_size, topk)
-    if workspace is None:
-        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q_I.device)
+    workspace = _ws(workspace, need, q_I.device)
     _check(lib().dsa_index_topk_decode_paged(_ptr(q_I), _ptr(q_scale), _ptr(w), _ptr(k_pool), _ptr(k_scale_pool),
                                              _ptr(block_table), _ptr(lens), B, max_blocks, page_size, pool_rows,
                                              H_I, d_I, topk, _ptr(idx), _ptr(workspace),
