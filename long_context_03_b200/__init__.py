@@ -196,8 +196,7 @@ def index_topk_chunk_paged(q_I, q_scale, w, k_pool, k_scale_pool, block_table, q
         idx = torch.empty((Tq, topk), dtype=torch.int32, device=q_I.device)
     _req(idx, "idx", torch.int32, (Tq, topk))
     need = index_topk_workspace_size(Tq, H_I, d_I, topk)
-    if workspace is None:
-        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q_I.device)
+    workspace = _ws(workspace, need, q_I.device)
     _check(lib().dsa_index_topk_chunk_paged(_ptr(q_I), _ptr(q_scale), _ptr(w), _ptr(k_pool), _ptr(k_scale_pool),
                                             _ptr(bt), bt.numel(), page_size, pool_rows, q0, Tq, L, H_I, d_I, topk,
                                             _ptr(idx), _ptr(workspace), workspace.numel() * workspace.element_size(),
