@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <algorithm>
+#include <atomic>
 #include <vector>
 #include <cstdio>
 #include <cstring>
@@ -311,7 +312,10 @@ dsa_status launch_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
   auto kern = pg.block_table ? sparse_mla_kernel<true> : sparse_mla_kernel<false>;
   dsa_status s = set_smem(kern, MlaCfg::SMEM_BYTES);
   if (s != DSA_OK) return s;
-  static int max_clusters = 0;  // the same for both instances (same resources)
+  // co-resident clusters, looked up once (the same for both instances: same
+  // resources); concurrent first calls compute the same value
+  static std::atomic<int> max_clusters_cache{0};
+  int max_clusters = max_clusters_cache.load(std::memory_order_relaxed);
   if (max_clusters == 0) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * 512, 1, 1);
@@ -323,6 +327,7 @@ dsa_status launch_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
       n = num_sms() / 2;
     }
     max_clusters = n;
+    max_clusters_cache.store(n, std::memory_order_relaxed);
   }
   const int nclusters = T < max_clusters ? T : max_clusters;
   kern<<<2 * nclusters, MlaCfg::NTHREADS, MlaCfg::SMEM_BYTES, st>>>(p);

@@ -155,3 +155,26 @@ def test_paged_prefill_chunk_argument_checks(lib):
 def test_error_strings_cover_every_status(lib):
     for st in (0, -1, -2, -3, -4, -5, -6):
         assert lib.dsa_status_string(st) not in (None, b"unknown status")
+
+
+def _declared_arity():
+    """Number of parameters of every function declared in include/dsa.h."""
+    src = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for name, args in re.findall(r"\b(dsa_[a-z_0-9]+)\s*\(([^)]*)\)\s*;", src):
+        args = args.strip()
+        out[name] = 0 if args in ("", "void") else args.count(",") + 1
+    return out
+
+
+def test_binding_declares_every_entry_with_its_arity(lib):
+    # the ctypes binding sets argtypes for each ABI call, with as many arguments as the header
+    import long_context_03_b200 as m
+    L = m.lib()
+    arity = _declared_arity()
+    assert len(arity) >= 20
+    for name, n in arity.items():
+        fn = getattr(L, name)
+        assert fn.argtypes is not None, name
+        assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
