@@ -264,12 +264,14 @@ dsa_status decode_scores(const uint8_t* q_I, const float* q_scale, const float* 
   return fail(DSA_ERR_UNSUPPORTED, "decode: H_I=%d d_I=%d not supported", H_I, d_I);
 }
 
+// Selection and ranking of every sequence's top-k: one CTA per sequence
+// selects, then sorts its keys in shared memory and writes idx.
 dsa_status launch_decode_select(const float* scores, const int32_t* lens, int L_max, int topk, const uint32_t* hist,
-                                uint64_t* sel, int B, cudaStream_t st) {
+                                uint64_t* sel, int32_t* idx, int B, cudaStream_t st) {
   const int smem = kDecodeSelBinCap * 8 + (2048 + select_scratch_ints(kDecodeSelThreads)) * 4;
   dsa_status s = set_smem(decode_select_kernel, smem);
   if (s != DSA_OK) return s;
-  decode_select_kernel<<<B, kDecodeSelThreads, smem, st>>>(scores, lens, L_max, topk, hist, sel);
+  decode_select_kernel<<<B, kDecodeSelThreads, smem, st>>>(scores, lens, L_max, topk, hist, sel, idx);
   return check_launch("decode_select_kernel");
 }
 
@@ -730,9 +732,7 @@ dsa_status dsa_index_topk_decode(const uint8_t* q_I, const float* q_scale, const
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(histogram)");
   s = decode_scores(q_I, q_scale, w, k_cache, k_scale, lens, B, L_max, H_I, d_I, scores, hist, st);
   if (s != DSA_OK) return s;
-  s = launch_decode_select(scores, lens, L_max, topk, hist, sel, B, st);
-  if (s != DSA_OK) return s;
-  return launch_rank_sort(sel, idx, topk, B, st);
+  return launch_decode_select(scores, lens, L_max, topk, hist, sel, idx, B, st);
 }
 
 dsa_status dsa_index_topk_decode_paged(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_pool,
@@ -770,9 +770,7 @@ dsa_status dsa_index_topk_decode_paged(const uint8_t* q_I, const float* q_scale,
   pg.pool_pages = pool_rows / page_size;
   s = decode_scores(q_I, q_scale, w, k_pool, k_scale_pool, lens, B, L_max, H_I, d_I, scores, hist, st, pg);
   if (s != DSA_OK) return s;
-  s = launch_decode_select(scores, lens, L_max, topk, hist, sel, B, st);
-  if (s != DSA_OK) return s;
-  return launch_rank_sort(sel, idx, topk, B, st);
+  return launch_decode_select(scores, lens, L_max, topk, hist, sel, idx, B, st);
 }
 
 dsa_status dsa_index_scores_decode(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
@@ -849,9 +847,7 @@ dsa_status dsa_index_topk_decode_noalloc(const uint8_t* q_I, const float* q_scal
   uint64_t* sel = reinterpret_cast<uint64_t*>(reinterpret_cast<char*>(base) + kNoAllocScoreBytes);
   s = decode_scores(q_I, q_scale, w, k_cache, k_scale, lens, B, L_max, H_I, d_I, scores, nullptr, st);
   if (s != DSA_OK) return s;
-  s = launch_decode_select(scores, lens, L_max, topk, nullptr, sel, B, st);
-  if (s != DSA_OK) return s;
-  return launch_rank_sort(sel, idx, topk, B, st);
+  return launch_decode_select(scores, lens, L_max, topk, nullptr, sel, idx, B, st);
 }
 
 dsa_status dsa_get_device_error(void* stream, unsigned int* detail) {
