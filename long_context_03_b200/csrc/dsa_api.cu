@@ -85,6 +85,23 @@ dsa_status make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_
   return DSA_OK;
 }
 
+// Queries [T, Hq, 576] bf16 as a 3-D map {576, Hq, T}; boxes of 64 values x
+// 128 heads x 1 token, 128-byte swizzled (heads >= Hq lie outside the map and
+// load as zeros).
+dsa_status make_map_q_bf16(CUtensorMap* m, const void* base, int T, int Hq) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[3] = {576, static_cast<cuuint64_t>(Hq), static_cast<cuuint64_t>(T)};
+  const cuuint64_t strides[2] = {576 * 2, static_cast<cuuint64_t>(Hq) * 576 * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled(q) failed (%d)", static_cast<int>(r));
+  return DSA_OK;
+}
+
 template <typename K>
 dsa_status set_smem(K kernel, int bytes) {
   const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -311,8 +328,11 @@ dsa_status launch_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
   p.page_shift = pg.page_shift;
   p.pool_rows = pg.pool_rows;
   p.scale_log2 = scale * 1.4426950408889634f;
+  CUtensorMap tmQ;
+  dsa_status s = make_map_q_bf16(&tmQ, q, T, Hq);
+  if (s != DSA_OK) return s;
   auto kern = pg.block_table ? sparse_mla_kernel<true> : sparse_mla_kernel<false>;
-  dsa_status s = set_smem(kern, MlaCfg::SMEM_BYTES);
+  s = set_smem(kern, MlaCfg::SMEM_BYTES);
   if (s != DSA_OK) return s;
   // co-resident clusters, looked up once (the same for both instances: same
   // resources); concurrent first calls compute the same value
@@ -332,7 +352,7 @@ dsa_status launch_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
     max_clusters_cache.store(n, std::memory_order_relaxed);
   }
   const int nclusters = T < max_clusters ? T : max_clusters;
-  kern<<<2 * nclusters, MlaCfg::NTHREADS, MlaCfg::SMEM_BYTES, st>>>(p);
+  kern<<<2 * nclusters, MlaCfg::NTHREADS, MlaCfg::SMEM_BYTES, st>>>(tmQ, p);
   return check_launch("sparse_mla_kernel");
 }
 
