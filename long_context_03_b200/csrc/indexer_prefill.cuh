@@ -120,22 +120,32 @@ struct IdxPrefillParams {
 };
 
 // sum_j w[j] * max(x_j, 0) over the H_I accumulator values of one token
-// (registers loaded from TMEM), into eight independent partial sums (head j
-// goes to sum j % 8) added in a fixed order at the end. Scalar FMAs: the
-// packed two-lane form needs its operands in aligned register pairs, which
-// cost a register move per ReLU output. Shared by both modes so their scores
-// are bit-identical.
+// (registers loaded from TMEM), written as (sum_j w[j]*x_j + sum_j w[j]*|x_j|)/2
+// so that both sums run on the FMA pipe: acc[0..3] take w*x as two packed
+// float pairs (fma.rn.f32x2 on register pairs straight from the TMEM load),
+// acc[4..7] take w*|x| with the absolute value folded into the scalar FMA.
+// The halves cancel exactly where every head is negative (an exact zero stays
+// zero). Shared by both modes so their scores are bit-identical.
 template <int HI>
 __device__ __forceinline__ void relu_weighted_acc(float (&acc)[8], const uint32_t* x, const float* __restrict__ w) {
-  static_assert(HI % 8 == 0, "a multiple of 8 heads");
+  static_assert(HI % 4 == 0, "a multiple of 4 heads");
 #pragma unroll
-  for (int j = 0; j < HI; j += 8) {
+  for (int j = 0; j < HI; j += 4) {
 #pragma unroll
-    for (int a = 0; a < 8; ++a) acc[a] = __fmaf_rn(w[j + a], fmaxf(__uint_as_float(x[j + a]), 0.f), acc[a]);
+    for (int pr = 0; pr < 2; ++pr) {
+      uint64_t d, wa, xa, ca;
+      asm("mov.b64 %0, {%1, %2};" : "=l"(wa) : "f"(w[j + 2 * pr]), "f"(w[j + 2 * pr + 1]));
+      asm("mov.b64 %0, {%1, %2};" : "=l"(xa) : "r"(x[j + 2 * pr]), "r"(x[j + 2 * pr + 1]));
+      asm("mov.b64 %0, {%1, %2};" : "=l"(ca) : "f"(acc[2 * pr]), "f"(acc[2 * pr + 1]));
+      asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(wa), "l"(xa), "l"(ca));
+      asm("mov.b64 {%0, %1}, %2;" : "=f"(acc[2 * pr]), "=f"(acc[2 * pr + 1]) : "l"(d));
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a) acc[4 + a] = __fmaf_rn(w[j + a], fabsf(__uint_as_float(x[j + a])), acc[4 + a]);
   }
 }
 __device__ __forceinline__ float relu_weighted_finish(const float (&acc)[8]) {
-  return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+  return 0.5f * (((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7])));
 }
 
 // Key tile of step i of a row block's sequence: with sampling, steps
