@@ -6,6 +6,7 @@ benchmark's allocations.
     python -m long_context_03_b200.run_kernel attention --L 16384
     python -m long_context_03_b200.run_kernel decode --B 64 --L 65536
     python -m long_context_03_b200.run_kernel decode_paged --B 64 --L 65536 --page 64
+    python -m long_context_03_b200.run_kernel rope --B 64        # RoPE + E4M3 of B appended query rows
 
 Prints the mean CUDA-event time of the calls after the warm-up ones. Inputs come from the seeded
 generators of the benchmark (`workloads`); the indexer case uses a single
@@ -45,7 +46,7 @@ def _time(fn, repeat):
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("op", choices=["indexer", "attention", "decode", "decode_paged"])
+    ap.add_argument("op", choices=["indexer", "attention", "decode", "decode_paged", "rope"])
     ap.add_argument("--L", type=int, default=65536)
     ap.add_argument("--B", type=int, default=64)
     ap.add_argument("--topk", type=int, default=2048)
@@ -64,6 +65,18 @@ def main(argv=None):
         idx = dsa.index_topk(P.q_I, P.q_scale, P.w, P.k_cache, P.k_scale, a.topk)
         out = torch.empty((a.L, 128, 512), dtype=torch.bfloat16, device=dev)
         ms = _time(lambda: dsa.sparse_mla_attn(P.q, P.kv, idx, P.scale, out=out), a.repeat)
+    elif a.op == "rope":
+        # B appended tokens: indexer queries [B, 64, 128] and keys [B, 128], rotated and quantised
+        g = torch.Generator(device=dev).manual_seed(0)
+        xq = torch.randn((a.B, 64, 128), generator=g, device=dev)
+        xk = torch.randn((a.B, 128), generator=g, device=dev)
+        pos = torch.randint(0, a.L, (a.B,), generator=g, device=dev, dtype=torch.int32)
+
+        def step():
+            dsa.rope_quantize_e4m3_rows(xq, pos)
+            dsa.rope_quantize_e4m3_rows(xk, pos)
+
+        ms = _time(step, a.repeat)
     elif a.op == "decode_paged":
         # both caches in one shuffled pool of pages (every sequence full length)
         D = workloads.make_decode(a.B, a.L, 64, 128, 128, a.topk, seed=0, device=dev)
