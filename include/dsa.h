@@ -172,6 +172,9 @@ dsa_status dsa_index_scores(const uint8_t* q_I, const float* q_scale, const floa
  *   scale    softmax scale, finite and > 0 (1/sqrt(576) for the latent row)
  * No workspace.
  * ------------------------------------------------------------------------ */
+dsa_status dsa_sparse_mla_attn(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int T, int L, int Hq,
+                               int topk, float scale, uint16_t* out, float* lse, void* stream);
+
 /* Sparse MQA attention over a paged latent cache: kv_pool [pool_rows, 576]
  * holds pages of page_size rows (a power of two, 16..4096); logical row r of
  * token t is physical row block_table[t * bt_stride + r / page_size] *
@@ -222,9 +225,6 @@ dsa_status dsa_rope_quantize_e4m3_rows(const float* x, const int32_t* pos, int n
  * L > DSA_MAX_TOPK, otherwise as dsa_sparse_mla_attn. */
 dsa_status dsa_dense_mla_attn_causal(const uint16_t* q, const uint16_t* kv, int T, int L, int q0, int Hq, float scale,
                                      uint16_t* out, float* lse, void* stream);
-
-dsa_status dsa_sparse_mla_attn(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int T, int L, int Hq,
-                               int topk, float scale, uint16_t* out, float* lse, void* stream);
 
 /* ------------------------------------------------------------------------
  * Decode: B sequences, one new query each, at position t = lens[b]-1 of its
@@ -320,8 +320,12 @@ dsa_status dsa_selftest_wait_timeout(void* stream);
  * the raw word, may be NULL); DSA_ERR_CUDA if the synchronisation fails. */
 dsa_status dsa_get_device_error(void* stream, unsigned int* detail);
 
+/* Static, NUL-terminated name of a status code ("unknown status" for any
+ * other value); never NULL, never to be freed. */
 const char* dsa_status_string(dsa_status s);
-/* Message of the last failing call on this host thread ("" if none). */
+/* Message of the last failing call on this host thread ("" if none); the
+ * buffer belongs to the library and is overwritten by the thread's next
+ * failing call. */
 const char* dsa_last_error(void);
 
 #ifdef __cplusplus

@@ -106,3 +106,20 @@ def test_fp8_gemm_probe_reports_instead_of_raising():
     import bench
     r = bench.measure_fp8_gemm(torch.device("cpu"), seconds=0.01, n=32)
     assert isinstance(r, dict) and ("error" in r or "burst_tflops" in r)
+
+
+def test_roofline_work_counts():
+    # the algorithmic work behind `achieved`: causal pairs for the indexer, min(k, t+1) rows per
+    # query for the attention, compulsory bytes for a decode step
+    import bench
+    for L, k in [(1, 4), (5, 4), (37, 8), (300, 64)]:
+        pairs = sum(t + 1 for t in range(L))
+        sel = sum(min(k, t + 1) for t in range(L))
+        idx_flop, attn_flop = bench.prefill_work(L, 8, 64, 16, k)
+        assert idx_flop == 2 * 8 * 64 * pairs
+        assert attn_flop == sel * 16 * 2 * (576 + 512)
+    idx_flop, attn_flop = bench.prefill_work(131072, 64, 128, 128, 2048)
+    assert idx_flop == pytest.approx(1.407e14, rel=1e-3) and attn_flop == pytest.approx(7.42e13, rel=1e-3)
+    keys, gather, small = bench.decode_bytes(64, 65536, 64, 128, 128, 2048)
+    assert keys == 64 * 65536 * 132 and gather == 64 * 2048 * 1152
+    assert (keys + gather + small) / 1e6 == pytest.approx(723.5, abs=0.1)
