@@ -66,6 +66,8 @@ def parse(argv=None):
     ap.add_argument("--decode-B", type=int, default=64)
     ap.add_argument("--decode-L", type=int, default=65536)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-chunks", type=int, default=8,
+                    help="query-row chunks whose copies overlap the compute in the e2e leg (1: no overlap)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-rows", type=int, default=240)
     ap.add_argument("--no-fp8-probe", action="store_true",
@@ -420,23 +422,50 @@ def run_e2e(a, dsa, P, idx, out, ws_p, ws, dev):
     dev_bufs = {n: getattr(P, n) for n in host}
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = out.numel() * out.element_size()
-    stream = torch.cuda.current_stream(dev)
+    # Query rows in nch chunks: chunk c's inputs copy in on s_in while chunk
+    # c-1 computes on s_cmp and chunk c-2's output copies out on s_out. The
+    # chunked selection equals the whole-sequence one row for row, so the
+    # result is the same as one call over all rows.
+    nch = max(1, min(a.e2e_chunks, P.L))
+    bounds = [(P.L * c) // nch for c in range(nch + 1)]
+    per_row = ("q_I", "q_scale", "w", "q")  # the cache-wide inputs copy first
+    s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    tq_max = max(bounds[c + 1] - bounds[c] for c in range(nch))
+    ws_c = torch.empty(max(dsa.index_topk_workspace_size(tq_max, P.H_I, P.d_I, P.topk), 16), dtype=torch.uint8,
+                       device=dev)
     times = []
     for s in range(a.warmup + a.steps):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for n, t in host.items():
-            dev_bufs[n].copy_(t, non_blocking=True)
-        dsa.index_topk(P.q_I, P.q_scale, P.w, P.k_cache, P.k_scale, P.topk, idx=idx, workspace=ws_p)
-        dsa.sparse_mla_attn(P.q, P.kv, idx, P.scale, out=out)
-        out_h.copy_(out, non_blocking=True)
-        e1.record(stream)
+        torch.cuda.synchronize()
+        e0.record(s_in)
+        with torch.cuda.stream(s_in):
+            for n in ("k_cache", "k_scale", "kv"):
+                dev_bufs[n].copy_(host[n], non_blocking=True)
+        for c in range(nch):
+            r0, r1 = bounds[c], bounds[c + 1]
+            with torch.cuda.stream(s_in):
+                for n in per_row:
+                    dev_bufs[n][r0:r1].copy_(host[n][r0:r1], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(ev)
+                dsa.index_topk_chunk(P.q_I[r0:r1], P.q_scale[r0:r1], P.w[r0:r1], P.k_cache[:r1], P.k_scale[:r1],
+                                     r0, P.topk, idx=idx[r0:r1], workspace=ws_c)
+                dsa.sparse_mla_attn(P.q[r0:r1], P.kv[:r1], idx[r0:r1], P.scale, out=out[r0:r1])
+                done = torch.cuda.Event()
+                done.record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done)
+                out_h[r0:r1].copy_(out[r0:r1], non_blocking=True)
+        e1.record(s_out)  # s_out waited on every chunk's compute, which waited on its inputs
         torch.cuda.synchronize()
         if s >= a.warmup:
             times.append(e0.elapsed_time(e1))
     t = max_over_ranks(float(np.mean(times)), ws)
     return {"value": ws * P.L / (t * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": t, "scope": "prefill (the headline metric)"}
+            "d2h_bytes_per_step": d2h, "ms_per_step": t, "scope": "prefill (the headline metric)",
+            "pipeline": f"{nch} query-row chunks; copies in, compute and copies out on three streams"}
 
 
 # ------------------------------------------------------- reference (oracle)

@@ -100,6 +100,21 @@ dsa_status dsa_index_topk_chunk(const uint8_t* q_I, const float* q_scale, const 
                                 const float* k_scale, int q0, int Tq, int L, int H_I, int d_I, int topk, int32_t* idx,
                                 void* workspace, size_t ws_bytes, void* stream);
 
+/* Chunked prefill over a paged FP8 key cache (one sequence): k_pool
+ * [pool_rows, d_I] e4m3 and k_scale_pool [pool_rows] f32 hold pages of
+ * page_size rows (a power of two, 16..4096; pool_rows a multiple of it); key
+ * s is pool row block_table[s / page_size] * page_size + s % page_size
+ * (block_table [max_blocks] int32, device, max_blocks * page_size >= L).
+ * Same result as dsa_index_topk_chunk over the gathered contiguous cache, bit
+ * for bit; same workspace. A page entry outside [0, pool_rows / page_size)
+ * for a key below L gives that page's keys zero codes and zero scale and is
+ * reported as DSA_ERR_BAD_INDEX by dsa_get_device_error. H_I = 64 only.
+ * Serving layout, no counterpart step in the pages. */
+dsa_status dsa_index_topk_chunk_paged(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_pool,
+                                      const float* k_scale_pool, const int32_t* block_table, int max_blocks,
+                                      int page_size, int pool_rows, int q0, int Tq, int L, int H_I, int d_I, int topk,
+                                      int32_t* idx, void* workspace, size_t ws_bytes, void* stream);
+
 /* Packed batch of sequences (cu_seqlens form): sequence b owns query rows
  * [cu_q[b], cu_q[b+1]) of q_I / q_scale / w and keys [cu_k[b], cu_k[b+1]) of
  * k_cache / k_scale; its queries sit at positions q_pos0[b] .. q_pos0[b] +
@@ -292,6 +307,14 @@ dsa_status dsa_index_topk_decode_noalloc(const uint8_t* q_I, const float* q_scal
 /* ------------------------------------------------------------------------
  * Errors.
  * ------------------------------------------------------------------------ */
+/* Failure-path self-test: enqueues on `stream` one small kernel that waits,
+ * with the same bounded wait every kernel here uses, on a barrier nothing
+ * completes. After about 2^31 SM cycles (~1 s) the wait gives up, records
+ * DSA_ERR_TIMEOUT with site 99 and the kernel exits; the next
+ * dsa_get_device_error reports it and the context stays usable. Returns the
+ * launch status. No counterpart in the pages. */
+dsa_status dsa_selftest_wait_timeout(void* stream);
+
 /* Synchronises `stream`, then reads and clears the device error word of the
  * current device: DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_BAD_INDEX (*detail gets
  * the raw word, may be NULL); DSA_ERR_CUDA if the synchronisation fails. */

@@ -53,6 +53,7 @@ def lib() -> ctypes.CDLL:
             L.dsa_index_scores.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P]
             L.dsa_index_topk_rerun_count.argtypes = [P, I, I, I, I, ctypes.POINTER(I), P]
             L.dsa_index_topk_chunk.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P, SZ, P]
+            L.dsa_index_topk_chunk_paged.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, P, P, SZ, P]
             L.dsa_index_topk_varlen_workspace_size.argtypes = [I, I, I, I, I]
             L.dsa_index_topk_varlen_workspace_size.restype = SZ
             L.dsa_index_topk_varlen.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, P, P, SZ, P]
@@ -69,17 +70,20 @@ def lib() -> ctypes.CDLL:
             L.dsa_sparse_mla_attn_decode.argtypes = [P, P, P, I, I, I, I, F, P, P, P]
             L.dsa_index_topk_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P, P]
             L.dsa_get_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_uint)]
+            L.dsa_selftest_wait_timeout.argtypes = [P]
             L.dsa_status_string.argtypes = [I]
             L.dsa_status_string.restype = ctypes.c_char_p
             L.dsa_last_error.argtypes = []
             L.dsa_last_error.restype = ctypes.c_char_p
             for name in ("dsa_index_topk", "dsa_index_topk_rerun_count", "dsa_index_topk_chunk",
+                         "dsa_index_topk_chunk_paged",
                          "dsa_index_topk_varlen", "dsa_dense_mla_attn_causal", "dsa_quantize_e4m3_rows",
                          "dsa_rope_quantize_e4m3_rows",
                          "dsa_sparse_mla_attn_paged",
                          "dsa_index_scores", "dsa_sparse_mla_attn", "dsa_index_topk_decode",
                          "dsa_index_scores_decode", "dsa_sparse_mla_attn_decode", "dsa_get_device_error",
-                         "dsa_index_topk_decode_noalloc", "dsa_index_topk_decode_paged"):
+                         "dsa_index_topk_decode_noalloc", "dsa_index_topk_decode_paged",
+                         "dsa_selftest_wait_timeout"):
                 getattr(L, name).restype = I
             _lib = L
     return _lib
@@ -170,6 +174,33 @@ def index_topk_chunk(q_I, q_scale, w, k_cache, k_scale, q0: int, topk: int, *, i
     _check(lib().dsa_index_topk_chunk(_ptr(q_I), _ptr(q_scale), _ptr(w), _ptr(k_cache), _ptr(k_scale), q0, Tq, L,
                                       H_I, d_I, topk, _ptr(idx), _ptr(workspace),
                                       workspace.numel() * workspace.element_size(), _stream(q_I.device)))
+    return idx
+
+
+def index_topk_chunk_paged(q_I, q_scale, w, k_pool, k_scale_pool, block_table, q0: int, L: int, topk: int, *,
+                          page_size: int = 64, idx=None, workspace=None):
+    """Chunked prefill over a paged key cache: k_pool [pool_rows, d_I] e4m3 and k_scale_pool
+    [pool_rows] f32 in pages of page_size rows; key s is in page block_table[s // page_size]
+    (block_table [max_blocks] int32). Same idx as index_topk_chunk over the gathered cache."""
+    q_I, k_pool = _u8(q_I), _u8(k_pool)
+    Tq, H_I, d_I = q_I.shape
+    pool_rows = k_pool.shape[0]
+    bt = block_table.reshape(-1)
+    _req(q_I, "q_I", torch.uint8)
+    _req(q_scale, "q_scale", torch.float32, (Tq,))
+    _req(w, "w", torch.float32, (Tq, H_I))
+    _req(k_pool, "k_pool", torch.uint8, (pool_rows, d_I))
+    _req(k_scale_pool, "k_scale_pool", torch.float32, (pool_rows,))
+    _req(bt, "block_table", torch.int32, (bt.numel(),))
+    if idx is None:
+        idx = torch.empty((Tq, topk), dtype=torch.int32, device=q_I.device)
+    _req(idx, "idx", torch.int32, (Tq, topk))
+    need = index_topk_workspace_size(Tq, H_I, d_I, topk)
+    workspace = _ws(workspace, need, q_I.device)
+    _check(lib().dsa_index_topk_chunk_paged(_ptr(q_I), _ptr(q_scale), _ptr(w), _ptr(k_pool), _ptr(k_scale_pool),
+                                            _ptr(bt), bt.numel(), page_size, pool_rows, q0, Tq, L, H_I, d_I, topk,
+                                            _ptr(idx), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                            _stream(q_I.device)))
     return idx
 
 
@@ -459,6 +490,12 @@ def device_error(device=None) -> Tuple[int, int]:
     detail = ctypes.c_uint(0)
     st = lib().dsa_get_device_error(_stream(device), ctypes.byref(detail))
     return int(st), int(detail.value)
+
+
+def selftest_wait_timeout(device=None):
+    """Enqueue the failure-path self-test: a kernel whose bounded wait runs out
+    (~1 s) and records DSA_ERR_TIMEOUT; read it with device_error()."""
+    _check(lib().dsa_selftest_wait_timeout(_stream(device)))
 
 
 def check_device_error(device=None):

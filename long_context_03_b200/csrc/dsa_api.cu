@@ -85,6 +85,23 @@ dsa_status make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_
   return DSA_OK;
 }
 
+// Queries [T, Hq, 576] bf16 as a 3-D map {576, Hq, T}; boxes of 64 values x
+// 128 heads x 1 token, 128-byte swizzled (heads >= Hq lie outside the map and
+// load as zeros).
+dsa_status make_map_q_bf16(CUtensorMap* m, const void* base, int T, int Hq) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[3] = {576, static_cast<cuuint64_t>(Hq), static_cast<cuuint64_t>(T)};
+  const cuuint64_t strides[2] = {576 * 2, static_cast<cuuint64_t>(Hq) * 576 * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled(q) failed (%d)", static_cast<int>(r));
+  return DSA_OK;
+}
+
 template <typename K>
 dsa_status set_smem(K kernel, int bytes) {
   const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -133,16 +150,23 @@ WsPrefill prefill_ws_layout(void* base, int L, int H_I, int topk, int grid) {
 // capacity: shorter rows rarely cut their lists anyway).
 int spec_min_row(int topk) { return 2 * select_cap(topk) > 4096 ? 2 * select_cap(topk) : 4096; }
 
-template <int HI, int DI, bool kSelect, int MQ>
+template <int HI, int DI, bool kSelect, int MQ, bool kPaged = false>
 dsa_status launch_prefill(const uint8_t* q_I, const uint8_t* k_cache, const IdxPrefillParams& p, int grid,
                           cudaStream_t st) {
   using C = IdxPrefillCfg<HI, DI>;
   CUtensorMap tmQ, tmK;
   dsa_status s = make_map_u8(&tmQ, q_I, DI, static_cast<uint64_t>(p.Tq) * HI, DI, C::NCOL);
   if (s != DSA_OK) return s;
-  s = make_map_u8(&tmK, k_cache, DI, static_cast<uint64_t>(p.L), DI, C::BM);
+  if (kPaged) {
+    // the pool's rows, one page (at most one key tile) per box
+    const int page = 1 << p.page_shift;
+    s = make_map_u8(&tmK, k_cache, DI, static_cast<uint64_t>(p.pool_pages) * page, DI,
+                    static_cast<uint32_t>(page < C::BM ? page : C::BM));
+  } else {
+    s = make_map_u8(&tmK, k_cache, DI, static_cast<uint64_t>(p.L), DI, C::BM);
+  }
   if (s != DSA_OK) return s;
-  auto kern = indexer_prefill_kernel<HI, DI, kSelect, MQ>;
+  auto kern = indexer_prefill_kernel<HI, DI, kSelect, MQ, kPaged>;
   s = set_smem(kern, C::SMEM_BYTES);
   if (s != DSA_OK) return s;
   kern<<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(tmQ, tmK, p);
@@ -152,6 +176,13 @@ dsa_status launch_prefill(const uint8_t* q_I, const uint8_t* k_cache, const IdxP
 template <bool kSelect, int MQ>
 dsa_status dispatch_prefill(int H_I, int d_I, const uint8_t* q_I, const uint8_t* k_cache, const IdxPrefillParams& p,
                             int grid, cudaStream_t st) {
+  if constexpr (kSelect) {
+    if (p.block_table) {  // paged key cache: the H_I = 64 shapes
+      if (H_I == 64 && d_I == 128) return launch_prefill<64, 128, true, MQ, true>(q_I, k_cache, p, grid, st);
+      if (H_I == 64 && d_I == 64) return launch_prefill<64, 64, true, MQ, true>(q_I, k_cache, p, grid, st);
+      return fail(DSA_ERR_UNSUPPORTED, "paged keys: H_I=%d d_I=%d not supported", H_I, d_I);
+    }
+  }
   if (H_I == 64 && d_I == 128) return launch_prefill<64, 128, kSelect, MQ>(q_I, k_cache, p, grid, st);
   if (H_I == 64 && d_I == 64) return launch_prefill<64, 64, kSelect, MQ>(q_I, k_cache, p, grid, st);
   if (H_I == 8 && d_I == 128) return launch_prefill<8, 128, kSelect, MQ>(q_I, k_cache, p, grid, st);
@@ -174,6 +205,26 @@ __global__ void fill_f32_kernel(float* p, size_t n, float v) {
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<size_t>(gridDim.x) * blockDim.x)
     p[i] = v;
+}
+
+// ---- failure-path self-test ----
+// One CTA waits, with the library's bounded wait, on an mbarrier that no
+// thread arrives on: the wait gives up after its bound (~2^31 cycles), records
+// a timeout with site kSelftestSite in the device error word and the kernel
+// returns, leaving the context usable.
+constexpr unsigned int kSelftestSite = 99;
+__global__ void selftest_wait_timeout_kernel() {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const AbortFlag ab{&abort_flag};
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, ab, kSelftestSite);
+  __syncthreads();
 }
 
 // ---- decode ----
@@ -230,12 +281,14 @@ dsa_status decode_scores(const uint8_t* q_I, const float* q_scale, const float* 
   return fail(DSA_ERR_UNSUPPORTED, "decode: H_I=%d d_I=%d not supported", H_I, d_I);
 }
 
+// Selection and ranking of every sequence's top-k: one CTA per sequence
+// selects, then sorts its keys in shared memory and writes idx.
 dsa_status launch_decode_select(const float* scores, const int32_t* lens, int L_max, int topk, const uint32_t* hist,
-                                uint64_t* sel, int B, cudaStream_t st) {
+                                uint64_t* sel, int32_t* idx, int B, cudaStream_t st) {
   const int smem = kDecodeSelBinCap * 8 + (2048 + select_scratch_ints(kDecodeSelThreads)) * 4;
   dsa_status s = set_smem(decode_select_kernel, smem);
   if (s != DSA_OK) return s;
-  decode_select_kernel<<<B, kDecodeSelThreads, smem, st>>>(scores, lens, L_max, topk, hist, sel);
+  decode_select_kernel<<<B, kDecodeSelThreads, smem, st>>>(scores, lens, L_max, topk, hist, sel, idx);
   return check_launch("decode_select_kernel");
 }
 
@@ -275,8 +328,11 @@ dsa_status launch_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
   p.page_shift = pg.page_shift;
   p.pool_rows = pg.pool_rows;
   p.scale_log2 = scale * 1.4426950408889634f;
+  CUtensorMap tmQ;
+  dsa_status s = make_map_q_bf16(&tmQ, q, T, Hq);
+  if (s != DSA_OK) return s;
   auto kern = pg.block_table ? sparse_mla_kernel<true> : sparse_mla_kernel<false>;
-  dsa_status s = set_smem(kern, MlaCfg::SMEM_BYTES);
+  s = set_smem(kern, MlaCfg::SMEM_BYTES);
   if (s != DSA_OK) return s;
   // co-resident clusters, looked up once (the same for both instances: same
   // resources); concurrent first calls compute the same value
@@ -296,7 +352,7 @@ dsa_status launch_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
     max_clusters_cache.store(n, std::memory_order_relaxed);
   }
   const int nclusters = T < max_clusters ? T : max_clusters;
-  kern<<<2 * nclusters, MlaCfg::NTHREADS, MlaCfg::SMEM_BYTES, st>>>(p);
+  kern<<<2 * nclusters, MlaCfg::NTHREADS, MlaCfg::SMEM_BYTES, st>>>(tmQ, p);
   return check_launch("sparse_mla_kernel");
 }
 
@@ -324,9 +380,15 @@ size_t dsa_index_topk_workspace_size(int L, int H_I, int d_I, int topk) {
 }
 
 // Queries r = 0..Tq-1 at positions q0 + r against keys 0..L-1 (q0 + Tq <= L).
+struct PrefillKeyPaging {
+  const int32_t* block_table = nullptr;
+  int page_shift = 0, pool_pages = 0;
+};
+
 static dsa_status index_topk_impl(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
                            const float* k_scale, int q0, int Tq, int L, int H_I, int d_I, int topk, int32_t* idx,
-                           void* workspace, size_t ws_bytes, cudaStream_t st) {
+                           void* workspace, size_t ws_bytes, cudaStream_t st,
+                           PrefillKeyPaging pg = PrefillKeyPaging()) {
   if (!q_I || !q_scale || !w || !k_cache || !k_scale || !idx) return fail(DSA_ERR_INVALID_ARG, "null pointer");
   if (L <= 0 || Tq <= 0 || q0 < 0 || static_cast<long long>(q0) + Tq > L)
     return fail(DSA_ERR_INVALID_ARG, "q0=%d Tq=%d L=%d (need q0 >= 0, Tq >= 1, q0 + Tq <= L)", q0, Tq, L);
@@ -357,6 +419,9 @@ static dsa_status index_topk_impl(const uint8_t* q_I, const float* q_scale, cons
   p.spec_min_t = spec_min_row(topk);
   p.redo_count = ws.redo;
   p.redo_list = ws.redo + 4;
+  p.block_table = pg.block_table;
+  p.page_shift = pg.page_shift;
+  p.pool_pages = pg.pool_pages;
   const cudaError_t me = cudaMemsetAsync(ws.redo, 0, sizeof(int), st);
   if (me != cudaSuccess) return cuda_fail(me, "cudaMemsetAsync");
   dsa_status s = (select_mq(topk) == 1) ? dispatch_prefill<true, 1>(H_I, d_I, q_I, k_cache, p, grid, st)
@@ -389,6 +454,26 @@ dsa_status dsa_index_topk_chunk(const uint8_t* q_I, const float* q_scale, const 
                                 void* workspace, size_t ws_bytes, void* stream) {
   return index_topk_impl(q_I, q_scale, w, k_cache, k_scale, q0, Tq, L, H_I, d_I, topk, idx, workspace, ws_bytes,
                          static_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_index_topk_chunk_paged(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_pool,
+                                      const float* k_scale_pool, const int32_t* block_table, int max_blocks,
+                                      int page_size, int pool_rows, int q0, int Tq, int L, int H_I, int d_I, int topk,
+                                      int32_t* idx, void* workspace, size_t ws_bytes, void* stream) {
+  if (!block_table) return fail(DSA_ERR_INVALID_ARG, "null pointer");
+  if (page_size < 16 || page_size > 4096 || (page_size & (page_size - 1)))
+    return fail(DSA_ERR_INVALID_ARG, "page_size=%d must be a power of two in [16, 4096]", page_size);
+  if (pool_rows <= 0 || pool_rows % page_size)
+    return fail(DSA_ERR_INVALID_ARG, "pool_rows=%d (a positive multiple of page_size)", pool_rows);
+  if (max_blocks <= 0 || static_cast<long long>(max_blocks) * page_size < L)
+    return fail(DSA_ERR_INVALID_ARG, "max_blocks=%d pages of %d rows do not cover L=%d", max_blocks, page_size, L);
+  if (H_I != 64) return fail(DSA_ERR_UNSUPPORTED, "paged keys: H_I=%d not supported", H_I);
+  PrefillKeyPaging pg;
+  pg.block_table = block_table;
+  pg.page_shift = __builtin_ctz(static_cast<unsigned>(page_size));
+  pg.pool_pages = pool_rows / page_size;
+  return index_topk_impl(q_I, q_scale, w, k_pool, k_scale_pool, q0, Tq, L, H_I, d_I, topk, idx, workspace, ws_bytes,
+                         static_cast<cudaStream_t>(stream), pg);
 }
 
 // ---- packed batch of sequences (cu_seqlens) ----
@@ -667,9 +752,7 @@ dsa_status dsa_index_topk_decode(const uint8_t* q_I, const float* q_scale, const
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(histogram)");
   s = decode_scores(q_I, q_scale, w, k_cache, k_scale, lens, B, L_max, H_I, d_I, scores, hist, st);
   if (s != DSA_OK) return s;
-  s = launch_decode_select(scores, lens, L_max, topk, hist, sel, B, st);
-  if (s != DSA_OK) return s;
-  return launch_rank_sort(sel, idx, topk, B, st);
+  return launch_decode_select(scores, lens, L_max, topk, hist, sel, idx, B, st);
 }
 
 dsa_status dsa_index_topk_decode_paged(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_pool,
@@ -707,9 +790,7 @@ dsa_status dsa_index_topk_decode_paged(const uint8_t* q_I, const float* q_scale,
   pg.pool_pages = pool_rows / page_size;
   s = decode_scores(q_I, q_scale, w, k_pool, k_scale_pool, lens, B, L_max, H_I, d_I, scores, hist, st, pg);
   if (s != DSA_OK) return s;
-  s = launch_decode_select(scores, lens, L_max, topk, hist, sel, B, st);
-  if (s != DSA_OK) return s;
-  return launch_rank_sort(sel, idx, topk, B, st);
+  return launch_decode_select(scores, lens, L_max, topk, hist, sel, idx, B, st);
 }
 
 dsa_status dsa_index_scores_decode(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
@@ -786,9 +867,7 @@ dsa_status dsa_index_topk_decode_noalloc(const uint8_t* q_I, const float* q_scal
   uint64_t* sel = reinterpret_cast<uint64_t*>(reinterpret_cast<char*>(base) + kNoAllocScoreBytes);
   s = decode_scores(q_I, q_scale, w, k_cache, k_scale, lens, B, L_max, H_I, d_I, scores, nullptr, st);
   if (s != DSA_OK) return s;
-  s = launch_decode_select(scores, lens, L_max, topk, nullptr, sel, B, st);
-  if (s != DSA_OK) return s;
-  return launch_rank_sort(sel, idx, topk, B, st);
+  return launch_decode_select(scores, lens, L_max, topk, nullptr, sel, idx, B, st);
 }
 
 dsa_status dsa_get_device_error(void* stream, unsigned int* detail) {
@@ -806,6 +885,11 @@ dsa_status dsa_get_device_error(void* stream, unsigned int* detail) {
   const unsigned int code = h & 0xFFu;
   if (code == kErrTimeout) return fail(DSA_ERR_TIMEOUT, "a kernel gave up waiting (site %u)", h >> 8);
   return fail(DSA_ERR_BAD_INDEX, "an index or page-table entry was outside its cache (site %u)", h >> 8);
+}
+
+dsa_status dsa_selftest_wait_timeout(void* stream) {
+  selftest_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+  return check_launch("selftest_wait_timeout_kernel");
 }
 
 const char* dsa_status_string(dsa_status s) {

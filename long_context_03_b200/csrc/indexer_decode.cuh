@@ -362,9 +362,9 @@ __global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS)
 constexpr int kDecodeSelThreads = 1024;
 constexpr int kDecodeSelBinCap = 16384;  // boundary-bin keys kept in shared memory (128 KB)
 
-__global__ void __launch_bounds__(kDecodeSelThreads)
-    decode_select_kernel(const float* __restrict__ scores, const int32_t* __restrict__ lens, int L_max, int K,
-                         const uint32_t* __restrict__ hist_in, uint64_t* __restrict__ sel_keys) {
+__device__ __forceinline__ void decode_select_body(const float* __restrict__ scores, const int32_t* __restrict__ lens,
+                                                   int L_max, int K, const uint32_t* __restrict__ hist_in,
+                                                   uint64_t* __restrict__ sel_keys) {
   constexpr int NT = kDecodeSelThreads;
   extern __shared__ __align__(16) uint8_t dsmem[];
   uint64_t* bin_keys = reinterpret_cast<uint64_t*>(dsmem);                          // [kDecodeSelBinCap]
@@ -543,6 +543,51 @@ __global__ void __launch_bounds__(kDecodeSelThreads)
   for (int i = tid; i < n; i += NT) {
     const uint64_t x = rank_key(sc[i], static_cast<uint32_t>(i));
     if (key_bin11(x) == dbin && x >= prefix) dst[atomicAdd(&wpos, 1)] = x;
+  }
+}
+
+// The k selected keys of one sequence in ranked order: a bitonic sort of the
+// keys (padded with 0 to a power of two <= 2048) in shared memory into
+// descending 64-bit order (score descending, then index ascending), written
+// as token indices, -1 for padding keys.
+template <int NT>
+__device__ __forceinline__ void sort_keys_to_idx(uint64_t* s, const uint64_t* src, int K, int32_t* out) {
+  const int tid = threadIdx.x;
+  int P = 1;
+  while (P < K) P <<= 1;
+  for (int i = tid; i < P; i += NT) s[i] = (i < K) ? src[i] : 0ull;
+  __syncthreads();
+  for (int k = 2; k <= P; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = tid; i < P; i += NT) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const uint64_t a = s[i], c = s[ixj];
+          // blocks with (i & k) == 0 run descending; the last stage (k = P) is all descending
+          if (((i & k) == 0) ? (a < c) : (a > c)) {
+            s[i] = c;
+            s[ixj] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = tid; i < K; i += NT) out[i] = (s[i] == 0ull) ? -1 : rank_key_index(s[i]);
+}
+
+// Exact top-k of sequence blockIdx.x; with idx set, also ranks the keys and
+// writes the sequence's index row (no separate sort launch).
+__global__ void __launch_bounds__(kDecodeSelThreads)
+    decode_select_kernel(const float* __restrict__ scores, const int32_t* __restrict__ lens, int L_max, int K,
+                         const uint32_t* __restrict__ hist_in, uint64_t* __restrict__ sel_keys,
+                         int32_t* __restrict__ idx) {
+  decode_select_body(scores, lens, L_max, K, hist_in, sel_keys);
+  if (idx) {
+    extern __shared__ __align__(16) uint8_t dsmem[];
+    __syncthreads();  // the selected keys (global, this CTA's writes) are complete; the bin buffer is free
+    const size_t row = static_cast<size_t>(blockIdx.x) * K;
+    sort_keys_to_idx<kDecodeSelThreads>(reinterpret_cast<uint64_t*>(dsmem), sel_keys + row, K, idx + row);
   }
 }
 

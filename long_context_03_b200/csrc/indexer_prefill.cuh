@@ -112,25 +112,40 @@ struct IdxPrefillParams {
   // score mode (test hook)
   float* scores;         // [nrows][L]; rows t in [row0, row0 + nrows)
   int row0, nrows;
+  // Paged key cache (the kernel's paged instance, one sequence): key s is pool
+  // row block_table[s >> page_shift] * page + (s & (page - 1)) of the FP8 keys
+  // and of k_scale; the pool holds pool_pages pages.
+  const int32_t* block_table;
+  int page_shift, pool_pages;
 };
 
 // sum_j w[j] * max(x_j, 0) over the H_I accumulator values of one token
-// (registers loaded from TMEM), into eight independent partial sums (head j
-// goes to sum j % 8) added in a fixed order at the end. Scalar FMAs: the
-// packed two-lane form needs its operands in aligned register pairs, which
-// cost a register move per ReLU output. Shared by both modes so their scores
-// are bit-identical.
+// (registers loaded from TMEM), written as (sum_j w[j]*x_j + sum_j w[j]*|x_j|)/2
+// so that both sums run on the FMA pipe: acc[0..3] take w*x as two packed
+// float pairs (fma.rn.f32x2 on register pairs straight from the TMEM load),
+// acc[4..7] take w*|x| with the absolute value folded into the scalar FMA.
+// The halves cancel exactly where every head is negative (an exact zero stays
+// zero). Shared by both modes so their scores are bit-identical.
 template <int HI>
 __device__ __forceinline__ void relu_weighted_acc(float (&acc)[8], const uint32_t* x, const float* __restrict__ w) {
-  static_assert(HI % 8 == 0, "a multiple of 8 heads");
+  static_assert(HI % 4 == 0, "a multiple of 4 heads");
 #pragma unroll
-  for (int j = 0; j < HI; j += 8) {
+  for (int j = 0; j < HI; j += 4) {
 #pragma unroll
-    for (int a = 0; a < 8; ++a) acc[a] = __fmaf_rn(w[j + a], fmaxf(__uint_as_float(x[j + a]), 0.f), acc[a]);
+    for (int pr = 0; pr < 2; ++pr) {
+      uint64_t d, wa, xa, ca;
+      asm("mov.b64 %0, {%1, %2};" : "=l"(wa) : "f"(w[j + 2 * pr]), "f"(w[j + 2 * pr + 1]));
+      asm("mov.b64 %0, {%1, %2};" : "=l"(xa) : "r"(x[j + 2 * pr]), "r"(x[j + 2 * pr + 1]));
+      asm("mov.b64 %0, {%1, %2};" : "=l"(ca) : "f"(acc[2 * pr]), "f"(acc[2 * pr + 1]));
+      asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(wa), "l"(xa), "l"(ca));
+      asm("mov.b64 {%0, %1}, %2;" : "=f"(acc[2 * pr]), "=f"(acc[2 * pr + 1]) : "l"(d));
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a) acc[4 + a] = __fmaf_rn(w[j + a], fabsf(__uint_as_float(x[j + a])), acc[4 + a]);
   }
 }
 __device__ __forceinline__ float relu_weighted_finish(const float (&acc)[8]) {
-  return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+  return 0.5f * (((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7])));
 }
 
 // Key tile of step i of a row block's sequence: with sampling, steps
@@ -154,7 +169,22 @@ __device__ __forceinline__ int sample_rank(int topk, int sampled_keys, int t, in
   return static_cast<int>(r);
 }
 
-template <int HI, int DI, bool kSelect, int MQ>
+// Paged key cache: the page-table entry of key s (-1 past the cache), and the
+// pool row a box starting at key s reads (the pool's end, which TMA fills
+// with zeros, past the cache or behind a bad entry).
+__device__ __forceinline__ int prefill_page_entry(const IdxPrefillParams& p, int s, int L) {
+  return (s < L) ? __ldg(p.block_table + (s >> p.page_shift)) : -1;
+}
+__device__ __forceinline__ int prefill_pool_row(const IdxPrefillParams& p, int s, int L, int page) {
+  if (s >= L) return p.pool_pages << p.page_shift;
+  if (page < 0 || page >= p.pool_pages) {
+    set_device_error(kErrBadIndex, 3);
+    return p.pool_pages << p.page_shift;
+  }
+  return (page << p.page_shift) + (s & ((1 << p.page_shift) - 1));
+}
+
+template <int HI, int DI, bool kSelect, int MQ, bool kPaged = false>
 __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
     indexer_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                            const IdxPrefillParams p) {
@@ -260,11 +290,41 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
         for (int b = 0; b < C::NACC; ++b)
           tma_load_2d(q_s + b * C::QBUF_BYTES, &tmQ, q_full, 0, (r0 + b * C::TB) * HI);
         bool ok = true;
+        // paged: one box of R = min(page, BM) rows per page of the tile; the
+        // next tile's page entries load before the wait for this tile's slot
+        constexpr int MAXB = C::BM / 16;
+        [[maybe_unused]] const int R = kPaged ? min(1 << p.page_shift, C::BM) : C::BM;
+        [[maybe_unused]] int nxt[MAXB];
+        if constexpr (kPaged) {
+#pragma unroll
+          for (int q = 0; q < MAXB; ++q)
+            nxt[q] = (q * R < C::BM) ? prefill_page_entry(p, tile_at<C::NSAMPLE>(0, nkt, spec) * C::BM + q * R, bk.L)
+                                     : -1;
+        }
         for (int i = 0; i < nsteps; ++i) {
+          [[maybe_unused]] int cur[MAXB];
+          if constexpr (kPaged) {
+#pragma unroll
+            for (int q = 0; q < MAXB; ++q) cur[q] = nxt[q];
+            if (i + 1 < nsteps) {
+              const int sn = tile_at<C::NSAMPLE>(i + 1, nkt, spec) * C::BM;
+#pragma unroll
+              for (int q = 0; q < MAXB; ++q) nxt[q] = (q * R < C::BM) ? prefill_page_entry(p, sn + q * R, bk.L) : -1;
+            }
+          }
           if (!mbar_wait(k_empty + kslot, ke_phase, ab, 2)) { ok = false; break; }
           mbar_arrive_expect_tx(k_full + kslot, C::KTILE_BYTES);
-          tma_load_2d(k_s + kslot * C::KTILE_BYTES, &tmK, k_full + kslot, 0,
-                      bk.kbase + tile_at<C::NSAMPLE>(i, nkt, spec) * C::BM);
+          if constexpr (kPaged) {
+            const int sc = tile_at<C::NSAMPLE>(i, nkt, spec) * C::BM;
+#pragma unroll
+            for (int q = 0; q < MAXB; ++q)
+              if (q * R < C::BM)
+                tma_load_2d(k_s + kslot * C::KTILE_BYTES + q * R * DI, &tmK, k_full + kslot, 0,
+                            prefill_pool_row(p, sc + q * R, bk.L, cur[q]));
+          } else {
+            tma_load_2d(k_s + kslot * C::KTILE_BYTES, &tmK, k_full + kslot, 0,
+                        bk.kbase + tile_at<C::NSAMPLE>(i, nkt, spec) * C::BM);
+          }
           if (++kslot == C::KST) { kslot = 0; ke_phase ^= 1; }
         }
         if (!ok) break;
@@ -368,9 +428,20 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
       named_bar_sync(1, C::NET);
       bool ok = true;
       float ks_next = 0.f;
+      // paged: page entry of the key two steps ahead, its scale one step ahead
+      // (no dependent load waits inside a step)
+      [[maybe_unused]] int pg_next = -1;
       {
         const int s0 = tile_at<C::NSAMPLE>(0, nkt, spec) * C::BM + quarter * 32 + static_cast<int>(lane);
-        ks_next = (s0 < bk.L) ? __ldg(p.k_scale + bk.kbase + s0) : 0.f;
+        if constexpr (kPaged) {
+          const int r = prefill_pool_row(p, s0, bk.L, prefill_page_entry(p, s0, bk.L));
+          ks_next = (s0 < bk.L && r < (p.pool_pages << p.page_shift)) ? __ldg(p.k_scale + r) : 0.f;
+          if (1 < nsteps)
+            pg_next = prefill_page_entry(
+                p, tile_at<C::NSAMPLE>(1, nkt, spec) * C::BM + quarter * 32 + static_cast<int>(lane), bk.L);
+        } else {
+          ks_next = (s0 < bk.L) ? __ldg(p.k_scale + bk.kbase + s0) : 0.f;
+        }
       }
       for (int i = 0; i < nsteps && ok; ++i) {
         const int kt = tile_at<C::NSAMPLE>(i, nkt, spec);
@@ -378,7 +449,15 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
         const float ks = ks_next;
         if (i + 1 < nsteps) {
           const int sn = tile_at<C::NSAMPLE>(i + 1, nkt, spec) * C::BM + quarter * 32 + static_cast<int>(lane);
-          ks_next = (sn < bk.L) ? __ldg(p.k_scale + bk.kbase + sn) : 0.f;
+          if constexpr (kPaged) {
+            const int r = prefill_pool_row(p, sn, bk.L, pg_next);
+            ks_next = (sn < bk.L && r < (p.pool_pages << p.page_shift)) ? __ldg(p.k_scale + r) : 0.f;
+            if (i + 2 < nsteps)
+              pg_next = prefill_page_entry(
+                  p, tile_at<C::NSAMPLE>(i + 2, nkt, spec) * C::BM + quarter * 32 + static_cast<int>(lane), bk.L);
+          } else {
+            ks_next = (sn < bk.L) ? __ldg(p.k_scale + bk.kbase + sn) : 0.f;
+          }
         }
         for (int b = 0; b < C::NACC; ++b) {
           if (!mbar_wait(acc_full + b, af_phase[b], ab, 8)) { ok = false; break; }

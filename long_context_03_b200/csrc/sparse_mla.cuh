@@ -11,7 +11,9 @@
 // The fp32 output tile of one token (128 heads x 512 values) needs all 512
 // TMEM columns of an SM, so each token runs on a 2-CTA cluster:
 //   CTA 0 (score CTA) keeps all of Q[t] in TMEM (288 columns of bf16 pairs,
-//     the A operand of TMEM-sourced MMAs) and computes S = Q C^T for chunks
+//     the A operand of TMEM-sourced MMAs; Q arrives as nine TMA tiles through
+//     the same ring as the gathered rows and the MMA warp copies each into
+//     TMEM with tcgen05.cp) and computes S = Q C^T for chunks
 //     of 128 selected rows (M = 128 heads, N = 128 rows: a full-rate tcgen05
 //     shape) into a single 128-column S buffer. The rows are gathered slab by
 //     slab (64 values = 128 bytes of each row, 16 KB per slab tile) through a
@@ -88,7 +90,7 @@ struct MlaCfg {
   static constexpr int B_RING_EMPTY = B_RING_FULL + NRING;  // [NRING]
   static constexpr int B_S_FULL = B_RING_EMPTY + NRING;     // [NSB]  (score CTA)
   static constexpr int B_S_EMPTY = B_S_FULL + NSB;          // [NSB]  (score CTA)
-  static constexpr int B_Q_READY = B_S_EMPTY + NSB;         // score CTA
+  static constexpr int B_Q_READY = B_S_EMPTY + NSB;         // score CTA (unused: Q arrives through the ring)
   static constexpr int B_Q_FREE = B_Q_READY + 1;            // score CTA
   static constexpr int B_P_FREE = B_Q_FREE + 1;             // [NPB] score CTA, arrived by the value CTA's MMA
   static constexpr int B_P_FULL = B_P_FREE + NPB;           // [NPB] value CTA, completed by the bulk copy
@@ -285,7 +287,7 @@ __device__ __forceinline__ void stage_index_row(int32_t* idx_s, const int32_t* _
 
 template <bool kPaged>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
-    sparse_mla_kernel(const MlaParams p) {
+    sparse_mla_kernel(const __grid_constant__ CUtensorMap tmQ, const MlaParams p) {
   using C = MlaCfg;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -353,6 +355,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       int slot = 0;
       uint32_t ph = 1;
       int n = 0;  // tokens done by this cluster
+      // thread 0: where the last token's Q tiles start in the ring and how
+      // many it loaded, so that an abort can still wait for its copies in flight
+      int q_slot0 = 0;
+      uint32_t q_ph0 = 1;
+      int q_issued = 0;
       for (int tk = cluster_id; tk < p.T; tk += nclusters, ++n) {
         const __nv_bfloat16* kv_tok = p.kv + tk * p.kv_token_stride;
         // the softmax warps are done with this mask buffer (two tokens back)
@@ -375,6 +382,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(bars + C::B_MASK_FULL + mb);
         bool ok = true;
+        // Q[tk] first: nine 16 KB tiles (128 heads x 64 values, 128-byte
+        // swizzled, heads >= Hq zero) through the ring by TMA; the MMA warp
+        // copies them into TMEM. Thread 0 arms the slot with the bytes, the
+        // other producer threads arrive, as for a gathered tile.
+        q_slot0 = slot;
+        q_ph0 = ph;
+        q_issued = 0;
+        for (int i = 0; i < C::NSLAB_QK; ++i) {
+          if (!mbar_wait(bars + C::B_RING_EMPTY + slot, ph, ab, 29)) { ok = false; break; }
+          if (ptid == 0) {
+            mbar_arrive_expect_tx(bars + C::B_RING_FULL + slot, C::SLAB_TILE);
+            tma_load_3d(smem + C::OFF_RING + slot * C::SLAB_TILE, &tmQ, bars + C::B_RING_FULL + slot, i * 64, 0, tk);
+            q_issued = i + 1;
+          } else {
+            mbar_arrive(bars + C::B_RING_FULL + slot);
+          }
+          if (++slot == C::NSST) { slot = 0; ph ^= 1; }
+        }
         for (int j = 0; j < nchunk && ok; ++j) {
           const ChunkRows cr = chunk_rows<kPaged>(p, kv_tok, tk, idx_s, j, p.K, p.rows, ptid);
           for (int i = 0; i < C::NSLAB_QK; ++i) {
@@ -387,18 +412,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
         if (!ok) break;
       }
       asm volatile("cp.async.wait_all;" ::: "memory");
+      if (ptid == 0 && ab.raised()) {
+        // aborted: the token's Q tiles may still be landing in the ring; wait
+        // for them (bounded, whatever the abort flag says) before leaving
+        int never = 0;
+        const AbortFlag no_abort{&never};
+        // only the latest use of each slot can still be in flight (a tile that
+        // reused a slot was issued after the earlier one had been consumed)
+        for (int i = (q_issued > C::NSST ? q_issued - C::NSST : 0); i < q_issued; ++i) {
+          const int pos = q_slot0 + i;  // ring position of Q tile i; the parity flips at each wrap
+          const uint32_t full_par = (q_ph0 ^ static_cast<uint32_t>((pos / C::NSST) & 1)) ^ 1u;
+          mbar_wait(bars + C::B_RING_FULL + pos % C::NSST, full_par, no_abort, 28);
+        }
+      }
     } else if (warp == C::W_MMA) {
       // The whole warp runs the loop and waits converged; one elected lane
       // issues each slab's MMAs together with every commit that covers them.
       int slot = 0;
       uint32_t ph = 0;
       uint32_t sph = 1;
-      uint32_t qph = 0;
+      uint32_t qfree_ph = 1;
       bool ok = true;
       for (int tk = cluster_id; tk < p.T && ok; tk += nclusters) {
-        if (!mbar_wait_warp(bars + C::B_Q_READY, qph, ab, 32)) break;
-        qph ^= 1;
+        // Q[tk] into TMEM once the previous token's QK^T has read the old Q
+        if (!mbar_wait_warp(bars + C::B_Q_FREE, qfree_ph, ab, 32)) break;
+        qfree_ph ^= 1;
         tc_fence_after();
+        for (int i = 0; i < C::NSLAB_QK; ++i) {
+          if (!mbar_wait_warp(bars + C::B_RING_FULL + slot, ph, ab, 37)) { ok = false; break; }
+          tc_fence_after();
+          if (elect_one()) {
+            const uint32_t tile = ring + slot * C::SLAB_TILE;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              tc_cp_128x256b(tmem + C::Q_COL + (4 * i + kk) * 8, smem_desc(tile + kk * 32, 16, 1024, kSw128));
+            tc_commit(bars + C::B_RING_EMPTY + slot);
+          }
+          __syncwarp();
+          if (++slot == C::NSST) { slot = 0; ph ^= 1; }
+        }
+        if (!ok) break;
         for (int j = 0; j < nchunk && ok; ++j) {
           if (!mbar_wait_warp(bars + C::B_S_EMPTY, sph, ab, 34)) { ok = false; break; }
           sph ^= 1;
@@ -434,48 +487,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       const uint32_t peer_msg = map_to_peer(msg, 1);
       const uint32_t peer_pfull = map_to_peer(smem_u32(bars + C::B_P_FULL), 1);
       uint32_t sph = 0;
-      uint32_t qfree_ph = 1;
       int pb = 0;
       uint32_t pfree_ph = 1;
       uint32_t stage_ph = 0;
       bool ok = true;
       int n = 0;  // tokens done by this cluster
       for (int tk = cluster_id; tk < p.T && ok; tk += nclusters, ++n) {
-        // --- Q[tk]: values 0..511 to TMEM, 512..575 to shared memory, once
-        //     the previous token's QK^T is done ---
-        if (!mbar_wait(bars + C::B_Q_FREE, qfree_ph, ab, 35)) break;
-        qfree_ph ^= 1;
-        tc_fence_after();
-        {
-          // the head's 1152-byte row in 9 blocks of 64 values, each to 32 TMEM
-          // columns, loaded three blocks at a time so each round trip has 24
-          // loads in flight
-          const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(tk) * p.Hq + h) * C::D);
-#pragma unroll
-          for (int rnd = 0; rnd < 3; ++rnd) {
-            uint4 x[24];
-#pragma unroll
-            for (int i = 0; i < 24; ++i) x[i] = (h < p.Hq) ? __ldg(qrow + rnd * 24 + i) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int bb = 0; bb < 3; ++bb) {
-              const int cb = rnd * 3 + bb;
-              uint32_t r[32];
-#pragma unroll
-              for (int v = 0; v < 8; ++v) {
-                r[4 * v + 0] = x[bb * 8 + v].x;
-                r[4 * v + 1] = x[bb * 8 + v].y;
-                r[4 * v + 2] = x[bb * 8 + v].z;
-                r[4 * v + 3] = x[bb * 8 + v].w;
-              }
-              tmem_st32(tmem + lane_addr + C::Q_COL + cb * 32, r);
-            }
-          }
-          tmem_st_wait();
-        }
-        fence_async_shared();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bars + C::B_Q_READY);
+        // Q[tk] reaches TMEM through the ring (TMA + tcgen05.cp by the MMA warp)
         if (tk + nclusters < p.T && h == 0) {
           // warm L2 with the next token's queries
           const char* nq = reinterpret_cast<const char*>(p.q + static_cast<size_t>(tk + nclusters) * p.Hq * C::D);

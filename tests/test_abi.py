@@ -137,6 +137,26 @@ def test_rope_quantiser_argument_checks(lib):
     assert lib.dsa_rope_quantize_e4m3_rows(None, None, 0, 64, 128, 64, b, 1, None, None, None, None) == 0  # empty
 
 
+def test_paged_prefill_chunk_argument_checks(lib):
+    p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    # (q_I, q_scale, w, k_pool, k_scale_pool, table, max_blocks, page, pool_rows, q0, Tq, L, H_I, d_I, topk,
+    #  idx, workspace, ws_bytes, stream)
+    args = [p, p, p, p, p, p, 16, 64, 1024, 0, 1000, 1000, 64, 128, 64, p, p, 1 << 30, None]
+    bad_table = list(args); bad_table[5] = None
+    assert lib.dsa_index_topk_chunk_paged(*bad_table) == -1
+    bad_page = list(args); bad_page[7] = 100
+    assert lib.dsa_index_topk_chunk_paged(*bad_page) == -1
+    short_table = list(args); short_table[6] = 15  # 15 pages of 64 rows < L = 1000
+    assert lib.dsa_index_topk_chunk_paged(*short_table) == -1
+    heads8 = list(args); heads8[12] = 8
+    assert lib.dsa_index_topk_chunk_paged(*heads8) == -2
+
+
+def test_error_strings_cover_every_status(lib):
+    for st in (0, -1, -2, -3, -4, -5, -6):
+        assert lib.dsa_status_string(st) not in (None, b"unknown status")
+
+
 def _declared_arity():
     """Number of parameters of every function declared in include/dsa.h."""
     src = open(os.path.join(ROOT, "include", "dsa.h")).read()

@@ -156,3 +156,53 @@ def test_decode_indexer_bad_page_is_reported(dsa):
     idx = dsa.index_topk_decode_paged(D.q_I, D.q_scale, D.w, k_pool, ks_pool, bad, D.lens, 2048, page_size=page)
     dsa.device_error()
     assert torch.equal(idx[0], ref[0])
+
+
+def _page_one(k_cache, k_scale, page, gen, spare=3):
+    """One sequence's keys [L, d] and scales [L] in a shuffled pool; table [max_blocks]."""
+    L, d = k_cache.shape
+    npg = (L + page - 1) // page
+    perm = torch.randperm(npg + spare, generator=gen)[:npg].to(k_cache.device)
+    k_pool = torch.zeros(((npg + spare) * page, d), dtype=torch.uint8, device=k_cache.device)
+    ks_pool = torch.full(((npg + spare) * page,), 5.0, dtype=torch.float32, device=k_cache.device)
+    kc = torch.zeros((npg * page, d), dtype=torch.uint8, device=k_cache.device)
+    kc[:L] = k_cache.view(torch.uint8)
+    ks = torch.zeros((npg * page,), dtype=torch.float32, device=k_cache.device)
+    ks[:L] = k_scale
+    rows = (perm[:, None] * page + torch.arange(page, device=k_cache.device)[None]).reshape(-1)
+    k_pool[rows] = kc
+    ks_pool[rows] = ks
+    return k_pool, ks_pool, perm.to(torch.int32)
+
+
+@pytest.mark.parametrize("page", [16, 64, 256])
+def test_prefill_chunk_paged_keys_match_contiguous(dsa, page):
+    L = 20480  # long enough for the sampled starting thresholds
+    P = workloads.make_prefill(L, 64, 128, 1, 2048, seed=51, device="cuda")
+    k_pool, ks_pool, table = _page_one(P.k_cache, P.k_scale, page, torch.Generator().manual_seed(page))
+    for q0, Tq in [(0, L), (17000, 3000), (4095, 1)]:
+        sl = slice(q0, q0 + Tq)
+        ref = dsa.index_topk_chunk(P.q_I[sl], P.q_scale[sl], P.w[sl], P.k_cache[:q0 + Tq], P.k_scale[:q0 + Tq],
+                                   q0, 2048)
+        idx = dsa.index_topk_chunk_paged(P.q_I[sl], P.q_scale[sl], P.w[sl], k_pool, ks_pool, table, q0, q0 + Tq,
+                                         2048, page_size=page)
+        dsa.check_device_error()
+        assert torch.equal(idx, ref), (q0, Tq)
+
+
+def test_prefill_chunk_bad_page_is_reported(dsa):
+    L = 4096
+    P = workloads.make_prefill(L, 64, 128, 1, 2048, seed=53, device="cuda")
+    k_pool, ks_pool, table = _page_one(P.k_cache, P.k_scale, 64, torch.Generator().manual_seed(1))
+    dsa.check_device_error()
+    bad = table.clone()
+    bad[10] = -7
+    dsa.index_topk_chunk_paged(P.q_I, P.q_scale, P.w, k_pool, ks_pool, bad, 0, L, 2048, page_size=64)
+    st, _ = dsa.device_error()
+    assert st == -6  # DSA_ERR_BAD_INDEX
+    # rows before the bad page never read it
+    ref = dsa.index_topk_chunk(P.q_I[:640], P.q_scale[:640], P.w[:640], P.k_cache[:640], P.k_scale[:640], 0, 2048)
+    idx = dsa.index_topk_chunk_paged(P.q_I[:640], P.q_scale[:640], P.w[:640], k_pool, ks_pool, bad, 0, 640, 2048,
+                                     page_size=64)
+    assert dsa.device_error()[0] == 0
+    assert torch.equal(idx, ref)
