@@ -309,11 +309,13 @@ dsa_status dsa_index_topk_decode_noalloc(const uint8_t* q_I, const float* q_scal
  * ------------------------------------------------------------------------ */
 /* Failure-path self-test: enqueues on `stream` one small kernel that waits,
  * with the same bounded wait every kernel here uses, on a barrier nothing
- * completes. After about 2^31 SM cycles (~1 s) the wait gives up, records
+ * completes. After wait_cycles SM cycles (0: the library's own bound of 2^31
+ * cycles, about a second; at most 2^31) the wait gives up, records
  * DSA_ERR_TIMEOUT with site 99 and the kernel exits; the next
  * dsa_get_device_error reports it and the context stays usable. Returns the
- * launch status. No counterpart in the pages. */
-dsa_status dsa_selftest_wait_timeout(void* stream);
+ * launch status, or DSA_ERR_INVALID_ARG for wait_cycles outside [0, 2^31].
+ * No counterpart in the pages. */
+dsa_status dsa_selftest_wait_timeout(long long wait_cycles, void* stream);
 
 /* Synchronises `stream`, then reads and clears the device error word of the
  * current device: DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_BAD_INDEX (*detail gets

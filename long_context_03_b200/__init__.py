@@ -70,7 +70,7 @@ def lib() -> ctypes.CDLL:
             L.dsa_sparse_mla_attn_decode.argtypes = [P, P, P, I, I, I, I, F, P, P, P]
             L.dsa_index_topk_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P, P]
             L.dsa_get_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_uint)]
-            L.dsa_selftest_wait_timeout.argtypes = [P]
+            L.dsa_selftest_wait_timeout.argtypes = [ctypes.c_longlong, P]
             L.dsa_status_string.argtypes = [I]
             L.dsa_status_string.restype = ctypes.c_char_p
             L.dsa_last_error.argtypes = []
@@ -492,10 +492,11 @@ def device_error(device=None) -> Tuple[int, int]:
     return int(st), int(detail.value)
 
 
-def selftest_wait_timeout(device=None):
+def selftest_wait_timeout(wait_cycles: int = 0, device=None):
     """Enqueue the failure-path self-test: a kernel whose bounded wait runs out
-    (~1 s) and records DSA_ERR_TIMEOUT; read it with device_error()."""
-    _check(lib().dsa_selftest_wait_timeout(_stream(device)))
+    after wait_cycles SM cycles (0: the library's ~1 s bound) and records
+    DSA_ERR_TIMEOUT; read it with device_error()."""
+    _check(lib().dsa_selftest_wait_timeout(int(wait_cycles), _stream(device)))
 
 
 def check_device_error(device=None):

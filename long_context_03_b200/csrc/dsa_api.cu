@@ -126,9 +126,10 @@ int rows_per_block(int H_I) { return 2 * (256 / H_I); }
 
 bool prefill_shape_ok(int H_I, int d_I) { return (H_I == 8 || H_I == 64) && (d_I == 64 || d_I == 128); }
 
+// Workspace of the prefill selection: the persistent CTAs' candidate lists,
+// then the re-run list.
 struct WsPrefill {
   uint64_t* cand;
-  uint64_t* sel;
   int* redo;  // [0]: count, [4 ..]: row blocks to re-run
   size_t bytes;
 };
@@ -137,12 +138,10 @@ WsPrefill prefill_ws_layout(void* base, int L, int H_I, int topk, int grid) {
   WsPrefill w;
   const int nrb = (L + rows_per_block(H_I) - 1) / rows_per_block(H_I);
   const size_t cand_bytes = static_cast<size_t>(grid) * rows_per_block(H_I) * select_cap(topk) * 8;
-  const size_t sel_bytes = static_cast<size_t>(L) * topk * 8;
   const size_t redo_bytes = (static_cast<size_t>(nrb) + 4) * 4;
   w.cand = reinterpret_cast<uint64_t*>(base);
-  w.sel = reinterpret_cast<uint64_t*>(reinterpret_cast<char*>(base) + cand_bytes);
-  w.redo = reinterpret_cast<int*>(reinterpret_cast<char*>(base) + cand_bytes + sel_bytes);
-  w.bytes = cand_bytes + sel_bytes + redo_bytes;
+  w.redo = reinterpret_cast<int*>(reinterpret_cast<char*>(base) + cand_bytes);
+  w.bytes = cand_bytes + redo_bytes;
   return w;
 }
 
@@ -155,7 +154,7 @@ dsa_status launch_prefill(const uint8_t* q_I, const uint8_t* k_cache, const IdxP
                           cudaStream_t st) {
   using C = IdxPrefillCfg<HI, DI>;
   CUtensorMap tmQ, tmK;
-  dsa_status s = make_map_u8(&tmQ, q_I, DI, static_cast<uint64_t>(p.Tq) * HI, DI, C::NCOL);
+  dsa_status s = make_map_u8(&tmQ, q_I, DI, static_cast<uint64_t>(p.Tq) * HI, DI, C::QBOX);
   if (s != DSA_OK) return s;
   if (kPaged) {
     // the pool's rows, one page (at most one key tile) per box
@@ -190,17 +189,6 @@ dsa_status dispatch_prefill(int H_I, int d_I, const uint8_t* q_I, const uint8_t*
   return fail(DSA_ERR_UNSUPPORTED, "H_I=%d d_I=%d not supported", H_I, d_I);
 }
 
-dsa_status launch_rank_sort(const uint64_t* keys, int32_t* idx, int K, int rows, cudaStream_t st) {
-  if (rows <= 0) return DSA_OK;
-  if (K <= 64) rank_sort_kernel<64><<<rows, 256, 0, st>>>(keys, idx, K, rows);
-  else if (K <= 128) rank_sort_kernel<128><<<rows, 256, 0, st>>>(keys, idx, K, rows);
-  else if (K <= 256) rank_sort_reg_kernel<256><<<rows, 32, 0, st>>>(keys, idx, K, rows);
-  else if (K <= 512) rank_sort_reg_kernel<512><<<rows, 64, 0, st>>>(keys, idx, K, rows);
-  else if (K <= 1024) rank_sort_reg_kernel<1024><<<rows, 128, 0, st>>>(keys, idx, K, rows);
-  else rank_sort_reg_kernel<2048><<<rows, 256, 0, st>>>(keys, idx, K, rows);
-  return check_launch("rank_sort_kernel");
-}
-
 __global__ void fill_f32_kernel(float* p, size_t n, float v) {
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<size_t>(gridDim.x) * blockDim.x)
@@ -209,11 +197,11 @@ __global__ void fill_f32_kernel(float* p, size_t n, float v) {
 
 // ---- failure-path self-test ----
 // One CTA waits, with the library's bounded wait, on an mbarrier that no
-// thread arrives on: the wait gives up after its bound (~2^31 cycles), records
-// a timeout with site kSelftestSite in the device error word and the kernel
-// returns, leaving the context usable.
+// thread arrives on: the wait gives up after `bound` cycles, records a timeout
+// with site kSelftestSite in the device error word and the kernel returns,
+// leaving the context usable.
 constexpr unsigned int kSelftestSite = 99;
-__global__ void selftest_wait_timeout_kernel() {
+__global__ void selftest_wait_timeout_kernel(long long bound) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
   if (threadIdx.x == 0) {
@@ -223,7 +211,7 @@ __global__ void selftest_wait_timeout_kernel() {
   }
   __syncthreads();
   const AbortFlag ab{&abort_flag};
-  if (threadIdx.x == 0) mbar_wait(&bar, 0, ab, kSelftestSite);
+  if (threadIdx.x == 0) mbar_wait_bounded(&bar, 0, ab, kSelftestSite, bound);
   __syncthreads();
 }
 
@@ -415,7 +403,7 @@ static dsa_status index_topk_impl(const uint8_t* q_I, const float* q_scale, cons
   p.rb_end = nrb;
   p.cand = ws.cand;
   p.cap = select_cap(topk);
-  p.sel_keys = ws.sel;
+  p.idx = idx;
   p.spec_min_t = spec_min_row(topk);
   p.redo_count = ws.redo;
   p.redo_list = ws.redo + 4;
@@ -436,10 +424,8 @@ static dsa_status index_topk_impl(const uint8_t* q_I, const float* q_scale, cons
   r.list_count = ws.redo;
   r.redo_count = nullptr;
   r.redo_list = nullptr;
-  s = (select_mq(topk) == 1) ? dispatch_prefill<true, 1>(H_I, d_I, q_I, k_cache, r, grid, st)
-                             : dispatch_prefill<true, 4>(H_I, d_I, q_I, k_cache, r, grid, st);
-  if (s != DSA_OK) return s;
-  return launch_rank_sort(ws.sel, idx, topk, Tq, st);
+  return (select_mq(topk) == 1) ? dispatch_prefill<true, 1>(H_I, d_I, q_I, k_cache, r, grid, st)
+                                : dispatch_prefill<true, 4>(H_I, d_I, q_I, k_cache, r, grid, st);
 }
 
 dsa_status dsa_index_topk(const uint8_t* q_I, const float* q_scale, const float* w, const uint8_t* k_cache,
@@ -477,10 +463,10 @@ dsa_status dsa_index_topk_chunk_paged(const uint8_t* q_I, const float* q_scale, 
 }
 
 // ---- packed batch of sequences (cu_seqlens) ----
-// Workspace: candidate lists and selected keys as for total_q rows, then the
-// re-run list and the row-block table (upper bound on the block count).
+// Workspace: candidate lists as for one sequence, then the re-run list and
+// the row-block table (upper bound on the block count).
 struct WsVarlen {
-  WsPrefill base;
+  uint64_t* cand;
   int* redo;
   int* table;  // blk_seq[nb_max], blk_lrb[nb_max], cuq[nseq+1], cuk[nseq+1], q0[nseq]
   size_t bytes;
@@ -489,16 +475,14 @@ static int varlen_max_blocks(int total_q, int nseq, int H_I) { return total_q / 
 static WsVarlen varlen_ws_layout(void* base, int total_q, int nseq, int H_I, int topk, int grid) {
   WsVarlen w;
   const size_t cand_bytes = static_cast<size_t>(grid) * rows_per_block(H_I) * select_cap(topk) * 8;
-  const size_t sel_bytes = static_cast<size_t>(total_q) * topk * 8;
   const int nbm = varlen_max_blocks(total_q, nseq, H_I);
   const size_t redo_bytes = (static_cast<size_t>(nbm) + 4) * 4;
   const size_t table_bytes = (2 * static_cast<size_t>(nbm) + 3 * static_cast<size_t>(nseq) + 2) * 4;
   char* c = reinterpret_cast<char*>(base);
-  w.base.cand = reinterpret_cast<uint64_t*>(c);
-  w.base.sel = reinterpret_cast<uint64_t*>(c + cand_bytes);
-  w.redo = reinterpret_cast<int*>(c + cand_bytes + sel_bytes);
-  w.table = reinterpret_cast<int*>(c + cand_bytes + sel_bytes + redo_bytes);
-  w.bytes = cand_bytes + sel_bytes + redo_bytes + table_bytes;
+  w.cand = reinterpret_cast<uint64_t*>(c);
+  w.redo = reinterpret_cast<int*>(c + cand_bytes);
+  w.table = reinterpret_cast<int*>(c + cand_bytes + redo_bytes);
+  w.bytes = cand_bytes + redo_bytes + table_bytes;
   return w;
 }
 
@@ -580,9 +564,9 @@ dsa_status dsa_index_topk_varlen(const uint8_t* q_I, const float* q_scale, const
   p.topk = topk;
   p.rb_begin = 0;
   p.rb_end = nblk;
-  p.cand = ws.base.cand;
+  p.cand = ws.cand;
   p.cap = select_cap(topk);
-  p.sel_keys = ws.base.sel;
+  p.idx = idx;
   p.spec_min_t = spec_min_row(topk);
   p.redo_count = ws.redo;
   p.redo_list = ws.redo + 4;
@@ -601,10 +585,8 @@ dsa_status dsa_index_topk_varlen(const uint8_t* q_I, const float* q_scale, const
   r.list_count = ws.redo;
   r.redo_count = nullptr;
   r.redo_list = nullptr;
-  s = (select_mq(topk) == 1) ? dispatch_prefill<true, 1>(H_I, d_I, q_I, k_cache, r, g, st)
-                             : dispatch_prefill<true, 4>(H_I, d_I, q_I, k_cache, r, g, st);
-  if (s != DSA_OK) return s;
-  return launch_rank_sort(ws.base.sel, idx, topk, total_q, st);
+  return (select_mq(topk) == 1) ? dispatch_prefill<true, 1>(H_I, d_I, q_I, k_cache, r, g, st)
+                                : dispatch_prefill<true, 4>(H_I, d_I, q_I, k_cache, r, g, st);
 }
 
 dsa_status dsa_index_topk_rerun_count(const void* workspace, int L, int H_I, int d_I, int topk, int* count,
@@ -887,8 +869,11 @@ dsa_status dsa_get_device_error(void* stream, unsigned int* detail) {
   return fail(DSA_ERR_BAD_INDEX, "an index or page-table entry was outside its cache (site %u)", h >> 8);
 }
 
-dsa_status dsa_selftest_wait_timeout(void* stream) {
-  selftest_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+dsa_status dsa_selftest_wait_timeout(long long wait_cycles, void* stream) {
+  if (wait_cycles < 0 || wait_cycles > kWaitBoundCycles)
+    return fail(DSA_ERR_INVALID_ARG, "wait_cycles=%lld not in [0, %lld]", wait_cycles, kWaitBoundCycles);
+  selftest_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(wait_cycles ? wait_cycles
+                                                                                         : kWaitBoundCycles);
   return check_launch("selftest_wait_timeout_kernel");
 }
 

@@ -77,22 +77,26 @@ struct AbortFlag {
   __device__ __forceinline__ void raise() const { *flag = 1; }
 };
 
-// Wait for the phase with the given parity to complete. Bounded: on timeout
-// records kErrTimeout (with `where`), raises the CTA abort flag, returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, AbortFlag ab,
-                                          unsigned int where) {
+// Wait for the phase with the given parity to complete. Bounded: after
+// `bound` SM cycles it records kErrTimeout (with `where`), raises the CTA abort
+// flag and returns false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, AbortFlag ab, unsigned int where,
+                                                  long long bound) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(a, parity)) return true;
     if (ab.raised()) return false;
-    if (clock64() - t0 > kWaitBoundCycles) {
+    if (clock64() - t0 > bound) {
       set_device_error(kErrTimeout, where);
       ab.raise();
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, AbortFlag ab, unsigned int where) {
+  return mbar_wait_bounded(bar, parity, ab, where, kWaitBoundCycles);
 }
 
 // Warp-wide wait: every lane of the (converged) warp waits, and the result is
@@ -388,5 +392,33 @@ __device__ __forceinline__ int32_t rank_key_index(uint64_t key) {
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
+
+// A named barrier shared by a group of whole warps inside a CTA whose other
+// waits are bounded. bar.sync itself cannot time out, so the group keeps this
+// rule: a warp that has seen the CTA's abort flag never waits at the barrier
+// again and, when it stops, calls leave() exactly once. Every member then
+// either waits at the next barrier or has left, so that barrier completes;
+// members leaving it see the flag and stop too, and the barrier after it has
+// nobody waiting. The flag is read by lane 0 and broadcast, so a warp never
+// splits at a barrier.
+struct GroupBar {
+  uint32_t id, nthreads;
+  AbortFlag ab;
+  __device__ __forceinline__ bool aborted() const {
+    return __shfl_sync(0xffffffffu, ab.raised() ? 1 : 0, 0) != 0;
+  }
+  // Wait for the group; false (without waiting, or after it) once the CTA aborted.
+  __device__ __forceinline__ bool sync() const {
+    if (aborted()) return false;
+    named_bar_sync(id, nthreads);
+    return !aborted();
+  }
+  // The calling warp stops for good: count it in at the barrier the others
+  // may be waiting at.
+  __device__ __forceinline__ void leave() const {
+    __threadfence_block();
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+  }
+};
 
 }  // namespace dsa

@@ -17,8 +17,8 @@
 // the sequence's global histogram when the CTA moves to another sequence.
 //
 // Selection kernel: one CTA per sequence runs an exact radix select over the
-// 64-bit ranking keys (score, then lower index) of its scores and writes the
-// top-k keys unordered; rank_sort_kernel orders them.
+// 64-bit ranking keys (score, then lower index) of its scores, then ranks the
+// selected keys in shared memory and writes the sequence's index row.
 #pragma once
 
 #include "dsa_common.cuh"
@@ -484,7 +484,12 @@ __device__ __forceinline__ void decode_select_body(const float* __restrict__ sco
       v[j] = (i < inb) ? bin_keys[i] : 0ull;
     }
     uint64_t floor = 1ull;
-    if (need < inb) floor = radix_select_floor<NT, kDecodeSelBinCap / NT>(v, need, scr, tid, 1);
+    // no bounded waits in this kernel: the group barrier never sees an abort
+    __shared__ int never_aborts;
+    if (tid == 0) never_aborts = 0;
+    __syncthreads();
+    const GroupBar bar{1, NT, AbortFlag{&never_aborts}};
+    if (need < inb) floor = radix_select_floor<NT, kDecodeSelBinCap / NT>(v, need, scr, tid, bar);
 #pragma unroll
     for (int j = 0; j < kDecodeSelBinCap / NT; ++j)
       if (v[j] != 0 && v[j] >= floor) dst[atomicAdd(&wpos, 1)] = v[j];

@@ -26,8 +26,8 @@
 // to exactly topk keys by a cooperative radix select and the threshold rises
 // to the cut. Nothing that could still rank in the top-k is ever dropped, and
 // the L x L score matrix never exists anywhere. At the end of a row block each
-// row's exact top-k keys go to `sel_keys` (unordered); rank_sort_kernel then
-// orders them.
+// row's exact top-k keys are ranked in shared memory and written as token
+// indices.
 #pragma once
 
 #include "dsa_common.cuh"
@@ -38,17 +38,20 @@ namespace dsa {
 template <int HI, int DI>
 struct IdxPrefillCfg {
   static constexpr int BM = 128;               // keys per tile (MMA M, TMEM lanes)
-  static constexpr int NCOL = 256;             // accumulator columns per buffer (MMA N)
+  static constexpr int NCOL = 128;             // accumulator columns per buffer (MMA N)
+  static constexpr int NACC = 4;               // accumulator buffers: all 512 TMEM columns
   static constexpr int TB = NCOL / HI;         // tokens per accumulator buffer
-  static constexpr int NACC = 2;               // accumulator buffers
   static constexpr int RB = TB * NACC;         // tokens per row block
   static constexpr int KST = 4;                // key-tile ring depth
-  static constexpr int QBUF_BYTES = NCOL * DI; // one Q half: 256 (token, head) rows x d_I bytes
+  static constexpr int QROWS = RB * HI;        // (token, head) query rows of a row block
+  static constexpr int QBOX = 256;             // query rows per TMA box
+  static constexpr int QBYTES = QROWS * DI;
   static constexpr int KTILE_BYTES = BM * DI;
-  static constexpr int NEPI = 16;              // epilogue warps (4 per TMEM lane quarter)
+  static constexpr int NEPI = 16;              // epilogue warps: 4 per buffer, one per TMEM lane quarter
   static constexpr int NTHREADS = (2 + NEPI) * 32;
   static constexpr int NET = NEPI * 32;        // epilogue threads
-  static constexpr int TOK_PER_WARP = TB / 4;  // tokens of a buffer per epilogue warp (64 columns)
+  static constexpr int TOK_PER_WARP = TB;      // an epilogue warp scores every token of its buffer
+  static constexpr int TPH = 64 / HI;          // tokens per 64-column half of a buffer
   static constexpr int CHECK_EVERY = 4;        // key tiles between list-capacity checks
   static constexpr int NSAMPLE = 8;            // key tiles scored first to set a row's starting threshold
   static constexpr SwizzleMode SW = (DI == 128) ? kSw128 : kSw64;
@@ -58,22 +61,30 @@ struct IdxPrefillCfg {
 
   // shared memory carve-up (offsets from a 1024-byte aligned base)
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + NACC * QBUF_BYTES;
+  static constexpr int OFF_K = OFF_Q + QBYTES;
   static constexpr int OFF_W = OFF_K + KST * KTILE_BYTES;  // f32 [RB][HI]
   static constexpr int OFF_QS = OFF_W + RB * HI * 4;       // f32 [RB]
   static constexpr int OFF_THR = OFF_QS + RB * 4;          // u64 [RB]
   static constexpr int OFF_CNT = OFF_THR + RB * 8;         // i32 [RB][4] sub-list counts
   static constexpr int OFF_SCR = OFF_CNT + RB * 16;        // i32 select scratch
-  static constexpr int SCR_INTS = (select_scratch_ints(NEPI * 32) > cut_scratch_ints()) ? select_scratch_ints(NEPI * 32)
-                                                                                        : cut_scratch_ints();
-  static constexpr int OFF_BAR = (OFF_SCR + SCR_INTS * 4 + 7) / 8 * 8;
+  // select scratch: [0, 2048) bin counts, [2048, 2112) the cuts' small fields,
+  // [2112, 4160) bin starts and [4160, 4224) small fields of the final ranking;
+  // the radix select's per-warp histograms overlay [0, 4112)
+  static constexpr int SCR_START = cut_scratch_ints();
+  static constexpr int SCR_SMALL = SCR_START + 2048;
+  static constexpr int SCR_INTS = SCR_SMALL + 64;
+  static_assert(SCR_INTS >= select_scratch_ints(NEPI * 32), "radix select scratch");
+  static constexpr int SRT_N = 4096;                                       // keys of the final ranking buffer
+  static constexpr int OFF_SRT = (OFF_SCR + SCR_INTS * 4 + 15) / 16 * 16;  // u64 [SRT_N]
+  static constexpr int OFF_BAR = OFF_SRT + SRT_N * 8;
   static constexpr int NBAR = 2 + 2 * KST + 2 * NACC;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;      // tmem base, abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
 
-  static_assert(HI * TB == NCOL, "heads must divide 256");
-  static_assert(TB % 4 == 0, "four epilogue warps per lane quarter split a buffer's tokens");
-  static_assert(TOK_PER_WARP * HI == 64, "one 64-column slice per warp and buffer");
+  static_assert(HI * TB == NCOL && HI <= 64, "heads must divide a buffer's 128 columns");
+  static_assert(QROWS % QBOX == 0, "whole query boxes per row block");
+  static_assert(RB <= 64, "one bit per row in the 64-bit cut mask");
+  static_assert(NACC * NCOL == 512, "the buffers fill TMEM");
 };
 
 struct IdxPrefillParams {
@@ -87,7 +98,7 @@ struct IdxPrefillParams {
   // selection mode
   uint64_t* cand;        // [gridDim.x][RB][cap] candidate lists
   int cap;
-  uint64_t* sel_keys;    // [L][topk] exact top-k keys per row, unordered, 0-padded
+  int32_t* idx;          // [Tq][topk] token indices per row, ranked, -1 padded
   // Sampled starting thresholds: row blocks with t0 >= spec_min_t (0: never)
   // first score NSAMPLE evenly spread key tiles and start from the sample's
   // r-th largest score (r ~ 2.5 * topk * sampled keys / (t+1)). A row that
@@ -119,34 +130,52 @@ struct IdxPrefillParams {
   int page_shift, pool_pages;
 };
 
-// sum_j w[j] * max(x_j, 0) over the H_I accumulator values of one token
-// (registers loaded from TMEM), written as (sum_j w[j]*x_j + sum_j w[j]*|x_j|)/2
-// so that both sums run on the FMA pipe: acc[0..3] take w*x as two packed
-// float pairs (fma.rn.f32x2 on register pairs straight from the TMEM load),
-// acc[4..7] take w*|x| with the absolute value folded into the scalar FMA.
-// The halves cancel exactly where every head is negative (an exact zero stays
-// zero). Shared by both modes so their scores are bit-identical.
+// sum_j w[j] * ReLU(x_j) over the H_I accumulator values of one token
+// (registers loaded from TMEM), in eight partial sums held as four float pairs
+// and accumulated with the packed two-lane FMA: head j of each group of eight
+// goes to partial sum j. In a group the first six ReLUs are max(x, 0) (ALU
+// pipe) and the last two x + |x| = 2 ReLU(x) (FMA pipe), so both pipes carry
+// part of the work; that last pair accumulates exactly twice the plain sums
+// (scaling by two is exact in binary floating point) and is halved at the
+// end, so the result is bit-identical to using max(x, 0) throughout. A token
+// whose heads all ReLU to zero gets exactly 0. The weights come from shared
+// memory as 16-byte vectors. Shared by both modes, so scores are identical.
 template <int HI>
-__device__ __forceinline__ void relu_weighted_acc(float (&acc)[8], const uint32_t* x, const float* __restrict__ w) {
-  static_assert(HI % 4 == 0, "a multiple of 4 heads");
+__device__ __forceinline__ float head_sum(const uint32_t* x, const float* __restrict__ w) {
+  static_assert(HI % 8 == 0, "groups of eight heads");
+  float2 acc[4];
 #pragma unroll
-  for (int j = 0; j < HI; j += 4) {
+  for (int a = 0; a < 4; ++a) acc[a] = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int pr = 0; pr < 2; ++pr) {
-      uint64_t d, wa, xa, ca;
-      asm("mov.b64 %0, {%1, %2};" : "=l"(wa) : "f"(w[j + 2 * pr]), "f"(w[j + 2 * pr + 1]));
-      asm("mov.b64 %0, {%1, %2};" : "=l"(xa) : "r"(x[j + 2 * pr]), "r"(x[j + 2 * pr + 1]));
-      asm("mov.b64 %0, {%1, %2};" : "=l"(ca) : "f"(acc[2 * pr]), "f"(acc[2 * pr + 1]));
-      asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(wa), "l"(xa), "l"(ca));
-      asm("mov.b64 {%0, %1}, %2;" : "=f"(acc[2 * pr]), "=f"(acc[2 * pr + 1]) : "l"(d));
+  for (int j = 0; j < HI; j += 8) {
+    const float4 w0 = *reinterpret_cast<const float4*>(w + j);
+    const float4 w1 = *reinterpret_cast<const float4*>(w + j + 4);
+    float r[8];
+#pragma unroll
+    for (int a = 0; a < 6; ++a) r[a] = fmaxf(__uint_as_float(x[j + a]), 0.f);
+#pragma unroll
+    for (int a = 6; a < 8; ++a) {
+      const float v = __uint_as_float(x[j + a]);
+      r[a] = __fadd_rn(v, fabsf(v));
     }
-#pragma unroll
-    for (int a = 0; a < 4; ++a) acc[4 + a] = __fmaf_rn(w[j + a], fabsf(__uint_as_float(x[j + a])), acc[4 + a]);
+    acc[0] = __ffma2_rn(make_float2(w0.x, w0.y), make_float2(r[0], r[1]), acc[0]);
+    acc[1] = __ffma2_rn(make_float2(w0.z, w0.w), make_float2(r[2], r[3]), acc[1]);
+    acc[2] = __ffma2_rn(make_float2(w1.x, w1.y), make_float2(r[4], r[5]), acc[2]);
+    acc[3] = __ffma2_rn(make_float2(w1.z, w1.w), make_float2(r[6], r[7]), acc[3]);
   }
+  return ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + 0.5f * (acc[3].x + acc[3].y));
 }
-__device__ __forceinline__ float relu_weighted_finish(const float (&acc)[8]) {
-  return 0.5f * (((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7])));
+
+// Threshold of a row as a float: a score s can pass only if s >= this value
+// (the score part of the 64-bit threshold; -inf for the empty threshold 0).
+__device__ __forceinline__ float thr_score(uint64_t thr) {
+  const uint32_t hi = static_cast<uint32_t>(thr >> 32);
+  return hi == 0 ? -INFINITY : order_key_float(hi);
 }
+
+// Largest bin the final ranking scans key by key (more: the exact select and
+// the bitonic ranking take over).
+constexpr int kBinRankMax = 96;
 
 // Key tile of step i of a row block's sequence: with sampling, steps
 // 0..NSAMPLE-1 are tiles at the middles of NSAMPLE equal strata of the
@@ -200,6 +229,7 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
   uint64_t* thr_s = reinterpret_cast<uint64_t*>(smem + C::OFF_THR);
   int* cnt_s = reinterpret_cast<int*>(smem + C::OFF_CNT);
   int* scr_s = reinterpret_cast<int*>(smem + C::OFF_SCR);
+  uint64_t* srt_s = reinterpret_cast<uint64_t*>(smem + C::OFF_SRT);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
@@ -211,7 +241,7 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
   int* abort_s = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
   // bit tl: a sub-list of row tl may overflow before the next check (set by
   // the appending warp, read at the capacity checks)
-  int* cutmask_s = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
+  unsigned long long* cutmask_s = reinterpret_cast<unsigned long long*>(smem + C::OFF_MISC + 8);
   const AbortFlag ab{abort_s};
 
   const uint32_t warp = warp_id();
@@ -227,7 +257,7 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
     }
     for (int i = 0; i < C::NACC; ++i) {
       mbar_init(acc_full + i, 1);
-      mbar_init(acc_empty + i, C::NEPI);
+      mbar_init(acc_empty + i, C::NEPI / C::NACC);
     }
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
@@ -286,9 +316,9 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
         const int nsteps = nkt + (spec ? C::NSAMPLE : 0);
         if (!mbar_wait(q_empty, qe_phase, ab, 1)) break;
         qe_phase ^= 1;
-        mbar_arrive_expect_tx(q_full, C::NACC * C::QBUF_BYTES);
-        for (int b = 0; b < C::NACC; ++b)
-          tma_load_2d(q_s + b * C::QBUF_BYTES, &tmQ, q_full, 0, (r0 + b * C::TB) * HI);
+        mbar_arrive_expect_tx(q_full, C::QBYTES);
+        for (int b = 0; b < C::QROWS / C::QBOX; ++b)
+          tma_load_2d(q_s + b * C::QBOX * DI, &tmQ, q_full, 0, r0 * HI + b * C::QBOX);
         bool ok = true;
         // paged: one box of R = min(page, BM) rows per page of the tile; the
         // next tile's page entries load before the wait for this tile's slot
@@ -340,12 +370,14 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer: the warp waits converged, one elected lane issues ----------------
+    // Per key tile: one accumulator buffer after the other (tokens b * TB ..
+    // b * TB + TB - 1 into buffer b), each as soon as its four epilogue warps
+    // have released it.
     {
       uint32_t qf_phase = 0;
       int kslot = 0;
       uint32_t kf_phase = 0;
-      uint32_t ae_phase[C::NACC];
-      for (int b = 0; b < C::NACC; ++b) ae_phase[b] = 1;
+      uint32_t ae_bits = (1u << C::NACC) - 1u;  // bit b: parity of buffer b's next release
       const uint32_t q_base = smem_u32(q_s);
       const uint32_t k_base = smem_u32(k_s);
       for (int j = blockIdx.x; j < nrb; j += G) {
@@ -361,25 +393,28 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
           if (!mbar_wait_warp(k_full + kslot, kf_phase, ab, 6)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = k_base + kslot * C::KTILE_BYTES;
-          for (int b = 0; b < C::NACC; ++b) {
-            if (!mbar_wait_warp(acc_empty + b, ae_phase[b], ab, 7)) { ok = false; break; }
-            ae_phase[b] ^= 1;
-            tc_fence_after();
-            if (elect_one()) {
-              const uint32_t b_addr = q_base + b * C::QBUF_BYTES;
 #pragma unroll
-              for (int kk = 0; kk < C::KSTEPS; ++kk) {
-                const uint64_t ad = smem_desc(a_addr + kk * 32, 16, C::SBO, C::SW);
-                const uint64_t bd = smem_desc(b_addr + kk * 32, 16, C::SBO, C::SW);
-                mma_f8(tmem + b * C::NCOL, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
+          for (int b = 0; b < C::NACC; ++b) {
+            if (ok && !mbar_wait_warp(acc_empty + b, (ae_bits >> b) & 1u, ab, 7)) ok = false;
+            if (ok) {
+              ae_bits ^= 1u << b;
+              tc_fence_after();
+              if (elect_one()) {
+                const uint32_t b_addr = q_base + b * C::NCOL * DI;
+#pragma unroll
+                for (int kk = 0; kk < C::KSTEPS; ++kk) {
+                  const uint64_t ad = smem_desc(a_addr + kk * 32, 16, C::SBO, C::SW);
+                  const uint64_t bd = smem_desc(b_addr + kk * 32, 16, C::SBO, C::SW);
+                  mma_f8(tmem + b * C::NCOL, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
+                }
+                tc_commit(acc_full + b);
+                if (b == C::NACC - 1) {
+                  tc_commit(k_empty + kslot);
+                  if (kt == nsteps - 1) tc_commit(q_empty);
+                }
               }
-              tc_commit(acc_full + b);
-              if (b == C::NACC - 1) {
-                tc_commit(k_empty + kslot);
-                if (kt == nsteps - 1) tc_commit(q_empty);
-              }
+              __syncwarp();
             }
-            __syncwarp();
           }
           if (!ok) break;
           if (++kslot == C::KST) { kslot = 0; kf_phase ^= 1; }
@@ -392,17 +427,20 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
     const int e = static_cast<int>(warp) - 2;          // 0..NEPI-1
     const int et = e * 32 + static_cast<int>(lane);    // 0..NET-1
     const int quarter = static_cast<int>(warp & 3);    // TMEM lane quarter this warp may access
-    const int half = e / 4;                            // which quarter of a buffer's tokens
+    const int grp = e / 4;                             // the accumulator buffer this warp drains
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t lanemask_lt = (1u << lane) - 1u;
-    uint32_t af_phase[C::NACC];
-    for (int b = 0; b < C::NACC; ++b) af_phase[b] = 0;
+    constexpr int TPW = C::TOK_PER_WARP;
+    constexpr int NR = TPW;  // rows this warp scores: the tokens of its buffer
+    const GroupBar bar{1, C::NET, ab};
+    uint32_t af_phase = 0;  // parity of this warp's buffer's next completed fill
     // Row tl's list is four quarter sub-lists of capq keys; sub-list q only
     // receives keys from TMEM lane quarter q, so exactly one warp appends to
-    // it and its count needs no atomics.
+    // it: its count lives in that warp's registers between cuts.
     const int capq = p.cap / 4;
     uint64_t* my_cand = p.cand + static_cast<size_t>(blockIdx.x) * C::RB * p.cap;
-    int* pos_s = scr_s + cut_scratch_ints() - 16;  // 9 ints: warp sums of the block scan
+    int* pos_s = scr_s + cut_scratch_ints() - 16;  // 16 ints: warp sums of the block scan
+    auto row_of = [&](int r) { return grp * C::TB + r; };
 
     for (int j = blockIdx.x; j < nrb; j += G) {
       const int rb = block_of(j);
@@ -413,6 +451,7 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
       const int nkt = tlast / C::BM + 1;
       const bool spec = samples(t0, nkt);
       const int nsteps = nkt + (spec ? C::NSAMPLE : 0);
+      const bool ragged = r0 + C::RB > bk.rend;  // the block runs past its sequence's last query row
       // per-row-block state
       for (int i = et; i < C::RB * HI; i += C::NET) {
         const int r = r0 + i / HI;
@@ -425,11 +464,36 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
       }
       for (int i = et; i < 4 * C::RB; i += C::NET) cnt_s[i] = 0;
       if (et == 0) *cutmask_s = 0;
-      named_bar_sync(1, C::NET);
+      if (!bar.sync()) break;
+      // this warp's rows in registers: query scale, threshold (exact and as a
+      // score), and its sub-list's count
+      float qs_r[NR], thf_r[NR];
+      uint64_t th_r[NR];
+      int cnt_r[NR];
+#pragma unroll
+      for (int r = 0; r < NR; ++r) {
+        qs_r[r] = qs_s[row_of(r)];
+        th_r[r] = 0ull;
+        thf_r[r] = -INFINITY;
+        cnt_r[r] = 0;
+      }
+      // cuts happen in shared memory: publish the counts before, reload after
+      auto publish_counts = [&]() {
+        if (lane == 0) {
+#pragma unroll
+          for (int r = 0; r < NR; ++r) cnt_s[row_of(r) * 4 + quarter] = cnt_r[r];
+        }
+      };
+      auto reload_rows = [&]() {
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+          th_r[r] = thr_s[row_of(r)];
+          thf_r[r] = thr_score(th_r[r]);
+          cnt_r[r] = cnt_s[row_of(r) * 4 + quarter];
+        }
+      };
       bool ok = true;
       float ks_next = 0.f;
-      // paged: page entry of the key two steps ahead, its scale one step ahead
-      // (no dependent load waits inside a step)
       [[maybe_unused]] int pg_next = -1;
       {
         const int s0 = tile_at<C::NSAMPLE>(0, nkt, spec) * C::BM + quarter * 32 + static_cast<int>(lane);
@@ -459,101 +523,60 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
             ks_next = (sn < bk.L) ? __ldg(p.k_scale + bk.kbase + sn) : 0.f;
           }
         }
-        for (int b = 0; b < C::NACC; ++b) {
-          if (!mbar_wait(acc_full + b, af_phase[b], ab, 8)) { ok = false; break; }
-          af_phase[b] ^= 1;
-          tc_fence_after();
-          // this warp's tokens are 128 consecutive accumulator columns
-          // this warp's 64 columns in two halves: the second half loads while
-          // the first is reduced
-          const uint32_t cbase = tmem + lane_addr + b * C::NCOL + half * 64;
-          uint32_t xa[32], xb[32];
-          tmem_ld32_nowait(cbase, xa);
-          tmem_ld_wait_fence(xa);
-          tmem_ld32_nowait(cbase + 32, xb);
-          // row state first (its loads overlap the arithmetic), every token's
-          // score next (independent chains), then the filter
-          uint64_t thr_r[C::TOK_PER_WARP];
-          int base_r[C::TOK_PER_WARP];
+        // only a tile reaching past the block's first position (the causal
+        // diagonal, or keys past the cache) or a ragged block needs masking
+        const bool masked = ragged || (kt * C::BM + C::BM - 1 > t0);
+        if (!mbar_wait(acc_full + grp, af_phase, ab, 8)) { ok = false; break; }
+        af_phase ^= 1u;
+        tc_fence_after();
+        // this warp's 128 columns of the buffer (TPW tokens of HI heads) in
+        // two halves of 64
+        float raw[TPW];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t x[64];
+          tmem_ld64(tmem + lane_addr + grp * C::NCOL + hh * 64, x);
+#pragma unroll
+          for (int q = 0; q < C::TPH; ++q)
+            raw[hh * C::TPH + q] = head_sum<HI>(x + q * HI, w_s + row_of(hh * C::TPH + q) * HI);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty + grp);  // the tensor core may refill this buffer now
+#pragma unroll
+        for (int r = 0; r < TPW; ++r) {
+          const int tl = row_of(r);
+          const float score = __fmul_rn(__fmul_rn(raw[r], qs_r[r]), ks);
           if constexpr (kSelect) {
-#pragma unroll
-            for (int q = 0; q < C::TOK_PER_WARP; ++q) {
-              const int tl = b * C::TB + half * C::TOK_PER_WARP + q;
-              thr_r[q] = thr_s[tl];
-              base_r[q] = cnt_s[tl * 4 + quarter];
+            // a key can only pass if its score reaches the threshold's score
+            bool pass = score >= thf_r[r];
+            if (masked) pass = pass && (r0 + tl < bk.rend) && (s <= t0 + tl);
+            if (__any_sync(0xffffffffu, pass)) {
+              const uint64_t key = (static_cast<uint64_t>(float_order_key(score)) << 32) |
+                                   static_cast<uint64_t>(~static_cast<uint32_t>(s));
+              const bool pred = pass && key > th_r[r];
+              const uint32_t m = __ballot_sync(0xffffffffu, pred);
+              if (pred)
+                my_cand[static_cast<size_t>(tl) * p.cap + static_cast<size_t>(quarter) * capq + cnt_r[r] +
+                        __popc(m & lanemask_lt)] = key;
+              cnt_r[r] += __popc(m);
             }
-          }
-          float score[C::TOK_PER_WARP];
-          {
-            // columns [0,32) then [32,64) of the slice; a token spans HI columns
-            constexpr int TPH = (HI >= 32) ? 1 : 32 / HI;  // tokens per 32-column half
-            float acc[C::TOK_PER_WARP][8];
-#pragma unroll
-            for (int q = 0; q < C::TOK_PER_WARP; ++q)
-#pragma unroll
-              for (int a = 0; a < 8; ++a) acc[q][a] = 0.f;
-            const int tl0 = b * C::TB + half * C::TOK_PER_WARP;
-            if constexpr (HI >= 32) {
-              relu_weighted_acc<32>(acc[0], xa, w_s + tl0 * HI);
-              tmem_ld_wait_fence(xb);
-              relu_weighted_acc<32>(acc[0], xb, w_s + tl0 * HI + 32);
-            } else {
-#pragma unroll
-              for (int q = 0; q < TPH; ++q) relu_weighted_acc<HI>(acc[q], xa + q * HI, w_s + (tl0 + q) * HI);
-              tmem_ld_wait_fence(xb);
-#pragma unroll
-              for (int q = 0; q < TPH; ++q)
-                relu_weighted_acc<HI>(acc[TPH + q], xb + q * HI, w_s + (tl0 + TPH + q) * HI);
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty + b);  // the tensor core may refill this buffer now
-#pragma unroll
-            for (int q = 0; q < C::TOK_PER_WARP; ++q)
-              score[q] = __fmul_rn(__fmul_rn(relu_weighted_finish(acc[q]), qs_s[tl0 + q]), ks);
-          }
-#pragma unroll
-          for (int q = 0; q < C::TOK_PER_WARP; ++q) {
-            const int tl = b * C::TB + half * C::TOK_PER_WARP + q;
+          } else {
             const int t = t0 + tl;
-            const bool valid = (r0 + tl < bk.rend) && (s <= t);
-            if constexpr (kSelect) {
-              // a key can only pass if its score reaches the threshold's score
-              const uint32_t sk = float_order_key(score[q]);
-              const bool maybe = valid && sk >= static_cast<uint32_t>(thr_r[q] >> 32);
-              if (__any_sync(0xffffffffu, maybe)) {
-                int* cnt = cnt_s + tl * 4 + quarter;
-                const int base = base_r[q];
-                const uint64_t key = (static_cast<uint64_t>(sk) << 32) | static_cast<uint64_t>(~static_cast<uint32_t>(s));
-                const bool pred = maybe && key > thr_r[q];
-                const uint32_t m = __ballot_sync(0xffffffffu, pred);
-                if (pred)
-                  my_cand[static_cast<size_t>(tl) * p.cap + static_cast<size_t>(quarter) * capq + base +
-                          __popc(m & lanemask_lt)] = key;
-                __syncwarp();
-                if (lane == 0 && m) {
-                  *cnt = base + __popc(m);
-                  if (base + __popc(m) > capq - 32 * C::CHECK_EVERY) atomicOr(cutmask_s, 1 << tl);
-                }
-              }
-            } else {
-              if (valid && t >= p.row0 && t < p.row0 + p.nrows)
-                p.scores[static_cast<size_t>(t - p.row0) * p.L + s] = score[q];
-            }
+            if ((r0 + tl < bk.rend) && (s <= t) && t >= p.row0 && t < p.row0 + p.nrows)
+              p.scores[static_cast<size_t>(t - p.row0) * p.L + s] = score;
           }
         }
+        if (!ok) break;
         if constexpr (kSelect) {
-          // Every CHECK_EVERY tiles, cut any list whose sub-list could
-          // overflow before the next check (at most 32 appends per sub-list
-          // and tile): one histogram pass keeps every key in or above the bin
-          // of the k-th largest; if that keeps too many, an exact select
-          // keeps exactly k.
           if (spec && i == C::NSAMPLE - 1) {
             // End of the sample: each row's threshold starts at the score of
-            // its r-th largest sampled key (keys scoring at least that pass;
-            // index bits cleared so equal scores are kept), and the list is
-            // emptied: the sampled tiles come round again in order.
-            named_bar_sync(1, C::NET);
+            // the lower edge of the histogram bin holding its r-th largest
+            // sampled key (keys scoring at least that pass; index bits cleared
+            // so equal scores are kept), and the list is emptied: the sampled
+            // tiles come round again in order.
+            publish_counts();
+            if (!bar.sync()) { ok = false; break; }
             for (int tl = 0; tl < C::RB; ++tl) {
               const int t = t0 + tl;
               if (r0 + tl >= bk.rend) break;
@@ -564,31 +587,39 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
               uint64_t* row = my_cand + static_cast<size_t>(tl) * p.cap;
               uint64_t v[4 * MQ];
               load_sublists<C::NET, MQ>(row, capq, cn, et, v);
+              // the lower edge of the bin holding the r-th largest sampled key:
+              // at most a bin's width below that key, so no fewer keys pass
               int above = 0, inb = 0;
-              uint64_t floor = histogram_cut<C::NET, 4 * MQ>(v, r, scr_s, et, 1, &above, &inb);
-              if (above + inb > r) {
-#pragma unroll
-                for (int q = 0; q < 4 * MQ; ++q) v[q] = (v[q] >= floor) ? v[q] : 0ull;
-                floor = radix_select_floor<C::NET, 4 * MQ>(v, r, scr_s, et, 1);
-              }
+              const uint64_t floor = histogram_cut<C::NET, 4 * MQ>(v, r, scr_s, et, bar, &above, &inb);
               if (et == 0) {
                 const uint64_t hi = floor >> 32;
                 thr_s[tl] = (hi == 0) ? 0ull : (hi << 32) - 1;
               }
-              named_bar_sync(1, C::NET);
+              if (!bar.sync()) break;
             }
             if (et < 4 * C::RB) cnt_s[et] = 0;
-            if (et == 0) *cutmask_s = 0;
-            named_bar_sync(1, C::NET);
+            if (!bar.sync()) { ok = false; break; }
+            reload_rows();
             continue;
           }
+          // Every CHECK_EVERY tiles, cut any list whose sub-list could
+          // overflow before the next check (at most 32 appends per sub-list
+          // and tile): one histogram pass keeps every key in or above the bin
+          // of the k-th largest; if that keeps too many, an exact select
+          // keeps exactly k.
           if ((i % C::CHECK_EVERY) != C::CHECK_EVERY - 1) continue;
-          named_bar_sync(1, C::NET);
-          const uint32_t cmask = static_cast<uint32_t>(*cutmask_s);
+          unsigned long long near = 0;  // rows of this warp whose sub-list is near capacity
+#pragma unroll
+          for (int r = 0; r < NR; ++r)
+            if (cnt_r[r] > capq - 32 * C::CHECK_EVERY) near |= 1ull << row_of(r);
+          if (lane == 0 && near) atomicOr(cutmask_s, near);
+          publish_counts();
+          if (!bar.sync()) { ok = false; break; }
+          const unsigned long long cmask = *cutmask_s;
           if (cmask == 0) continue;
           for (int tl = 0; tl < C::RB; ++tl) {
             const int* cn = cnt_s + tl * 4;
-            if ((cmask >> tl) & 1u) {
+            if ((cmask >> tl) & 1ull) {
               uint64_t* row = my_cand + static_cast<size_t>(tl) * p.cap;
               const int n = cn[0] + cn[1] + cn[2] + cn[3];
               uint64_t v[4 * MQ];
@@ -596,29 +627,32 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
               uint64_t floor = 1ull;  // fewer than topk keys: only rebalance the sub-lists
               if (n > p.topk) {
                 int above = 0, inb = 0;
-                floor = histogram_cut<C::NET, 4 * MQ>(v, p.topk, scr_s, et, 1, &above, &inb);
+                floor = histogram_cut<C::NET, 4 * MQ>(v, p.topk, scr_s, et, bar, &above, &inb);
                 if (above + inb > p.cap / 2) {
                   // keys below the boundary bin can go now; exact select on the rest
 #pragma unroll
-                  for (int i = 0; i < 4 * MQ; ++i) v[i] = (v[i] >= floor) ? v[i] : 0ull;
-                  floor = radix_select_floor<C::NET, 4 * MQ>(v, p.topk, scr_s, et, 1);
+                  for (int q = 0; q < 4 * MQ; ++q) v[q] = (v[q] >= floor) ? v[q] : 0ull;
+                  floor = radix_select_floor<C::NET, 4 * MQ>(v, p.topk, scr_s, et, bar);
                 }
               }
-              store_sublists<C::NET, MQ>(row, capq, cnt_s + tl * 4, v, floor, pos_s, et, 1);
+              store_sublists<C::NET, MQ>(row, capq, cnt_s + tl * 4, v, floor, pos_s, et, bar);
               if (et == 0 && floor - 1 > thr_s[tl]) thr_s[tl] = floor - 1;
-              named_bar_sync(1, C::NET);
+              if (!bar.sync()) break;
             }
           }
           // every flagged row was cut; all threads read the mask before the cuts' barriers
           if (et == 0) *cutmask_s = 0;
-          named_bar_sync(1, C::NET);
+          if (!bar.sync()) { ok = false; break; }
+          reload_rows();
         }
       }
       if (!ok) break;
       if constexpr (kSelect) {
         // exact top-k of each row: the histogram pass finds the boundary bin,
-        // a radix select over that bin's keys alone finds the exact cut
-        named_bar_sync(1, C::NET);
+        // a radix select over that bin's keys alone finds the exact cut; the
+        // row's keys are then ranked in shared memory and its indices written
+        publish_counts();
+        if (!bar.sync()) break;
         bool redo = false;
         for (int tl = 0; tl < C::RB; ++tl) {
           const int t = t0 + tl;
@@ -630,35 +664,33 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
           uint64_t* row = my_cand + static_cast<size_t>(tl) * p.cap;
           uint64_t v[4 * MQ];
           load_sublists<C::NET, MQ>(row, capq, cn, et, v);
-          uint64_t floor = 1ull;  // keep every valid key
-          if (n > p.topk) {
-            int above = 0, inb = 0;
-            floor = histogram_cut<C::NET, 4 * MQ>(v, p.topk, scr_s, et, 1, &above, &inb);
-            if (above + inb > p.topk) {
-              // the k-th largest lies in the boundary bin: exact select among keys >= its lower edge
+          int32_t* dst = p.idx + static_cast<size_t>(r0 + tl) * p.topk;
+          if (!topk_rank_by_bins<C::NET, 4 * MQ>(v, p.topk, scr_s, scr_s + C::SCR_START, scr_s + C::SCR_SMALL, srt_s,
+                                                 C::SRT_N, kBinRankMax, et, bar, dst)) {
+            // a crowded bin: exact select, then the bitonic ranking
+            uint64_t floor = 1ull;  // keep every valid key
+            if (n > p.topk) {
+              int above = 0, inb = 0;
+              floor = histogram_cut<C::NET, 4 * MQ>(v, p.topk, scr_s, et, bar, &above, &inb);
+              if (above + inb > p.topk) {
 #pragma unroll
-              for (int i = 0; i < 4 * MQ; ++i) v[i] = (v[i] >= floor) ? v[i] : 0ull;
-              floor = radix_select_floor<C::NET, 4 * MQ>(v, p.topk, scr_s, et, 1);
+                for (int q = 0; q < 4 * MQ; ++q) v[q] = (v[q] >= floor) ? v[q] : 0ull;
+                floor = radix_select_floor<C::NET, 4 * MQ>(v, p.topk, scr_s, et, bar);
+              }
             }
+            sort_selected_to_idx<C::NET, 4 * MQ>(v, floor, srt_s, pos_s, et, bar, p.topk, dst);
           }
-          // write the row's selected keys (unordered) and zero-pad to topk
-          uint64_t* dst = p.sel_keys + static_cast<size_t>(r0 + tl) * p.topk;  // row r0 + tl of the output
-          int mine = 0;
-#pragma unroll
-          for (int i = 0; i < 4 * MQ; ++i) mine += (v[i] != 0 && v[i] >= floor) ? 1 : 0;
-          int kept = 0;
-          int pos = block_exclusive_scan<C::NET>(mine, pos_s, et, 1, &kept);
-#pragma unroll
-          for (int i = 0; i < 4 * MQ; ++i)
-            if (v[i] != 0 && v[i] >= floor) dst[pos++] = v[i];
-          for (int i = kept + et; i < p.topk; i += C::NET) dst[i] = 0ull;
+          if (bar.aborted()) break;
         }
+        if (bar.aborted()) break;
         if (redo && et == 0) p.redo_list[atomicAdd(p.redo_count, 1)] = rb;
       }
-      named_bar_sync(1, C::NET);
+      if (!bar.sync()) break;
     }
+    // a warp that stopped on the abort flag counts itself in at the barrier
+    // the others may be waiting at
+    if (bar.aborted()) bar.leave();
   }
-
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();

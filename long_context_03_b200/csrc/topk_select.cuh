@@ -14,7 +14,7 @@ namespace dsa {
 
 // Cooperative radix select over keys held in registers.
 //
-// `NT` threads (thread index `et`, synchronised with named barrier `bar_id`)
+// `NT` threads (thread index `et`, synchronised with the group barrier `bar`)
 // hold up to MAXPER keys each in v[] (0 = empty). Finds `floor`, the smallest
 // key value such that exactly K keys are >= floor (K < number of valid keys),
 // by walking 8-bit digits from the first bit where the keys differ. Each warp
@@ -25,7 +25,7 @@ __host__ __device__ constexpr int select_scratch_ints(int nt) { return (nt / 32)
 
 template <int NT, int MAXPER>
 __device__ __forceinline__ uint64_t radix_select_floor(const uint64_t (&v)[MAXPER], int K, int* scratch, int et,
-                                                       uint32_t bar_id) {
+                                                       const GroupBar& bar) {
   constexpr int NW = NT / 32;
   int* hist = scratch;                                   // [NW][256]
   unsigned long long* mm = reinterpret_cast<unsigned long long*>(scratch + NW * 256);  // min, max
@@ -51,12 +51,12 @@ __device__ __forceinline__ uint64_t radix_select_floor(const uint64_t (&v)[MAXPE
     mm[0] = ~0ull;
     mm[1] = 0ull;
   }
-  named_bar_sync(bar_id, NT);
+  bar.sync();
   if ((et & 31) == 0) {
     atomicMin(&mm[0], kmin);
     atomicMax(&mm[1], kmax);
   }
-  named_bar_sync(bar_id, NT);
+  bar.sync();
   kmin = mm[0];
   kmax = mm[1];
   const uint64_t diff = kmin ^ kmax;
@@ -66,21 +66,21 @@ __device__ __forceinline__ uint64_t radix_select_floor(const uint64_t (&v)[MAXPE
   int remaining = K;
   while (true) {
     for (int i = et; i < NW * 256; i += NT) hist[i] = 0;
-    named_bar_sync(bar_id, NT);
+    bar.sync();
 #pragma unroll
     for (int j = 0; j < MAXPER; ++j) {
       const uint64_t x = v[j];
       const bool match = (x != 0) && ((shift + 8 >= 64) || ((x >> (shift + 8)) == (prefix >> (shift + 8))));
       if (match) atomicAdd(&my_hist[(x >> shift) & 255u], 1);
     }
-    named_bar_sync(bar_id, NT);
+    bar.sync();
     for (int i = et; i < 256; i += NT) {
       int tot = 0;
 #pragma unroll
       for (int w = 0; w < NW; ++w) tot += hist[w * 256 + i];
       hist[i] = tot;
     }
-    named_bar_sync(bar_id, NT);
+    bar.sync();
     if (et < 32) {
       const int l = et;
       int c[8];
@@ -112,7 +112,7 @@ __device__ __forceinline__ uint64_t radix_select_floor(const uint64_t (&v)[MAXPE
         }
       }
     }
-    named_bar_sync(bar_id, NT);
+    bar.sync();
     const int d = misc[0];
     const int above = misc[1];
     const int inb = misc[2];
@@ -124,36 +124,11 @@ __device__ __forceinline__ uint64_t radix_select_floor(const uint64_t (&v)[MAXPE
   return prefix;  // bits below `shift` are zero
 }
 
-// Compact row `c[0..n)` (global memory, keys) to exactly K keys (K < n) in
-// c[0..K), unordered. Returns the floor used (every kept key >= floor).
-template <int NT, int MAXPER>
-__device__ __forceinline__ uint64_t compact_top_k(uint64_t* c, int n, int K, int* scratch, int et, uint32_t bar_id) {
-  uint64_t v[MAXPER];
-#pragma unroll
-  for (int j = 0; j < MAXPER; ++j) {
-    const int i = et + j * NT;
-    v[j] = (i < n) ? c[i] : 0ull;
-  }
-  const uint64_t floor = radix_select_floor<NT, MAXPER>(v, K, scratch, et, bar_id);
-  int* wpos = scratch + (NT / 32) * 256 + 8;
-  if (et == 0) *wpos = 0;
-  named_bar_sync(bar_id, NT);
-#pragma unroll
-  for (int j = 0; j < MAXPER; ++j) {
-    if (v[j] != 0 && v[j] >= floor) {
-      const int pos = atomicAdd(wpos, 1);
-      c[pos] = v[j];
-    }
-  }
-  named_bar_sync(bar_id, NT);
-  return floor;
-}
-
 // Exclusive prefix sum of one int per thread over NT threads (named barrier
-// bar_id). wsum: NT/32 + 1 ints of shared memory. Returns the prefix;
+// bar). wsum: NT/32 + 1 ints of shared memory. Returns the prefix;
 // *total gets the sum over all threads.
 template <int NT>
-__device__ __forceinline__ int block_exclusive_scan(int x, int* wsum, int et, uint32_t bar_id, int* total) {
+__device__ __forceinline__ int block_exclusive_scan(int x, int* wsum, int et, const GroupBar& bar, int* total) {
   constexpr int NW = NT / 32;
   const int l = et & 31, w = et >> 5;
   int incl = x;
@@ -162,9 +137,9 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int* wsum, int et, ui
     const int y = __shfl_up_sync(0xffffffffu, incl, off);
     if (l >= off) incl += y;
   }
-  named_bar_sync(bar_id, NT);  // wsum may still be read by a previous scan
+  bar.sync();  // wsum may still be read by a previous scan
   if (l == 31) wsum[w] = incl;
-  named_bar_sync(bar_id, NT);
+  bar.sync();
   int base = 0, tot = 0;
 #pragma unroll
   for (int i = 0; i < NW; ++i) {
@@ -189,7 +164,7 @@ __host__ __device__ constexpr int cut_scratch_ints() { return 2048 + 64; }  // w
 // *inb = keys in that bin (so keys >= floor number *above + *inb >= K).
 template <int NT, int M>
 __device__ __forceinline__ uint64_t histogram_cut(const uint64_t (&v)[M], int K, int* scratch, int et,
-                                                  uint32_t bar_id, int* above_out, int* inb_out) {
+                                                  const GroupBar& bar, int* above_out, int* inb_out) {
   constexpr int NW = NT / 32;
   static_assert(NT == 256 || NT == 512, "the 2048-bin scan takes 256 or 512 threads");
   constexpr int BPT = 2048 / NT;  // bins per thread
@@ -217,12 +192,12 @@ __device__ __forceinline__ uint64_t histogram_cut(const uint64_t (&v)[M], int K,
     mm[1] = 0ull;
   }
   for (int i = et; i < 2048; i += NT) hist[i] = 0;
-  named_bar_sync(bar_id, NT);
+  bar.sync();
   if ((et & 31) == 0) {
     atomicMin(&mm[0], kmin);
     atomicMax(&mm[1], kmax);
   }
-  named_bar_sync(bar_id, NT);
+  bar.sync();
   kmin = mm[0];
   kmax = mm[1];
   const uint64_t diff = kmin ^ kmax;
@@ -232,7 +207,7 @@ __device__ __forceinline__ uint64_t histogram_cut(const uint64_t (&v)[M], int K,
 #pragma unroll
   for (int j = 0; j < M; ++j)
     if (v[j] != 0) atomicAdd(&hist[(v[j] >> shift) & 2047u], 1);
-  named_bar_sync(bar_id, NT);
+  bar.sync();
   // descending scan: thread et owns bins 2047-BPT*et .. 2048-BPT*(et+1)
   int c[BPT];
   int tot = 0;
@@ -249,7 +224,7 @@ __device__ __forceinline__ uint64_t histogram_cut(const uint64_t (&v)[M], int K,
     if (l >= off) incl += y;
   }
   if (l == 31) wsum[w] = incl;
-  named_bar_sync(bar_id, NT);
+  bar.sync();
   int wbase = 0;
 #pragma unroll
   for (int i = 0; i < NW; ++i) wbase += (i < w) ? wsum[i] : 0;
@@ -267,10 +242,154 @@ __device__ __forceinline__ uint64_t histogram_cut(const uint64_t (&v)[M], int K,
       cum += c[i];
     }
   }
-  named_bar_sync(bar_id, NT);
+  bar.sync();
   *above_out = res[1];
   *inb_out = res[2];
   return prefix | (static_cast<uint64_t>(res[0]) << shift);
+}
+
+// Exact top-K of one row, ranked, in one histogram pass. The NT threads hold
+// the row's keys in v[] (0 = empty). Every key's 11-bit digit below the
+// keys' common prefix puts it in one of 2048 bins; bins are ordered like the
+// keys, so a descending prefix sum over the bin counts gives each bin's first
+// rank, and a key's rank is that plus the number of larger keys in its own
+// bin. The K-th largest key lies in bin b*: keys in higher bins all rank below
+// K, keys of b* are kept by their rank, lower bins are dropped. The keys of
+// bins >= b* go to buf (at most bufn) grouped by bin; dst[0..K) gets the
+// token indices in rank order, -1 past the row's valid keys.
+// Returns false, with nothing written, when a bin >= b* holds more than cmax
+// keys or more than bufn keys lie in bins >= b*: the caller then ranks with
+// the exact select and the bitonic sort. Scratch (ints, shared): hist[2048],
+// start[2048], small[64].
+template <int NT, int M>
+__device__ __forceinline__ bool topk_rank_by_bins(const uint64_t (&v)[M], int K, int* hist, int* start, int* small,
+                                                  uint64_t* buf, int bufn, int cmax, int et, const GroupBar& bar,
+                                                  int32_t* __restrict__ dst) {
+  constexpr int NW = NT / 32;
+  static_assert(NT == 512, "four bins per thread");
+  constexpr int BPT = 2048 / NT;
+  int* wsum = small;                                                        // [NW]
+  unsigned long long* mm = reinterpret_cast<unsigned long long*>(small + 16);  // min, max
+  int* res = small + 24;  // b*, keys above b*, keys in b*, largest bin count, valid keys
+  bar.sync();  // every thread is done with the previous row's hist, start and buf
+  unsigned long long kmin = ~0ull, kmax = 0ull;
+  int nv = 0;
+#pragma unroll
+  for (int j = 0; j < M; ++j) {
+    if (v[j] != 0) {
+      kmin = v[j] < kmin ? v[j] : kmin;
+      kmax = v[j] > kmax ? v[j] : kmax;
+      ++nv;
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const unsigned long long a = __shfl_xor_sync(0xffffffffu, kmin, off);
+    const unsigned long long b = __shfl_xor_sync(0xffffffffu, kmax, off);
+    kmin = a < kmin ? a : kmin;
+    kmax = b > kmax ? b : kmax;
+    nv += __shfl_xor_sync(0xffffffffu, nv, off);
+  }
+  if (et == 0) {
+    mm[0] = ~0ull;
+    mm[1] = 0ull;
+    res[0] = 0;
+    res[1] = 0;
+    res[2] = 0;
+    res[3] = 0;
+    res[4] = 0;
+  }
+  for (int i = et; i < 2048; i += NT) hist[i] = 0;
+  bar.sync();
+  if ((et & 31) == 0) {
+    atomicMin(&mm[0], kmin);
+    atomicMax(&mm[1], kmax);
+    atomicAdd(&res[4], nv);
+  }
+  bar.sync();
+  kmin = mm[0];
+  kmax = mm[1];
+  const int n = res[4];
+  const uint64_t diff = kmin ^ kmax;
+  const int hi_bit = diff ? 63 - __clzll(static_cast<long long>(diff)) : 0;
+  const int shift = hi_bit >= 10 ? hi_bit - 10 : 0;
+#pragma unroll
+  for (int j = 0; j < M; ++j)
+    if (v[j] != 0) atomicAdd(&hist[(v[j] >> shift) & 2047u], 1);
+  bar.sync();
+  // descending scan: thread et owns bins 2047 - BPT*et - i, i < BPT
+  int c[BPT];
+  int tot = 0;
+#pragma unroll
+  for (int i = 0; i < BPT; ++i) {
+    c[i] = hist[2047 - BPT * et - i];
+    tot += c[i];
+  }
+  const int l = et & 31, w = et >> 5;
+  int incl = tot;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (l >= off) incl += y;
+  }
+  if (l == 31) wsum[w] = incl;
+  bar.sync();
+  int wbase = 0;
+#pragma unroll
+  for (int i = 0; i < NW; ++i) wbase += (i < w) ? wsum[i] : 0;
+  const int excl = wbase + incl - tot;
+  const int keff = K < n ? K : n;  // the K-th largest, or the smallest valid key
+  {
+    int cum = excl;
+#pragma unroll
+    for (int i = 0; i < BPT; ++i) {
+      start[2047 - BPT * et - i] = cum;
+      if (keff > 0 && cum < keff && cum + c[i] >= keff) {
+        res[0] = 2047 - BPT * et - i;
+        res[1] = cum;
+        res[2] = c[i];
+      }
+      cum += c[i];
+    }
+  }
+  bar.sync();
+  const int bstar = res[0];
+  const int total = res[1] + res[2];  // keys in bins >= b*
+  int cm = 0;
+#pragma unroll
+  for (int i = 0; i < BPT; ++i)
+    if (2047 - BPT * et - i >= bstar) cm = c[i] > cm ? c[i] : cm;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const int y = __shfl_xor_sync(0xffffffffu, cm, off);
+    cm = y > cm ? y : cm;
+  }
+  if (l == 0 && cm > 0) atomicMax(&res[3], cm);
+  bar.sync();
+  if (res[3] > cmax || total > bufn) return false;  // the same answer on every thread
+  // group the keys of bins >= b* by bin (start[] then points past each bin)
+#pragma unroll
+  for (int j = 0; j < M; ++j) {
+    if (v[j] != 0) {
+      const int b = static_cast<int>((v[j] >> shift) & 2047u);
+      if (b >= bstar) {
+        const int p = atomicAdd(&start[b], 1);
+        if (p < bufn) buf[p] = v[j];
+      }
+    }
+  }
+  bar.sync();
+  for (int i = et; i < total; i += NT) {
+    const uint64_t key = buf[i];
+    const int b = static_cast<int>((key >> shift) & 2047u);
+    const int cb = hist[b];
+    const int s0 = start[b] - cb;
+    int r = s0;
+    for (int q = s0; q < s0 + cb; ++q) r += (buf[q] > key) ? 1 : 0;
+    if (r < K) dst[r] = rank_key_index(key);
+  }
+  for (int i = (total > 0 ? total : 0) + et; i < K; i += NT) dst[i] = -1;
+  return true;
 }
 
 // Load a row's four quarter sub-lists (counts cnt[0..3], capacity capq each)
@@ -294,135 +413,128 @@ __device__ __forceinline__ void load_sublists(const uint64_t* row, int capq, con
 // per-thread survivor counts (no atomics). Returns the number kept.
 template <int NT, int MQ>
 __device__ __forceinline__ int store_sublists(uint64_t* row, int capq, int* cnt, const uint64_t (&v)[4 * MQ],
-                                              uint64_t floor, int* wsum, int et, uint32_t bar_id) {
+                                              uint64_t floor, int* wsum, int et, const GroupBar& bar) {
   int mine = 0;
 #pragma unroll
   for (int j = 0; j < 4 * MQ; ++j) mine += (v[j] != 0 && v[j] >= floor) ? 1 : 0;
   int kept = 0;
-  int pos = block_exclusive_scan<NT>(mine, wsum, et, bar_id, &kept);
+  int pos = block_exclusive_scan<NT>(mine, wsum, et, bar, &kept);
 #pragma unroll
   for (int j = 0; j < 4 * MQ; ++j) {
     if (v[j] != 0 && v[j] >= floor) {
-      row[static_cast<size_t>(pos & 3) * capq + (pos >> 2)] = v[j];
+      if (pos < 4 * capq) row[static_cast<size_t>(pos & 3) * capq + (pos >> 2)] = v[j];
       ++pos;
     }
   }
+  kept = min(kept, 4 * capq);
   if (et < 4) cnt[et] = (kept + 3 - et) / 4;
   return kept;
 }
 
-// One CTA per row (small K): sort the row's K keys descending (bitonic, in
-// shared memory) and write the token indices; empty slots (key 0) become -1.
-// keys [rows, K] (row r at keys + r*K), idx [rows, K].
-template <int P>  // power of two >= K
-__global__ void __launch_bounds__(256) rank_sort_kernel(const uint64_t* __restrict__ keys, int32_t* __restrict__ idx,
-                                                        int K, int rows) {
-  __shared__ uint64_t s[P];
-  const int r = blockIdx.x;
-  if (r >= rows) return;
-  const uint64_t* src = keys + static_cast<size_t>(r) * K;
-  for (int i = threadIdx.x; i < P; i += blockDim.x) s[i] = (i < K) ? src[i] : 0ull;
-  __syncthreads();
-  for (int size = 2; size <= P; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = threadIdx.x; i < P / 2; i += blockDim.x) {
-        const int lo = 2 * i - (i & (stride - 1));
-        const int hi = lo + stride;
-        const bool desc = ((lo & size) == 0);  // final merge (size == P) is descending everywhere
-        const uint64_t a = s[lo], b = s[hi];
-        if ((a < b) == desc) {
-          s[lo] = b;
-          s[hi] = a;
+// Rank the selected keys of one row and write its token indices, inside the
+// kernel that selected them: the keys v[i] != 0 && v[i] >= floor (at most K
+// over the NT cooperating threads) are compacted into `srt` (shared memory,
+// P = the power of two >= K keys), padded with empty keys (0) and sorted into
+// descending 64-bit order (score descending, then index ascending) by a
+// bitonic network; dst[0..K) gets their token indices and -1 past them.
+// With P == 4 * NT each thread keeps four consecutive keys in registers:
+// strides 1 and 2 stay in the thread, strides 4..64 are warp shuffles and
+// only strides >= 128 go through shared memory. Group barrier `bar` over the
+// NT threads; wsum as for block_exclusive_scan. Writes stay inside srt and
+// dst even if the group aborted and the positions are stale.
+template <int NT, int M>
+__device__ __forceinline__ void sort_selected_to_idx(const uint64_t (&v)[M], uint64_t floor, uint64_t* srt, int* wsum,
+                                                     int et, const GroupBar& bar, int K, int32_t* __restrict__ dst) {
+  int mine = 0;
+#pragma unroll
+  for (int i = 0; i < M; ++i) mine += (v[i] != 0 && v[i] >= floor) ? 1 : 0;
+  int kept = 0;
+  int pos = block_exclusive_scan<NT>(mine, wsum, et, bar, &kept);
+#pragma unroll
+  int P = 1;
+  while (P < K) P <<= 1;
+#pragma unroll
+  for (int i = 0; i < M; ++i)
+    if (v[i] != 0 && v[i] >= floor) {
+      if (pos < P) srt[pos] = v[i];
+      ++pos;
+    }
+  for (int i = max(kept, 0) + et; i < P; i += NT) srt[i] = 0ull;
+  bar.sync();
+  if (P == 4 * NT) {
+    uint64_t a[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) a[u] = srt[4 * et + u];
+#pragma unroll 1
+    for (int k = 2; k <= P; k <<= 1) {
+#pragma unroll 1
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        if (j >= 128) {  // the partner sits in another warp
+          bar.sync();  // every thread has read what the last exchange wrote
+#pragma unroll
+          for (int u = 0; u < 4; ++u) srt[4 * et + u] = a[u];
+          bar.sync();
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int e = 4 * et + u;
+            const uint64_t b = srt[e ^ j];
+            const bool keep_max = ((e & j) == 0) == ((e & k) == 0);
+            a[u] = keep_max ? (a[u] > b ? a[u] : b) : (a[u] > b ? b : a[u]);
+          }
+        } else if (j >= 4) {  // the partner is lane (et ^ j/4) of this warp
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int e = 4 * et + u;
+            const uint64_t b = __shfl_xor_sync(0xffffffffu, a[u], j >> 2);
+            const bool keep_max = ((e & j) == 0) == ((e & k) == 0);
+            a[u] = keep_max ? (a[u] > b ? a[u] : b) : (a[u] > b ? b : a[u]);
+          }
+        } else {  // both keys are this thread's
+          // for k >= 4 the direction bit (e & k) is the same for the four keys
+          // 4et..4et+3; for k = 2 the pairs (0,1) and (2,3) run opposite ways
+          const bool desc = ((4 * et) & k) == 0;
+          auto cx = [&](uint64_t& lo, uint64_t& hi, bool d) {
+            const uint64_t mx = lo > hi ? lo : hi, mn = lo > hi ? hi : lo;
+            lo = d ? mx : mn;
+            hi = d ? mn : mx;
+          };
+          if (j == 2) {
+            cx(a[0], a[2], desc);
+            cx(a[1], a[3], desc);
+          } else if (k == 2) {
+            cx(a[0], a[1], true);
+            cx(a[2], a[3], false);
+          } else {
+            cx(a[0], a[1], desc);
+            cx(a[2], a[3], desc);
+          }
         }
       }
-      __syncthreads();
     }
-  }
-  int32_t* dst = idx + static_cast<size_t>(r) * K;
-  for (int i = threadIdx.x; i < K; i += blockDim.x) {
-    const uint64_t k = s[i];
-    dst[i] = (k == 0ull) ? -1 : rank_key_index(k);
-  }
-}
-
-// Compare-exchange of the in-thread pairs (a, a | S), a & S == 0, of a
-// thread's 8 consecutive elements 8i..8i+7 within bitonic blocks of `size`.
-template <int S>
-__device__ __forceinline__ void bitonic_reg_step(uint64_t (&v)[8], int i, int size) {
 #pragma unroll
-  for (int a = 0; a < 8; ++a) {
-    if ((a & S) == 0) {
-      const int b = a | S;
-      const bool desc = ((8 * i + a) & size) == 0;
-      const uint64_t mx = v[a] > v[b] ? v[a] : v[b], mn = v[a] > v[b] ? v[b] : v[a];
-      v[a] = desc ? mx : mn;
-      v[b] = desc ? mn : mx;
+    for (int u = 0; u < 4; ++u) {
+      const int e = 4 * et + u;
+      if (e < K) dst[e] = (a[u] == 0ull) ? -1 : rank_key_index(a[u]);
     }
-  }
-}
-
-// One CTA of P/8 threads per row, 8 keys per thread in registers: a bitonic
-// sort into descending key order (= score descending, index ascending).
-// Strides below 8 stay inside a thread, strides 8..128 go through warp
-// shuffles, larger strides through shared memory. Writes the token indices;
-// empty slots (key 0) become -1.
-template <int P>
-__global__ void __launch_bounds__(P / 8) rank_sort_reg_kernel(const uint64_t* __restrict__ keys,
-                                                               int32_t* __restrict__ idx, int K, int rows) {
-  static_assert(P >= 256 && P <= 2048, "8 keys per thread, at least one warp");
-  __shared__ uint64_t sm[P];
-  const int r = blockIdx.x;
-  if (r >= rows) return;
-  const int i = threadIdx.x;
-  const uint64_t* src = keys + static_cast<size_t>(r) * K;
-  uint64_t v[8];
-#pragma unroll
-  for (int a = 0; a < 8; ++a) {
-    const int e = 8 * i + a;
-    v[a] = (e < K) ? src[e] : 0ull;
-  }
+  } else {
 #pragma unroll 1
-  for (int size = 2; size <= P; size <<= 1) {
+    for (int k = 2; k <= P; k <<= 1) {
 #pragma unroll 1
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      if (stride >= 256) {
-        __syncthreads();
-#pragma unroll
-        for (int a = 0; a < 8; ++a) sm[8 * i + a] = v[a];
-        __syncthreads();
-#pragma unroll
-        for (int a = 0; a < 8; ++a) {
-          const int e = 8 * i + a;
-          const uint64_t o = sm[e ^ stride];
-          const bool lower = (e & stride) == 0;
-          const bool desc = (e & size) == 0;
-          const uint64_t mx = v[a] > o ? v[a] : o, mn = v[a] > o ? o : v[a];
-          v[a] = (lower == desc) ? mx : mn;
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        for (int i = et; i < P / 2; i += NT) {
+          const int lo = 2 * i - (i & (j - 1));
+          const int hi = lo + j;
+          const bool desc = (lo & k) == 0;
+          const uint64_t a = srt[lo], b = srt[hi];
+          if ((a < b) == desc) {
+            srt[lo] = b;
+            srt[hi] = a;
+          }
         }
-      } else if (stride >= 8) {
-#pragma unroll
-        for (int a = 0; a < 8; ++a) {
-          const int e = 8 * i + a;
-          const uint64_t o = __shfl_xor_sync(0xffffffffu, v[a], stride >> 3);
-          const bool lower = (e & stride) == 0;
-          const bool desc = (e & size) == 0;
-          const uint64_t mx = v[a] > o ? v[a] : o, mn = v[a] > o ? o : v[a];
-          v[a] = (lower == desc) ? mx : mn;
-        }
-      } else if (stride == 4) {
-        bitonic_reg_step<4>(v, i, size);
-      } else if (stride == 2) {
-        bitonic_reg_step<2>(v, i, size);
-      } else {
-        bitonic_reg_step<1>(v, i, size);
+        bar.sync();
       }
     }
-  }
-  int32_t* dst = idx + static_cast<size_t>(r) * K;
-#pragma unroll
-  for (int a = 0; a < 8; ++a) {
-    const int e = 8 * i + a;
-    if (e < K) dst[e] = (v[a] == 0ull) ? -1 : rank_key_index(v[a]);
+    for (int i = et; i < K; i += NT) dst[i] = (srt[i] == 0ull) ? -1 : rank_key_index(srt[i]);
   }
 }
 
