@@ -17,6 +17,16 @@ ranks and `value` counts every rank's tokens.
 
 --impl reference times the float64 CPU oracle (the checker, not a competing
 system) on a bounded sample of the same workload on this host's cores.
+
+--kernel OP runs one hot-path call repeatedly on seeded inputs instead (for
+timing or profiling a single kernel, e.g. under ncu with -k and -s/-c) and
+prints its mean CUDA-event time as one JSON line:
+
+    python bench.py --kernel indexer --prefill-L 65536 --repeat 5
+    python bench.py --kernel attention --prefill-L 16384
+    python bench.py --kernel decode --decode-B 64 --decode-L 65536
+    python bench.py --kernel decode_paged --decode-B 64 --decode-L 65536 --page 64
+    python bench.py --kernel rope --decode-B 64      # RoPE + E4M3 of B appended indexer rows
 """
 from __future__ import annotations
 
@@ -42,15 +52,15 @@ METRIC = "DSA prefill tokens/s @128K & decode tok/s, % of FP8/BF16/HBM roofline"
 
 # DRAM bytes (read + write) per timed unit of the default workload, from one
 # single-pass ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of
-# this benchmark on B200. Valid only for the kernels they were taken on: set
-# an entry to None when its kernels change. Units: the prefill indexer entry
-# covers its main pass, re-run pass and rank sort; decode entries cover one
+# this benchmark on B200. Valid only for the kernels they were taken on: an
+# entry is None until the current kernels are captured. Units: the prefill
+# indexer entry covers its main and re-run passes; decode entries cover one
 # decode batch.
 MEASURED_TRAFFIC = {
-    "prefill_indexer": 1.6947e9 + 5.2533e9 + 0.0001e9 + 2.1494e9 + 1.0408e9,
-    "prefill_attention": 75.2040e9 + 17.1771e9,
-    "decode_step": 0.5543e9 + 0.0140e9 + 0.0173e9 + 0.0011e9 + 0.1610e9 + 0.0002e9,
-    "decode_indexer": 0.5543e9 + 0.0140e9 + 0.0173e9 + 0.0011e9,
+    "prefill_indexer": None,
+    "prefill_attention": None,
+    "decode_step": None,
+    "decode_indexer": None,
 }
 DEFAULT_SIZES = (131072, 64, 65536)  # prefill L, decode B, decode L the traffic was measured on
 D_QK, D_V = 576, 512
@@ -70,6 +80,10 @@ def parse(argv=None):
                     help="query-row chunks whose copies overlap the compute in the e2e leg (1: no overlap)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-rows", type=int, default=240)
+    ap.add_argument("--kernel", default=None, choices=["indexer", "attention", "decode", "decode_paged", "rope"],
+                    help="time one hot-path call instead of the whole step (see the module docstring)")
+    ap.add_argument("--repeat", type=int, default=5, help="calls in --kernel mode (the first min(3, repeat-1) warm up)")
+    ap.add_argument("--page", type=int, default=64, help="page size of --kernel decode_paged")
     ap.add_argument("--no-fp8-probe", action="store_true",
                     help="skip the library FP8 GEMM measured after the timed work (context for the indexer's peak)")
     return ap.parse_args(argv)
@@ -357,7 +371,7 @@ def run_ours(a, ws, rank):
     rl = {
         "prefill_indexer": {"bound": "tensor", "achieved": idx_tf, "peak": fp8_peak, "unit": "TFLOP/s",
                             "frac": idx_tf / fp8_peak, "traffic": None,
-                            "note": "FP8 peak = 2 x measured sustained bf16 (nominal fp8:bf16 ratio); time includes the rank sort"},
+                            "note": "FP8 peak = 2 x measured sustained bf16 (nominal fp8:bf16 ratio); time includes the in-kernel ranking"},
         "prefill_attention": {"bound": "tensor", "achieved": attn_tf, "peak": pk["bf16_tflops_sustained"],
                               "unit": "TFLOP/s", "frac": attn_tf / pk["bf16_tflops_sustained"], "traffic": None},
         "decode_step": {"bound": "hbm", "achieved": dec_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
@@ -367,7 +381,8 @@ def run_ours(a, ws, rank):
     }
     if (L, D.B, D.L) == DEFAULT_SIZES:
         for key, val in MEASURED_TRAFFIC.items():
-            rl[key]["traffic"] = val
+            if val is not None:
+                rl[key]["traffic"] = val
     dom = "prefill_indexer" if t_idx >= t_attn else "prefill_attention"
     res = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": a.steps, "warmup": a.warmup,
@@ -379,12 +394,13 @@ def run_ours(a, ws, rank):
         "roofline": dict(rl[dom], kernel=dom),
         "roofline_all": rl,
         "peaks": {"source": pk["source"], "fp8": "2 x bf16_tflops_sustained"},
-        "gpu_launches": 8 * a.steps,  # prefill: indexer (main + re-run), rank sort, attention; decode: scores, select, rank sort, attention
+        "gpu_launches": 6 * a.steps,  # prefill: indexer (main + re-run pass), attention; decode: scores, select, attention
         "clocks": clocks,
         "wall_s_timed": t_wall,
     }
     if not a.no_e2e:
         res["e2e"] = run_e2e(a, dsa, P, idx, out, ws_p, ws, dev)
+        res["e2e"]["decode"] = run_e2e_decode(a, dsa, D, didx, dout, ws_d, ws, dev)
     if rank == 0 and not a.no_cpu_baseline:
         tps, dt, rows, cores = cpu_oracle_prefill(P, a.cpu_sample_rows)
         dtps, ddt = cpu_oracle_decode(D, 2)
@@ -468,6 +484,40 @@ def run_e2e(a, dsa, P, idx, out, ws_p, ws, dev):
             "pipeline": f"{nch} query-row chunks; copies in, compute and copies out on three streams"}
 
 
+def run_e2e_decode(a, dsa, D, didx, dout, ws_d, ws, dev):
+    """Decode tokens/s through the public API with host buffers: every step
+    copies the step's new-token inputs (indexer query, its scale and head
+    weights, the attention query) host->device and the output back; the key
+    and latent caches stay resident on the device, as in serving."""
+    names = ("q_I", "q_scale", "w", "q")
+    try:
+        host = {n: getattr(D, n).cpu().pin_memory() for n in names}
+        out_h = torch.empty(dout.shape, dtype=dout.dtype).pin_memory()
+    except Exception as e:
+        return {"value": None, "unit": "tokens/s", "error": f"{type(e).__name__}: {e}"}
+    dev_bufs = {n: getattr(D, n) for n in names}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = dout.numel() * dout.element_size()
+    stream = torch.cuda.current_stream(dev)
+    times = []
+    for s in range(a.warmup + 4 * a.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for n, t in host.items():
+            dev_bufs[n].copy_(t, non_blocking=True)
+        dsa.index_topk_decode(D.q_I, D.q_scale, D.w, D.k_cache, D.k_scale, D.lens, D.topk, idx=didx, workspace=ws_d)
+        dsa.sparse_mla_attn_decode(D.q, D.kv, didx, D.scale, out=dout)
+        out_h.copy_(dout, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if s >= a.warmup:
+            times.append(e0.elapsed_time(e1))
+    t = max_over_ranks(float(np.mean(times)), ws)
+    return {"value": ws * D.B / (t * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": t,
+            "scope": "decode: new-token inputs in, output out; caches resident"}
+
+
 # ------------------------------------------------------- reference (oracle)
 
 def run_reference(a, ws, rank):
@@ -479,7 +529,9 @@ def run_reference(a, ws, rank):
     # the sample needs only a few query rows of the 128-head queries
     g = torch.Generator().manual_seed(7)
     import oracle
-    rows_per_step = max(4, oracle.num_threads())
+    # eight rows per host thread and step keep every core busy while the
+    # per-row cost varies with t (rows are drawn uniformly over the prefill)
+    rows_per_step = 8 * max(1, oracle.num_threads())
     q_rows = torch.randn((rows_per_step * (a.warmup + a.steps), 128, D_QK), generator=g).to(torch.bfloat16)
     times = []
     rng = np.random.default_rng(1)
@@ -505,8 +557,91 @@ def run_reference(a, ws, rank):
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def _time_calls(fn, repeat, dsa):
+    """Mean CUDA-event time (ms) of the calls after the first min(3, repeat - 1)."""
+    warm = min(3, repeat - 1)
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(repeat - warm):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    dsa.check_device_error()
+    return e0.elapsed_time(e1) / (repeat - warm), repeat - warm
+
+
+def run_kernel(a):
+    """One hot-path call, repeated on seeded synthetic inputs of the benchmark's shapes."""
+    import long_context_03_b200 as dsa
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    L, B, DL, k = a.prefill_L, a.decode_B, a.decode_L, 2048
+    if a.kernel == "indexer":
+        # the indexer never reads the attention queries: one query head keeps the inputs small
+        P = workloads.make_prefill(L, 64, 128, 1, k, seed=0, device=dev)
+        ws = torch.empty(dsa.index_topk_workspace_size(L, 64, 128, k), dtype=torch.uint8, device=dev)
+        idx = torch.empty((L, k), dtype=torch.int32, device=dev)
+        fn = lambda: dsa.index_topk(P.q_I, P.q_scale, P.w, P.k_cache, P.k_scale, k, idx=idx, workspace=ws)
+        shape = {"L": L}
+    elif a.kernel == "attention":
+        P = workloads.make_prefill(L, 64, 128, 128, k, seed=0, device=dev)
+        idx = dsa.index_topk(P.q_I, P.q_scale, P.w, P.k_cache, P.k_scale, k)
+        out = torch.empty((L, 128, D_V), dtype=torch.bfloat16, device=dev)
+        fn = lambda: dsa.sparse_mla_attn(P.q, P.kv, idx, P.scale, out=out)
+        shape = {"L": L}
+    elif a.kernel == "rope":
+        g = torch.Generator(device=dev).manual_seed(0)
+        xq = torch.randn((B, 64, 128), generator=g, device=dev)
+        xk = torch.randn((B, 128), generator=g, device=dev)
+        pos = torch.randint(0, L, (B,), generator=g, device=dev, dtype=torch.int32)
+
+        def fn():
+            dsa.rope_quantize_e4m3_rows(xq, pos)
+            dsa.rope_quantize_e4m3_rows(xk, pos)
+        shape = {"B": B}
+    elif a.kernel == "decode_paged":
+        # both caches in one shuffled pool of pages (every sequence full length)
+        D = workloads.make_decode(B, DL, 64, 128, 128, k, seed=0, device=dev)
+        npg = DL // a.page
+        perm = torch.randperm(B * npg, device=dev)
+        k_pool = torch.empty((B * DL, 128), dtype=torch.uint8, device=dev)
+        k_pool.view(-1, a.page, 128)[perm] = D.k_cache.view(torch.uint8).reshape(-1, a.page, 128)
+        ks_pool = torch.empty((B * DL,), dtype=torch.float32, device=dev)
+        ks_pool.view(-1, a.page)[perm] = D.k_scale.reshape(-1, a.page)
+        kv_pool = torch.empty((B * DL, D_QK), dtype=torch.bfloat16, device=dev)
+        kv_pool.view(-1, a.page, D_QK)[perm] = D.kv.reshape(-1, a.page, D_QK)
+        table = perm.to(torch.int32).view(B, npg)
+        ws = torch.empty(dsa.index_topk_decode_workspace_size(B, DL, k), dtype=torch.uint8, device=dev)
+        idx = torch.empty((B, k), dtype=torch.int32, device=dev)
+        out = torch.empty((B, 128, D_V), dtype=torch.bfloat16, device=dev)
+
+        def fn():
+            dsa.index_topk_decode_paged(D.q_I, D.q_scale, D.w, k_pool, ks_pool, table, D.lens, k,
+                                        page_size=a.page, idx=idx, workspace=ws)
+            dsa.sparse_mla_attn_paged(D.q, kv_pool, table, idx, DL, D.scale, page_size=a.page, out=out)
+        shape = {"B": B, "L": DL, "page": a.page}
+    else:
+        D = workloads.make_decode(B, DL, 64, 128, 128, k, seed=0, device=dev)
+        ws = torch.empty(dsa.index_topk_decode_workspace_size(B, DL, k), dtype=torch.uint8, device=dev)
+        idx = torch.empty((B, k), dtype=torch.int32, device=dev)
+        out = torch.empty((B, 128, D_V), dtype=torch.bfloat16, device=dev)
+
+        def fn():
+            dsa.index_topk_decode(D.q_I, D.q_scale, D.w, D.k_cache, D.k_scale, D.lens, k, idx=idx, workspace=ws)
+            dsa.sparse_mla_attn_decode(D.q, D.kv, idx, D.scale, out=out)
+        shape = {"B": B, "L": DL}
+    ms, n = _time_calls(fn, a.repeat, dsa)
+    return {"kernel": a.kernel, "ms": ms, "calls_timed": n, "calls": a.repeat, **shape}
+
+
 def main():
     a = parse()
+    if a.kernel is not None:
+        print(json.dumps(run_kernel(a)))
+        return
     if a.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
         ws = int(os.environ.get("WORLD_SIZE", "1"))

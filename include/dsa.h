@@ -175,6 +175,23 @@ dsa_status dsa_index_scores(const uint8_t* q_I, const float* q_scale, const floa
 dsa_status dsa_sparse_mla_attn(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int T, int L, int Hq,
                                int topk, float scale, uint16_t* out, float* lse, void* stream);
 
+/* Sparse MQA attention over a packed batch of sequences (cu_seqlens form),
+ * the attention that follows dsa_index_topk_varlen: sequence b owns query
+ * tokens cu_q[b] .. cu_q[b+1]-1 of q / idx / out / lse and latent rows
+ * cu_k[b] .. cu_k[b+1]-1 of kv [total_k, 576]; idx holds row numbers local to
+ * the token's sequence (as dsa_index_topk_varlen returns them). cu_q and cu_k
+ * [nseq+1] int32 are DEVICE arrays (the indexer's varlen call takes host
+ * arrays), non-decreasing, cu_q[0] = cu_k[0] = 0, cu_q[nseq] = T, cu_k[nseq]
+ * <= total_k; each token finds its sequence on the device. A local index at
+ * or past its sequence's row count is skipped and reported as
+ * DSA_ERR_BAD_INDEX; offsets outside [0, total_k] are clamped into it, so no
+ * read leaves kv. Per token the result equals dsa_sparse_mla_attn over that
+ * sequence's rows. Serving layout (continuous batching), no counterpart step
+ * in the pages. */
+dsa_status dsa_sparse_mla_attn_varlen(const uint16_t* q, const uint16_t* kv, const int32_t* idx, const int32_t* cu_q,
+                                      const int32_t* cu_k, int nseq, int T, int total_k, int Hq, int topk, float scale,
+                                      uint16_t* out, float* lse, void* stream);
+
 /* Sparse MQA attention over a paged latent cache: kv_pool [pool_rows, 576]
  * holds pages of page_size rows (a power of two, 16..4096); logical row r of
  * token t is physical row block_table[t * bt_stride + r / page_size] *
@@ -195,7 +212,8 @@ dsa_status dsa_sparse_mla_attn_paged(const uint16_t* q, const uint16_t* kv_pool,
  * and codes[r, i] = E4M3(x[r, i] / scale[r]), nearest with ties to even,
  * saturating to +-448 ("Lightning Indexer 的计算过程", step 2 <2>, FP8 量化).
  * Bit-identical to that definition evaluated in fp32. x [n, d] f32, codes
- * [n, d] e4m3 bytes, scale [n] f32, all device memory. n = 0 is a no-op. */
+ * [n, d] e4m3 bytes, scale [n] f32, all device memory; codes and scale must
+ * not overlap x (DSA_ERR_INVALID_ARG). n = 0 is a no-op. */
 dsa_status dsa_quantize_e4m3_rows(const float* x, int n, int d, uint8_t* codes, float* scale, void* stream);
 
 /* RoPE + FP8 quantiser for newly appended indexer queries or keys
@@ -209,7 +227,10 @@ dsa_status dsa_quantize_e4m3_rows(const float* x, int n, int d, uint8_t* codes, 
  * quantised exactly as by dsa_quantize_e4m3_rows with one scale over its
  * heads * d values. codes [n, heads * d] e4m3, scale [n] f32, rotated
  * [n, heads * d] f32 or NULL (receives the fp32 rotated rows). rope_dim even,
- * 2 <= rope_dim <= min(d, 128); base finite and > 0. n = 0 is a no-op. */
+ * 2 <= rope_dim <= min(d, 128); base finite and > 0. Each row is read twice
+ * and a thread reads values other threads rotate, so rotated, codes and
+ * scale must not overlap x: an in-place call returns DSA_ERR_INVALID_ARG.
+ * n = 0 is a no-op. */
 dsa_status dsa_rope_quantize_e4m3_rows(const float* x, const int32_t* pos, int n, int heads, int d, int rope_dim,
                                        double base, int interleaved, uint8_t* codes, float* scale, float* rotated,
                                        void* stream);
@@ -290,7 +311,10 @@ dsa_status dsa_sparse_mla_attn_decode(const uint16_t* q, const uint16_t* kv, con
  * enqueued) with the limit in dsa_last_error().
  * The first call on each device looks up the array's device address (a
  * runtime query, no allocation); make that first call before any stream
- * capture. Every call shares the one array: calls whose work overlaps on the
+ * capture. The address is kept for the life of the process, so after a
+ * cudaDeviceReset (or anything else that re-creates a device's primary
+ * context) this entry point must not be called on that device again. Every
+ * call shares the one array: calls whose work overlaps on the
  * GPU (different streams, or several host threads) race and must be ordered
  * by the caller. Nothing in the array needs to start at zero: each call
  * writes every element it later reads. No cudaMalloc, cudaFree or

@@ -62,6 +62,7 @@ def lib() -> ctypes.CDLL:
             L.dsa_quantize_e4m3_rows.argtypes = [P, I, I, P, P, P]
             L.dsa_rope_quantize_e4m3_rows.argtypes = [P, P, I, I, I, I, ctypes.c_double, I, P, P, P, P]
             L.dsa_sparse_mla_attn_paged.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, F, P, P, P]
+            L.dsa_sparse_mla_attn_varlen.argtypes = [P, P, P, P, P, I, I, I, I, I, F, P, P, P]
             L.dsa_index_topk_decode_workspace_size.argtypes = [I, I, I]
             L.dsa_index_topk_decode_workspace_size.restype = SZ
             L.dsa_index_topk_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P, P, SZ, P]
@@ -79,7 +80,7 @@ def lib() -> ctypes.CDLL:
                          "dsa_index_topk_chunk_paged",
                          "dsa_index_topk_varlen", "dsa_dense_mla_attn_causal", "dsa_quantize_e4m3_rows",
                          "dsa_rope_quantize_e4m3_rows",
-                         "dsa_sparse_mla_attn_paged",
+                         "dsa_sparse_mla_attn_paged", "dsa_sparse_mla_attn_varlen",
                          "dsa_index_scores", "dsa_sparse_mla_attn", "dsa_index_topk_decode",
                          "dsa_index_scores_decode", "dsa_sparse_mla_attn_decode", "dsa_get_device_error",
                          "dsa_index_topk_decode_noalloc", "dsa_index_topk_decode_paged",
@@ -315,6 +316,33 @@ def sparse_mla_attn_paged(q, kv_pool, block_table, idx, rows: int, scale: float,
     _check(lib().dsa_sparse_mla_attn_paged(_ptr(q), _ptr(kv_pool), _ptr(block_table), _ptr(idx), T, rows, pool_rows,
                                            bt_stride, max_blocks, page_size, Hq, topk, float(scale), _ptr(out),
                                            _ptr(lse), _stream(q.device)))
+    return out, lse
+
+
+def sparse_mla_attn_varlen(q, kv, idx, cu_q, cu_k, scale: float, *, out=None, lse=None, want_lse: bool = False):
+    """Attention over a packed batch: sequence b owns query tokens cu_q[b]:cu_q[b+1] and latent rows
+    cu_k[b]:cu_k[b+1] of kv; idx holds sequence-local rows (as index_topk_varlen returns them).
+    cu_q / cu_k: int32 [nseq+1] on the device (lists are copied there)."""
+    T, Hq, D = q.shape
+    total_k = kv.shape[0]
+    topk = idx.shape[1]
+    cu_q = torch.as_tensor(cu_q, dtype=torch.int32, device=q.device).contiguous()
+    cu_k = torch.as_tensor(cu_k, dtype=torch.int32, device=q.device).contiguous()
+    nseq = cu_q.numel() - 1
+    _req(q, "q", torch.bfloat16, (T, Hq, D_QK))
+    _req(kv, "kv", torch.bfloat16, (total_k, D_QK))
+    _req(idx, "idx", torch.int32, (T, topk))
+    _req(cu_q, "cu_q", torch.int32, (nseq + 1,))
+    _req(cu_k, "cu_k", torch.int32, (nseq + 1,))
+    if out is None:
+        out = torch.empty((T, Hq, D_V), dtype=torch.bfloat16, device=q.device)
+    _req(out, "out", torch.bfloat16, (T, Hq, D_V))
+    if lse is None and want_lse:
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _req(lse, "lse", torch.float32, (T, Hq))
+    _check(lib().dsa_sparse_mla_attn_varlen(_ptr(q), _ptr(kv), _ptr(idx), _ptr(cu_q), _ptr(cu_k), nseq, T, total_k,
+                                            Hq, topk, float(scale), _ptr(out), _ptr(lse), _stream(q.device)))
     return out, lse
 
 

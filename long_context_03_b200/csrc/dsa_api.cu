@@ -41,6 +41,13 @@ dsa_status cuda_fail(cudaError_t e, const char* what) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Whether the byte ranges [a, a + na) and [b, b + nb) share a byte.
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
 int num_sms() {
   int dev = 0;
   cudaGetDevice(&dev);
@@ -296,10 +303,15 @@ struct MlaPaging {
   const int32_t* block_table = nullptr;
   int bt_stride = 0, page_shift = 0, pool_rows = 0;
 };
+struct MlaPacked {  // packed batch: device cu_seqlens of the queries and of the cache rows
+  const int32_t* cu_q = nullptr;
+  const int32_t* cu_k = nullptr;
+  int nseq = 0;
+};
 dsa_status launch_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int T, int rows, long long kv_stride,
                       int Hq, int topk, float scale, uint16_t* out, float* lse, cudaStream_t st, int causal_q0 = 0,
-                      MlaPaging pg = MlaPaging()) {
-  MlaParams p;
+                      MlaPaging pg = MlaPaging(), MlaPacked pk = MlaPacked()) {
+  MlaParams p = {};
   p.q = reinterpret_cast<const __nv_bfloat16*>(q);
   p.kv = reinterpret_cast<const __nv_bfloat16*>(kv);
   p.idx = idx;
@@ -315,6 +327,9 @@ dsa_status launch_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
   p.bt_stride = pg.bt_stride;
   p.page_shift = pg.page_shift;
   p.pool_rows = pg.pool_rows;
+  p.seq_cu_q = pk.cu_q;
+  p.seq_cu_k = pk.cu_k;
+  p.nseq = pk.nseq;
   p.scale_log2 = scale * 1.4426950408889634f;
   CUtensorMap tmQ;
   dsa_status s = make_map_q_bf16(&tmQ, q, T, Hq);
@@ -663,6 +678,9 @@ dsa_status dsa_quantize_e4m3_rows(const float* x, int n, int d, uint8_t* codes, 
   if (n < 0 || d <= 0) return fail(DSA_ERR_INVALID_ARG, "n=%d d=%d", n, d);
   if (n == 0) return DSA_OK;
   if (!x || !codes || !scale) return fail(DSA_ERR_INVALID_ARG, "null pointer");
+  const size_t nx = static_cast<size_t>(n) * d;
+  if (overlaps(x, nx * 4, codes, nx) || overlaps(x, nx * 4, scale, static_cast<size_t>(n) * 4))
+    return fail(DSA_ERR_INVALID_ARG, "codes / scale overlap x");
   const int grid = n < 8 * num_sms() ? n : 8 * num_sms();
   quantize_e4m3_rows_kernel<<<grid, kQuantThreads, 0, static_cast<cudaStream_t>(stream)>>>(x, n, d, codes, scale);
   return check_launch("quantize_e4m3_rows_kernel");
@@ -678,6 +696,10 @@ dsa_status dsa_rope_quantize_e4m3_rows(const float* x, const int32_t* pos, int n
   if (!std::isfinite(base) || !(base > 0.0)) return fail(DSA_ERR_INVALID_ARG, "base must be finite and > 0");
   if (n == 0) return DSA_OK;
   if (!x || !pos || !codes || !scale) return fail(DSA_ERR_INVALID_ARG, "null pointer");
+  const size_t nx = static_cast<size_t>(n) * heads * d;
+  if (overlaps(x, nx * 4, rotated, nx * 4) || overlaps(x, nx * 4, codes, nx) ||
+      overlaps(x, nx * 4, scale, static_cast<size_t>(n) * 4))
+    return fail(DSA_ERR_INVALID_ARG, "rotated / codes / scale overlap x (no in-place rotation)");
   const int grid = n < 8 * num_sms() ? n : 8 * num_sms();
   rope_quantize_e4m3_rows_kernel<<<grid, kQuantThreads, 0, static_cast<cudaStream_t>(stream)>>>(
       x, pos, n, heads, d, rope_dim, base, interleaved, codes, scale, rotated);
@@ -697,6 +719,22 @@ dsa_status dsa_dense_mla_attn_causal(const uint16_t* q, const uint16_t* kv, int 
   if (!std::isfinite(scale) || !(scale > 0.f)) return fail(DSA_ERR_INVALID_ARG, "scale must be finite and > 0");
   if (T == 0) return DSA_OK;
   return launch_mla(q, kv, nullptr, T, L, 0, Hq, L, scale, out, lse, static_cast<cudaStream_t>(stream), q0);
+}
+
+dsa_status dsa_sparse_mla_attn_varlen(const uint16_t* q, const uint16_t* kv, const int32_t* idx, const int32_t* cu_q,
+                                      const int32_t* cu_k, int nseq, int T, int total_k, int Hq, int topk, float scale,
+                                      uint16_t* out, float* lse, void* stream) {
+  dsa_status s = check_mla_args(q, kv, idx, T, total_k, Hq, topk, scale, out);
+  if (s != DSA_OK) return s;
+  if (nseq < 1) return fail(DSA_ERR_INVALID_ARG, "nseq=%d", nseq);
+  if (!cu_q || !cu_k) return fail(DSA_ERR_INVALID_ARG, "null pointer");
+  if (T == 0) return DSA_OK;
+  MlaPacked pk;
+  pk.cu_q = cu_q;
+  pk.cu_k = cu_k;
+  pk.nseq = nseq;
+  return launch_mla(q, kv, idx, T, total_k, 0, Hq, topk, scale, out, lse, static_cast<cudaStream_t>(stream), 0,
+                    MlaPaging(), pk);
 }
 
 dsa_status dsa_sparse_mla_attn(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int T, int L, int Hq,

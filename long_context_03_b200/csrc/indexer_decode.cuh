@@ -581,19 +581,168 @@ __device__ __forceinline__ void sort_keys_to_idx(uint64_t* s, const uint64_t* sr
   for (int i = tid; i < K; i += NT) out[i] = (s[i] == 0ull) ? -1 : rank_key_index(s[i]);
 }
 
-// Exact top-k of sequence blockIdx.x; with idx set, also ranks the keys and
-// writes the sequence's index row (no separate sort launch).
+// Largest histogram bin the decode ranking scans key by key.
+constexpr int kDecodeBinRankMax = 256;
+
+// The fast path of the decode selection: the candidates (keys in bins above
+// the boundary bin of the scoring kernel's 11-bit histogram, plus the
+// boundary bin's own keys) are gathered in shared memory and ranked by one
+// finer histogram pass (topk_rank_by_bins), which writes the sequence's
+// index row. False when the boundary bin is too large for shared memory or a
+// finer bin is too crowded; nothing is written to idx then.
+__device__ __forceinline__ bool decode_rank_fast(const float* __restrict__ scores, const int32_t* __restrict__ lens,
+                                                 int L_max, int K, const uint32_t* __restrict__ hist_in,
+                                                 int32_t* __restrict__ idx) {
+  constexpr int NT = kDecodeSelThreads;
+  constexpr int NV = (2048 + kDecodeSelBinCap) / NT;  // candidate slots per thread
+  extern __shared__ __align__(16) uint8_t dsmem[];
+  uint64_t* bin_keys = reinterpret_cast<uint64_t*>(dsmem);  // [kDecodeSelBinCap]; the ranking buffer afterwards
+  uint64_t* abv = bin_keys + kDecodeSelBinCap;              // [2048] keys above the boundary bin
+  int* hist = reinterpret_cast<int*>(abv + 2048);           // [2048]
+  int* start = hist + 2048;                                 // [2048]
+  int* small = start + 2048;                                // [64]
+  __shared__ int wsum[32];
+  __shared__ int res[4];
+  __shared__ int npos, bpos;
+  __shared__ int never_aborts;  // no bounded waits in this kernel
+  const int b = blockIdx.x;
+  const int n = min(lens[b], L_max);
+  const float* sc = scores + static_cast<size_t>(b) * L_max;
+  int32_t* out = idx + static_cast<size_t>(b) * K;
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    never_aborts = 0;
+    npos = 0;
+    bpos = 0;
+  }
+  const GroupBar bar{1, NT, AbortFlag{&never_aborts}};
+  if (n <= K) {  // every key is selected: rank them all (K <= 2048 = 2 per thread)
+    uint64_t v[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int i = tid + j * NT;
+      v[j] = (i < n) ? rank_key(sc[i], static_cast<uint32_t>(i)) : 0ull;
+    }
+    __syncthreads();
+    return topk_rank_by_bins<NT, 2>(v, K, hist, start, small, bin_keys, kDecodeSelBinCap, kDecodeBinRankMax, tid,
+                                    bar, out);
+  }
+  // 1. the scoring kernel's 2048-bin histogram of the top 11 key bits
+  if (hist_in) {
+    for (int i = tid; i < 2048; i += NT) hist[i] = static_cast<int>(hist_in[static_cast<size_t>(b) * 2048 + i]);
+  } else {
+    for (int i = tid; i < 2048; i += NT) hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < n; i += NT) atomicAdd(hist + key_bin11(rank_key(sc[i], static_cast<uint32_t>(i))), 1);
+  }
+  __syncthreads();
+  // 2. the bin of the K-th largest key: descending scan, 2 bins per thread
+  {
+    const int c0 = hist[2047 - 2 * tid], c1 = hist[2046 - 2 * tid];
+    const int tot = c0 + c1;
+    const int l = tid & 31, w = tid >> 5;
+    int incl = tot;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (l >= off) incl += y;
+    }
+    if (l == 31) wsum[w] = incl;
+    __syncthreads();
+    int wbase = 0;
+    for (int i = 0; i < w; ++i) wbase += wsum[i];
+    const int excl = wbase + incl - tot;
+    if (excl < K && excl + tot >= K) {
+      if (excl + c0 >= K) {
+        res[0] = 2047 - 2 * tid; res[1] = excl; res[2] = c0;
+      } else {
+        res[0] = 2046 - 2 * tid; res[1] = excl + c0; res[2] = c1;
+      }
+    }
+    __syncthreads();
+  }
+  const uint32_t dbin = static_cast<uint32_t>(res[0]);
+  const int above = res[1], inb = res[2];
+  if (inb > kDecodeSelBinCap || above > 2048) return false;
+  // 3. one pass over the scores: keys above the bin and the bin's keys to
+  //    shared memory (4 keys per thread per round, warp-aggregated appends)
+  const int lane = tid & 31;
+  const bool vec = ((L_max & 3) == 0) && ((reinterpret_cast<uintptr_t>(scores) & 15) == 0);
+  const int nround = (n + 4 * NT - 1) / (4 * NT);
+  for (int rd = 0; rd < nround; ++rd) {
+    const int i0 = 4 * (rd * NT + tid);
+    float f[4];
+    if (vec && i0 + 3 < n) {
+      const float4 x = *reinterpret_cast<const float4*>(sc + i0);
+      f[0] = x.x; f[1] = x.y; f[2] = x.z; f[3] = x.w;
+    } else {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) f[u] = (i0 + u < n) ? sc[i0 + u] : 0.f;
+    }
+    uint64_t key[4];
+    uint32_t hi = 0, eq = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      key[u] = rank_key(f[u], static_cast<uint32_t>(i0 + u));
+      const uint32_t bin = key_bin11(key[u]);
+      const bool in = i0 + u < n;
+      hi |= (in && bin > dbin) ? (1u << u) : 0u;
+      eq |= (in && bin == dbin) ? (1u << u) : 0u;
+    }
+    const int mine = __popc(hi) | (__popc(eq) << 16);
+    int incl = mine;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    int base = 0;
+    if (lane == 31 && incl != 0) {
+      const int th = incl & 0xffff, te = incl >> 16;
+      base = (th ? atomicAdd(&npos, th) : 0) | ((te ? atomicAdd(&bpos, te) : 0) << 16);
+    }
+    base = __shfl_sync(0xffffffffu, base, 31);
+    int ph = (base & 0xffff) + ((incl - mine) & 0xffff);
+    int pe = (base >> 16) + ((incl - mine) >> 16);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if ((hi >> u) & 1u) {
+        if (ph < 2048) abv[ph] = key[u];
+        ++ph;
+      }
+      if ((eq >> u) & 1u) {
+        if (pe < kDecodeSelBinCap) bin_keys[pe] = key[u];
+        ++pe;
+      }
+    }
+  }
+  __syncthreads();
+  // 4. rank the candidates (the ranking buffer reuses the bin keys' space
+  //    once every thread holds its candidates)
+  uint64_t v[NV];
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int i = tid + j * NT;
+    v[j] = (i < above) ? abv[i] : ((i - above < inb) ? bin_keys[i - above] : 0ull);
+  }
+  return topk_rank_by_bins<NT, NV>(v, K, hist, start, small, bin_keys, kDecodeSelBinCap, kDecodeBinRankMax, tid,
+                                   bar, out);
+}
+
+// Exact top-k of sequence blockIdx.x, ranked, as its index row idx[b, 0..K):
+// the fast path above, else (a crowded bin) the exact select into sel_keys
+// and a bitonic ranking of those keys.
 __global__ void __launch_bounds__(kDecodeSelThreads)
     decode_select_kernel(const float* __restrict__ scores, const int32_t* __restrict__ lens, int L_max, int K,
                          const uint32_t* __restrict__ hist_in, uint64_t* __restrict__ sel_keys,
                          int32_t* __restrict__ idx) {
+  if (decode_rank_fast(scores, lens, L_max, K, hist_in, idx)) return;  // the same answer on every thread
+  __syncthreads();
   decode_select_body(scores, lens, L_max, K, hist_in, sel_keys);
-  if (idx) {
-    extern __shared__ __align__(16) uint8_t dsmem[];
-    __syncthreads();  // the selected keys (global, this CTA's writes) are complete; the bin buffer is free
-    const size_t row = static_cast<size_t>(blockIdx.x) * K;
-    sort_keys_to_idx<kDecodeSelThreads>(reinterpret_cast<uint64_t*>(dsmem), sel_keys + row, K, idx + row);
-  }
+  extern __shared__ __align__(16) uint8_t dsmem[];
+  __syncthreads();  // the selected keys (global, this CTA's writes) are complete; the bin buffer is free
+  const size_t row = static_cast<size_t>(blockIdx.x) * K;
+  sort_keys_to_idx<kDecodeSelThreads>(reinterpret_cast<uint64_t*>(dsmem), sel_keys + row, K, idx + row);
 }
 
 }  // namespace dsa

@@ -52,7 +52,7 @@ struct IdxPrefillCfg {
   static constexpr int NET = NEPI * 32;        // epilogue threads
   static constexpr int TOK_PER_WARP = TB;      // an epilogue warp scores every token of its buffer
   static constexpr int TPH = 64 / HI;          // tokens per 64-column half of a buffer
-  static constexpr int CHECK_EVERY = 4;        // key tiles between list-capacity checks
+  static constexpr int CHECK_EVERY = 16;       // key tiles between list-capacity checks
   static constexpr int NSAMPLE = 8;            // key tiles scored first to set a row's starting threshold
   static constexpr SwizzleMode SW = (DI == 128) ? kSw128 : kSw64;
   static constexpr uint32_t SBO = 8 * DI;      // bytes between 8-row core groups

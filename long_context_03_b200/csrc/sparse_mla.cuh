@@ -122,8 +122,35 @@ struct MlaParams {
   // of kv (a pool of pool_rows rows); bt_stride 0 shares one table row.
   const int32_t* block_table;
   int bt_stride, page_shift, pool_rows;
+  // Packed batch (cu_seqlens, device arrays): when seq_cu_q is set, token i
+  // belongs to the sequence b with seq_cu_q[b] <= i < seq_cu_q[b+1] and reads
+  // kv rows seq_cu_k[b] .. seq_cu_k[b+1]-1 (its indices are local to the
+  // sequence); rows then holds the packed cache's row count, and every
+  // sequence's rows are clamped into it.
+  const int32_t* seq_cu_q;
+  const int32_t* seq_cu_k;
+  int nseq;
   float scale_log2;          // softmax scale * log2(e)
 };
+
+// First row and row count of token tk's cache.
+__device__ __forceinline__ void token_cache(const MlaParams& p, int tk, const __nv_bfloat16*& kv_tok, int& rows) {
+  if (p.seq_cu_q) {
+    int lo = 0, hi = p.nseq - 1;  // the last sequence whose first query is at or before tk
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (__ldg(p.seq_cu_q + mid) <= tk) lo = mid;
+      else hi = mid - 1;
+    }
+    const int k0 = min(max(__ldg(p.seq_cu_k + lo), 0), p.rows);
+    const int k1 = min(max(__ldg(p.seq_cu_k + lo + 1), k0), p.rows);
+    kv_tok = p.kv + static_cast<long long>(k0) * MlaCfg::D;
+    rows = k1 - k0;
+  } else {
+    kv_tok = p.kv + tk * p.kv_token_stride;
+    rows = p.rows;
+  }
+}
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -361,7 +388,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       uint32_t q_ph0 = 1;
       int q_issued = 0;
       for (int tk = cluster_id; tk < p.T; tk += nclusters, ++n) {
-        const __nv_bfloat16* kv_tok = p.kv + tk * p.kv_token_stride;
+        const __nv_bfloat16* kv_tok;
+        int trows;
+        token_cache(p, tk, kv_tok, trows);
         // the softmax warps are done with this mask buffer (two tokens back)
         const int mb = n & 1;
         if (!mbar_wait(bars + C::B_MASK_FREE + mb, ((n >> 1) & 1) ^ 1, ab, 30)) break;
@@ -370,7 +399,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
         for (int wd = static_cast<int>(warp); wd < nchunk * (C::NK / 32); wd += C::NPROD) {
           const int e = wd * 32 + static_cast<int>(lane);
           const int row = (e < p.K) ? idx_s[e] : -1;
-          bool present = row >= 0 && row < p.rows;
+          bool present = row >= 0 && row < trows;
           if (kPaged && present) {  // paged: the page must lie inside the pool
             const int page = p.block_table[static_cast<long long>(tk) * p.bt_stride + (row >> p.page_shift)];
             present = page >= 0 && (static_cast<long long>(page) << p.page_shift) +
@@ -401,7 +430,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
           if (++slot == C::NSST) { slot = 0; ph ^= 1; }
         }
         for (int j = 0; j < nchunk && ok; ++j) {
-          const ChunkRows cr = chunk_rows<kPaged>(p, kv_tok, tk, idx_s, j, p.K, p.rows, ptid);
+          const ChunkRows cr = chunk_rows<kPaged>(p, kv_tok, tk, idx_s, j, p.K, trows, ptid);
           for (int i = 0; i < C::NSLAB_QK; ++i) {
             if (!mbar_wait(bars + C::B_RING_EMPTY + slot, ph, ab, 31)) { ok = false; break; }
             gather_slab_tile(ring + slot * C::SLAB_TILE, cr, i, ptid);
@@ -617,13 +646,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       int slot = 0;
       uint32_t ph = 1;
       for (int tk = cluster_id; tk < p.T; tk += nclusters) {
-        const __nv_bfloat16* kv_tok = p.kv + tk * p.kv_token_stride;
+        const __nv_bfloat16* kv_tok;
+        int trows;
+        token_cache(p, tk, kv_tok, trows);
         stage_index_row(idx_s, p.idx ? p.idx + static_cast<size_t>(tk) * p.K : nullptr, p.K, ptid, p.causal_q0 + tk);
         bool ok = true;
         for (int j = 0; j < nchunk && ok; ++j) {
           for (int u = 0; u < C::NK / C::VROWS; ++u) {
             if (!mbar_wait(bars + C::B_RING_EMPTY + slot, ph, ab, 41)) { ok = false; break; }
-            gather_value_tile<kPaged>(ring + slot * C::V_TILE, p, kv_tok, tk, idx_s, j, u, p.K, p.rows, ptid);
+            gather_value_tile<kPaged>(ring + slot * C::V_TILE, p, kv_tok, tk, idx_s, j, u, p.K, trows, ptid);
             cp_async_mbar_arrive(bars + C::B_RING_FULL + slot);
             if (++slot == C::NVST) { slot = 0; ph ^= 1; }
           }

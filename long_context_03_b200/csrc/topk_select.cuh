@@ -266,11 +266,11 @@ __device__ __forceinline__ bool topk_rank_by_bins(const uint64_t (&v)[M], int K,
                                                   uint64_t* buf, int bufn, int cmax, int et, const GroupBar& bar,
                                                   int32_t* __restrict__ dst) {
   constexpr int NW = NT / 32;
-  static_assert(NT == 512, "four bins per thread");
+  static_assert(NT == 512 || NT == 1024, "two or four bins per thread");
   constexpr int BPT = 2048 / NT;
   int* wsum = small;                                                        // [NW]
-  unsigned long long* mm = reinterpret_cast<unsigned long long*>(small + 16);  // min, max
-  int* res = small + 24;  // b*, keys above b*, keys in b*, largest bin count, valid keys
+  unsigned long long* mm = reinterpret_cast<unsigned long long*>(small + 32);  // min, max
+  int* res = small + 40;  // b*, keys above b*, keys in b*, largest bin count, valid keys
   bar.sync();  // every thread is done with the previous row's hist, start and buf
   unsigned long long kmin = ~0ull, kmax = 0ull;
   int nv = 0;

@@ -137,6 +137,26 @@ def test_rope_quantiser_argument_checks(lib):
     assert lib.dsa_rope_quantize_e4m3_rows(None, None, 0, 64, 128, 64, b, 1, None, None, None, None) == 0  # empty
 
 
+def test_quantisers_refuse_outputs_that_overlap_the_input(lib):
+    # pointers are only compared, never dereferenced: the overlap check fails first
+    x = 1 << 20
+    n, heads, d = 4, 64, 128
+    row_bytes = heads * d * 4
+    other = ctypes.c_void_p(x + 64 * n * row_bytes)
+    b = ctypes.c_double(10000.0)
+    X = ctypes.c_void_p(x)
+    inside = ctypes.c_void_p(x + row_bytes)  # the second row of x
+    # (x, pos, n, heads, d, rope_dim, base, interleaved, codes, scale, rotated, stream)
+    assert lib.dsa_rope_quantize_e4m3_rows(X, other, n, heads, d, 64, b, 1, other, other, X, None) == -1  # in place
+    assert lib.dsa_rope_quantize_e4m3_rows(X, other, n, heads, d, 64, b, 1, other, other, inside, None) == -1
+    assert lib.dsa_rope_quantize_e4m3_rows(X, other, n, heads, d, 64, b, 1, inside, other, None, None) == -1
+    assert lib.dsa_rope_quantize_e4m3_rows(X, other, n, heads, d, 64, b, 1, other, inside, None, None) == -1
+    assert b"overlap" in lib.dsa_last_error()
+    # (x, n, d, codes, scale, stream)
+    assert lib.dsa_quantize_e4m3_rows(X, n, heads * d, inside, other, None) == -1
+    assert lib.dsa_quantize_e4m3_rows(X, n, heads * d, other, X, None) == -1
+
+
 def test_paged_prefill_chunk_argument_checks(lib):
     p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
     # (q_I, q_scale, w, k_pool, k_scale_pool, table, max_blocks, page, pool_rows, q0, Tq, L, H_I, d_I, topk,

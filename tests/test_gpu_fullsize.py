@@ -87,8 +87,14 @@ def test_prefill_L131072(dsa):
     P = workloads.make_config("prefill_L131072", device="cuda")
     idx, out = _run_prefill(dsa, P)
     g = np.random.default_rng(7)
-    rows = [0, 2047, 2048, 65535, 131070, 131071] + g.choice(131072, 2, replace=False).tolist()
-    _check_prefill_rows(dsa, P, idx, out, rows, score_block_rows=[131068])
+    # rows from every class of row block: short rows (t < 2048, all keys
+    # selected), the streamed range below the sampled starting thresholds,
+    # the sampled range t >= 16384 (most of the work), the block edges around
+    # the score-hook blocks, and the last block
+    rows = ([0, 1, 2046, 2047, 2048, 2049] + g.choice(np.arange(2050, 16384), 8, replace=False).tolist()
+            + g.choice(np.arange(16384, 131064), 40, replace=False).tolist()
+            + [16383, 16384, 16385, 65535, 65536, 65537, 99999, 100000] + list(range(131064, 131072)))
+    _check_prefill_rows(dsa, P, idx, out, rows, score_block_rows=[1024, 16384, 65536, 131068])
     del P, idx, out
     torch.cuda.empty_cache()
 

@@ -206,3 +206,71 @@ def test_prefill_chunk_bad_page_is_reported(dsa):
                                      page_size=64)
     assert dsa.device_error()[0] == 0
     assert torch.equal(idx, ref)
+
+
+def test_paged_decode_step_matches_the_oracle(dsa):
+    """Paged decode (keys and latent rows in one shuffled pool) against the
+    oracle on the logical caches: selection bit-exact against a CPU top-k of
+    the GPU's own scores and >= 99.9% overlap with the oracle's, attention
+    within tolerance, for ragged lengths."""
+    import oracle
+    from gpu_helpers import attn_close, cpu_topk_of, overlap_excluding_ties
+    B, L, page = 5, 20000, 64
+    lens = [20000, 2049, 1, 13333, 2048]
+    D = workloads.make_decode(B, L, 64, 128, 128, 2048, seed=45, lens=lens, device="cuda")
+    k_pool, ks_pool, table = _page_keys(D.k_cache, D.k_scale, D.lens, page, torch.Generator().manual_seed(11))
+    kv_pool = torch.zeros((k_pool.shape[0], 576), dtype=torch.bfloat16, device="cuda")
+    for b in range(B):
+        n = (lens[b] + page - 1) // page
+        rows = (table[b, :n].long()[:, None] * page + torch.arange(page, device="cuda")[None]).reshape(-1)
+        src = torch.zeros((n * page, 576), dtype=torch.bfloat16, device="cuda")
+        m = min(n * page, L)
+        src[:m] = D.kv[b, :m]
+        kv_pool[rows] = src
+    idx = dsa.index_topk_decode_paged(D.q_I, D.q_scale, D.w, k_pool, ks_pool, table, D.lens, 2048, page_size=page)
+    out, lse = dsa.sparse_mla_attn_paged(D.q, kv_pool, table, idx, L, D.scale, page_size=page, want_lse=True)
+    sc = dsa.index_scores_decode(D.q_I, D.q_scale, D.w, D.k_cache, D.k_scale, D.lens)
+    dsa.check_device_error()
+    host = workloads.DecodeInputs(B, L, 64, 128, 128, 2048, D.scale,
+                                  *[getattr(D, n).cpu() for n in ("q_I", "q_scale", "w", "k_cache", "k_scale", "q",
+                                                                  "kv", "lens")])
+    res = oracle.decode_seqs(host, range(B))
+    gidx = idx.cpu().numpy()
+    gsc = sc.cpu().numpy()
+    for b in range(B):
+        ref_sc, ref_idx, _, _ = res[b]
+        t = lens[b] - 1
+        assert np.array_equal(gidx[b], cpu_topk_of(gsc[b:b + 1, :t + 1], [t], 2048)[0]), b
+        assert overlap_excluding_ties(gidx[b:b + 1], ref_idx[None], ref_sc[None], [t], 2048) >= 0.999, b
+        ref_o, ref_l = oracle.sparse_mla(oracle._bf16_bits(host.q[b:b + 1]), host.kv[b, :lens[b]], gidx[b:b + 1],
+                                         D.scale)
+        ok, mx, rl = attn_close(out[b:b + 1], ref_o)
+        assert ok, (b, mx, rl)
+        np.testing.assert_allclose(lse[b].cpu().numpy(), ref_l[0], rtol=1e-4, atol=1e-4)
+
+
+def test_paged_prefill_keys_and_latent_rows_match_the_oracle(dsa):
+    """A chunk of a prefill over a paged FP8 key cache, then attention over a
+    paged latent cache (one shared table), against the oracle on sampled rows."""
+    import oracle
+    from gpu_helpers import attn_close, overlap_excluding_ties
+    L, page, q0, Tq = 20480, 64, 16000, 2000
+    P = workloads.make_prefill(L, 64, 128, 16, 2048, seed=57, device="cuda")
+    k_pool, ks_pool, table = _page_one(P.k_cache, P.k_scale, page, torch.Generator().manual_seed(12))
+    sl = slice(q0, q0 + Tq)
+    idx = dsa.index_topk_chunk_paged(P.q_I[sl], P.q_scale[sl], P.w[sl], k_pool, ks_pool, table, q0, q0 + Tq, 2048,
+                                     page_size=page)
+    kv_pool, kv_table = _page(P.kv[:q0 + Tq], page, torch.Generator().manual_seed(13))
+    out, _ = dsa.sparse_mla_attn_paged(P.q[sl].contiguous(), kv_pool, kv_table.cuda()[None], idx, q0 + Tq, P.scale,
+                                       page_size=page)
+    dsa.check_device_error()
+    local = [0, 1, 999, 1998, 1999]
+    rows = np.asarray([q0 + r for r in local], dtype=np.int64)
+    h = {n: getattr(P, n).cpu() for n in ("q_I", "q_scale", "w", "k_cache", "k_scale")}
+    ref_sc = oracle.index_scores(h["q_I"][rows], h["q_scale"][rows], h["w"][rows], h["k_cache"], h["k_scale"], rows,
+                                 query_rows=np.arange(len(rows)))
+    gidx = idx[local].cpu().numpy()
+    assert overlap_excluding_ties(gidx, oracle.topk(ref_sc, rows, 2048), ref_sc, rows, 2048) >= 0.999
+    ref_o, _ = oracle.sparse_mla(P.q[rows.tolist()].cpu(), P.kv.cpu(), gidx, P.scale)
+    ok, mx, rl = attn_close(out[local], ref_o)
+    assert ok, (mx, rl)
