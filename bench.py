@@ -24,6 +24,7 @@ prints its mean CUDA-event time as one JSON line:
 
     python bench.py --kernel indexer --prefill-L 65536 --repeat 5
     python bench.py --kernel attention --prefill-L 16384
+    python bench.py --kernel attention_chunk --chunk-T 2048   # last 2048 rows of the 128K prefill
     python bench.py --kernel decode --decode-B 64 --decode-L 65536
     python bench.py --kernel decode_paged --decode-B 64 --decode-L 65536 --page 64
     python bench.py --kernel rope --decode-B 64      # RoPE + E4M3 of B appended indexer rows
@@ -80,10 +81,13 @@ def parse(argv=None):
                     help="query-row chunks whose copies overlap the compute in the e2e leg (1: no overlap)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-rows", type=int, default=240)
-    ap.add_argument("--kernel", default=None, choices=["indexer", "attention", "decode", "decode_paged", "rope"],
+    ap.add_argument("--kernel", default=None,
+                    choices=["indexer", "attention", "attention_chunk", "decode", "decode_paged", "rope"],
                     help="time one hot-path call instead of the whole step (see the module docstring)")
     ap.add_argument("--repeat", type=int, default=5, help="calls in --kernel mode (the first min(3, repeat-1) warm up)")
     ap.add_argument("--page", type=int, default=64, help="page size of --kernel decode_paged")
+    ap.add_argument("--chunk-T", type=int, default=2048,
+                    help="--kernel attention_chunk: the last T query rows of the prefill attend over its whole cache")
     ap.add_argument("--no-fp8-probe", action="store_true",
                     help="skip the library FP8 GEMM measured after the timed work (context for the indexer's peak)")
     return ap.parse_args(argv)
@@ -592,6 +596,20 @@ def run_kernel(a):
         out = torch.empty((L, 128, D_V), dtype=torch.bfloat16, device=dev)
         fn = lambda: dsa.sparse_mla_attn(P.q, P.kv, idx, P.scale, out=out)
         shape = {"L": L}
+    elif a.kernel == "attention_chunk":
+        # the attention of the last T rows of an L-token prefill: their real
+        # selections (the chunked indexer) over the whole latent cache, with
+        # queries only for those rows (the full query tensor would be 19 GB)
+        T = min(a.chunk_T, L)
+        P = workloads.make_prefill(L, 64, 128, 1, k, seed=0, device=dev)
+        q0 = L - T
+        idx = dsa.index_topk_chunk(P.q_I[q0:].contiguous(), P.q_scale[q0:].contiguous(), P.w[q0:].contiguous(),
+                                   P.k_cache, P.k_scale, q0, k)
+        g = torch.Generator(device=dev).manual_seed(1)
+        q = torch.randn((T, 128, D_QK), generator=g, device=dev).to(torch.bfloat16)
+        out = torch.empty((T, 128, D_V), dtype=torch.bfloat16, device=dev)
+        fn = lambda: dsa.sparse_mla_attn(q, P.kv, idx, P.scale, out=out)
+        shape = {"L": L, "T": T}
     elif a.kernel == "rope":
         g = torch.Generator(device=dev).manual_seed(0)
         xq = torch.randn((B, 64, 128), generator=g, device=dev)

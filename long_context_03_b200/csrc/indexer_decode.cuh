@@ -84,7 +84,7 @@ __device__ __forceinline__ int paged_key_row(const IdxDecodeParams& p, int b, in
 __device__ __forceinline__ uint32_t key_bin11(uint64_t key) { return static_cast<uint32_t>(key >> 53); }
 
 template <int HI, int DI, bool kPaged>
-__global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS)
+__global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS, 2)
     indexer_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const IdxDecodeParams p) {
   using C = IdxDecodeCfg<HI, DI>;
@@ -285,27 +285,49 @@ __global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS)
     int g = 0;
     int cur_b = -1;
     bool ok = true;
+    const GroupBar bar{1, 128, ab};  // the four epilogue warps (abort-safe: see GroupBar)
+    // Per-key scales of an item's tiles (this thread's key in each), loaded one
+    // item ahead so their DRAM latency hides behind a whole item.
+    auto load_scales = [&](int it, float (&ks)[C::NKT]) {
+      int b, s0, nkt, n;
+      const bool v = it < it1 && item(it, b, s0, nkt, n);
+#pragma unroll
+      for (int kt = 0; kt < C::NKT; ++kt) {
+        ks[kt] = 0.f;
+        if (v && kt < nkt) {
+          const int s = s0 + kt * C::BM + quarter * 32 + static_cast<int>(lane);
+          if constexpr (kPaged) {
+            const int r = (s < n) ? paged_key_row(p, b, s) : -1;
+            if (r >= 0) ks[kt] = __ldg(p.k_scale + r);
+          } else {
+            if (s < n) ks[kt] = __ldg(p.k_scale + static_cast<size_t>(b) * p.L_max + s);
+          }
+        }
+      }
+    };
+    float ks_cur[C::NKT], ks_nxt[C::NKT];
+    load_scales(it0, ks_nxt);
     for (int it = it0; it < it1 && ok; ++it) {
+#pragma unroll
+      for (int kt = 0; kt < C::NKT; ++kt) ks_cur[kt] = ks_nxt[kt];
+      load_scales(it + 1, ks_nxt);
       int b, s0, nkt, n;
       if (!item(it, b, s0, nkt, n)) continue;
       if (b != cur_b) {
-        named_bar_sync(1, 128);  // the previous sequence's weights and counts are done with
+        if (!bar.sync()) { ok = false; break; }  // the previous sequence's weights and counts are done with
         if (p.hist && cur_b >= 0) flush_hist(cur_b);
         for (int i = et; i < HI; i += 128) w_s[i] = p.w[static_cast<size_t>(b) * HI + i];
-        named_bar_sync(1, 128);
+        if (!bar.sync()) { ok = false; break; }
         cur_b = b;
       }
       const float qs = p.q_scale[b];
+#pragma unroll 1
       for (int kt = 0; kt < nkt; ++kt, ++g) {
         const int buf = g % C::NACC;
         const int s = s0 + kt * C::BM + quarter * 32 + static_cast<int>(lane);
-        float ks = 0.f;
-        if constexpr (kPaged) {
-          const int r = (s < n) ? paged_key_row(p, b, s) : -1;
-          if (r >= 0) ks = p.k_scale[r];
-        } else {
-          if (s < n) ks = p.k_scale[static_cast<size_t>(b) * p.L_max + s];
-        }
+        float ks = ks_cur[0];
+#pragma unroll
+        for (int u = 1; u < C::NKT; ++u) ks = (kt == u) ? ks_cur[u] : ks;  // no dynamic register indexing
         if (!mbar_wait(acc_full + buf, (g / C::NACC) & 1, ab, 16)) { ok = false; break; }
         tc_fence_after();
         // eight independent partial sums (head j to sum j % 8), added in a
@@ -338,10 +360,8 @@ __global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS)
         }
       }
     }
-    if (p.hist && cur_b >= 0) {
-      named_bar_sync(1, 128);
-      flush_hist(cur_b);
-    }
+    if (ok && p.hist && cur_b >= 0 && bar.sync()) flush_hist(cur_b);
+    if (bar.aborted()) bar.leave();  // count this warp in at the barrier the others may wait at
   }
   __syncthreads();
   if (warp == 1) {

@@ -30,6 +30,8 @@
 // indices.
 #pragma once
 
+#include <type_traits>
+
 #include "dsa_common.cuh"
 #include "topk_select.cuh"
 
@@ -441,6 +443,11 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
     uint64_t* my_cand = p.cand + static_cast<size_t>(blockIdx.x) * C::RB * p.cap;
     int* pos_s = scr_s + cut_scratch_ints() - 16;  // 16 ints: warp sums of the block scan
     auto row_of = [&](int r) { return grp * C::TB + r; };
+    // this warp's sub-list of each of its rows in the CTA's candidate lists
+    uint64_t* row_ptr[TPW];
+#pragma unroll
+    for (int r = 0; r < TPW; ++r)
+      row_ptr[r] = my_cand + static_cast<size_t>(row_of(r)) * p.cap + static_cast<size_t>(quarter) * capq;
 
     for (int j = blockIdx.x; j < nrb; j += G) {
       const int rb = block_of(j);
@@ -507,7 +514,12 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
           ks_next = (s0 < bk.L) ? __ldg(p.k_scale + bk.kbase + s0) : 0.f;
         }
       }
-      for (int i = 0; i < nsteps && ok; ++i) {
+      // One key tile (step i of the block's sequence) for this warp: wait for
+      // its buffer, reduce the heads of its tokens, release the buffer, then
+      // filter and append. kMasked: the tile reaches past the block's first
+      // position (the causal diagonal or past the cache) or the block is ragged.
+      auto tile_step = [&](int i, auto masked_c) -> bool {
+        constexpr bool kMasked = decltype(masked_c)::value;
         const int kt = tile_at<C::NSAMPLE>(i, nkt, spec);
         const int s = kt * C::BM + quarter * 32 + static_cast<int>(lane);
         const float ks = ks_next;
@@ -523,10 +535,7 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
             ks_next = (sn < bk.L) ? __ldg(p.k_scale + bk.kbase + sn) : 0.f;
           }
         }
-        // only a tile reaching past the block's first position (the causal
-        // diagonal, or keys past the cache) or a ragged block needs masking
-        const bool masked = ragged || (kt * C::BM + C::BM - 1 > t0);
-        if (!mbar_wait(acc_full + grp, af_phase, ab, 8)) { ok = false; break; }
+        if (!mbar_wait(acc_full + grp, af_phase, ab, 8)) return false;
         af_phase ^= 1u;
         tc_fence_after();
         // this warp's 128 columns of the buffer (TPW tokens of HI heads) in
@@ -550,15 +559,13 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
           if constexpr (kSelect) {
             // a key can only pass if its score reaches the threshold's score
             bool pass = score >= thf_r[r];
-            if (masked) pass = pass && (r0 + tl < bk.rend) && (s <= t0 + tl);
+            if constexpr (kMasked) pass = pass && (r0 + tl < bk.rend) && (s <= t0 + tl);
             if (__any_sync(0xffffffffu, pass)) {
               const uint64_t key = (static_cast<uint64_t>(float_order_key(score)) << 32) |
                                    static_cast<uint64_t>(~static_cast<uint32_t>(s));
               const bool pred = pass && key > th_r[r];
               const uint32_t m = __ballot_sync(0xffffffffu, pred);
-              if (pred)
-                my_cand[static_cast<size_t>(tl) * p.cap + static_cast<size_t>(quarter) * capq + cnt_r[r] +
-                        __popc(m & lanemask_lt)] = key;
+              if (pred) row_ptr[r][cnt_r[r] + __popc(m & lanemask_lt)] = key;
               cnt_r[r] += __popc(m);
             }
           } else {
@@ -567,7 +574,10 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
               p.scores[static_cast<size_t>(t - p.row0) * p.L + s] = score;
           }
         }
-        if (!ok) break;
+        return true;
+      };
+      // After step i: the end of the sample, or a capacity checkpoint.
+      auto after_step = [&](int i) -> bool {
         if constexpr (kSelect) {
           if (spec && i == C::NSAMPLE - 1) {
             // End of the sample: each row's threshold starts at the score of
@@ -576,7 +586,7 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
             // so equal scores are kept), and the list is emptied: the sampled
             // tiles come round again in order.
             publish_counts();
-            if (!bar.sync()) { ok = false; break; }
+            if (!bar.sync()) return false;
             for (int tl = 0; tl < C::RB; ++tl) {
               const int t = t0 + tl;
               if (r0 + tl >= bk.rend) break;
@@ -598,25 +608,25 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
               if (!bar.sync()) break;
             }
             if (et < 4 * C::RB) cnt_s[et] = 0;
-            if (!bar.sync()) { ok = false; break; }
+            if (!bar.sync()) return false;
             reload_rows();
-            continue;
+            return true;
           }
           // Every CHECK_EVERY tiles, cut any list whose sub-list could
           // overflow before the next check (at most 32 appends per sub-list
           // and tile): one histogram pass keeps every key in or above the bin
           // of the k-th largest; if that keeps too many, an exact select
           // keeps exactly k.
-          if ((i % C::CHECK_EVERY) != C::CHECK_EVERY - 1) continue;
+          if ((i % C::CHECK_EVERY) != C::CHECK_EVERY - 1) return true;
           unsigned long long near = 0;  // rows of this warp whose sub-list is near capacity
 #pragma unroll
           for (int r = 0; r < NR; ++r)
             if (cnt_r[r] > capq - 32 * C::CHECK_EVERY) near |= 1ull << row_of(r);
           if (lane == 0 && near) atomicOr(cutmask_s, near);
           publish_counts();
-          if (!bar.sync()) { ok = false; break; }
+          if (!bar.sync()) return false;
           const unsigned long long cmask = *cutmask_s;
-          if (cmask == 0) continue;
+          if (cmask == 0) return true;
           for (int tl = 0; tl < C::RB; ++tl) {
             const int* cn = cnt_s + tl * 4;
             if ((cmask >> tl) & 1ull) {
@@ -642,10 +652,18 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
           }
           // every flagged row was cut; all threads read the mask before the cuts' barriers
           if (et == 0) *cutmask_s = 0;
-          if (!bar.sync()) { ok = false; break; }
+          if (!bar.sync()) return false;
           reload_rows();
         }
-      }
+        return true;
+      };
+      // the sampled tiles, then the tiles wholly at or before the block's
+      // first position (no masking), then the masked tail
+      const int ns = spec ? C::NSAMPLE : 0;
+      const int kt_m = ragged ? 0 : min(nkt, (t0 + 1) / C::BM);
+      for (int i = 0; i < ns && ok; ++i) ok = tile_step(i, std::true_type{}) && after_step(i);
+      for (int i = ns; i < ns + kt_m && ok; ++i) ok = tile_step(i, std::false_type{}) && after_step(i);
+      for (int i = ns + kt_m; i < nsteps && ok; ++i) ok = tile_step(i, std::true_type{}) && after_step(i);
       if (!ok) break;
       if constexpr (kSelect) {
         // exact top-k of each row: the histogram pass finds the boundary bin,

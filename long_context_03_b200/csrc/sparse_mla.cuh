@@ -295,11 +295,12 @@ __device__ __forceinline__ void gather_value_tile(uint32_t tile, const MlaParams
 }
 
 // The producer warps copy a token's index row into shared memory once
-// (named barrier 1 among the 128 producer threads on both sides). Without
-// an index row (dense causal mode) entry e is row e for e <= pos, else absent.
-__device__ __forceinline__ void stage_index_row(int32_t* idx_s, const int32_t* __restrict__ idx_tok, int K, int ptid,
-                                                int pos) {
-  named_bar_sync(1, MlaCfg::NPROD * 32);  // everyone is done with the previous row
+// (group barrier `bar` among the 128 producer threads on either side).
+// Without an index row (dense causal mode) entry e is row e for e <= pos,
+// else absent. False once the CTA aborted (nothing is staged then).
+__device__ __forceinline__ bool stage_index_row(int32_t* idx_s, const int32_t* __restrict__ idx_tok, int K, int ptid,
+                                                int pos, const GroupBar& bar) {
+  if (!bar.sync()) return false;  // everyone is done with the previous row
   if (idx_tok == nullptr) {
     for (int i = ptid; i < K; i += MlaCfg::NPROD * 32) idx_s[i] = (i <= pos) ? i : -1;
   } else if ((K & 3) == 0 && (reinterpret_cast<uintptr_t>(idx_tok) & 15) == 0) {
@@ -309,7 +310,7 @@ __device__ __forceinline__ void stage_index_row(int32_t* idx_s, const int32_t* _
   } else {
     for (int i = ptid; i < K; i += MlaCfg::NPROD * 32) idx_s[i] = __ldg(idx_tok + i);
   }
-  named_bar_sync(1, MlaCfg::NPROD * 32);
+  return bar.sync();
 }
 
 template <bool kPaged>
@@ -382,6 +383,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       int slot = 0;
       uint32_t ph = 1;
       int n = 0;  // tokens done by this cluster
+      const GroupBar pbar{1, C::NPROD * 32, ab};  // the producer warps (abort-safe: see GroupBar)
       // thread 0: where the last token's Q tiles start in the ring and how
       // many it loaded, so that an abort can still wait for its copies in flight
       int q_slot0 = 0;
@@ -394,7 +396,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
         // the softmax warps are done with this mask buffer (two tokens back)
         const int mb = n & 1;
         if (!mbar_wait(bars + C::B_MASK_FREE + mb, ((n >> 1) & 1) ^ 1, ab, 30)) break;
-        stage_index_row(idx_s, p.idx ? p.idx + static_cast<size_t>(tk) * p.K : nullptr, p.K, ptid, p.causal_q0 + tk);
+        if (!stage_index_row(idx_s, p.idx ? p.idx + static_cast<size_t>(tk) * p.K : nullptr, p.K, ptid,
+                             p.causal_q0 + tk, pbar))
+          break;
         // validity bits of every selection entry, 32 per word (entry e -> word e/32)
         for (int wd = static_cast<int>(warp); wd < nchunk * (C::NK / 32); wd += C::NPROD) {
           const int e = wd * 32 + static_cast<int>(lane);
@@ -454,6 +458,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
           mbar_wait(bars + C::B_RING_FULL + pos % C::NSST, full_par, no_abort, 28);
         }
       }
+      __syncwarp();
+      if (pbar.aborted()) pbar.leave();  // count this warp in at the barrier the others may wait at
     } else if (warp == C::W_MMA) {
       // The whole warp runs the loop and waits converged; one elected lane
       // issues each slab's MMAs together with every commit that covers them.
@@ -645,11 +651,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       const int ptid = threadIdx.x;
       int slot = 0;
       uint32_t ph = 1;
+      const GroupBar pbar{1, C::NPROD * 32, ab};  // the producer warps (abort-safe: see GroupBar)
       for (int tk = cluster_id; tk < p.T; tk += nclusters) {
         const __nv_bfloat16* kv_tok;
         int trows;
         token_cache(p, tk, kv_tok, trows);
-        stage_index_row(idx_s, p.idx ? p.idx + static_cast<size_t>(tk) * p.K : nullptr, p.K, ptid, p.causal_q0 + tk);
+        if (!stage_index_row(idx_s, p.idx ? p.idx + static_cast<size_t>(tk) * p.K : nullptr, p.K, ptid,
+                             p.causal_q0 + tk, pbar))
+          break;
         bool ok = true;
         for (int j = 0; j < nchunk && ok; ++j) {
           for (int u = 0; u < C::NK / C::VROWS; ++u) {
@@ -662,6 +671,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
         if (!ok) break;
       }
       asm volatile("cp.async.wait_all;" ::: "memory");
+      if (pbar.aborted()) pbar.leave();  // count this warp in at the barrier the others may wait at
     } else if (warp == C::W_MMA) {
       // whole warp waits converged; one elected lane issues and commits
       int slot = 0;
