@@ -86,12 +86,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   if (mbar_try_wait(a, parity)) return true;
   const long long t0 = clock64();
   while (true) {
-    // a few probes between the abort and clock checks: each probe may
-    // suspend the thread for a while, and the checks cost issue slots that
-    // the warps doing work share
-#pragma unroll 1
-    for (int k = 0; k < 8; ++k)
-      if (mbar_try_wait(a, parity)) return true;
+    if (mbar_try_wait(a, parity)) return true;
     if (ab.raised()) return false;
     if (clock64() - t0 > bound) {
       set_device_error(kErrTimeout, where);

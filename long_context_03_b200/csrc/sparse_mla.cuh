@@ -100,7 +100,8 @@ struct MlaCfg {
   static constexpr int B_QUIESCE = B_STAGE + 1;             // value CTA: all PV issued so far complete
   static constexpr int B_MASK_FULL = B_QUIESCE + 1;         // [2] score CTA: producers wrote a token's masks
   static constexpr int B_MASK_FREE = B_MASK_FULL + 2;       // [2] score CTA: softmax is done with them
-  static constexpr int NBAR = B_MASK_FREE + 2;
+  static constexpr int B_PSTAGE = B_MASK_FREE + 2;          // both CTAs: the producers' index-row staging
+  static constexpr int NBAR = B_PSTAGE + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 32;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -294,13 +295,17 @@ __device__ __forceinline__ void gather_value_tile(uint32_t tile, const MlaParams
   }
 }
 
-// The producer warps copy a token's index row into shared memory once
-// (group barrier `bar` among the 128 producer threads on either side).
-// Without an index row (dense causal mode) entry e is row e for e <= pos,
-// else absent. False once the CTA aborted (nothing is staged then).
+// The producer warps copy a token's index row into shared memory once. The
+// 128 producer threads of a CTA meet twice per token on the mbarrier
+// `stage` (everyone is done with the previous row; the new row is written),
+// with bounded waits, so a producer that gives up never leaves the others
+// waiting. Without an index row (dense causal mode) entry e is row e for
+// e <= pos, else absent. False once the CTA aborted.
 __device__ __forceinline__ bool stage_index_row(int32_t* idx_s, const int32_t* __restrict__ idx_tok, int K, int ptid,
-                                                int pos, const GroupBar& bar) {
-  if (!bar.sync()) return false;  // everyone is done with the previous row
+                                                int pos, uint64_t* stage, uint32_t& phase, AbortFlag ab) {
+  mbar_arrive(stage);
+  if (!mbar_wait(stage, phase, ab, 26)) return false;  // everyone is done with the previous row
+  phase ^= 1u;
   if (idx_tok == nullptr) {
     for (int i = ptid; i < K; i += MlaCfg::NPROD * 32) idx_s[i] = (i <= pos) ? i : -1;
   } else if ((K & 3) == 0 && (reinterpret_cast<uintptr_t>(idx_tok) & 15) == 0) {
@@ -310,7 +315,10 @@ __device__ __forceinline__ bool stage_index_row(int32_t* idx_s, const int32_t* _
   } else {
     for (int i = ptid; i < K; i += MlaCfg::NPROD * 32) idx_s[i] = __ldg(idx_tok + i);
   }
-  return bar.sync();
+  mbar_arrive(stage);
+  if (!mbar_wait(stage, phase, ab, 27)) return false;
+  phase ^= 1u;
+  return true;
 }
 
 template <bool kPaged>
@@ -359,6 +367,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       mbar_init(bars + C::B_MASK_FULL + i, C::NPROD);
       mbar_init(bars + C::B_MASK_FREE + i, 4);
     }
+    mbar_init(bars + C::B_PSTAGE, C::NPROD * 32);
     fence_mbar_init();
   }
   if (warp == C::W_MMA) tmem_alloc(tmem_base_s, 512);
@@ -383,7 +392,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       int slot = 0;
       uint32_t ph = 1;
       int n = 0;  // tokens done by this cluster
-      const GroupBar pbar{1, C::NPROD * 32, ab};  // the producer warps (abort-safe: see GroupBar)
+      uint32_t stage_ph = 0;  // phase of the producers' staging barrier
       // thread 0: where the last token's Q tiles start in the ring and how
       // many it loaded, so that an abort can still wait for its copies in flight
       int q_slot0 = 0;
@@ -397,7 +406,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
         const int mb = n & 1;
         if (!mbar_wait(bars + C::B_MASK_FREE + mb, ((n >> 1) & 1) ^ 1, ab, 30)) break;
         if (!stage_index_row(idx_s, p.idx ? p.idx + static_cast<size_t>(tk) * p.K : nullptr, p.K, ptid,
-                             p.causal_q0 + tk, pbar))
+                             p.causal_q0 + tk, bars + C::B_PSTAGE, stage_ph, ab))
           break;
         // validity bits of every selection entry, 32 per word (entry e -> word e/32)
         for (int wd = static_cast<int>(warp); wd < nchunk * (C::NK / 32); wd += C::NPROD) {
@@ -458,8 +467,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
           mbar_wait(bars + C::B_RING_FULL + pos % C::NSST, full_par, no_abort, 28);
         }
       }
-      __syncwarp();
-      if (pbar.aborted()) pbar.leave();  // count this warp in at the barrier the others may wait at
     } else if (warp == C::W_MMA) {
       // The whole warp runs the loop and waits converged; one elected lane
       // issues each slab's MMAs together with every commit that covers them.
@@ -651,13 +658,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       const int ptid = threadIdx.x;
       int slot = 0;
       uint32_t ph = 1;
-      const GroupBar pbar{1, C::NPROD * 32, ab};  // the producer warps (abort-safe: see GroupBar)
+      uint32_t stage_ph = 0;  // phase of the producers' staging barrier
       for (int tk = cluster_id; tk < p.T; tk += nclusters) {
         const __nv_bfloat16* kv_tok;
         int trows;
         token_cache(p, tk, kv_tok, trows);
         if (!stage_index_row(idx_s, p.idx ? p.idx + static_cast<size_t>(tk) * p.K : nullptr, p.K, ptid,
-                             p.causal_q0 + tk, pbar))
+                             p.causal_q0 + tk, bars + C::B_PSTAGE, stage_ph, ab))
           break;
         bool ok = true;
         for (int j = 0; j < nchunk && ok; ++j) {
@@ -671,7 +678,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
         if (!ok) break;
       }
       asm volatile("cp.async.wait_all;" ::: "memory");
-      if (pbar.aborted()) pbar.leave();  // count this warp in at the barrier the others may wait at
     } else if (warp == C::W_MMA) {
       // whole warp waits converged; one elected lane issues and commits
       int slot = 0;
