@@ -10,15 +10,17 @@
 //
 // Mapping onto tcgen05 (kind::f8f6f4, fp32 accumulator in TMEM):
 //   D[key, (token, head)] = K_tile[128 keys x d_I] * Q_half[(token, head) x d_I]^T
-// i.e. keys in M (128 TMEM lanes) and (token, head) in N (256 columns). Each
+// i.e. keys in M (128 TMEM lanes) and (token, head) in N (128 columns, two
+// tokens of 64 heads). Four such accumulator buffers fill the 512 TMEM
+// columns; each is drained by its own four epilogue warps (one per TMEM lane
+// quarter), so the tensor core fills one buffer while the others drain. Each
 // epilogue thread owns one key (one TMEM lane) and reduces the H_I heads of a
-// token inside its own registers: no shuffles. Two 256-column accumulators
-// alternate so the tensor core fills one while the epilogue drains the other.
+// token inside its own registers: no shuffles.
 //
-// A CTA is persistent and owns "row blocks" of RB = 2 * 256 / H_I consecutive
-// query tokens, taken longest-first. For a row block it streams every key tile
-// up to the block's last token (TMA, 4-stage ring), so each key tile is reused
-// by RB tokens from shared memory.
+// A CTA is persistent and owns "row blocks" of RB = 4 * 128 / H_I consecutive
+// query tokens (8 at H_I = 64), taken longest-first. For a row block it
+// streams every key tile up to the block's last token (TMA, 4-stage ring), so
+// each key tile is reused by RB tokens from shared memory.
 //
 // Selection (same page, step 4 <1>; deepseek.csdn.net section 2.2): each row
 // keeps a candidate list in the workspace, admitting a key only if its 64-bit
@@ -26,8 +28,8 @@
 // to exactly topk keys by a cooperative radix select and the threshold rises
 // to the cut. Nothing that could still rank in the top-k is ever dropped, and
 // the L x L score matrix never exists anywhere. At the end of a row block each
-// row's exact top-k keys are ranked in shared memory and written as token
-// indices.
+// row's exact top-k keys are ranked in shared memory (a histogram of the
+// keys' high bits, then ranks inside each bin) and written as token indices.
 #pragma once
 
 #include <type_traits>
