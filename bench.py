@@ -323,6 +323,7 @@ def run_ours(a, ws, rank):
     didx = torch.empty((D.B, k), dtype=torch.int32, device=dev)
     dout = torch.empty((D.B, D.Hq, D_V), dtype=torch.bfloat16, device=dev)
     ws_d = torch.empty(dsa.index_topk_decode_workspace_size(D.B, D.L, k), dtype=torch.uint8, device=dev)
+    ws_a = torch.empty(dsa.split_workspace_size(D.B, k), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step(ev=None):
@@ -337,7 +338,7 @@ def run_ours(a, ws, rank):
         dsa.index_topk_decode(D.q_I, D.q_scale, D.w, D.k_cache, D.k_scale, D.lens, k, idx=didx, workspace=ws_d)
         if ev:
             ev[3].record(stream)
-        dsa.sparse_mla_attn_decode(D.q, D.kv, didx, D.scale, out=dout)
+        dsa.sparse_mla_attn_decode(D.q, D.kv, didx, D.scale, out=dout, workspace=ws_a)
         if ev:
             ev[4].record(stream)
 
@@ -398,7 +399,7 @@ def run_ours(a, ws, rank):
         "roofline": dict(rl[dom], kernel=dom),
         "roofline_all": rl,
         "peaks": {"source": pk["source"], "fp8": "2 x bf16_tflops_sustained"},
-        "gpu_launches": 6 * a.steps,  # prefill: indexer (main + re-run pass), attention; decode: scores, select, attention
+        "gpu_launches": 7 * a.steps,  # prefill: indexer (main + re-run pass), attention; decode: scores, select, attention, combine
         "clocks": clocks,
         "wall_s_timed": t_wall,
     }
@@ -500,6 +501,7 @@ def run_e2e_decode(a, dsa, D, didx, dout, ws_d, ws, dev):
     except Exception as e:
         return {"value": None, "unit": "tokens/s", "error": f"{type(e).__name__}: {e}"}
     dev_bufs = {n: getattr(D, n) for n in names}
+    ws_a = torch.empty(dsa.split_workspace_size(D.B, D.topk), dtype=torch.uint8, device=dev)
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = dout.numel() * dout.element_size()
     stream = torch.cuda.current_stream(dev)
@@ -510,7 +512,7 @@ def run_e2e_decode(a, dsa, D, didx, dout, ws_d, ws, dev):
         for n, t in host.items():
             dev_bufs[n].copy_(t, non_blocking=True)
         dsa.index_topk_decode(D.q_I, D.q_scale, D.w, D.k_cache, D.k_scale, D.lens, D.topk, idx=didx, workspace=ws_d)
-        dsa.sparse_mla_attn_decode(D.q, D.kv, didx, D.scale, out=dout)
+        dsa.sparse_mla_attn_decode(D.q, D.kv, didx, D.scale, out=dout, workspace=ws_a)
         out_h.copy_(dout, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
@@ -633,23 +635,26 @@ def run_kernel(a):
         kv_pool.view(-1, a.page, D_QK)[perm] = D.kv.reshape(-1, a.page, D_QK)
         table = perm.to(torch.int32).view(B, npg)
         ws = torch.empty(dsa.index_topk_decode_workspace_size(B, DL, k), dtype=torch.uint8, device=dev)
+        ws_a = torch.empty(dsa.split_workspace_size(B, k), dtype=torch.uint8, device=dev)
         idx = torch.empty((B, k), dtype=torch.int32, device=dev)
         out = torch.empty((B, 128, D_V), dtype=torch.bfloat16, device=dev)
 
         def fn():
             dsa.index_topk_decode_paged(D.q_I, D.q_scale, D.w, k_pool, ks_pool, table, D.lens, k,
                                         page_size=a.page, idx=idx, workspace=ws)
-            dsa.sparse_mla_attn_paged(D.q, kv_pool, table, idx, DL, D.scale, page_size=a.page, out=out)
+            dsa.sparse_mla_attn_paged(D.q, kv_pool, table, idx, DL, D.scale, page_size=a.page, out=out,
+                                      split=True, workspace=ws_a)
         shape = {"B": B, "L": DL, "page": a.page}
     else:
         D = workloads.make_decode(B, DL, 64, 128, 128, k, seed=0, device=dev)
         ws = torch.empty(dsa.index_topk_decode_workspace_size(B, DL, k), dtype=torch.uint8, device=dev)
+        ws_a = torch.empty(dsa.split_workspace_size(B, k), dtype=torch.uint8, device=dev)
         idx = torch.empty((B, k), dtype=torch.int32, device=dev)
         out = torch.empty((B, 128, D_V), dtype=torch.bfloat16, device=dev)
 
         def fn():
             dsa.index_topk_decode(D.q_I, D.q_scale, D.w, D.k_cache, D.k_scale, D.lens, k, idx=idx, workspace=ws)
-            dsa.sparse_mla_attn_decode(D.q, D.kv, idx, D.scale, out=out)
+            dsa.sparse_mla_attn_decode(D.q, D.kv, idx, D.scale, out=out, workspace=ws_a)
         shape = {"B": B, "L": DL}
     ms, n = _time_calls(fn, a.repeat, dsa)
     return {"kernel": a.kernel, "ms": ms, "calls_timed": n, "calls": a.repeat, **shape}

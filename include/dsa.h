@@ -200,12 +200,14 @@ dsa_status dsa_sparse_mla_attn_varlen(const uint16_t* q, const uint16_t* kv, con
  * per token, as in decode). idx [T, topk] holds logical rows < rows, with
  * rows <= max_blocks * page_size. Same results as dsa_sparse_mla_attn over
  * the contiguous cache; a page entry outside the pool skips its rows and is
- * reported as DSA_ERR_BAD_INDEX by dsa_get_device_error. Serving layout, no
+ * reported as DSA_ERR_BAD_INDEX by dsa_get_device_error. workspace /
+ * ws_bytes as for dsa_sparse_mla_attn_decode (NULL: whole tokens per
+ * cluster, the better choice for long prefills). Serving layout, no
  * counterpart step in the pages. */
 dsa_status dsa_sparse_mla_attn_paged(const uint16_t* q, const uint16_t* kv_pool, const int32_t* block_table,
                                      const int32_t* idx, int T, int rows, int pool_rows, int bt_stride,
                                      int max_blocks, int page_size, int Hq, int topk, float scale, uint16_t* out,
-                                     float* lse, void* stream);
+                                     float* lse, void* workspace, size_t ws_bytes, void* stream);
 
 /* FP8 quantiser for newly appended tokens (indexer keys or queries): for each
  * of n rows of d fp32 values, scale[r] = absmax/448 (1 for an all-zero row)
@@ -289,9 +291,26 @@ dsa_status dsa_index_scores_decode(const uint8_t* q_I, const float* q_scale, con
                                    float* scores, void* stream);
 
 /*   q [B, Hq, 576] bf16, kv [B, L_max, 576] bf16, idx [B, topk] int32 (rows of
- *   sequence b's cache, -1 = none), out [B, Hq, 512] bf16, lse [B, Hq] f32 or NULL. */
+ *   sequence b's cache, -1 = none), out [B, Hq, 512] bf16, lse [B, Hq] f32 or NULL.
+ *
+ * Split selections (flash-decoding): with a workspace of at least
+ * dsa_sparse_mla_attn_split_workspace_size(B, topk) bytes (device, 16-byte
+ * aligned), a batch small enough to leave at least half of the GPU's 2-SM
+ * clusters idle (2 * B <= clusters; 74 clusters on a 148-SM B200) has its
+ * B x ceil(topk/128) (sequence, 128-entry chunk) units cut into one
+ * contiguous range per cluster, so it still uses every SM; a sequence whose
+ * chunks fall to several clusters gets, from each, its unnormalised output
+ * and softmax statistics in the workspace, and a combine step merges them
+ * (the softmax over the union of the rows). The result equals the unsplit
+ * one up to fp32 rounding order. Larger batches, and workspace NULL, run one
+ * cluster per sequence with no combine step. A workspace given but too small
+ * returns DSA_ERR_WORKSPACE. No counterpart step in the pages (the decode
+ * regime of the cost figure (b) is what it serves). */
+size_t dsa_sparse_mla_attn_split_workspace_size(int T, int topk);
+
 dsa_status dsa_sparse_mla_attn_decode(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int L_max,
-                                      int Hq, int topk, float scale, uint16_t* out, float* lse, void* stream);
+                                      int Hq, int topk, float scale, uint16_t* out, float* lse, void* workspace,
+                                      size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * Decode indexer + top-k with no caller workspace and no allocation.

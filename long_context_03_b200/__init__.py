@@ -61,14 +61,16 @@ def lib() -> ctypes.CDLL:
             L.dsa_dense_mla_attn_causal.argtypes = [P, P, I, I, I, I, F, P, P, P]
             L.dsa_quantize_e4m3_rows.argtypes = [P, I, I, P, P, P]
             L.dsa_rope_quantize_e4m3_rows.argtypes = [P, P, I, I, I, I, ctypes.c_double, I, P, P, P, P]
-            L.dsa_sparse_mla_attn_paged.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, F, P, P, P]
+            L.dsa_sparse_mla_attn_paged.argtypes = [P, P, P, P, I, I, I, I, I, I, I, I, F, P, P, P, SZ, P]
             L.dsa_sparse_mla_attn_varlen.argtypes = [P, P, P, P, P, I, I, I, I, I, F, P, P, P]
             L.dsa_index_topk_decode_workspace_size.argtypes = [I, I, I]
             L.dsa_index_topk_decode_workspace_size.restype = SZ
             L.dsa_index_topk_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P, P, SZ, P]
             L.dsa_index_topk_decode_paged.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, SZ, P]
             L.dsa_index_scores_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, P, P]
-            L.dsa_sparse_mla_attn_decode.argtypes = [P, P, P, I, I, I, I, F, P, P, P]
+            L.dsa_sparse_mla_attn_split_workspace_size.argtypes = [I, I]
+            L.dsa_sparse_mla_attn_split_workspace_size.restype = SZ
+            L.dsa_sparse_mla_attn_decode.argtypes = [P, P, P, I, I, I, I, F, P, P, P, SZ, P]
             L.dsa_index_topk_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P, P]
             L.dsa_get_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_uint)]
             L.dsa_selftest_wait_timeout.argtypes = [ctypes.c_longlong, P]
@@ -291,10 +293,26 @@ def sparse_mla_attn(q, kv, idx, scale: float, *, out=None, lse=None, want_lse: b
     return out, lse
 
 
+def split_workspace_size(T: int, topk: int) -> int:
+    """Bytes of the workspace that lets an attention call split the selections over every SM."""
+    return int(lib().dsa_sparse_mla_attn_split_workspace_size(T, topk))
+
+
+def _split_ws(split: bool, workspace, T: int, topk: int, device):
+    if not split or T == 0:
+        return None, 0
+    if workspace is None:
+        workspace = torch.empty(split_workspace_size(T, topk), dtype=torch.uint8, device=device)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous device tensor")
+    return workspace, workspace.numel() * workspace.element_size()
+
+
 def sparse_mla_attn_paged(q, kv_pool, block_table, idx, rows: int, scale: float, *, page_size: int = 64,
-                          out=None, lse=None, want_lse: bool = False):
+                          out=None, lse=None, want_lse: bool = False, split: bool = False, workspace=None):
     """Attention over a paged latent cache. block_table [T, max_blocks] (one table row per token)
-    or [1, max_blocks] (shared by all tokens); idx holds logical rows < rows."""
+    or [1, max_blocks] (shared by all tokens); idx holds logical rows < rows. split: spread the
+    selections over every SM with a combine step (decode batches; see sparse_mla_attn_decode)."""
     T, Hq, D = q.shape
     pool_rows = kv_pool.shape[0]
     topk = idx.shape[1]
@@ -313,9 +331,10 @@ def sparse_mla_attn_paged(q, kv_pool, block_table, idx, rows: int, scale: float,
         lse = torch.empty((T, Hq), dtype=torch.float32, device=q.device)
     if lse is not None:
         _req(lse, "lse", torch.float32, (T, Hq))
+    ws, ws_bytes = _split_ws(split, workspace, T, topk, q.device)
     _check(lib().dsa_sparse_mla_attn_paged(_ptr(q), _ptr(kv_pool), _ptr(block_table), _ptr(idx), T, rows, pool_rows,
                                            bt_stride, max_blocks, page_size, Hq, topk, float(scale), _ptr(out),
-                                           _ptr(lse), _stream(q.device)))
+                                           _ptr(lse), _ptr(ws), ws_bytes, _stream(q.device)))
     return out, lse
 
 
@@ -493,8 +512,11 @@ def index_scores_decode(q_I, q_scale, w, k_cache, k_scale, lens, *, scores=None)
     return scores
 
 
-def sparse_mla_attn_decode(q, kv, idx, scale: float, *, out=None, lse=None, want_lse: bool = False):
-    """Decode sparse MQA: q [B, Hq, 576], kv [B, L_max, 576] -> out [B, Hq, 512] bf16 (and lse)."""
+def sparse_mla_attn_decode(q, kv, idx, scale: float, *, out=None, lse=None, want_lse: bool = False,
+                           split: bool = True, workspace=None):
+    """Decode sparse MQA: q [B, Hq, 576], kv [B, L_max, 576] -> out [B, Hq, 512] bf16 (and lse).
+    split (default): the (sequence, chunk) work is spread over every SM and a combine step merges
+    the parts; workspace (optional, split_workspace_size(B, topk) bytes) avoids an allocation."""
     B, Hq, D = q.shape
     L_max = kv.shape[1]
     topk = idx.shape[1]
@@ -508,8 +530,9 @@ def sparse_mla_attn_decode(q, kv, idx, scale: float, *, out=None, lse=None, want
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
     if lse is not None:
         _req(lse, "lse", torch.float32, (B, Hq))
+    ws, ws_bytes = _split_ws(split, workspace, B, topk, q.device)
     _check(lib().dsa_sparse_mla_attn_decode(_ptr(q), _ptr(kv), _ptr(idx), B, L_max, Hq, topk, float(scale),
-                                            _ptr(out), _ptr(lse), _stream(q.device)))
+                                            _ptr(out), _ptr(lse), _ptr(ws), ws_bytes, _stream(q.device)))
     return out, lse
 
 

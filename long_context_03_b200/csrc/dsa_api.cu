@@ -109,6 +109,40 @@ dsa_status make_map_q_bf16(CUtensorMap* m, const void* base, int T, int Hq) {
   return DSA_OK;
 }
 
+// Output [T, Hq, 512] bf16 as a 3-D map {512, Hq, T} for bulk tensor
+// stores: boxes of 32 values x 32 heads x 1 token, 64-byte swizzled (heads
+// >= Hq lie outside the map and are not written).
+dsa_status make_map_out_bf16(CUtensorMap* m, const void* base, int T, int Hq) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[3] = {512, static_cast<cuuint64_t>(Hq), static_cast<cuuint64_t>(T)};
+  const cuuint64_t strides[2] = {512 * 2, static_cast<cuuint64_t>(Hq) * 512 * 2};
+  const cuuint32_t box[3] = {32, 32, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled(out) failed (%d)", static_cast<int>(r));
+  return DSA_OK;
+}
+
+// The partial slots' numerators [slots][Hq rows of 512] f32 (slot stride
+// kMlaPartFloats) as a 3-D map {512, Hq, slots}: boxes of 16 values x 32
+// heads x 1 slot, 64-byte swizzled.
+dsa_status make_map_part_f32(CUtensorMap* m, const float* base, int slots, int Hq) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[3] = {512, static_cast<cuuint64_t>(Hq), static_cast<cuuint64_t>(slots)};
+  const cuuint64_t strides[2] = {512 * 4, static_cast<cuuint64_t>(kMlaPartFloats) * 4};
+  const cuuint32_t box[3] = {16, 32, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled(part) failed (%d)", static_cast<int>(r));
+  return DSA_OK;
+}
+
 template <typename K>
 dsa_status set_smem(K kernel, int bytes) {
   const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -120,6 +154,26 @@ dsa_status check_launch(const char* what) {
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, what);
   return DSA_OK;
+}
+
+// Launch as a programmatic dependent of the previous kernel in the stream
+// (programmatic stream serialization): the kernel may be scheduled while
+// that kernel finishes and waits for it (griddep_wait) before touching
+// global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
 // ---- prefill indexer ----
@@ -283,7 +337,9 @@ dsa_status launch_decode_select(const float* scores, const int32_t* lens, int L_
   const int smem = kDecodeSelBinCap * 8 + (2048 + select_scratch_ints(kDecodeSelThreads)) * 4;
   dsa_status s = set_smem(decode_select_kernel, smem);
   if (s != DSA_OK) return s;
-  decode_select_kernel<<<B, kDecodeSelThreads, smem, st>>>(scores, lens, L_max, topk, hist, sel, idx);
+  const cudaError_t e = launch_dependent(decode_select_kernel, dim3(B), dim3(kDecodeSelThreads), smem, st, scores,
+                                         lens, L_max, topk, hist, sel, idx);
+  if (e != cudaSuccess) return cuda_fail(e, "decode_select_kernel launch");
   return check_launch("decode_select_kernel");
 }
 
@@ -308,9 +364,42 @@ struct MlaPacked {  // packed batch: device cu_seqlens of the queries and of the
   const int32_t* cu_k = nullptr;
   int nseq = 0;
 };
+// Co-resident 2-CTA clusters of the attention kernel, looked up once (the
+// same for both instances: same resources); concurrent first calls compute
+// the same value.
+int mla_max_clusters() {
+  static std::atomic<int> cache{0};
+  int n = cache.load(std::memory_order_relaxed);
+  if (n == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * 512, 1, 1);
+    cfg.blockDim = dim3(MlaCfg::NTHREADS, 1, 1);
+    cfg.dynamicSmemBytes = MlaCfg::SMEM_BYTES;
+    if (set_smem(sparse_mla_kernel<false>, MlaCfg::SMEM_BYTES) != DSA_OK ||
+        cudaOccupancyMaxActiveClusters(&n, sparse_mla_kernel<false>, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = num_sms() / 2;
+    }
+    if (n > num_sms() / 2) n = num_sms() / 2;
+    if (n < 1) n = 1;
+    cache.store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
+
+// Partial slots of a split attention call over T tokens: two per cluster.
+size_t mla_split_bytes(int T, int topk) {
+  const long long units = static_cast<long long>(T) * ((topk + MlaCfg::NK - 1) / MlaCfg::NK);
+  const long long gmax = num_sms() / 2 > 1 ? num_sms() / 2 : 1;
+  const long long g = units < gmax ? units : gmax;
+  return static_cast<size_t>(2 * g) * kMlaPartFloats * 4;
+}
+
+// part != null: split the selections over all clusters (flash-decoding) with
+// partial slots in `part` (mla_split_bytes), then the combine step.
 dsa_status launch_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int T, int rows, long long kv_stride,
                       int Hq, int topk, float scale, uint16_t* out, float* lse, cudaStream_t st, int causal_q0 = 0,
-                      MlaPaging pg = MlaPaging(), MlaPacked pk = MlaPacked()) {
+                      MlaPaging pg = MlaPaging(), MlaPacked pk = MlaPacked(), float* part = nullptr) {
   MlaParams p = {};
   p.q = reinterpret_cast<const __nv_bfloat16*>(q);
   p.kv = reinterpret_cast<const __nv_bfloat16*>(kv);
@@ -331,32 +420,55 @@ dsa_status launch_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx,
   p.seq_cu_k = pk.cu_k;
   p.nseq = pk.nseq;
   p.scale_log2 = scale * 1.4426950408889634f;
-  CUtensorMap tmQ;
+  CUtensorMap tmQ, tmO, tmP;
   dsa_status s = make_map_q_bf16(&tmQ, q, T, Hq);
   if (s != DSA_OK) return s;
+  s = make_map_out_bf16(&tmO, out, T, Hq);
+  if (s != DSA_OK) return s;
+  std::memset(&tmP, 0, sizeof(tmP));  // used only by split calls
   auto kern = pg.block_table ? sparse_mla_kernel<true> : sparse_mla_kernel<false>;
   s = set_smem(kern, MlaCfg::SMEM_BYTES);
   if (s != DSA_OK) return s;
-  // co-resident clusters, looked up once (the same for both instances: same
-  // resources); concurrent first calls compute the same value
-  static std::atomic<int> max_clusters_cache{0};
-  int max_clusters = max_clusters_cache.load(std::memory_order_relaxed);
-  if (max_clusters == 0) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * 512, 1, 1);
-    cfg.blockDim = dim3(MlaCfg::NTHREADS, 1, 1);
-    cfg.dynamicSmemBytes = MlaCfg::SMEM_BYTES;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
-      cudaGetLastError();
-      n = num_sms() / 2;
-    }
-    max_clusters = n;
-    max_clusters_cache.store(n, std::memory_order_relaxed);
+  const int max_clusters = mla_max_clusters();
+  const int nchunk = (topk + MlaCfg::NK - 1) / MlaCfg::NK;
+  const long long units = static_cast<long long>(T) * nchunk;
+  // Split only batches that leave at least half of the clusters idle: with
+  // more tokens the whole-token schedule already fills the GPU and a split
+  // would only add partial writes and the combine step.
+  if (2 * T > max_clusters) part = nullptr;
+  p.part = part;
+  const int nclusters = part ? static_cast<int>(units < max_clusters ? units : max_clusters)
+                             : (T < max_clusters ? T : max_clusters);
+  if (part) {
+    s = make_map_part_f32(&tmP, part, 2 * nclusters, Hq);
+    if (s != DSA_OK) return s;
   }
-  const int nclusters = T < max_clusters ? T : max_clusters;
-  kern<<<2 * nclusters, MlaCfg::NTHREADS, MlaCfg::SMEM_BYTES, st>>>(tmQ, p);
-  return check_launch("sparse_mla_kernel");
+  const cudaError_t e = launch_dependent(kern, dim3(2 * nclusters), dim3(MlaCfg::NTHREADS), MlaCfg::SMEM_BYTES, st,
+                                         tmQ, tmO, tmP, p);
+  if (e != cudaSuccess) return cuda_fail(e, "sparse_mla_kernel launch");
+  s = check_launch("sparse_mla_kernel");
+  if (s != DSA_OK || !part) return s;
+  const int nsplit = mla_split_tokens(T, nchunk, nclusters, -1, nullptr);
+  if (nsplit == 0) return DSA_OK;  // every token was held whole by one cluster
+  const dim3 cgrid(nsplit, (Hq + kCombineHeads - 1) / kCombineHeads);
+  const cudaError_t e2 = launch_dependent(mla_combine_kernel, cgrid, dim3(256), 0, st, part, T, nchunk, nclusters,
+                                          Hq, p.out, lse);
+  if (e2 != cudaSuccess) return cuda_fail(e2, "mla_combine_kernel launch");
+  return check_launch("mla_combine_kernel");
+}
+
+// Optional workspace of a split attention call: NULL (unsplit) or at least
+// mla_split_bytes(T, topk) bytes, 16-byte aligned.
+dsa_status check_split_workspace(void* workspace, size_t ws_bytes, int T, int topk, float** part) {
+  *part = nullptr;
+  if (!workspace) return DSA_OK;
+  if (static_cast<long long>(T) * ((topk + MlaCfg::NK - 1) / MlaCfg::NK) >= (1ll << 31))
+    return fail(DSA_ERR_UNSUPPORTED, "T=%d too large for a split call", T);
+  const size_t need = mla_split_bytes(T, topk);
+  if (ws_bytes < need) return fail(DSA_ERR_WORKSPACE, "workspace %zu bytes, need %zu", ws_bytes, need);
+  if (!aligned16(workspace)) return fail(DSA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+  *part = static_cast<float*>(workspace);
+  return DSA_OK;
 }
 
 dsa_status check_mla_args(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int T, int L, int Hq, int topk,
@@ -655,7 +767,7 @@ dsa_status dsa_index_scores(const uint8_t* q_I, const float* q_scale, const floa
 dsa_status dsa_sparse_mla_attn_paged(const uint16_t* q, const uint16_t* kv_pool, const int32_t* block_table,
                                      const int32_t* idx, int T, int rows, int pool_rows, int bt_stride,
                                      int max_blocks, int page_size, int Hq, int topk, float scale, uint16_t* out,
-                                     float* lse, void* stream) {
+                                     float* lse, void* workspace, size_t ws_bytes, void* stream) {
   dsa_status s = check_mla_args(q, kv_pool, idx, T, rows, Hq, topk, scale, out);
   if (s != DSA_OK) return s;
   if (!block_table && T > 0) return fail(DSA_ERR_INVALID_ARG, "null pointer");
@@ -666,12 +778,16 @@ dsa_status dsa_sparse_mla_attn_paged(const uint16_t* q, const uint16_t* kv_pool,
     return fail(DSA_ERR_INVALID_ARG, "pool_rows=%d bt_stride=%d max_blocks=%d page_size=%d rows=%d", pool_rows,
                 bt_stride, max_blocks, page_size, rows);
   if (T == 0) return DSA_OK;
+  float* part = nullptr;
+  s = check_split_workspace(workspace, ws_bytes, T, topk, &part);
+  if (s != DSA_OK) return s;
   MlaPaging pg;
   pg.block_table = block_table;
   pg.bt_stride = bt_stride;
   pg.page_shift = __builtin_ctz(static_cast<unsigned>(page_size));
   pg.pool_rows = pool_rows;
-  return launch_mla(q, kv_pool, idx, T, rows, 0, Hq, topk, scale, out, lse, static_cast<cudaStream_t>(stream), 0, pg);
+  return launch_mla(q, kv_pool, idx, T, rows, 0, Hq, topk, scale, out, lse, static_cast<cudaStream_t>(stream), 0, pg,
+                    MlaPacked(), part);
 }
 
 dsa_status dsa_quantize_e4m3_rows(const float* x, int n, int d, uint8_t* codes, float* scale, void* stream) {
@@ -823,13 +939,22 @@ dsa_status dsa_index_scores_decode(const uint8_t* q_I, const float* q_scale, con
                        static_cast<cudaStream_t>(stream));
 }
 
+size_t dsa_sparse_mla_attn_split_workspace_size(int T, int topk) {
+  if (T <= 0 || topk <= 0) return 0;
+  return mla_split_bytes(T, topk);
+}
+
 dsa_status dsa_sparse_mla_attn_decode(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int L_max,
-                                      int Hq, int topk, float scale, uint16_t* out, float* lse, void* stream) {
+                                      int Hq, int topk, float scale, uint16_t* out, float* lse, void* workspace,
+                                      size_t ws_bytes, void* stream) {
   dsa_status s = check_mla_args(q, kv, idx, B, L_max, Hq, topk, scale, out);
   if (s != DSA_OK) return s;
   if (B == 0) return DSA_OK;
+  float* part = nullptr;
+  s = check_split_workspace(workspace, ws_bytes, B, topk, &part);
+  if (s != DSA_OK) return s;
   return launch_mla(q, kv, idx, B, L_max, static_cast<long long>(L_max) * DSA_D_QK, Hq, topk, scale, out, lse,
-                    static_cast<cudaStream_t>(stream));
+                    static_cast<cudaStream_t>(stream), 0, MlaPaging(), MlaPacked(), part);
 }
 
 // ---- decode indexer + top-k with library-owned scratch ----

@@ -88,6 +88,7 @@ __global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS, 2)
     indexer_decode_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const IdxDecodeParams p) {
   using C = IdxDecodeCfg<HI, DI>;
+  griddep_launch_dependents();  // the selection may be scheduled now; it waits for this grid
   // Persistent: work item i is chunk i % nch of sequence i / nch; each CTA
   // takes a contiguous range of items (so its sequence rarely changes) and
   // keeps its barriers, TMEM and ring phases from one item to the next.
@@ -154,6 +155,9 @@ __global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS, 2)
   };
 
   if (warp == 0) {
+    // the keys stream through once: let them leave L2 first, so the scores
+    // this kernel writes are still there for the selection that reads them
+    const uint64_t kpol = l2_evict_first();
     if constexpr (kPaged) {
       // Paged producer: the whole warp first stages the pool row of the first
       // key of every page the item touches (one round trip for all of them),
@@ -199,7 +203,7 @@ __global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS, 2)
                 const int base = pg_s[(sk >> shift) - fp];
                 if (base >= 0) prow = base + (sk & ((1 << shift) - 1));
               }
-              tma_load_2d(k_s + slot * C::KTILE_BYTES + i * DI, &tmK, k_full + slot, 0, prow);
+              tma_load_2d_hint(k_s + slot * C::KTILE_BYTES + i * DI, &tmK, k_full + slot, 0, prow, kpol);
             }
           }
         }
@@ -227,7 +231,7 @@ __global__ void __launch_bounds__(IdxDecodeCfg<HI, DI>::NTHREADS, 2)
           const int slot = g % C::KST;
           if (!mbar_wait(k_empty + slot, ((g / C::KST) & 1) ^ 1, ab, 11)) { ok = false; break; }
           mbar_arrive_expect_tx(k_full + slot, C::KTILE_BYTES);
-          tma_load_2d(k_s + slot * C::KTILE_BYTES, &tmK, k_full + slot, 0, row0 + kt * C::BM);
+          tma_load_2d_hint(k_s + slot * C::KTILE_BYTES, &tmK, k_full + slot, 0, row0 + kt * C::BM, kpol);
         }
         if (!ok) break;
       }
@@ -623,7 +627,7 @@ __device__ __forceinline__ bool decode_rank_fast(const float* __restrict__ score
   int* small = start + 2048;                                // [64]
   __shared__ int wsum[32];
   __shared__ int res[4];
-  __shared__ int npos, bpos;
+  __shared__ int npos;  // slots taken: keys above the bin (low 16 bits), the bin's keys (high 16)
   __shared__ int never_aborts;  // no bounded waits in this kernel
   const int b = blockIdx.x;
   const int n = min(lens[b], L_max);
@@ -633,7 +637,6 @@ __device__ __forceinline__ bool decode_rank_fast(const float* __restrict__ score
   if (tid == 0) {
     never_aborts = 0;
     npos = 0;
-    bpos = 0;
   }
   const GroupBar bar{1, NT, AbortFlag{&never_aborts}};
   if (n <= K) {  // every key is selected: rank them all (K <= 2048 = 2 per thread)
@@ -685,54 +688,74 @@ __device__ __forceinline__ bool decode_rank_fast(const float* __restrict__ score
   const int above = res[1], inb = res[2];
   if (inb > kDecodeSelBinCap || above > 2048) return false;
   // 3. one pass over the scores: keys above the bin and the bin's keys to
-  //    shared memory (4 keys per thread per round, warp-aggregated appends)
+  //    shared memory (4 keys per thread per round). The loads of PF rounds
+  //    are issued together so their latencies overlap, and a warp reserves
+  //    space for all PF rounds with one shared atomic: keys above the bin
+  //    count in the low 16 bits of `pos`, the bin's keys in the high 16
+  //    (above <= 2048 and inb <= kDecodeSelBinCap were checked, so neither
+  //    field overflows).
   const int lane = tid & 31;
   const bool vec = ((L_max & 3) == 0) && ((reinterpret_cast<uintptr_t>(scores) & 15) == 0);
   const int nround = (n + 4 * NT - 1) / (4 * NT);
-  for (int rd = 0; rd < nround; ++rd) {
-    const int i0 = 4 * (rd * NT + tid);
-    float f[4];
-    if (vec && i0 + 3 < n) {
-      const float4 x = *reinterpret_cast<const float4*>(sc + i0);
-      f[0] = x.x; f[1] = x.y; f[2] = x.z; f[3] = x.w;
-    } else {
+  constexpr int PF = 4;
+  for (int rd0 = 0; rd0 < nround; rd0 += PF) {
+    float f[PF][4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) f[u] = (i0 + u < n) ? sc[i0 + u] : 0.f;
+    for (int q = 0; q < PF; ++q) {
+      const int i0 = 4 * ((rd0 + q) * NT + tid);
+      if (vec && i0 + 3 < n) {
+        const float4 x = *reinterpret_cast<const float4*>(sc + i0);
+        f[q][0] = x.x; f[q][1] = x.y; f[q][2] = x.z; f[q][3] = x.w;
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) f[q][u] = (i0 + u < n) ? sc[i0 + u] : 0.f;
+      }
     }
-    uint64_t key[4];
-    uint32_t hi = 0, eq = 0;
+    uint32_t hi[PF], eq[PF];
+    int excl[PF];  // this lane's first slot of round q within the warp's batch (both fields)
+    int wtot = 0;  // the warp's keys of the batch (both fields)
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      key[u] = rank_key(f[u], static_cast<uint32_t>(i0 + u));
-      const uint32_t bin = key_bin11(key[u]);
-      const bool in = i0 + u < n;
-      hi |= (in && bin > dbin) ? (1u << u) : 0u;
-      eq |= (in && bin == dbin) ? (1u << u) : 0u;
-    }
-    const int mine = __popc(hi) | (__popc(eq) << 16);
-    int incl = mine;
+    for (int q = 0; q < PF; ++q) {
+      const int i0 = 4 * ((rd0 + q) * NT + tid);
+      hi[q] = 0;
+      eq[q] = 0;
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += y;
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t bin = key_bin11(rank_key(f[q][u], static_cast<uint32_t>(i0 + u)));
+        const bool in = i0 + u < n;
+        hi[q] |= (in && bin > dbin) ? (1u << u) : 0u;
+        eq[q] |= (in && bin == dbin) ? (1u << u) : 0u;
+      }
+      const int mine = __popc(hi[q]) | (__popc(eq[q]) << 16);
+      int incl = mine;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      excl[q] = wtot + incl - mine;
+      wtot += __shfl_sync(0xffffffffu, incl, 31);
     }
     int base = 0;
-    if (lane == 31 && incl != 0) {
-      const int th = incl & 0xffff, te = incl >> 16;
-      base = (th ? atomicAdd(&npos, th) : 0) | ((te ? atomicAdd(&bpos, te) : 0) << 16);
-    }
-    base = __shfl_sync(0xffffffffu, base, 31);
-    int ph = (base & 0xffff) + ((incl - mine) & 0xffff);
-    int pe = (base >> 16) + ((incl - mine) >> 16);
+    if (lane == 0 && wtot != 0) base = atomicAdd(&npos, wtot);
+    base = __shfl_sync(0xffffffffu, base, 0);
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      if ((hi >> u) & 1u) {
-        if (ph < 2048) abv[ph] = key[u];
-        ++ph;
-      }
-      if ((eq >> u) & 1u) {
-        if (pe < kDecodeSelBinCap) bin_keys[pe] = key[u];
-        ++pe;
+    for (int q = 0; q < PF; ++q) {
+      const int i0 = 4 * ((rd0 + q) * NT + tid);
+      int ph = (base & 0xffff) + (excl[q] & 0xffff);
+      int pe = (base >> 16) + (excl[q] >> 16);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (((hi[q] | eq[q]) >> u) & 1u) {
+          const uint64_t key = rank_key(f[q][u], static_cast<uint32_t>(i0 + u));
+          if ((hi[q] >> u) & 1u) {
+            if (ph < 2048) abv[ph] = key;
+            ++ph;
+          } else {
+            if (pe < kDecodeSelBinCap) bin_keys[pe] = key;
+            ++pe;
+          }
+        }
       }
     }
   }
@@ -756,6 +779,8 @@ __global__ void __launch_bounds__(kDecodeSelThreads)
     decode_select_kernel(const float* __restrict__ scores, const int32_t* __restrict__ lens, int L_max, int K,
                          const uint32_t* __restrict__ hist_in, uint64_t* __restrict__ sel_keys,
                          int32_t* __restrict__ idx) {
+  griddep_wait();               // launched as a programmatic dependent of the scoring kernel
+  griddep_launch_dependents();  // the attention may be scheduled now; it waits for this grid
   if (decode_rank_fast(scores, lens, L_max, K, hist_in, idx)) return;  // the same answer on every thread
   __syncthreads();
   decode_select_body(scores, lens, L_max, K, hist_in, sel_keys);

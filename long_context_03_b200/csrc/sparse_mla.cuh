@@ -40,6 +40,8 @@
 // also skipped and reported through the device error word.
 #pragma once
 
+#include <type_traits>
+
 #include "dsa_common.cuh"
 
 namespace dsa {
@@ -83,7 +85,11 @@ struct MlaCfg {
   static constexpr int OFF_MSG = OFF_RING + RING_BYTES;    // NPB x MSG_STRIDE (staging / receive)
   static constexpr int OFF_IDX = OFF_MSG + NPB * MSG_STRIDE;  // int32 [KMAX]: the token's index row
   static constexpr int OFF_VMASK = OFF_IDX + KMAX * 4;       // score CTA: u32 [2][KMAX/32] validity bits per token
-  static constexpr int OFF_BAR = OFF_VMASK + 2 * (KMAX / 32) * 4;
+  // value CTA: output staging for the bulk tensor stores, two 2 KB tiles
+  // (32 rows x 64 bytes, 64-byte swizzled) per epilogue warp
+  static constexpr int EPI_TILE = 2048;
+  static constexpr int OFF_EPI = (OFF_VMASK + 2 * (KMAX / 32) * 4 + 1023) / 1024 * 1024;
+  static constexpr int OFF_BAR = OFF_EPI + 4 * 2 * EPI_TILE;
   // barriers
   static constexpr int NRING = (NSST > NVST) ? NSST : NVST;
   static constexpr int B_RING_FULL = 0;                     // [NRING]
@@ -132,6 +138,85 @@ struct MlaParams {
   const int32_t* seq_cu_k;
   int nseq;
   float scale_log2;          // softmax scale * log2(e)
+  // Split selections (flash-decoding): when part is set, the T x nchunk
+  // (token, 128-entry chunk) units are cut into one contiguous range per
+  // cluster, so a token's chunks may be spread over several clusters. A
+  // cluster that holds only part of a token writes that part's unnormalised
+  // fp32 output and its softmax statistics to a partial slot (see
+  // mla_part_slot) instead of `out`; mla_combine_kernel merges the parts.
+  float* part;
+};
+
+// A partial slot: O[128 heads][512] f32 (softmax numerators, scaled by
+// 2^-m), then m[128] (reference maxima, log2 units) and l[128] (row sums).
+constexpr int kMlaPartFloats = 128 * 512 + 2 * 128;
+
+// First unit of cluster g when U units are cut into G contiguous ranges.
+__host__ __device__ __forceinline__ long long mla_unit_start(int g, long long U, int G) {
+  return (static_cast<long long>(g) * U) / G;
+}
+// The cluster whose range holds unit u.
+__host__ __device__ __forceinline__ int mla_unit_owner(long long u, long long U, int G) {
+  return static_cast<int>(((u + 1) * G - 1) / U);
+}
+
+// One piece of work of a cluster: token tk, chunks [c0, c1). slot < 0: the
+// cluster holds the whole token and writes its output; else the partial slot
+// it writes: 2g for its first piece, 2g + 1 for its last.
+struct MlaSeg {
+  int tk, c0, c1, slot;
+};
+// The pieces of cluster g in order. Whole tokens g, g + G, ... without
+// splitting; the range [start(g), start(g + 1)) of (token, chunk) units with it.
+struct MlaSegIter {
+  int u, u0, u1;  // units (T * nchunk < 2^31, checked by the host)
+  int g, G, nchunk, T;
+  bool split;
+  __device__ __forceinline__ MlaSegIter(const MlaParams& p, int g_, int G_, int nchunk_)
+      : g(g_), G(G_), nchunk(nchunk_), T(p.T), split(p.part != nullptr) {
+    if (split) {
+      const long long U = static_cast<long long>(p.T) * nchunk;
+      u0 = static_cast<int>(mla_unit_start(g, U, G));
+      u1 = static_cast<int>(mla_unit_start(g + 1, U, G));
+      u = u0;
+    } else {
+      u = g;
+      u0 = u1 = 0;
+    }
+  }
+  __device__ __forceinline__ bool next(MlaSeg& s) {
+    if (split) {
+      if (u >= u1) return false;
+      s.tk = u / nchunk;
+      s.c0 = u - s.tk * nchunk;
+      s.c1 = min(nchunk, s.c0 + (u1 - u));
+      s.slot = (s.c0 == 0 && s.c1 == nchunk) ? -1 : (u == u0 ? 2 * g : 2 * g + 1);
+      u += s.c1 - s.c0;
+      return true;
+    }
+    if (u >= T) return false;
+    s.tk = u;
+    s.c0 = 0;
+    s.c1 = nchunk;
+    s.slot = -1;
+    u += G;
+    return true;
+  }
+  // token of the piece next() returns next, or -1 at the end
+  __device__ __forceinline__ int next_token() const {
+    if (split) return u < u1 ? u / nchunk : -1;
+    return u < T ? u : -1;
+  }
+  // P messages (one per chunk) this cluster sends, and whether message i
+  // is the last chunk of its piece (it then carries the row sums and maxima)
+  __device__ __forceinline__ int messages() const {
+    return split ? u1 - u0 : (g < T ? ((T - 1 - g) / G + 1) * nchunk : 0);
+  }
+  __device__ __forceinline__ bool last_of_piece(int i) const {
+    if (!split) return (i % nchunk) == nchunk - 1;
+    const int uu = u0 + i;
+    return (uu % nchunk) == nchunk - 1 || uu == u1 - 1;
+  }
 };
 
 // First row and row count of token tk's cache.
@@ -321,9 +406,14 @@ __device__ __forceinline__ bool stage_index_row(int32_t* idx_s, const int32_t* _
   return true;
 }
 
+// tmO: out [T, Hq, 512] bf16 as {512, Hq, T}, boxes of 32 values x 32 heads,
+// 64-byte swizzled. tmP (split selections only): the partial slots'
+// numerators as {512, Hq, slots} f32 with a slot stride of kMlaPartFloats,
+// boxes of 16 values x 32 heads, 64-byte swizzled.
 template <bool kPaged>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
-    sparse_mla_kernel(const __grid_constant__ CUtensorMap tmQ, const MlaParams p) {
+    sparse_mla_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+                      const __grid_constant__ CUtensorMap tmP, const MlaParams p) {
   using C = MlaCfg;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -339,7 +429,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
   const int cluster_id = blockIdx.x >> 1;
   const int nclusters = gridDim.x >> 1;
   const int nchunk = (p.K + C::NK - 1) / C::NK;
-  const int total_msgs = ((p.T - 1 - cluster_id) / nclusters + 1) * nchunk;  // messages this cluster sends
+  const MlaSegIter segs0(p, cluster_id, nclusters, nchunk);  // every role walks its own copy
+  const int total_msgs = segs0.messages();                    // messages this cluster sends
 
   if (threadIdx.x == 0) {
     *abort_s = 0;
@@ -372,14 +463,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
   }
   if (warp == C::W_MMA) tmem_alloc(tmem_base_s, 512);
   __syncthreads();
+  griddep_launch_dependents();  // a combine step may be scheduled now; it waits for this grid
   // Value CTA: arm the first use of each P receive buffer before the peer can send.
   if (rank == 1 && threadIdx.x == 0) {
     for (int i = 0; i < C::NPB && i < total_msgs; ++i) {
-      const bool last = ((i % nchunk) == nchunk - 1);
+      const bool last = segs0.last_of_piece(i);
       mbar_arrive_expect_tx(bars + C::B_P_FULL + i, last ? C::MSG_BYTES_LAST : C::MSG_BYTES_MID);
     }
   }
   cluster_sync_all();
+  // Launched as a programmatic dependent, the kernel got here (barriers,
+  // TMEM, cluster) while the previous kernel was finishing; nothing of
+  // global memory is touched before this wait.
+  griddep_wait();
   tc_fence_after();
   const uint32_t tmem = *tmem_base_s;
   const uint32_t ring = smem_u32(smem + C::OFF_RING);
@@ -398,13 +494,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       int q_slot0 = 0;
       uint32_t q_ph0 = 1;
       int q_issued = 0;
-      for (int tk = cluster_id; tk < p.T; tk += nclusters, ++n) {
+      MlaSegIter segs = segs0;
+      MlaSeg sg;
+      for (; segs.next(sg); ++n) {
+        const int tk = sg.tk;
         const __nv_bfloat16* kv_tok;
         int trows;
         token_cache(p, tk, kv_tok, trows);
-        // the softmax warps are done with this mask buffer (two tokens back)
+        bool ok = true;
+        // Q[tk] first, before the index row (it does not depend on it): nine
+        // 16 KB tiles (128 heads x 64 values, 128-byte swizzled, heads >= Hq
+        // zero) through the ring by TMA; the MMA warp copies them into TMEM.
+        // Thread 0 arms the slot with the bytes, the other producer threads
+        // arrive, as for a gathered tile.
+        q_slot0 = slot;
+        q_ph0 = ph;
+        q_issued = 0;
+        for (int i = 0; i < C::NSLAB_QK; ++i) {
+          if (!mbar_wait(bars + C::B_RING_EMPTY + slot, ph, ab, 29)) { ok = false; break; }
+          if (ptid == 0) {
+            mbar_arrive_expect_tx(bars + C::B_RING_FULL + slot, C::SLAB_TILE);
+            tma_load_3d(smem + C::OFF_RING + slot * C::SLAB_TILE, &tmQ, bars + C::B_RING_FULL + slot, i * 64, 0, tk);
+            q_issued = i + 1;
+          } else {
+            mbar_arrive(bars + C::B_RING_FULL + slot);
+          }
+          if (++slot == C::NSST) { slot = 0; ph ^= 1; }
+        }
+        // the softmax warps are done with this mask buffer (two pieces back)
         const int mb = n & 1;
-        if (!mbar_wait(bars + C::B_MASK_FREE + mb, ((n >> 1) & 1) ^ 1, ab, 30)) break;
+        if (!ok || !mbar_wait(bars + C::B_MASK_FREE + mb, ((n >> 1) & 1) ^ 1, ab, 30)) break;
         if (!stage_index_row(idx_s, p.idx ? p.idx + static_cast<size_t>(tk) * p.K : nullptr, p.K, ptid,
                              p.causal_q0 + tk, bars + C::B_PSTAGE, stage_ph, ab))
           break;
@@ -423,26 +542,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(bars + C::B_MASK_FULL + mb);
-        bool ok = true;
-        // Q[tk] first: nine 16 KB tiles (128 heads x 64 values, 128-byte
-        // swizzled, heads >= Hq zero) through the ring by TMA; the MMA warp
-        // copies them into TMEM. Thread 0 arms the slot with the bytes, the
-        // other producer threads arrive, as for a gathered tile.
-        q_slot0 = slot;
-        q_ph0 = ph;
-        q_issued = 0;
-        for (int i = 0; i < C::NSLAB_QK; ++i) {
-          if (!mbar_wait(bars + C::B_RING_EMPTY + slot, ph, ab, 29)) { ok = false; break; }
-          if (ptid == 0) {
-            mbar_arrive_expect_tx(bars + C::B_RING_FULL + slot, C::SLAB_TILE);
-            tma_load_3d(smem + C::OFF_RING + slot * C::SLAB_TILE, &tmQ, bars + C::B_RING_FULL + slot, i * 64, 0, tk);
-            q_issued = i + 1;
-          } else {
-            mbar_arrive(bars + C::B_RING_FULL + slot);
-          }
-          if (++slot == C::NSST) { slot = 0; ph ^= 1; }
-        }
-        for (int j = 0; j < nchunk && ok; ++j) {
+        for (int j = sg.c0; j < sg.c1 && ok; ++j) {
           const ChunkRows cr = chunk_rows<kPaged>(p, kv_tok, tk, idx_s, j, p.K, trows, ptid);
           for (int i = 0; i < C::NSLAB_QK; ++i) {
             if (!mbar_wait(bars + C::B_RING_EMPTY + slot, ph, ab, 31)) { ok = false; break; }
@@ -475,8 +575,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       uint32_t sph = 1;
       uint32_t qfree_ph = 1;
       bool ok = true;
-      for (int tk = cluster_id; tk < p.T && ok; tk += nclusters) {
-        // Q[tk] into TMEM once the previous token's QK^T has read the old Q
+      MlaSegIter segs = segs0;
+      MlaSeg sg;
+      while (ok && segs.next(sg)) {
+        // Q[tk] into TMEM once the previous piece's QK^T has read the old Q
         if (!mbar_wait_warp(bars + C::B_Q_FREE, qfree_ph, ab, 32)) break;
         qfree_ph ^= 1;
         tc_fence_after();
@@ -494,7 +596,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
           if (++slot == C::NSST) { slot = 0; ph ^= 1; }
         }
         if (!ok) break;
-        for (int j = 0; j < nchunk && ok; ++j) {
+        for (int j = sg.c0; j < sg.c1 && ok; ++j) {
           if (!mbar_wait_warp(bars + C::B_S_EMPTY, sph, ab, 34)) { ok = false; break; }
           sph ^= 1;
           tc_fence_after();
@@ -512,7 +614,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
               tc_commit(bars + C::B_RING_EMPTY + slot);
               if (i == C::NSLAB_QK - 1) {
                 tc_commit(bars + C::B_S_FULL);
-                if (j == nchunk - 1) tc_commit(bars + C::B_Q_FREE);
+                if (j == sg.c1 - 1) tc_commit(bars + C::B_Q_FREE);
               }
             }
             __syncwarp();
@@ -533,12 +635,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       uint32_t pfree_ph = 1;
       uint32_t stage_ph = 0;
       bool ok = true;
-      int n = 0;  // tokens done by this cluster
-      for (int tk = cluster_id; tk < p.T && ok; tk += nclusters, ++n) {
+      int n = 0;  // pieces done by this cluster
+      MlaSegIter segs = segs0;
+      MlaSeg sg;
+      for (; ok && segs.next(sg); ++n) {
         // Q[tk] reaches TMEM through the ring (TMA + tcgen05.cp by the MMA warp)
-        if (tk + nclusters < p.T && h == 0) {
-          // warm L2 with the next token's queries
-          const char* nq = reinterpret_cast<const char*>(p.q + static_cast<size_t>(tk + nclusters) * p.Hq * C::D);
+        const int ntk = segs.next_token();
+        if (h == 0 && ntk >= 0 && ntk != sg.tk) {
+          // warm L2 with the next piece's queries
+          const char* nq = reinterpret_cast<const char*>(p.q + static_cast<size_t>(ntk) * p.Hq * C::D);
           const uint32_t qbytes = static_cast<uint32_t>(p.Hq) * C::D * 2;
           asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(nq), "r"(qbytes) : "memory");
         }
@@ -548,7 +653,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
         const int mb = n & 1;
         if (!mbar_wait(bars + C::B_MASK_FULL + mb, (n >> 1) & 1, ab, 39)) break;
         const uint4* vm_tok = reinterpret_cast<const uint4*>(vmask_s + mb * (C::KMAX / 32));
-        for (int j = 0; j < nchunk; ++j) {
+        for (int j = sg.c0; j < sg.c1; ++j) {
           // validity of the chunk's 128 entries (the same for every head)
           const uint4 vm4 = vm_tok[j];
           const uint32_t vmask[4] = {vm4.x, vm4.y, vm4.z, vm4.w};
@@ -590,7 +695,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
             m_ref = mc;
             l_sum *= alpha;
           }
-          const bool last = (j == nchunk - 1);
+          const bool last = (j == sg.c1 - 1);
           // staging buffer pb is free once the value CTA's MMA consumed its previous message
           if (!mbar_wait(bars + C::B_P_FREE + pb, pfree_ph, ab, 37)) { ok = false; break; }
           uint8_t* st = smem + C::OFF_MSG + pb * C::MSG_STRIDE;
@@ -659,7 +764,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       int slot = 0;
       uint32_t ph = 1;
       uint32_t stage_ph = 0;  // phase of the producers' staging barrier
-      for (int tk = cluster_id; tk < p.T; tk += nclusters) {
+      MlaSegIter segs = segs0;
+      MlaSeg sg;
+      while (segs.next(sg)) {
+        const int tk = sg.tk;
         const __nv_bfloat16* kv_tok;
         int trows;
         token_cache(p, tk, kv_tok, trows);
@@ -667,7 +775,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
                              p.causal_q0 + tk, bars + C::B_PSTAGE, stage_ph, ab))
           break;
         bool ok = true;
-        for (int j = 0; j < nchunk && ok; ++j) {
+        for (int j = sg.c0; j < sg.c1 && ok; ++j) {
           for (int u = 0; u < C::NK / C::VROWS; ++u) {
             if (!mbar_wait(bars + C::B_RING_EMPTY + slot, ph, ab, 41)) { ok = false; break; }
             gather_value_tile<kPaged>(ring + slot * C::V_TILE, p, kv_tok, tk, idx_s, j, u, p.K, trows, ptid);
@@ -686,14 +794,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       uint32_t pph = 0;
       int use = 0;  // messages consumed, to arm the receive barriers ahead
       bool ok = true;
-      for (int tk = cluster_id; tk < p.T && ok; tk += nclusters) {
-        for (int j = 0; j < nchunk && ok; ++j) {
+      MlaSegIter segs = segs0;
+      MlaSeg sg;
+      while (ok && segs.next(sg)) {
+        for (int j = sg.c0; j < sg.c1 && ok; ++j) {
           if (!mbar_wait_warp(bars + C::B_P_FULL + pb, pph, ab, 43)) { ok = false; break; }
           const uint32_t any_rs =
               reinterpret_cast<const volatile uint32_t*>(smem + C::OFF_MSG + pb * C::MSG_STRIDE + C::MSG_CTRL)[0];
           // A rescale needs O quiescent: commit everything issued so far to
           // QUIESCE; the correction warps wait on it, rescale, then signal O_READY.
-          if (any_rs && j > 0) {
+          if (any_rs && j > sg.c0) {
             if (elect_one()) tc_commit(bars + C::B_QUIESCE);
             __syncwarp();
           }
@@ -712,17 +822,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
 #pragma unroll
                 for (int nh = 0; nh < 2; ++nh) {
                   const uint64_t bd = smem_desc(vbase + nh * 4 * C::VSLAB + kk * 2048, C::VSLAB, 1024, kSw128);
-                  mma_bf16_ss(tmem + nh * 256, ad, bd, C::IDESC_PV, (j > 0 || u > 0 || kk > 0) ? 1u : 0u);
+                  mma_bf16_ss(tmem + nh * 256, ad, bd, C::IDESC_PV, (j > sg.c0 || u > 0 || kk > 0) ? 1u : 0u);
                 }
               }
               tc_commit(bars + C::B_RING_EMPTY + slot);
               if (u == C::NK / C::VROWS - 1) {
                 tc_commit_mc(bars + C::B_P_FREE + pb, 0x1);  // the score CTA's buffer pb is free
-                if (j == nchunk - 1) tc_commit(bars + C::B_PV_DONE);
+                if (j == sg.c1 - 1) tc_commit(bars + C::B_PV_DONE);
                 // re-arm this receive buffer for message use + NPB
                 const int nxt = use + C::NPB;
                 if (nxt < total_msgs) {
-                  const bool lastm = ((nxt % nchunk) == nchunk - 1);
+                  const bool lastm = segs0.last_of_piece(nxt);
                   mbar_arrive_expect_tx(bars + C::B_P_FULL + pb, lastm ? C::MSG_BYTES_LAST : C::MSG_BYTES_MID);
                 }
               }
@@ -744,18 +854,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
       uint32_t pph = 0;
       uint32_t pv_ph = 0;
       uint32_t qz_ph = 0;
+      uint32_t epi_n = 0;  // staging tiles used by this warp (tile epi_n & 1 is next)
       bool ok = true;
-      for (int tk = cluster_id; tk < p.T && ok; tk += nclusters) {
+      MlaSegIter segs = segs0;
+      MlaSeg sg;
+      while (ok && segs.next(sg)) {
+        const int tk = sg.tk;
         float l_fin = 0.f, m_fin = -INFINITY;
-        for (int j = 0; j < nchunk; ++j) {
+        for (int j = sg.c0; j < sg.c1; ++j) {
           if (!mbar_wait(bars + C::B_P_FULL + pb, pph, ab, 45)) { ok = false; break; }
           const uint8_t* mb = smem + C::OFF_MSG + pb * C::MSG_STRIDE;
           const uint32_t any_rs = reinterpret_cast<const volatile uint32_t*>(mb + C::MSG_CTRL)[0];
-          if (j == nchunk - 1) {
+          if (j == sg.c1 - 1) {
             l_fin = reinterpret_cast<const float*>(mb + C::MSG_L)[h];
             m_fin = reinterpret_cast<const float*>(mb + C::MSG_M)[h];
           }
-          if (any_rs && j > 0) {
+          if (any_rs && j > sg.c0) {
             const float alpha = reinterpret_cast<const float*>(mb + C::MSG_ALPHA)[h];
             if (!mbar_wait(bars + C::B_QUIESCE, qz_ph, ab, 46)) { ok = false; break; }
             qz_ph ^= 1;
@@ -780,38 +894,237 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg::NTHREADS, 1)
         if (!mbar_wait(bars + C::B_PV_DONE, pv_ph, ab, 47)) break;
         pv_ph ^= 1;
         tc_fence_after();
+        // The output leaves by bulk tensor stores: a warp writes 64-byte row
+        // segments of its 32 rows (heads) into one of its two staging tiles
+        // (64-byte swizzle: 16-byte chunk c of row r at c ^ ((r >> 1) & 3)),
+        // and one lane stores the tile, so the global writes take no
+        // load/store-unit issue and each staging tile is reused once its
+        // store has read it. A whole token gets u = O / l in bf16 (32 values
+        // per tile); part of a token (a split selection) gets its
+        // unnormalised fp32 numerators (16 values per tile) in the piece's
+        // partial slot and its statistics, for the combine step.
+        const bool partial = sg.slot >= 0;
         const bool empty = !(l_fin > 0.f);
-        const float inv = empty ? 0.f : 1.f / l_fin;
-        uint4* orow = reinterpret_cast<uint4*>(p.out + (static_cast<size_t>(tk) * p.Hq + (h < p.Hq ? h : 0)) * C::DV);
-#pragma unroll 1
-        for (int cb = 0; cb < C::DV / 32; ++cb) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_addr + cb * 32, r);  // whole warp (aligned op); only real heads store
-          if (h < p.Hq) {
+        const float inv = partial ? 1.f : (empty ? 0.f : 1.f / l_fin);
+        uint8_t* stage = smem + C::OFF_EPI + quarter * 2 * C::EPI_TILE;
+        const uint32_t swz = (lane >> 1) & 3u;
+        auto emit = [&](const uint32_t (&w4)[4][4], int x) {  // 64 bytes of this lane's row, at value x
+          uint8_t* buf = stage + (epi_n & 1) * C::EPI_TILE;
+          if (lane == 0) bulk_wait_read_1();  // the store issued from this tile two tiles ago has read it
+          __syncwarp();
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 o;
-              o.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]) * inv, __uint_as_float(r[8 * v + 1]) * inv);
-              o.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]) * inv, __uint_as_float(r[8 * v + 3]) * inv);
-              o.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]) * inv, __uint_as_float(r[8 * v + 5]) * inv);
-              o.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]) * inv, __uint_as_float(r[8 * v + 7]) * inv);
-              orow[cb * 4 + v] = o;
+          for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4*>(buf + lane * 64 + ((c ^ swz) << 4)) =
+                make_uint4(w4[c][0], w4[c][1], w4[c][2], w4[c][3]);
+          fence_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            if (quarter * 32 < p.Hq) {  // a box wholly past the last head has nothing to write
+              if (partial) tma_store_3d(&tmP, buf, x, quarter * 32, sg.slot);
+              else tma_store_3d(&tmO, buf, x, quarter * 32, tk);
             }
+            bulk_commit();
+          }
+          ++epi_n;
+        };
+        auto store_block = [&](int cb, const uint32_t (&r)[32]) {
+          uint32_t w4[4][4];
+          if (partial) {
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+              for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) w4[c][e] = r[16 * hf + 4 * c + e];
+              emit(w4, cb * 32 + 16 * hf);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                w4[c][e] = pack_bf16x2(__uint_as_float(r[8 * c + 2 * e]) * inv, __uint_as_float(r[8 * c + 2 * e + 1]) * inv);
+            emit(w4, cb * 32);
+          }
+        };
+        // the next block's TMEM load is in flight while a block is stored
+        uint32_t ra[32], rb[32];
+        tmem_ld32_nowait(tmem + lane_addr, ra);
+        tmem_ld_wait_fence(ra);
+#pragma unroll 1
+        for (int cb = 0; cb < C::DV / 32; cb += 2) {
+          tmem_ld32_nowait(tmem + lane_addr + (cb + 1) * 32, rb);
+          store_block(cb, ra);
+          tmem_ld_wait_fence(rb);
+          if (cb + 2 < C::DV / 32) tmem_ld32_nowait(tmem + lane_addr + (cb + 2) * 32, ra);
+          store_block(cb + 1, rb);
+          if (cb + 2 < C::DV / 32) tmem_ld_wait_fence(ra);
+        }
+        float* part = partial ? p.part + static_cast<size_t>(sg.slot) * kMlaPartFloats : nullptr;
+        if (h < p.Hq) {
+          if (partial) {
+            part[128 * C::DV + h] = m_fin;
+            part[128 * C::DV + 128 + h] = l_fin;
+          } else if (p.lse) {
+            p.lse[static_cast<size_t>(tk) * p.Hq + h] =
+                empty ? -INFINITY : (m_fin + log2f(l_fin)) * 0.69314718055994531f;
           }
         }
-        if (h < p.Hq && p.lse)
-          p.lse[static_cast<size_t>(tk) * p.Hq + h] = empty ? -INFINITY : (m_fin + log2f(l_fin)) * 0.69314718055994531f;
         tc_fence_before();
       }
     }
   }
 
+  // the value CTA's output stores have completed before the CTA leaves
+  if (rank == 1 && warp >= C::W_SM0 && lane == 0) bulk_wait_all();
   __syncthreads();
   cluster_sync_all();
   if (warp == C::W_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+}
+
+// Tokens whose chunks were spread over several clusters: exactly those that
+// hold a cluster boundary start(g), 0 < g < G, strictly inside them. Returns
+// how many there are and, for want >= 0, the want-th of them in *tk.
+__host__ __device__ __forceinline__ int mla_split_tokens(int T, int nchunk, int G, int want, int* tk) {
+  const long long U = static_cast<long long>(T) * nchunk;
+  int n = 0, last = -1;
+  for (int g = 1; g < G; ++g) {
+    const long long u = mla_unit_start(g, U, G);
+    if (u % nchunk == 0) continue;  // a boundary between tokens splits nothing
+    const int t = static_cast<int>(u / nchunk);
+    if (t == last) continue;        // several boundaries inside one token
+    last = t;
+    if (n == want) *tk = t;
+    ++n;
+  }
+  return n;
+}
+
+// Combine step of the split selections: block (j, y) merges the j-th split
+// token (mla_split_tokens) for heads 2y, 2y + 1. Each part i holds numerators
+// O_i = sum 2^(z - m_i) v, sums l_i = sum 2^(z - m_i) and its reference
+// maximum m_i (z = score * scale * log2 e); with M = max_i m_i,
+//     u = sum_i 2^(m_i - M) O_i / sum_i 2^(m_i - M) l_i,
+//     lse = (M + log2 sum_i 2^(m_i - M) l_i) * ln 2,
+// the softmax over the union of the parts' rows. A token whose parts hold no
+// valid row gets u = 0 and lse = -inf, as in the unsplit kernel.
+constexpr int kMlaMaxParts = MlaCfg::KMAX / MlaCfg::NK;  // a part holds at least one chunk
+constexpr int kCombineHeads = 2;                          // heads per block (128 threads each)
+__global__ void __launch_bounds__(256)
+    mla_combine_kernel(const float* __restrict__ part, int T, int nchunk, int G, int Hq,
+                       __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+  __shared__ float wgt[kCombineHeads][kMlaMaxParts];
+  __shared__ int slot_s[kMlaMaxParts];
+  __shared__ int tk_s, np_s;
+  griddep_wait();  // launched as a programmatic dependent of the attention kernel
+  const long long U = static_cast<long long>(T) * nchunk;
+  if (threadIdx.x < 32) {
+    // warp 0 finds the blockIdx.x-th split token: boundary g counts when it
+    // lies strictly inside a token that no earlier boundary lies in
+    const int lane = static_cast<int>(threadIdx.x);
+    int found = -1, seen = 0;
+    for (int g0 = 1; g0 < G && found < 0; g0 += 32) {
+      const int g = g0 + lane;
+      bool first = false;
+      int t = 0;
+      if (g < G) {
+        const long long u = mla_unit_start(g, U, G), up = mla_unit_start(g - 1, U, G);
+        t = static_cast<int>(u / nchunk);
+        first = (u % nchunk != 0) && (g == 1 || up / nchunk != t || up % nchunk == 0);
+      }
+      const uint32_t m = __ballot_sync(0xffffffffu, first);
+      const int want = static_cast<int>(blockIdx.x) - seen;
+      if (want < __popc(m)) {
+        // the want-th set bit of m
+        uint32_t mm = m;
+        for (int k = 0; k < want; ++k) mm &= mm - 1;
+        found = __shfl_sync(0xffffffffu, t, __ffs(mm) - 1);
+      }
+      seen += __popc(m);
+    }
+    int np = 0;
+    if (found >= 0) {
+      const long long a = static_cast<long long>(found) * nchunk;  // the token's units [a, a + nchunk)
+      const int g_lo = mla_unit_owner(a, U, G), g_hi = mla_unit_owner(a + nchunk - 1, U, G);
+      np = g_hi - g_lo + 1;
+      if (np > kMlaMaxParts) np = 0;  // cannot happen: every cluster holds at least one unit
+      if (lane < np) {
+        const int gi = g_lo + lane;
+        // the token is the first piece of a cluster that starts inside it,
+        // else the last piece of the cluster that started before it
+        slot_s[lane] = (mla_unit_start(gi, U, G) >= a) ? 2 * gi : 2 * gi + 1;
+      }
+    }
+    if (lane == 0) {
+      tk_s = found;
+      np_s = np;
+    }
+  }
+  __syncthreads();
+  const int tk = tk_s, np = np_s;
+  if (tk < 0 || np < 2) return;  // (cannot happen: the host launches one block per split token)
+  const int hl = static_cast<int>(threadIdx.x) >> 7;  // head of this thread within the block
+  const int h = blockIdx.y * kCombineHeads + hl;
+  const bool active = h < Hq;  // an odd Hq leaves the last block's second head empty
+  const int t = static_cast<int>(threadIdx.x) & 127;
+  if (active && t < 32) {
+    // the head's weights: lane i takes part i
+    const float* pi = part + static_cast<size_t>(slot_s[min(t, np - 1)]) * kMlaPartFloats + 128 * 512;
+    const float mi = (t < np) ? pi[h] : -INFINITY;
+    const float li = (t < np) ? pi[128 + h] : 0.f;
+    float M = mi;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    const float e = (mi == -INFINITY) ? 0.f : exp2f(mi - M);
+    float Lsum = e * li;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, off);
+    const bool empty = !(Lsum > 0.f);
+    if (t < np) wgt[hl][t] = empty ? 0.f : e / Lsum;
+    if (t == 0 && lse)
+      lse[static_cast<size_t>(tk) * Hq + h] = empty ? -INFINITY : (M + log2f(Lsum)) * 0.69314718055994531f;
+  }
+  __syncthreads();
+  if (!active) return;
+  // four values per thread (coalesced reads and writes); every part's load
+  // is issued before the sums (NP >= np loads, the ones past np re-read the
+  // last part with weight 0)
+  const int d = 4 * t;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  auto merge = [&](auto np_c) {
+    constexpr int NP = decltype(np_c)::value;
+    float4 o[NP];
+    // issued back to back (ordered asm), so all NP loads are in flight together
+#pragma unroll
+    for (int i = 0; i < NP; ++i) {
+      const float* src = part + static_cast<size_t>(slot_s[min(i, np - 1)]) * kMlaPartFloats +
+                         static_cast<size_t>(h) * 512 + d;
+      asm volatile("ld.global.v4.f32 {%0, %1, %2, %3}, [%4];"
+                   : "=f"(o[i].x), "=f"(o[i].y), "=f"(o[i].z), "=f"(o[i].w)
+                   : "l"(src));
+    }
+    // no use of a loaded value before the last load is issued
+#pragma unroll
+    for (int i = 0; i < NP; ++i) asm volatile("" : "+f"(o[i].x), "+f"(o[i].y), "+f"(o[i].z), "+f"(o[i].w));
+#pragma unroll
+    for (int i = 0; i < NP; ++i) {
+      const float wv = (i < np) ? wgt[hl][i] : 0.f;
+      acc.x = __fmaf_rn(wv, o[i].x, acc.x);
+      acc.y = __fmaf_rn(wv, o[i].y, acc.y);
+      acc.z = __fmaf_rn(wv, o[i].z, acc.z);
+      acc.w = __fmaf_rn(wv, o[i].w, acc.w);
+    }
+  };
+  if (np <= 2) merge(std::integral_constant<int, 2>{});
+  else if (np <= 4) merge(std::integral_constant<int, 4>{});
+  else if (np <= 8) merge(std::integral_constant<int, 8>{});
+  else merge(std::integral_constant<int, kMlaMaxParts>{});
+  __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(out + (static_cast<size_t>(tk) * Hq + h) * 512 + d);
+  dst[0] = __floats2bfloat162_rn(acc.x, acc.y);
+  dst[1] = __floats2bfloat162_rn(acc.z, acc.w);
 }
 
 }  // namespace dsa

@@ -105,8 +105,27 @@ def test_paged_attention_argument_checks(lib):
     p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
     f = ctypes.c_float(0.1)
     # page size not a power of two; table too small for the rows
-    assert lib.dsa_sparse_mla_attn_paged(p, p, p, p, 2, 1000, 4096, 16, 16, 48, 16, 8, f, p, None, None) == -2
-    assert lib.dsa_sparse_mla_attn_paged(p, p, p, p, 2, 1000, 4096, 15, 15, 64, 16, 8, f, p, None, None) == -1
+    assert lib.dsa_sparse_mla_attn_paged(p, p, p, p, 2, 1000, 4096, 16, 16, 48, 16, 8, f, p, None, None, 0,
+                                         None) == -2
+    assert lib.dsa_sparse_mla_attn_paged(p, p, p, p, 2, 1000, 4096, 15, 15, 64, 16, 8, f, p, None, None, 0,
+                                         None) == -1
+    # a split workspace that is too small
+    assert lib.dsa_sparse_mla_attn_paged(p, p, p, p, 2, 1000, 4096, 16, 16, 64, 16, 8, f, p, None, p, 16,
+                                         None) == -5
+
+
+def test_split_attention_workspace(lib):
+    p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    f = ctypes.c_float(0.1)
+    one_slot = (128 * 512 + 256) * 4
+    assert lib.dsa_sparse_mla_attn_split_workspace_size(0, 2048) == 0
+    # at least two partial slots, and never more than two per possible cluster
+    n = lib.dsa_sparse_mla_attn_split_workspace_size(64, 2048)
+    assert n >= 2 * one_slot and n % one_slot == 0
+    assert lib.dsa_sparse_mla_attn_split_workspace_size(1, 128) == 2 * one_slot  # one unit: one cluster
+    # (q, kv, idx, B, L_max, Hq, topk, scale, out, lse, workspace, ws_bytes, stream)
+    assert lib.dsa_sparse_mla_attn_decode(p, p, p, 4, 1000, 16, 256, f, p, None, p, 1024, None) == -5
+    assert lib.dsa_sparse_mla_attn_decode(p, p, p, 0, 1000, 16, 256, f, p, None, p, 1024, None) == 0  # nothing to do
 
 
 def test_paged_decode_indexer_argument_checks(lib):

@@ -63,3 +63,34 @@ def test_decode_selection_with_all_scores_tied(dsa):
         assert np.all(sc[b, :n] == sc[b, 0])
         assert np.array_equal(idx[b], np.arange(k, dtype=np.int32))
         assert np.array_equal(idx[b], cpu_topk_of(sc[b:b + 1, :n], [n - 1], k)[0])
+
+
+@pytest.mark.parametrize("B,Hq,lens", [
+    (1, 128, [3001]),                      # one sequence over 16 clusters
+    (3, 16, [2048, 1, 700]),               # a sequence with one row: its other parts are empty
+    (30, 128, None),                       # pieces of about six chunks, sequences over two or three clusters
+    (100, 128, None),                      # a batch that fills the GPU: one cluster per sequence
+])
+def test_split_selections_match_the_oracle(dsa, B, Hq, lens):
+    """Flash-decoding: the (sequence, chunk) work spread over every cluster and
+    combined equals the oracle, and the unsplit call up to rounding."""
+    L, k = 3072, 2048
+    inp = workloads.make_decode(B, L, 64, 128, Hq, k, seed=57, lens=lens)
+    d = inp.to("cuda")
+    idx = dsa.index_topk_decode(d.q_I, d.q_scale, d.w, d.k_cache, d.k_scale, d.lens, k)
+    ws = torch.empty(dsa.split_workspace_size(B, k), dtype=torch.uint8, device="cuda")
+    out, lse = dsa.sparse_mla_attn_decode(d.q, d.kv, idx, inp.scale, want_lse=True, workspace=ws)
+    out1, lse1 = dsa.sparse_mla_attn_decode(d.q, d.kv, idx, inp.scale, want_lse=True, split=False)
+    dsa.check_device_error()
+    ok, mx, rl = attn_close(out, out1.float().cpu().numpy().astype(np.float64), max_abs=8e-3, rel=4e-3)
+    assert ok, (mx, rl)
+    np.testing.assert_allclose(lse.cpu().numpy(), lse1.cpu().numpy(), rtol=1e-5, atol=1e-5)
+    idx_h = idx.cpu().numpy()
+    n_all = inp.lens.numpy() if hasattr(inp.lens, "numpy") else np.asarray(inp.lens)
+    for b in sorted({0, B // 2, B - 1}):
+        n = int(n_all[b])
+        ref_o, ref_l = oracle.sparse_mla(oracle._bf16_bits(inp.q[b:b + 1]), inp.kv[b, :n], idx_h[b:b + 1],
+                                         inp.scale)
+        ok, mx, rl = attn_close(out[b:b + 1], ref_o)
+        assert ok, (b, mx, rl)
+        np.testing.assert_allclose(lse[b].cpu().numpy(), ref_l[0], rtol=1e-4, atol=1e-4)

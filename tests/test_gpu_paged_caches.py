@@ -49,9 +49,15 @@ def test_decode_tables_match_contiguous(dsa):
         base += pool.shape[0] // page
     pool = torch.cat(pools)
     table = torch.stack(tables).cuda()
-    out, lse = dsa.sparse_mla_attn_paged(D.q, pool, table, idx, L, D.scale, page_size=page, want_lse=True)
+    out, lse = dsa.sparse_mla_attn_paged(D.q, pool, table, idx, L, D.scale, page_size=page, want_lse=True,
+                                         split=True)
     dsa.check_device_error()
     assert torch.equal(out, ref) and torch.equal(lse, ref_lse)
+    # one cluster per sequence (no split) in both forms
+    ref1, ref1_lse = dsa.sparse_mla_attn_decode(D.q, D.kv, idx, D.scale, want_lse=True, split=False)
+    out1, lse1 = dsa.sparse_mla_attn_paged(D.q, pool, table, idx, L, D.scale, page_size=page, want_lse=True)
+    dsa.check_device_error()
+    assert torch.equal(out1, ref1) and torch.equal(lse1, ref1_lse)
 
 
 def test_prefill_shared_table_and_bad_page(dsa):
@@ -135,7 +141,8 @@ def test_paged_decode_step_matches_contiguous(dsa):
         src[:m] = D.kv[b, :m]
         kv_pool[rows] = src
     idx = dsa.index_topk_decode_paged(D.q_I, D.q_scale, D.w, k_pool, ks_pool, table, D.lens, 2048, page_size=page)
-    out, lse = dsa.sparse_mla_attn_paged(D.q, kv_pool, table, idx, L, D.scale, page_size=page, want_lse=True)
+    out, lse = dsa.sparse_mla_attn_paged(D.q, kv_pool, table, idx, L, D.scale, page_size=page, want_lse=True,
+                                         split=True)
     dsa.check_device_error()
     assert torch.equal(idx, ref_idx)
     assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
@@ -228,7 +235,8 @@ def test_paged_decode_step_matches_the_oracle(dsa):
         src[:m] = D.kv[b, :m]
         kv_pool[rows] = src
     idx = dsa.index_topk_decode_paged(D.q_I, D.q_scale, D.w, k_pool, ks_pool, table, D.lens, 2048, page_size=page)
-    out, lse = dsa.sparse_mla_attn_paged(D.q, kv_pool, table, idx, L, D.scale, page_size=page, want_lse=True)
+    out, lse = dsa.sparse_mla_attn_paged(D.q, kv_pool, table, idx, L, D.scale, page_size=page, want_lse=True,
+                                         split=True)
     sc = dsa.index_scores_decode(D.q_I, D.q_scale, D.w, D.k_cache, D.k_scale, D.lens)
     dsa.check_device_error()
     host = workloads.DecodeInputs(B, L, 64, 128, 128, 2048, D.scale,
