@@ -105,7 +105,7 @@ struct IdxPrefillParams {
   int32_t* idx;          // [Tq][topk] token indices per row, ranked, -1 padded
   // Sampled starting thresholds: row blocks with t0 >= spec_min_t (0: never)
   // first score NSAMPLE evenly spread key tiles and start from the sample's
-  // r-th largest score (r ~ 2.5 * topk * sampled keys / (t+1)). A row that
+  // r-th largest score (r ~ 2 * topk * sampled keys / (t+1)). A row that
   // ends with fewer than topk keys at or above that start is re-run: its row
   // block index goes to redo_list[atomicAdd(redo_count, 1)].
   int spec_min_t;
@@ -190,12 +190,12 @@ __device__ __forceinline__ int tile_at(int i, int nkt, bool spec) {
   if (i < NS) return ((2 * i + 1) * nkt) / (2 * NS);
   return i - NS;
 }
-// Rank r of the sampled key whose score starts a row's threshold: about 2.5
-// times the row's share of topk among the sampled keys, so that the expected
-// count of keys at or above it is ~2.5 * topk; at least 1, at most n.
+// Rank r of the sampled key whose score starts a row's threshold: twice the
+// row's share of topk among the sampled keys, so that the expected count of
+// keys at or above it is ~2 * topk; at least 1, at most n.
 __device__ __forceinline__ int sample_rank(int topk, int sampled_keys, int t, int n) {
-  const long long num = 5ll * topk * sampled_keys;
-  const long long den = 2ll * (t + 1);
+  const long long num = 2ll * topk * sampled_keys;
+  const long long den = static_cast<long long>(t + 1);
   long long r = (num + den - 1) / den;
   if (r > n) r = n;
   if (r < 1) r = 1;
