@@ -337,6 +337,15 @@ dsa_status launch_decode_select(const float* scores, const int32_t* lens, int L_
   const int smem = kDecodeSelBinCap * 8 + (2048 + select_scratch_ints(kDecodeSelThreads)) * 4;
   dsa_status s = set_smem(decode_select_kernel, smem);
   if (s != DSA_OK) return s;
+  if (hist) {
+    // two CTAs per sequence (a cluster) split the pass over the scores
+    s = set_smem(decode_select_pair_kernel, smem);
+    if (s != DSA_OK) return s;
+    const cudaError_t e = launch_dependent(decode_select_pair_kernel, dim3(2 * B), dim3(kDecodeSelThreads), smem, st,
+                                           scores, lens, L_max, topk, hist, sel, idx);
+    if (e != cudaSuccess) return cuda_fail(e, "decode_select_pair_kernel launch");
+    return check_launch("decode_select_pair_kernel");
+  }
   const cudaError_t e = launch_dependent(decode_select_kernel, dim3(B), dim3(kDecodeSelThreads), smem, st, scores,
                                          lens, L_max, topk, hist, sel, idx);
   if (e != cudaSuccess) return cuda_fail(e, "decode_select_kernel launch");

@@ -140,6 +140,34 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uin
       : "memory");
 }
 
+// ---------------------------------------------------------------------------
+// Thread-block clusters
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Every thread of every CTA of the cluster; shared-memory writes before it
+// (local or to a peer) are visible to the whole cluster after it.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// The shared::cluster address of the same shared-memory location in CTA `peer`.
+__device__ __forceinline__ uint32_t map_to_peer(uint32_t local_saddr, uint32_t peer) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_saddr), "r"(peer));
+  return r;
+}
+__device__ __forceinline__ int atom_add_cluster(uint32_t saddr_cluster, int v) {
+  int old;
+  asm volatile("atom.shared::cluster.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(saddr_cluster), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ void st_cluster_u64(uint32_t saddr_cluster, uint64_t v) {
+  asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(saddr_cluster), "l"(v) : "memory");
+}
+
 // Programmatic dependent launch. A kernel launched as a programmatic
 // dependent may start while the previous kernel in the stream is still
 // running; griddep_wait() returns once that kernel has completed and its

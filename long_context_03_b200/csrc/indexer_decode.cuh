@@ -388,7 +388,7 @@ constexpr int kDecodeSelBinCap = 16384;  // boundary-bin keys kept in shared mem
 
 __device__ __forceinline__ void decode_select_body(const float* __restrict__ scores, const int32_t* __restrict__ lens,
                                                    int L_max, int K, const uint32_t* __restrict__ hist_in,
-                                                   uint64_t* __restrict__ sel_keys) {
+                                                   uint64_t* __restrict__ sel_keys, int b) {
   constexpr int NT = kDecodeSelThreads;
   extern __shared__ __align__(16) uint8_t dsmem[];
   uint64_t* bin_keys = reinterpret_cast<uint64_t*>(dsmem);                          // [kDecodeSelBinCap]
@@ -397,7 +397,6 @@ __device__ __forceinline__ void decode_select_body(const float* __restrict__ sco
   __shared__ int wsum[32];
   __shared__ int res[4];
   __shared__ int wpos, bpos;
-  const int b = blockIdx.x;
   const int n = min(lens[b], L_max);
   const float* sc = scores + static_cast<size_t>(b) * L_max;
   uint64_t* dst = sel_keys + static_cast<size_t>(b) * K;
@@ -614,6 +613,15 @@ constexpr int kDecodeBinRankMax = 256;
 // finer histogram pass (topk_rank_by_bins), which writes the sequence's
 // index row. False when the boundary bin is too large for shared memory or a
 // finer bin is too crowded; nothing is written to idx then.
+//
+// kPair: the two CTAs of a cluster share the sequence (blockIdx.x / 2, the
+// scoring kernel's histogram required): each takes half of the pass over
+// the scores and appends its candidates to CTA 0's shared memory (cluster
+// atomics and stores), and CTA 0 ranks. Both CTAs reach the same decisions
+// (same histogram), so they leave before the cluster barriers together when
+// the fast path does not apply; CTA 1 returns true without writing anything
+// (CTA 0 writes the row).
+template <bool kPair>
 __device__ __forceinline__ bool decode_rank_fast(const float* __restrict__ scores, const int32_t* __restrict__ lens,
                                                  int L_max, int K, const uint32_t* __restrict__ hist_in,
                                                  int32_t* __restrict__ idx) {
@@ -629,7 +637,8 @@ __device__ __forceinline__ bool decode_rank_fast(const float* __restrict__ score
   __shared__ int res[4];
   __shared__ int npos;  // slots taken: keys above the bin (low 16 bits), the bin's keys (high 16)
   __shared__ int never_aborts;  // no bounded waits in this kernel
-  const int b = blockIdx.x;
+  const int b = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const uint32_t crank = kPair ? cluster_ctarank() : 0u;
   const int n = min(lens[b], L_max);
   const float* sc = scores + static_cast<size_t>(b) * L_max;
   int32_t* out = idx + static_cast<size_t>(b) * K;
@@ -640,6 +649,7 @@ __device__ __forceinline__ bool decode_rank_fast(const float* __restrict__ score
   }
   const GroupBar bar{1, NT, AbortFlag{&never_aborts}};
   if (n <= K) {  // every key is selected: rank them all (K <= 2048 = 2 per thread)
+    if (kPair && crank != 0) return true;
     uint64_t v[2];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -687,6 +697,9 @@ __device__ __forceinline__ bool decode_rank_fast(const float* __restrict__ score
   const uint32_t dbin = static_cast<uint32_t>(res[0]);
   const int above = res[1], inb = res[2];
   if (inb > kDecodeSelBinCap || above > 2048) return false;
+  // a pair appends into CTA 0's buffers (addresses mapped where used) once
+  // its counter is set up
+  if constexpr (kPair) cluster_sync_all();
   // 3. one pass over the scores: keys above the bin and the bin's keys to
   //    shared memory (4 keys per thread per round). The loads of PF rounds
   //    are issued together so their latencies overlap, and a warp reserves
@@ -697,12 +710,18 @@ __device__ __forceinline__ bool decode_rank_fast(const float* __restrict__ score
   const int lane = tid & 31;
   const bool vec = ((L_max & 3) == 0) && ((reinterpret_cast<uintptr_t>(scores) & 15) == 0);
   const int nround = (n + 4 * NT - 1) / (4 * NT);
+  // a pair: CTA 0 takes rounds [0, h), CTA 1 rounds [h, nround)
+  const int rhalf = (nround + 1) / 2;
+  const int rbeg = (kPair && crank != 0) ? rhalf : 0;
+  const int rend = kPair ? (crank != 0 ? nround : rhalf) : nround;
+  // rounds past rend read nothing (their i0 is pushed past n)
+  auto first_key = [&](int rd) { return rd < rend ? 4 * (rd * NT + tid) : n; };
   constexpr int PF = 4;
-  for (int rd0 = 0; rd0 < nround; rd0 += PF) {
+  for (int rd0 = rbeg; rd0 < rend; rd0 += PF) {
     float f[PF][4];
 #pragma unroll
     for (int q = 0; q < PF; ++q) {
-      const int i0 = 4 * ((rd0 + q) * NT + tid);
+      const int i0 = first_key(rd0 + q);
       if (vec && i0 + 3 < n) {
         const float4 x = *reinterpret_cast<const float4*>(sc + i0);
         f[q][0] = x.x; f[q][1] = x.y; f[q][2] = x.z; f[q][3] = x.w;
@@ -716,7 +735,7 @@ __device__ __forceinline__ bool decode_rank_fast(const float* __restrict__ score
     int wtot = 0;  // the warp's keys of the batch (both fields)
 #pragma unroll
     for (int q = 0; q < PF; ++q) {
-      const int i0 = 4 * ((rd0 + q) * NT + tid);
+      const int i0 = first_key(rd0 + q);
       hi[q] = 0;
       eq[q] = 0;
 #pragma unroll
@@ -737,11 +756,11 @@ __device__ __forceinline__ bool decode_rank_fast(const float* __restrict__ score
       wtot += __shfl_sync(0xffffffffu, incl, 31);
     }
     int base = 0;
-    if (lane == 0 && wtot != 0) base = atomicAdd(&npos, wtot);
+    if (lane == 0 && wtot != 0) base = kPair ? atom_add_cluster(map_to_peer(smem_u32(&npos), 0), wtot) : atomicAdd(&npos, wtot);
     base = __shfl_sync(0xffffffffu, base, 0);
 #pragma unroll
     for (int q = 0; q < PF; ++q) {
-      const int i0 = 4 * ((rd0 + q) * NT + tid);
+      const int i0 = first_key(rd0 + q);
       int ph = (base & 0xffff) + (excl[q] & 0xffff);
       int pe = (base >> 16) + (excl[q] >> 16);
 #pragma unroll
@@ -749,15 +768,25 @@ __device__ __forceinline__ bool decode_rank_fast(const float* __restrict__ score
         if (((hi[q] | eq[q]) >> u) & 1u) {
           const uint64_t key = rank_key(f[q][u], static_cast<uint32_t>(i0 + u));
           if ((hi[q] >> u) & 1u) {
-            if (ph < 2048) abv[ph] = key;
+            if (ph < 2048) {
+              if (kPair) st_cluster_u64(map_to_peer(smem_u32(abv + ph), 0), key);
+              else abv[ph] = key;
+            }
             ++ph;
           } else {
-            if (pe < kDecodeSelBinCap) bin_keys[pe] = key;
+            if (pe < kDecodeSelBinCap) {
+              if (kPair) st_cluster_u64(map_to_peer(smem_u32(bin_keys + pe), 0), key);
+              else bin_keys[pe] = key;
+            }
             ++pe;
           }
         }
       }
     }
+  }
+  if constexpr (kPair) {
+    cluster_sync_all();  // CTA 1's candidates have landed in CTA 0
+    if (crank != 0) return true;
   }
   __syncthreads();
   // 4. rank the candidates (the ranking buffer reuses the bin keys' space
@@ -781,12 +810,33 @@ __global__ void __launch_bounds__(kDecodeSelThreads)
                          int32_t* __restrict__ idx) {
   griddep_wait();               // launched as a programmatic dependent of the scoring kernel
   griddep_launch_dependents();  // the attention may be scheduled now; it waits for this grid
-  if (decode_rank_fast(scores, lens, L_max, K, hist_in, idx)) return;  // the same answer on every thread
+  if (decode_rank_fast<false>(scores, lens, L_max, K, hist_in, idx)) return;  // the same answer on every thread
   __syncthreads();
-  decode_select_body(scores, lens, L_max, K, hist_in, sel_keys);
+  decode_select_body(scores, lens, L_max, K, hist_in, sel_keys, static_cast<int>(blockIdx.x));
   extern __shared__ __align__(16) uint8_t dsmem[];
   __syncthreads();  // the selected keys (global, this CTA's writes) are complete; the bin buffer is free
   const size_t row = static_cast<size_t>(blockIdx.x) * K;
+  sort_keys_to_idx<kDecodeSelThreads>(reinterpret_cast<uint64_t*>(dsmem), sel_keys + row, K, idx + row);
+}
+
+// The same selection with two CTAs per sequence (a cluster; the scoring
+// kernel's histogram required): the pass over the scores is split between
+// them (decode_rank_fast<true>); when the fast path does not apply, CTA 0
+// runs the single-CTA selection for the sequence alone.
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kDecodeSelThreads)
+    decode_select_pair_kernel(const float* __restrict__ scores, const int32_t* __restrict__ lens, int L_max, int K,
+                              const uint32_t* __restrict__ hist_in, uint64_t* __restrict__ sel_keys,
+                              int32_t* __restrict__ idx) {
+  griddep_wait();               // launched as a programmatic dependent of the scoring kernel
+  griddep_launch_dependents();  // the attention may be scheduled now; it waits for this grid
+  if (decode_rank_fast<true>(scores, lens, L_max, K, hist_in, idx)) return;  // the same answer on every thread
+  if (cluster_ctarank() != 0) return;
+  __syncthreads();
+  const int b = static_cast<int>(blockIdx.x >> 1);
+  decode_select_body(scores, lens, L_max, K, hist_in, sel_keys, b);
+  extern __shared__ __align__(16) uint8_t dsmem[];
+  __syncthreads();  // the selected keys (global, this CTA's writes) are complete; the bin buffer is free
+  const size_t row = static_cast<size_t>(b) * K;
   sort_keys_to_idx<kDecodeSelThreads>(reinterpret_cast<uint64_t*>(dsmem), sel_keys + row, K, idx + row);
 }
 
