@@ -122,7 +122,7 @@ def test_split_attention_workspace(lib):
     # at least two partial slots, and never more than two per possible cluster
     n = lib.dsa_sparse_mla_attn_split_workspace_size(64, 2048)
     assert n >= 2 * one_slot and n % one_slot == 0
-    assert lib.dsa_sparse_mla_attn_split_workspace_size(1, 128) == 2 * one_slot  # one unit: one cluster
+    assert lib.dsa_sparse_mla_attn_split_workspace_size(1, 64) == 2 * one_slot  # one chunk: one cluster
     # (q, kv, idx, B, L_max, Hq, topk, scale, out, lse, workspace, ws_bytes, stream)
     assert lib.dsa_sparse_mla_attn_decode(p, p, p, 4, 1000, 16, 256, f, p, None, p, 1024, None) == -5
     assert lib.dsa_sparse_mla_attn_decode(p, p, p, 0, 1000, 16, 256, f, p, None, p, 1024, None) == 0  # nothing to do
