@@ -322,7 +322,9 @@ __global__ void __launch_bounds__(IdxPrefillCfg<HI, DI>::NTHREADS, 1)
         qe_phase ^= 1;
         mbar_arrive_expect_tx(q_full, C::QBYTES);
         for (int b = 0; b < C::QROWS / C::QBOX; ++b)
-          tma_load_2d(q_s + b * C::QBOX * DI, &tmQ, q_full, 0, r0 * HI + b * C::QBOX);
+          // the query rows are read once: evict-first keeps L2 for the key
+          // tiles (read by every row block) and the candidate lists
+          tma_load_2d_hint(q_s + b * C::QBOX * DI, &tmQ, q_full, 0, r0 * HI + b * C::QBOX, l2_evict_first());
         bool ok = true;
         // paged: one box of R = min(page, BM) rows per page of the tile; the
         // next tile's page entries load before the wait for this tile's slot

@@ -386,9 +386,9 @@ __device__ __forceinline__ bool topk_rank_by_bins(const uint64_t (&v)[M], int K,
     const int s0 = start[b] - cb;
     int r = s0;
     for (int q = s0; q < s0 + cb; ++q) r += (buf[q] > key) ? 1 : 0;
-    if (r < K) dst[r] = rank_key_index(key);
+    if (r < K) __stcs(dst + r, rank_key_index(key));  // streaming store: the index rows are not read back here
   }
-  for (int i = (total > 0 ? total : 0) + et; i < K; i += NT) dst[i] = -1;
+  for (int i = (total > 0 ? total : 0) + et; i < K; i += NT) __stcs(dst + i, -1);
   return true;
 }
 
