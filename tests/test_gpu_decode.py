@@ -69,6 +69,7 @@ def test_decode_selection_with_all_scores_tied(dsa):
     (1, 128, [3001]),                      # one sequence over 16 clusters
     (3, 16, [2048, 1, 700]),               # a sequence with one row: its other parts are empty
     (30, 128, None),                       # pieces of about six chunks, sequences over two or three clusters
+    (5, 17, [3000, 1, 2048, 999, 2500]),   # an odd head count: partial output boxes and a half-used combine block
     (100, 128, None),                      # a batch that fills the GPU: one cluster per sequence
 ])
 def test_split_selections_match_the_oracle(dsa, B, Hq, lens):
