@@ -34,7 +34,7 @@ def test_tiny_all_rows(dsa, tiny):
     np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, rtol=1e-4, atol=1e-4)
 
 
-@pytest.mark.parametrize("Hq,k", [(128, 2048), (128, 96), (64, 256), (1, 32)])
+@pytest.mark.parametrize("Hq,k", [(128, 2048), (128, 96), (64, 256), (1, 32), (17, 200), (100, 2048)])
 def test_heads_and_chunks(dsa, Hq, k):
     L = 3000
     inp = workloads.make_prefill(L, 8, 64, Hq, k, seed=21)
