@@ -58,7 +58,7 @@ METRIC = "DSA prefill tokens/s @128K & decode tok/s, % of FP8/BF16/HBM roofline"
 # indexer entry covers its main and re-run passes; decode entries cover one
 # decode batch.
 MEASURED_TRAFFIC = {
-    "prefill_indexer": 1.2264e9 + 2.7398e9 + 0.0001e9,  # main pass + re-run pass
+    "prefill_indexer": 1.2733e9 + 3.0800e9 + 0.0001e9,  # main pass + re-run pass
     "prefill_attention": None,  # measured on a 2048-row chunk only; does not scale with the token count
     "decode_step": 0.5542e9 + 0.0027e9 + 0.0174e9 + 0.1611e9 + 0.0002e9,
     "decode_indexer": 0.5542e9 + 0.0027e9 + 0.0174e9,
